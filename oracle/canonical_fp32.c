@@ -1,0 +1,90 @@
+/*
+ * ORACLE — test infrastructure only. Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this code; the product path never does.
+ *
+ * fp32 canonical block selector: the single-precision arithmetic, in a fixed
+ * order, in which the selection decision (an integer result decided by floating
+ * point) is taken. Each statement below is one IEEE-754 binary32 operation with
+ * round-to-nearest-even; fmaf() is the correctly rounded fused multiply-add of
+ * C99 (F.10.10.1). Compile with -ffp-contract=off so that no other operation is
+ * fused.
+ *
+ * What it computes (COBS: Cumulant Order Block Sparse Attention, gist.science
+ * explainer of arXiv 2607.09052, §2.2 "Die Kumulanten-Expansion" and §2.3
+ * "Second-Order Scoring"; the per-channel variance form of the covariance term):
+ *
+ *   summaries  mu_{b,c}   = (1/L) sum_r k_{bL+r,c}
+ *              var_{b,c}  = (1/L) sum_r (k_{bL+r,c} - mu_{b,c})^2
+ *   group query  Qsum_c = sum_{h in g} q_{h,c},  Q2_c = sum_{h in g} q_{h,c}^2
+ *   score      S_{g,b} = (sum_c Qsum_c mu_{b,c}) * isd + c2 * (sum_c Q2_c var_{b,c})
+ *              with isd = RN(1/sqrt(d)), c2 = RN(alpha / (2 d)),
+ *   which equals sum_{h in g} [ q_h.mu_b / sqrt(d) + alpha/2 * sum_c q_{h,c}^2 var_{b,c} / d ].
+ *
+ * Order: every sum runs over its index in ascending order starting from +0.
+ */
+#include <math.h>
+#include <stdint.h>
+
+/*
+ * K: [T][d] float32 rows (exact bf16 or fp32 values). Writes out[j][0][c] = mu,
+ * out[j][1][c] = var for the complete blocks j < T / L.
+ */
+void cobs_oracle_summaries_f32(const float* K, int64_t T, int d, int L, float* out) {
+    const int64_t nB = T / L;
+    const float invL = 1.0f / (float)L; /* exact: L is a power of two */
+    for (int64_t j = 0; j < nB; ++j) {
+        for (int c = 0; c < d; ++c) {
+            float s = 0.0f;
+            for (int r = 0; r < L; ++r) s = s + K[(j * L + r) * d + c];
+            const float mu = s * invL;
+            float a = 0.0f;
+            for (int r = 0; r < L; ++r) {
+                const float t = K[(j * L + r) * d + c] - mu;
+                a = fmaf(t, t, a);
+            }
+            out[(j * 2 + 0) * d + c] = mu;
+            out[(j * 2 + 1) * d + c] = a * invL;
+        }
+    }
+}
+
+/* q: [G][d] query heads of one group. Writes qsum[d], q2[d]. */
+void cobs_oracle_group_query_f32(const float* q, int G, int d, float* qsum, float* q2) {
+    for (int c = 0; c < d; ++c) {
+        float s = 0.0f, s2 = 0.0f;
+        for (int h = 0; h < G; ++h) {
+            const float x = q[h * d + c];
+            s = s + x;
+            s2 = fmaf(x, x, s2);
+        }
+        qsum[c] = s;
+        q2[c] = s2;
+    }
+}
+
+/* Score constants: isd = RN32(1/sqrt(d)) (via double), c2 = RN32(alpha * 0.5 / d). */
+void cobs_oracle_score_constants(int d, float alpha, float* isd, float* c2) {
+    *isd = (float)(1.0 / sqrt((double)d));
+    *c2 = (float)((double)alpha * 0.5 / (double)d);
+}
+
+/*
+ * Scores of nq group queries against blocks [0, nb) of one unit.
+ * qsum, q2: [nq][d]; summ: [nb][2][d]; S: [nq][nb].
+ */
+void cobs_oracle_scores_f32(const float* qsum, const float* q2, const float* summ, int64_t nq,
+                            int64_t nb, int d, float isd, float c2, float* S) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nq; ++i) {
+        const float* qs = qsum + i * d;
+        const float* qq = q2 + i * d;
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* mu = summ + (b * 2 + 0) * d;
+            const float* var = summ + (b * 2 + 1) * d;
+            float a = 0.0f, v = 0.0f;
+            for (int c = 0; c < d; ++c) a = fmaf(qs[c], mu[c], a);
+            for (int c = 0; c < d; ++c) v = fmaf(qq[c], var[c], v);
+            S[i * nb + b] = fmaf(c2, v, a * isd);
+        }
+    }
+}

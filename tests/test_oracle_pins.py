@@ -1,0 +1,427 @@
+"""Pins of the oracle against what the pages and the mathematics fix (CPU only).
+
+Each test ties an oracle function to something other than the oracle itself:
+hand-computed or closed-form values, exact rational arithmetic, textbook attention
+from a library, or invariants. A plausible slip (a dropped 1/2, a wrong 1/sqrt(d),
+a transposed operand, a wrong tie rule, an off-by-one block range) fails one of them.
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import cobs_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+# ---------------------------------------------------------------- exact mass, OSA
+
+def test_exact_mass_hand_computed():
+    """COBS §2.1 mass m_b = sum_r exp(q.k_r/sqrt(d)) on a case computed by hand."""
+    rows = _golden_rows("exact_mass_tiny.txt")
+    L, d = 4, 2
+    K = np.zeros((L * len(rows), d))
+    expected = []
+    for j, r in enumerate(rows):
+        a = [float(x) for x in r[1:5]]
+        K[j * L:(j + 1) * L, 0] = np.log(a)
+        K[j * L:(j + 1) * L, 1] = [0.3, -1.0, 2.0, 5.0]   # orthogonal to q: must not matter
+        expected.append(float(r[5]))
+    q = np.array([math.sqrt(2.0), 0.0])
+    got = O.exact_log_mass(q, K, L)
+    np.testing.assert_allclose(got, expected, rtol=0, atol=1e-12)
+    # oracle sparse attention picks the blocks of largest mass (block 3, then the tie 0/2 -> 0)
+    assert list(O.osa_top_k(q[None], K, L, len(rows), 2)) == [0, 3]
+
+
+# ---------------------------------------------------------------- summaries
+
+def test_summaries_linear_rows_closed_form():
+    """Rows k_r = r + c0: mean (L-1)/2 + c0, population variance (L^2-1)/12 (COBS §2.2 kappa_1, kappa_2)."""
+    L, d = 64, 8
+    r = np.arange(2 * L, dtype=np.float64)
+    K = r[:, None] + np.arange(d)[None, :] * 0.5
+    mu, var = O.block_summaries(K, L)
+    for b in range(2):
+        np.testing.assert_allclose(mu[b], b * L + (L - 1) / 2 + np.arange(d) * 0.5, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(var[b], (L * L - 1) / 12.0, rtol=0, atol=1e-9)
+    s32 = O.canonical_summaries(K.astype(np.float32), L)
+    # every step is exact in float32 here, so the canonical summaries equal the closed form exactly
+    assert np.array_equal(s32[:, 0], mu.astype(np.float32))
+    assert np.all(s32[:, 1] == np.float32((L * L - 1) / 12.0))
+
+
+def test_summaries_identical_rows_and_shift():
+    rng = np.random.default_rng(0)
+    L, d = 64, 16
+    # bf16-valued row (as in the cache): 64 copies sum exactly in float32
+    row = synth.bf16_to_f32(synth.f32_to_bf16(rng.standard_normal(d).astype(np.float32)))
+    K = np.tile(row, (L, 1)).astype(np.float64)
+    mu, var = O.block_summaries(K, L)
+    s32 = O.canonical_summaries(K.astype(np.float32), L)
+    assert np.array_equal(s32[0, 0], row) and np.all(s32[0, 1] == 0)
+    np.testing.assert_allclose(mu[0], row, atol=1e-15)
+    assert np.all(var[0] == 0)
+    # variance is shift invariant, mean shifts
+    K2 = rng.standard_normal((3 * L, d))
+    c = rng.standard_normal(d) * 10
+    m1, v1 = O.block_summaries(K2, L)
+    m2, v2 = O.block_summaries(K2 + c, L)
+    np.testing.assert_allclose(v1, v2, rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(m2 - m1, np.tile(c, (3, 1)), atol=1e-12)
+    # and agree with numpy's own mean/var(ddof=0)
+    np.testing.assert_allclose(v1, K2.reshape(3, L, d).var(axis=1, ddof=0), rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- scores
+
+def test_identical_key_block_score_equals_exact_mass():
+    """Zero spread: the cumulant series stops after kappa_1, so score = ln m_b - ln L (COBS §2.2)."""
+    rng = np.random.default_rng(1)
+    L, d = 64, 32
+    rows = rng.standard_normal((5, d)) * 0.7
+    K = np.repeat(rows, L, axis=0)
+    mu, var = O.block_summaries(K, L)
+    for _ in range(4):
+        q = rng.standard_normal(d)
+        s = O.head_scores(q, mu, var, alpha=1.0)
+        np.testing.assert_allclose(s, O.exact_log_mass(q, K, L) - np.log(L), rtol=0, atol=1e-12)
+
+
+def test_gaussian_keys_lognormal_closed_form():
+    """Golden closed form: for Gaussian keys the second-order estimate is exact in the limit."""
+    (d, qs, ms, ss, exp) = _golden_rows("lognormal_closed_form.txt")[0]
+    d = int(d)
+    q = np.array([float(x) for x in qs.split(",")])
+    m = np.array([float(x) for x in ms.split(",")])
+    s = np.array([float(x) for x in ss.split(",")])
+    # the oracle's score with the population summaries (mean m, variance s^2)
+    got = O.head_scores(q, m[None], (s * s)[None], alpha=1.0)[0]
+    assert abs(got - float(exp)) < 1e-12
+    # and the exact mass of sampled blocks converges to it, error ~ L^(-1/2)
+    rng = np.random.default_rng(2)
+    errs = []
+    for logL in (10, 14, 18):
+        L = 1 << logL
+        K = m + s * rng.standard_normal((L, d))
+        errs.append(abs(O.exact_log_mass(q, K, L)[0] - np.log(L) - float(exp)))
+    assert errs[2] < 0.01, errs
+    assert errs[2] < errs[0], errs
+    # with alpha = 0 the estimate keeps a constant bias of variance/2 = 0.0925
+    first = O.head_scores(q, m[None], (s * s)[None], alpha=0.0)[0]
+    assert abs(first - float(exp)) > 0.09
+
+
+def test_gaussian_blocks_empirical_summaries_converge():
+    """Per-channel variance weighting: the score from the block's own summaries tracks ln(m_b/L)."""
+    rng = np.random.default_rng(3)
+    d = 8
+    q = rng.standard_normal(d)
+    m = rng.standard_normal(d) * 0.3
+    s = np.linspace(0.1, 0.5, d)
+    prev = None
+    for logL in (10, 14, 18):
+        L = 1 << logL
+        K = m + s * rng.standard_normal((L, d))
+        mu, var = O.block_summaries(K, L)
+        err = abs(O.exact_log_mass(q, K, L)[0] - np.log(L) - O.head_scores(q, mu, var, 1.0)[0])
+        err0 = abs(O.exact_log_mass(q, K, L)[0] - np.log(L) - O.head_scores(q, mu, var, 0.0)[0])
+        assert err < err0
+        prev = err
+    assert prev < 2e-3
+
+
+def test_alpha_zero_is_first_order_mean_pool():
+    """alpha = 0 ranks blocks by the mean-pooled key against the summed group query (NSA mean-pool)."""
+    rng = np.random.default_rng(4)
+    L, d, G, nB = 64, 64, 4, 40
+    K = rng.standard_normal((nB * L, d)) * rng.uniform(0.2, 2.0, size=(nB * L, 1))
+    qs = rng.standard_normal((G, d))
+    pooled = K.reshape(nB, L, d).mean(axis=1)
+    ref = np.sort(np.argsort(-(pooled @ qs.sum(axis=0)), kind="stable")[:8])
+    mu, var = O.block_summaries(K, L)
+    assert list(O.top_k(O.group_scores(qs, mu, var, 0.0), nB, 8)) == list(ref)
+    summ = O.canonical_summaries(K.astype(np.float32), L)
+    a, b = O.canonical_group_query(qs.astype(np.float32))
+    S = O.canonical_scores(a[None], b[None], summ, 0.0)[0]
+    assert list(O.top_k(S, nB, 8)) == list(ref)
+
+
+def test_group_sum_reading_internal_consistency():
+    """Group score = sum of head scores = collapsed form (reading; parity unpinned by the pages)."""
+    rng = np.random.default_rng(5)
+    L, d, G, nB = 64, 128, 4, 10
+    K = rng.standard_normal((nB * L, d))
+    qs = rng.standard_normal((G, d))
+    mu, var = O.block_summaries(K, L)
+    collapsed = (mu @ qs.sum(0)) / np.sqrt(d) + 0.7 * 0.5 * (var @ (qs * qs).sum(0)) / d
+    np.testing.assert_allclose(O.group_scores(qs, mu, var, 0.7), collapsed, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- canonical float32 arithmetic
+
+def _rn32(x: Fraction) -> Fraction:
+    """Round an exact rational to the nearest binary32 value, ties to even (normal range)."""
+    if x == 0:
+        return Fraction(0)
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 23)
+    n, rem = divmod(a, ulp)
+    n = int(n)
+    if rem * 2 > ulp or (rem * 2 == ulp and n % 2 == 1):
+        n += 1
+    return sign * n * ulp
+
+
+def test_canonical_selector_matches_exact_rational_emulation():
+    """Brute force: each canonical step as exact rational arithmetic rounded once to float32."""
+    rng = np.random.default_rng(6)
+    L, d, G, nB = 64, 32, 3, 3
+    K = synth.bf16_to_f32(synth.f32_to_bf16((rng.standard_normal((nB * L, d)) * 1.3).astype(np.float32)))
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    alpha = np.float32(0.83)
+    summ = O.canonical_summaries(K, L)
+    qsum, q2 = O.canonical_group_query(q)
+    S = O.canonical_scores(qsum[None], q2[None], summ, float(alpha))[0]
+    F = lambda v: Fraction(float(v))
+    for b in range(nB):
+        for c in range(d):
+            s = Fraction(0)
+            for r in range(L):
+                s = _rn32(s + F(K[b * L + r, c]))
+            mu = _rn32(s / L)
+            a = Fraction(0)
+            for r in range(L):
+                t = _rn32(F(K[b * L + r, c]) - mu)
+                a = _rn32(t * t + a)
+            assert F(summ[b, 0, c]) == mu
+            assert F(summ[b, 1, c]) == _rn32(a / L)
+    for c in range(d):
+        s, s2 = Fraction(0), Fraction(0)
+        for h in range(G):
+            s = _rn32(s + F(q[h, c]))
+            s2 = _rn32(F(q[h, c]) * F(q[h, c]) + s2)
+        assert F(qsum[c]) == s and F(q2[c]) == s2
+    isd = _rn32(Fraction(1.0 / math.sqrt(d)))
+    c2 = _rn32(F(alpha) / (2 * d))
+    for b in range(nB):
+        a, v = Fraction(0), Fraction(0)
+        for c in range(d):
+            a = _rn32(F(qsum[c]) * F(summ[b, 0, c]) + a)
+        for c in range(d):
+            v = _rn32(F(q2[c]) * F(summ[b, 1, c]) + v)
+        assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
+
+
+def test_canonical_scores_exact_on_dyadic_inputs():
+    """Dyadic inputs make every float32 step exact: canonical == float64 definition, bit for bit."""
+    rng = np.random.default_rng(7)
+    L, d, G, nB = 64, 64, 4, 12
+    # rows = centre + balanced deviations: mean = centre exactly, deviations in {0, +-1/2, +-1}
+    centre = rng.integers(-8, 9, size=(nB, 1, d)) / 4.0
+    half = rng.integers(-2, 3, size=(nB, L // 2, d)) / 2.0
+    dev = np.concatenate([half, -half], axis=1)
+    dev = np.take_along_axis(dev, rng.permuted(np.tile(np.arange(L)[None, :, None], (nB, 1, d)), axis=1), axis=1)
+    K = (centre + dev).reshape(nB * L, d)
+    qs = rng.integers(-1, 2, size=(G, d)).astype(np.float64)
+    mu, var = O.block_summaries(K, L)
+    ref = O.group_scores(qs, mu, var, 1.0)
+    summ = O.canonical_summaries(K.astype(np.float32), L)
+    a, b = O.canonical_group_query(qs.astype(np.float32))
+    S = O.canonical_scores(a[None], b[None], summ, 1.0)[0]
+    assert np.array_equal(S.astype(np.float64), ref)
+
+
+# ---------------------------------------------------------------- top-k
+
+def test_topk_tie_rule_padding_and_order():
+    S = np.array([1.0, 3.0, 3.0, -0.0, 0.0, 3.0, 2.0], np.float32)
+    assert list(O.top_k(S, 7, 2)) == [1, 2]            # equal scores: lower index wins
+    assert list(O.top_k(S, 7, 4)) == [1, 2, 5, 6]        # returned ascending
+    assert list(O.top_k(S, 5, 4)) == [0, 1, 2, 3]        # -0 == +0, lower index wins
+    assert list(O.top_k(S, 3, 5)) == [0, 1, 2, -1, -1]   # fewer candidates than k: -1 padding
+    assert list(O.top_k(S, 0, 2)) == [-1, -1]
+    # duplicated summaries: identical scores, the lower block index is kept
+    L, d = 64, 16
+    rng = np.random.default_rng(8)
+    blk = rng.standard_normal((L, d))
+    K = np.concatenate([rng.standard_normal((L, d)) * 0.1, blk, blk, rng.standard_normal((L, d)) * 0.1])
+    summ = O.canonical_summaries(K.astype(np.float32), L)
+    q = rng.standard_normal((2, d)).astype(np.float32)
+    a, b = O.canonical_group_query(q)
+    S = O.canonical_scores(a[None], b[None], summ, 1.0)[0]
+    assert S[1] == S[2]
+    sel = O.top_k(S, 4, 1)
+    assert sel[0] in (0, 1, 3) and sel[0] != 2
+
+
+def test_candidates_are_complete_blocks_before_position():
+    assert O.n_candidates(62, 64) == 0
+    assert O.n_candidates(63, 64) == 1
+    assert O.n_candidates(64, 64) == 1
+    assert O.n_candidates(32767, 64) == 512
+
+
+# ---------------------------------------------------------------- branches
+
+def _sdpa(q, K, V):
+    """Textbook attention from torch (float64, CPU)."""
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))[None, None]
+    return torch.nn.functional.scaled_dot_product_attention(t(q[None]), t(K), t(V))[0, 0, 0].numpy()
+
+
+def test_branches_reduce_to_dense_attention():
+    rng = np.random.default_rng(9)
+    L, d, T = 64, 32, 512
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    q = rng.standard_normal((1, d)) * 2
+    dense = _sdpa(q[0], K, V)
+    nB = T // L
+    Kc = O.compressed_tokens(K, None, 1, 1, "f32")
+    Vc = O.compressed_tokens(V, None, 1, 1, "f32")
+    all_blocks = np.arange(nB)
+    t = T - 1
+    # top-k = all blocks: the selected branch is dense attention
+    o = O.position_output(q, [[0, 1, 0]], K, V, Kc, Vc, all_blocks, t, L, 128, 1, 1)
+    np.testing.assert_allclose(o[0], dense, rtol=0, atol=1e-12)
+    # window covering the whole context: dense
+    o = O.position_output(q, [[0, 0, 1]], K, V, Kc, Vc, all_blocks[:1], t, L, T + 5, 1, 1)
+    np.testing.assert_allclose(o[0], dense, rtol=0, atol=1e-12)
+    # compression with block = stride = 1 and identity map: dense
+    o = O.position_output(q, [[1, 0, 0]], K, V, Kc, Vc, all_blocks[:1], t, L, 128, 1, 1)
+    np.testing.assert_allclose(o[0], dense, rtol=0, atol=1e-12)
+    # gates mix linearly
+    o1 = O.position_output(q, [[0.2, 0.3, 0.5]], K, V, Kc, Vc, all_blocks, t, L, T, 1, 1)
+    np.testing.assert_allclose(o1[0], dense, rtol=0, atol=1e-12)
+
+
+def test_window_and_selection_token_sets():
+    slc, win, cmp_ = O.branch_tokens(200, np.array([0, 2, -1]), 64, 128, 32, 16, 100)
+    assert list(slc) == list(range(0, 64)) + list(range(128, 192))
+    assert list(win) == list(range(73, 201))
+    # compressed token i covers rows 16i .. 16i+31 and is visible when 16i+31 <= t
+    assert list(cmp_) == list(range(0, 11))          # 16*10+31 = 191 <= 200 < 16*11+31
+    slc, win, cmp_ = O.branch_tokens(20, np.array([-1]), 64, 128, 32, 16, 100)
+    assert len(slc) == 0 and list(win) == list(range(0, 21)) and len(cmp_) == 0
+
+
+def test_attention_shift_invariance_and_empty_branch():
+    rng = np.random.default_rng(10)
+    K = rng.standard_normal((50, 16))
+    V = rng.standard_normal((50, 16))
+    q = rng.standard_normal(16)
+    o1 = O.attend(q, K, V)
+    o2 = O.attend(q, K + rng.standard_normal(16), V)     # q.k shifts by a constant
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+    assert np.all(O.attend(q, K[:0], V[:0]) == 0)
+
+
+def test_compressed_tokens_mean_pool_closed_form():
+    T, d = 256, 4
+    X = np.arange(T, dtype=np.float64)[:, None] * np.ones((1, d))
+    C = O.compressed_tokens(X, None, 32, 16, "f32")
+    assert C.shape == ((T - 32) // 16 + 1, d)
+    np.testing.assert_allclose(C[:, 0], 16 * np.arange(C.shape[0]) + 15.5, atol=0)
+    P = np.diag([1.0, 2.0, -1.0, 0.5])
+    Cp = O.compressed_tokens(X, P, 32, 16, "f32")
+    np.testing.assert_allclose(Cp, C * np.array([1.0, 2.0, -1.0, 0.5]), atol=0)
+
+
+def test_round_bf16_matches_bit_rounding():
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal(100000) * 10.0 ** rng.integers(-3, 4, 100000)).astype(np.float32)
+    # halfway cases: ties to even
+    x[:4] = np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 1.0 + 2 ** -9], np.float32)
+    ref = synth.bf16_to_f32(synth.f32_to_bf16(x)).astype(np.float64)
+    assert np.array_equal(O.round_bf16(x.astype(np.float64)), ref)
+    assert list(ref[:4]) == [1.0, 1.015625, -1.0, 1.0]
+
+
+# ---------------------------------------------------------------- whole path
+
+def test_decode_equals_prefill_last_row():
+    w = synth.WORKLOADS["tiny"]
+    K, V = synth.kv_cache(w)
+    Q = synth.queries_decode(w)
+    g = synth.gates_decode(w)
+    dec = O.decode(w, K, V, Q, g, None, None)
+    Qp = synth.queries_prefill(w, positions=[w.T - 1])
+    gp = synth.gates_prefill(w, positions=[w.T - 1])
+    assert np.array_equal(Qp[0, 0], Q[0])
+    Op, idxp = O.prefill_positions(w, K, V, Qp[0], gp[0], None, None, [w.T - 1])
+    assert np.array_equal(idxp[0], dec["idx"][0])
+    np.testing.assert_allclose(Op[0], dec["O"][0], rtol=0, atol=1e-13)
+
+
+def test_needle_recall_second_order_beats_first_order():
+    """Method claim (COBS §2.2/§2.3): the variance term finds high-spread blocks the mean misses."""
+    w = synth.WORKLOADS["decode32k"].replace(B=1, Hkv=2, Hq=8, T=8192)
+    K, V = synth.kv_cache(w)
+    Q = synth.queries_decode(w)
+    r1, r0 = [], []
+    for h in range(w.Hkv):
+        Kf = synth.to_f64(K[0, h], w.dtype)
+        qs = synth.to_f64(Q[0, h * w.G:(h + 1) * w.G], w.dtype)
+        summ = O.canonical_summaries(Kf.astype(np.float32), w.block)
+        a, b = O.canonical_group_query(qs.astype(np.float32))
+        ref = O.osa_top_k(qs, Kf, w.block, w.nB, w.topk)
+        s1 = O.top_k(O.canonical_scores(a[None], b[None], summ, 1.0)[0], w.nB, w.topk)
+        s0 = O.top_k(O.canonical_scores(a[None], b[None], summ, 0.0)[0], w.nB, w.topk)
+        r1.append(O.recall(s1, ref))
+        r0.append(O.recall(s0, ref))
+    assert np.mean(r1) > np.mean(r0), (r1, r0)
+
+
+def test_projection_orientation():
+    """Compressed token = P @ pooled (row j of the output is P[j] . m): constant rows e_0 give P[:, 0]."""
+    rng = np.random.default_rng(12)
+    d = 8
+    P = rng.standard_normal((d, d))
+    X = np.zeros((64, d))
+    X[:, 0] = 1.0
+    C = O.compressed_tokens(X, P, 32, 16, "f32")
+    np.testing.assert_allclose(C[0], P[:, 0], rtol=0, atol=1e-15)
+
+
+def test_gate_order_isolates_each_branch():
+    """Gates (cmp, slc, win): each unit gate picks exactly its branch, checked against library attention."""
+    rng = np.random.default_rng(13)
+    L, d, T, W = 64, 16, 1024, 96
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    P = rng.standard_normal((d, d)) / np.sqrt(d)
+    Kc = O.compressed_tokens(K, P, 32, 16, "f32")
+    Vc = O.compressed_tokens(V, P.T, 32, 16, "f32")
+    q = rng.standard_normal((1, d)) * 2
+    idx = np.array([1, 4, 9])
+    t = 700
+    sel_tok = np.concatenate([np.arange(b * L, (b + 1) * L) for b in idx])
+    n_vis = (t - 32 + 1) // 16 + 1
+    expect = {
+        0: _sdpa(q[0], Kc[:n_vis], Vc[:n_vis]),
+        1: _sdpa(q[0], K[sel_tok], V[sel_tok]),
+        2: _sdpa(q[0], K[t - W + 1:t + 1], V[t - W + 1:t + 1]),
+    }
+    for j in range(3):
+        g = np.zeros((1, 3))
+        g[0, j] = 1.0
+        o = O.position_output(q, g, K, V, Kc, Vc, idx, t, L, W, 32, 16)
+        np.testing.assert_allclose(o[0], expect[j], rtol=0, atol=1e-12)
+    assert not np.allclose(expect[0], expect[1]) and not np.allclose(expect[1], expect[2])
