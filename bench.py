@@ -1,0 +1,429 @@
+#!/usr/bin/env python3
+"""Benchmark of the COBS decode hot path on B200.
+
+One step = one decode step of the 32k decode workload (B=8, 32 query heads over 8 KV
+heads, d=128, T=32768, top-16, window 512): the summary update for the token appended at
+T-1 (cobs_build_summaries from T-1), the block selection (cobs_select) and the three-branch
+attention (cobs_sparse_attn_decode). Inputs are seeded synthetic tensors resident in HBM
+when the timed region starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs the whole workload on its own GPU (independent decode
+batches, no collective on the data path: weak scaling); the step time is the max over ranks.
+`--impl reference` times the CPU oracle (the reference arm) on host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode query-heads/s + achieved HBM GB/s at 32k ctx; prefill TFLOP/s"
+CSRC = os.path.join(ROOT, "block_sparse_long_summary_b200", "csrc")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k"])
+    ap.add_argument("--copies", type=int, default=6, help="KV-cache copies rotated between steps (L2 defeat)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
+    current sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(kernel)
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.flush()
+        self.out.seek(0)
+        rows = [ln.strip().split(", ") for ln in self.out.read().splitlines() if ln.strip()]
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ algorithmic bytes
+
+def decode_bytes(w, idx):
+    """Algorithmic HBM bytes of one decode step, from the selected blocks (idx [B, Hkv, k])."""
+    import numpy as np
+    d, esz = w.d, 2 if w.dtype == "bf16" else 4
+    t = w.T - 1
+    w0 = max(0, t - w.window + 1)
+    win = set(range(w0, t + 1))
+    ncv = min(w.nC, (t - w.cmp_block + 1) // w.cmp_stride + 1) if t >= w.cmp_block - 1 else 0
+    kv_tokens = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            toks = set(win)
+            for blk in idx[b, h]:
+                if blk >= 0:
+                    toks.update(range(blk * w.block, (blk + 1) * w.block))
+            kv_tokens += len(toks)
+    units = w.B * w.Hkv
+    attn = kv_tokens * 2 * d * esz + units * ncv * 2 * d * esz          # K/V union + compressed K/V
+    attn += w.B * w.Hq * d * esz * 2 + w.B * w.Hq * 3 * 4 + units * w.topk * 4   # Q, O, gates, idx
+    select = units * w.nB * 2 * d * 4 + w.B * w.Hq * d * esz + units * w.topk * 4
+    # summary update for the appended token: the completed block (64 K rows) and the last
+    # compressed token (cmp_block K and V rows), plus their outputs
+    update = units * (w.block * d * esz + 2 * d * 4 + 2 * w.cmp_block * d * esz + 2 * d * esz)
+    return {"attn": attn, "select": select, "update": update, "total": attn + select + update,
+            "kv_tokens_per_unit": kv_tokens / units}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units):
+    """Time the oracle (as it stands) on the listed units; returns (seconds, query heads)."""
+    from oracle import cobs_oracle as O
+    t0 = time.perf_counter()
+    O.decode(w, K, V, Q, g, Pk, Pv, units=units)
+    return time.perf_counter() - t0, len(units) * w.G
+
+
+def limit_threads():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=1)
+    except Exception:  # pragma: no cover
+        return None
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on host cores, bounded sample per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    lim = limit_threads()
+    units_all = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    K, V = synth.kv_cache(w)
+    Q, g = synth.queries_decode(w), synth.gates_decode(w)
+    Pk, Pv = synth.projections(w)
+    per_step = 1
+    for i in range(args.warmup):
+        oracle_decode_sample(w, K, V, Q, g, Pk, Pv, [units_all[i % len(units_all)]])
+    secs, heads = 0.0, 0
+    for i in range(args.steps):
+        s, hh = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, [units_all[i % len(units_all)]])
+        secs += s
+        heads += hh
+    value = heads / secs
+    sample = f"{per_step} (batch, KV-head) unit of {w.name} per step ({w.G} query heads), full oracle decode"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "query-heads/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
+                   "window": w.window},
+        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "query-heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del lim
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def to_dev(a, dtype, dev):
+    import numpy as np
+    import torch
+    if a is None:
+        return None
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from block_sparse_long_summary_b200 import build as B
+    if rank == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    from block_sparse_long_summary_b200 import cobs
+    import synth
+
+    w = synth.WORKLOADS[args.workload]
+    p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
+                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+    K, V = synth.kv_cache(w)
+    Q, g = synth.queries_decode(w), synth.gates_decode(w)
+    Pk, Pv = synth.projections(w)
+
+    R = max(1, args.copies)
+    tQ, tg = to_dev(Q, w.dtype, dev), torch.from_numpy(g).to(dev)
+    tPk, tPv = to_dev(Pk, "f32", dev), to_dev(Pv, "f32", dev)
+    Ks = [to_dev(K, w.dtype, dev) for _ in range(R)]
+    Vs = [to_dev(V, w.dtype, dev) for _ in range(R)]
+    bufs = [cobs.alloc(p, prefill=False, device=dev) for _ in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for r in range(R):   # cache state: full summaries of every copy
+            cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, 0, bufs[r].summaries, bufs[r].Kc, bufs[r].Vc)
+    stream.synchronize()
+    cobs.device_error(reset=True)
+
+    def step(r):
+        cobs.decode_step(p, tQ, Ks[r], Vs[r], tPk, tPv, tg, bufs[r], t_begin=w.T - 1)
+
+    # warm-up, then one CUDA graph per cache copy
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            step(i % R)
+    stream.synchronize()
+    launches0 = cobs.launch_count()
+    graphs = []
+    for r in range(R):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            step(r)
+        graphs.append(gr)
+    launches_per_step = (cobs.launch_count() - launches0) // R
+    for r in range(R):
+        graphs[r].replay()
+    stream.synchronize()
+
+    # parity spot check of what the bench runs: selected blocks of two units vs the oracle
+    idx0 = bufs[0].idx.cpu().numpy()
+    parity = None
+    if rank == 0:
+        from oracle import cobs_oracle as O
+        ok = True
+        for (b, h) in [(0, 0), (w.B - 1, w.Hkv - 1)]:
+            Kf = synth.to_f64(K[b, h], w.dtype)
+            summ = O.canonical_summaries(Kf.astype(np.float32), w.block)
+            qs = synth.to_f64(Q[b, h * w.G:(h + 1) * w.G], w.dtype).astype(np.float32)
+            sel, _ = O.select_decode(w, qs, summ)
+            ok &= bool(np.array_equal(sel, idx0[b, h]))
+        parity = "idx bit-exact on 2 sampled units" if ok else "IDX MISMATCH"
+
+    # ---- timed region: K graph replays, cache copies rotated (L2 defeat) ----
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[i % R].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    clocks = clk.summary()
+
+    # ---- per-call durations (same rotation, eager launches with events between the calls) ----
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            r = i % R
+            ev[i][0].record(stream)
+            cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc, bufs[r].Vc)
+            ev[i][1].record(stream)
+            cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select)
+            ev[i][2].record(stream)
+            cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg, bufs[r].O,
+                                         bufs[r].ws_attn)
+            ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    t_upd = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)) / args.steps
+    t_sel = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)) / args.steps
+    t_att = sum(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)) / args.steps
+
+    # ---- end to end through the public API: pinned host inputs in, output back, every step ----
+    hQ = torch.from_numpy(np.ascontiguousarray(Q).view(np.int16)).view(torch.bfloat16).pin_memory() \
+        if w.dtype == "bf16" else torch.from_numpy(Q).pin_memory()
+    hg = torch.from_numpy(g).pin_memory()
+    hk = Ks[0][:, :, w.T - 1].contiguous().cpu().pin_memory()   # the appended token's K/V rows
+    hv = Vs[0][:, :, w.T - 1].contiguous().cpu().pin_memory()
+    hO = torch.empty(bufs[0].O.shape, dtype=bufs[0].O.dtype).pin_memory()
+    dQ, dg = torch.empty_like(tQ), torch.empty_like(tg)
+    h2d = hQ.numel() * hQ.element_size() + hg.numel() * 4 + 2 * hk.numel() * hk.element_size()
+    d2h = hO.numel() * hO.element_size()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a0.record(stream)
+        for i in range(args.steps):
+            r = i % R
+            dQ.copy_(hQ, non_blocking=True)
+            dg.copy_(hg, non_blocking=True)
+            Ks[r][:, :, w.T - 1].copy_(hk, non_blocking=True)
+            Vs[r][:, :, w.T - 1].copy_(hv, non_blocking=True)
+            cobs.decode_step(p, dQ, Ks[r], Vs[r], tPk, tPv, dg, bufs[r], t_begin=w.T - 1)
+            hO.copy_(bufs[r].O, non_blocking=True)
+        a1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = a0.elapsed_time(a1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    dev_err = cobs.device_error()
+
+    qheads = w.B * w.Hq * world
+    by = decode_bytes(w, idx0)
+    peak, peak_kind = read_peaks()
+    att_gbs = by["attn"] / (t_att * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": qheads / (ms * 1e-3), "unit": "query-heads/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
+                   "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
+                   "step": "summary update at T-1 + select + decode attention, one CUDA graph",
+                   "l2": f"{R} KV-cache copies rotated between steps (working set {R} x step bytes > L2)",
+                   "parallelism": f"dp{world} (independent decode batches per GPU)"},
+        "hbm_gbs": by["total"] / (ms * 1e-3) / 1e9,
+        "hbm_bytes_per_step": by["total"],
+        "roofline": {"bound": "hbm", "kernel": "cobs_sparse_attn_decode (chunk + merge)",
+                     "achieved": att_gbs, "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
+                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": by["attn"],
+                     "traffic": recorded_traffic("decode_attention")},
+        "calls_ms": {"build_summaries_update": t_upd, "select": t_sel, "sparse_attn_decode": t_att,
+                     "select_gbs": by["select"] / (t_sel * 1e-3) / 1e9},
+        "e2e": {"value": qheads / (ms_e2e * 1e-3), "unit": "query-heads/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "parity": parity,
+        "device_error": dev_err,
+        "kv_tokens_per_unit": by["kv_tokens_per_unit"],
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        os.environ.setdefault("OMP_NUM_THREADS", "1")
+        lim = limit_threads()
+        units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:24]
+        secs, heads = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units)
+        result["cpu_baseline"] = {"value": heads / secs, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
+                                  "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
+                                            f"full oracle decode incl. summaries ({secs:.1f} s)"}
+        del lim
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        for gr in graphs:
+            del gr
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,252 @@
+// C ABI of the COBS library: host-side validation and launches on the caller's stream.
+// The library allocates nothing; every buffer and the workspace belong to the caller.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "dims.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+cobs_status fail(cobs_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+cobs_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(COBS_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// Device error flag: one int per device that loads this library. Host code cannot use
+// the symbol's name as a device address, so the address is looked up once per device.
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_flag_mutex;
+int* g_flag_addr[kMaxDevices] = {nullptr};
+
+cobs_status device_flag(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(COBS_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+    std::lock_guard<std::mutex> lock(g_flag_mutex);
+    if (g_flag_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_error);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        g_flag_addr[dev] = static_cast<int*>(p);
+    }
+    *out = g_flag_addr[dev];
+    return COBS_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cobs_status validate(const cobs_params* p) {
+    if (p == nullptr) return fail(COBS_ERR_INVALID_ARG, "params is NULL");
+    if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->T < 1)
+        return fail(COBS_ERR_INVALID_ARG, "B, Hq, Hkv and T must be >= 1 (got %d, %d, %d, %d)", p->B, p->Hq,
+                    p->Hkv, p->T);
+    if (p->Hq % p->Hkv != 0) return fail(COBS_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", p->Hq, p->Hkv);
+    if (p->Hq / p->Hkv > 16) return fail(COBS_ERR_UNSUPPORTED, "GQA group size %d > 16", p->Hq / p->Hkv);
+    if (p->d != 64 && p->d != 128) return fail(COBS_ERR_UNSUPPORTED, "head dimension %d (supported: 64, 128)", p->d);
+    if (p->block != 64) return fail(COBS_ERR_UNSUPPORTED, "selection block %d (supported: 64)", p->block);
+    if (p->topk < 1) return fail(COBS_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", p->topk);
+    if (p->topk > 32) return fail(COBS_ERR_UNSUPPORTED, "topk %d > 32", p->topk);
+    if (p->window < p->block)
+        return fail(COBS_ERR_INVALID_ARG, "window (%d) must be >= block (%d) so that the partial block is covered",
+                    p->window, p->block);
+    if (p->cmp_stride < 1 || p->cmp_block < p->cmp_stride)
+        return fail(COBS_ERR_INVALID_ARG, "need 1 <= cmp_stride <= cmp_block (got %d, %d)", p->cmp_stride,
+                    p->cmp_block);
+    if (p->dtype != COBS_F32 && p->dtype != COBS_BF16) return fail(COBS_ERR_INVALID_ARG, "dtype %d", p->dtype);
+    if (!isfinite(p->alpha)) return fail(COBS_ERR_INVALID_ARG, "alpha is not finite");
+    if ((long long)p->B * p->Hkv > 65535) return fail(COBS_ERR_UNSUPPORTED, "B * Hkv > 65535");
+    return COBS_OK;
+}
+
+cobs_status check_ptr(const void* ptr, const char* name, bool may_be_null = false) {
+    if (ptr == nullptr) {
+        if (may_be_null) return COBS_OK;
+        return fail(COBS_ERR_INVALID_ARG, "%s is NULL", name);
+    }
+    if (!aligned16(ptr)) return fail(COBS_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return COBS_OK;
+}
+
+#define COBS_TRY(x)                      \
+    do {                                 \
+        cobs_status _s = (x);            \
+        if (_s != COBS_OK) return _s;    \
+    } while (0)
+
+}  // namespace
+
+namespace cobs {
+static std::atomic<long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+void score_constants(int d, float alpha, float* isd, float* c2) {
+    *isd = (float)(1.0 / sqrt((double)d));
+    *c2 = (float)((double)alpha * 0.5 / (double)d);
+}
+}  // namespace cobs
+
+extern "C" {
+
+int32_t cobs_version(void) { return 100; }
+
+int64_t cobs_launch_count(int32_t reset) {
+    return reset ? cobs::g_launches.exchange(0) : cobs::g_launches.load();
+}
+
+const char* cobs_status_string(cobs_status s) {
+    switch (s) {
+        case COBS_OK: return "ok";
+        case COBS_ERR_INVALID_ARG: return "invalid argument";
+        case COBS_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case COBS_ERR_CUDA: return "CUDA error";
+        case COBS_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+const char* cobs_last_error(void) { return g_last_error.c_str(); }
+
+size_t cobs_summaries_elems(const cobs_params* p) {
+    if (p == nullptr || validate(p) != COBS_OK) return 0;
+    const cobs::Dims m = cobs::make_dims(*p);
+    return (size_t)m.units() * m.summ_unit_floats();
+}
+
+size_t cobs_workspace_bytes(const cobs_params* p, int32_t which) {
+    if (p == nullptr || validate(p) != COBS_OK) return 0;
+    const cobs::Dims m = cobs::make_dims(*p);
+    switch (which) {
+        case COBS_WS_SELECT: {
+            const size_t a = cobs::select_workspace_bytes(m, 0), b = cobs::select_workspace_bytes(m, 1);
+            return a > b ? a : b;
+        }
+        case COBS_WS_DECODE: return cobs::decode_workspace_bytes(m);
+        case COBS_WS_PREFILL: return cobs::prefill_workspace_bytes(m);
+    }
+    return 0;
+}
+
+int32_t cobs_device_error(int32_t reset) {
+    int* flag = nullptr;
+    if (device_flag(&flag) != COBS_OK) return -1;
+    int v = 0;
+    if (cudaMemcpy(&v, flag, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+    if (reset) {
+        const int zero = 0;
+        if (cudaMemcpy(flag, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return -1;
+    }
+    return v;
+}
+
+cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void* V, const float* Pk,
+                                 const float* Pv, int32_t t_begin, float* summaries, void* Kc, void* Vc,
+                                 cobs_stream_t stream) {
+    COBS_TRY(validate(p));
+    COBS_TRY(check_ptr(K, "K"));
+    COBS_TRY(check_ptr(V, "V"));
+    COBS_TRY(check_ptr(Pk, "Pk", true));
+    COBS_TRY(check_ptr(Pv, "Pv", true));
+    COBS_TRY(check_ptr(summaries, "summaries"));
+    const cobs::Dims m = cobs::make_dims(*p);
+    if (m.nC > 0) {
+        COBS_TRY(check_ptr(Kc, "Kc"));
+        COBS_TRY(check_ptr(Vc, "Vc"));
+    }
+    if (t_begin < 0 || t_begin > p->T) return fail(COBS_ERR_INVALID_ARG, "t_begin %d outside [0, T]", t_begin);
+    cudaError_t e = cobs::launch_summaries(m, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_build_summaries launch");
+    return COBS_OK;
+}
+
+cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summaries, int32_t prefill, int32_t* idx,
+                        void* workspace, size_t ws_bytes, cobs_stream_t stream) {
+    COBS_TRY(validate(p));
+    COBS_TRY(check_ptr(Q, "Q"));
+    COBS_TRY(check_ptr(summaries, "summaries"));
+    COBS_TRY(check_ptr(idx, "idx"));
+    if (prefill != 0 && prefill != 1) return fail(COBS_ERR_INVALID_ARG, "prefill must be 0 or 1");
+    const cobs::Dims m = cobs::make_dims(*p);
+    const size_t need = cobs::select_workspace_bytes(m, prefill);
+    if (need > 0) {
+        COBS_TRY(check_ptr(workspace, "workspace"));
+        if (ws_bytes < need) return fail(COBS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    }
+    int* flag = nullptr;
+    COBS_TRY(device_flag(&flag));
+    cudaError_t e = cobs::launch_select(m, Q, summaries, prefill, idx, workspace, (cudaStream_t)stream, flag);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_select launch");
+    return COBS_OK;
+}
+
+static cobs_status attn_common(const cobs_params* p, const void* Q, const void* K, const void* V, const void* Kc,
+                               const void* Vc, const int32_t* idx, const float* gates, void* O) {
+    COBS_TRY(validate(p));
+    COBS_TRY(check_ptr(Q, "Q"));
+    COBS_TRY(check_ptr(K, "K"));
+    COBS_TRY(check_ptr(V, "V"));
+    COBS_TRY(check_ptr(idx, "idx"));
+    COBS_TRY(check_ptr(gates, "gates"));
+    COBS_TRY(check_ptr(O, "O"));
+    const cobs::Dims m = cobs::make_dims(*p);
+    if (m.nC > 0) {
+        COBS_TRY(check_ptr(Kc, "Kc"));
+        COBS_TRY(check_ptr(Vc, "Vc"));
+    }
+    return COBS_OK;
+}
+
+cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const void* K, const void* V,
+                                    const void* Kc, const void* Vc, const int32_t* idx, const float* gates, void* O,
+                                    void* workspace, size_t ws_bytes, cobs_stream_t stream) {
+    COBS_TRY(attn_common(p, Q, K, V, Kc, Vc, idx, gates, O));
+    const cobs::Dims m = cobs::make_dims(*p);
+    const size_t need = cobs::decode_workspace_bytes(m);
+    if (need > 0) {
+        COBS_TRY(check_ptr(workspace, "workspace"));
+        if (ws_bytes < need) return fail(COBS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    }
+    int* flag = nullptr;
+    COBS_TRY(device_flag(&flag));
+    cudaError_t e = cobs::launch_decode(m, Q, K, V, Kc, Vc, idx, gates, O, workspace, (cudaStream_t)stream, flag);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_sparse_attn_decode launch");
+    return COBS_OK;
+}
+
+cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const void* K, const void* V,
+                                     const void* Kc, const void* Vc, const int32_t* idx, const float* gates,
+                                     void* O, void* workspace, size_t ws_bytes, cobs_stream_t stream) {
+    COBS_TRY(attn_common(p, Q, K, V, Kc, Vc, idx, gates, O));
+    const cobs::Dims m = cobs::make_dims(*p);
+    const size_t need = cobs::prefill_workspace_bytes(m);
+    if (need > 0) {
+        COBS_TRY(check_ptr(workspace, "workspace"));
+        if (ws_bytes < need) return fail(COBS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    }
+    int* flag = nullptr;
+    COBS_TRY(device_flag(&flag));
+    cudaError_t e = cobs::launch_prefill(m, Q, K, V, Kc, Vc, idx, gates, O, workspace, (cudaStream_t)stream, flag);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_sparse_attn_prefill launch");
+    return COBS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// Host-side derived sizes shared by the launchers (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/cobs.h"
+
+namespace cobs {
+
+struct Dims {
+    int B, Hq, Hkv, G, d, T, L, lc, sc, k, W;
+    int nB;       // complete selection blocks, T / L
+    int nG;       // 32-block summary groups, ceil(nB / 32) (at least 1)
+    int nC;       // compressed tokens, (T - lc) / sc + 1 (0 if T < lc)
+    float alpha;
+    int dtype;    // cobs_dtype
+    int units() const { return B * Hkv; }
+    size_t summ_unit_floats() const { return (size_t)nG * 2 * d * 32; }
+};
+
+inline Dims make_dims(const cobs_params& p) {
+    Dims m;
+    m.B = p.B; m.Hq = p.Hq; m.Hkv = p.Hkv; m.G = p.Hkv ? p.Hq / p.Hkv : 0; m.d = p.d; m.T = p.T;
+    m.L = p.block; m.lc = p.cmp_block; m.sc = p.cmp_stride; m.k = p.topk; m.W = p.window;
+    m.nB = p.block > 0 ? p.T / p.block : 0;
+    m.nG = m.nB > 0 ? (m.nB + 31) / 32 : 1;
+    m.nC = (p.cmp_stride > 0 && p.T >= p.cmp_block) ? (p.T - p.cmp_block) / p.cmp_stride + 1 : 0;
+    m.alpha = p.alpha; m.dtype = p.dtype;
+    return m;
+}
+
+// Count one kernel launch (read through cobs_launch_count).
+void count_launch(int n = 1);
+
+// Score constants of the canonical selector: isd = RN32(1/sqrt(d)) (through double),
+// c2 = RN32(alpha * 0.5 / d).
+void score_constants(int d, float alpha, float* isd, float* c2);
+
+// ---- launchers (return cudaSuccess or the launch error) ----
+cudaError_t launch_summaries(const Dims& m, const void* K, const void* V, const float* Pk,
+                             const float* Pv, int t_begin, float* summ, void* Kc, void* Vc,
+                             cudaStream_t s);
+
+size_t select_workspace_bytes(const Dims& m, int prefill);
+cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx,
+                          void* ws, cudaStream_t s, int* err);
+
+size_t decode_workspace_bytes(const Dims& m);
+cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                          const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
+                          cudaStream_t s, int* err);
+
+size_t prefill_workspace_bytes(const Dims& m);
+cudaError_t launch_prefill(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                           const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
+                           cudaStream_t s, int* err);
+
+}  // namespace cobs

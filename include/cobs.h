@@ -1,0 +1,179 @@
+/*
+ * cobs.h — C ABI of the B200 (sm_100a) library for block-sparse attention with
+ * cumulant-order block selection (COBS).
+ *
+ * Method sources (cited per call below):
+ *   [COBS]    "COBS: Cumulant Order Block Sparse Attention", gist.science explainer of
+ *             arXiv 2607.09052: §2.1 attention mass, §2.2 cumulant expansion,
+ *             §2.3 second-order scoring on the NSA branches.
+ *   [SKILL]   "cumulant-order-block-sparse-attention" skill card: "Method",
+ *             "Implementation steps".
+ *   [NSA-181] deepseek-ai/Janus issue #181 ("four dimensions regarding importance and
+ *             connection strength"): compression / selection / sliding-window paths and
+ *             their gates.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument except `p` is DEVICE memory owned by the caller; `p` is host
+ *   memory read during the call only. The library never allocates, frees or keeps
+ *   pointers past the call, and never synchronises: work is enqueued on `stream`
+ *   (NULL = legacy default stream) and the call returns at once.
+ * - Arguments are validated on the host before anything is launched. An invalid
+ *   argument returns COBS_ERR_INVALID_ARG (or COBS_ERR_UNSUPPORTED for a valid
+ *   but unsupported shape) and enqueues nothing; cobs_last_error() then holds a
+ *   message. A failed launch returns COBS_ERR_CUDA. Kernels never trap: an
+ *   out-of-range block index met on the device is skipped and recorded in a device
+ *   flag read by cobs_device_error().
+ * - Tensor layouts (row-major, contiguous, element type per `dtype`: bfloat16 or
+ *   float32; indices int32; gates and summaries float32):
+ *     K, V         [B, Hkv, T, d]
+ *     Q, O decode  [B, Hq, d]            (the query at position T-1)
+ *     Q, O prefill [B, T, Hq, d]
+ *     gates        decode [B, Hq, 3], prefill [B, T, Hq, 3]: (g_cmp, g_slc, g_win),
+ *                  already passed through the sigmoid
+ *     Kc, Vc       [B, Hkv, nC, d], nC = (T - cmp_block) / cmp_stride + 1 (0 if T < cmp_block)
+ *     idx          decode [B, Hkv, topk], prefill [B, T, Hkv, topk]
+ *     summaries    [B, Hkv, nG, 2, d/4, 32, 4] float32, nG = ceil(nB / 32), nB = T / block:
+ *                  block b of a unit lives in group b/32, lane b%32; entry [..., 0, c/4, b%32, c%4]
+ *                  is the key mean mu_{b,c}, [..., 1, ...] the key variance var_{b,c}.
+ *                  (32 consecutive blocks are interleaved channel-by-channel so that one
+ *                  warp reads one channel of 32 blocks in one 512-byte transaction.)
+ * - GQA: query head h belongs to KV head h / (Hq / Hkv).
+ * - Supported: d in {64, 128}; block = 64; 1 <= topk <= 32; window >= block;
+ *   Hq % Hkv == 0 and Hq / Hkv <= 16; cmp_block = 32, cmp_stride = 16 for bf16
+ *   (any cmp_block >= cmp_stride >= 1 for float32); T >= 1.
+ */
+#ifndef COBS_H_
+#define COBS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cobs_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    COBS_OK = 0,
+    COBS_ERR_INVALID_ARG = -1,
+    COBS_ERR_UNSUPPORTED = -2,
+    COBS_ERR_CUDA = -3,
+    COBS_ERR_WORKSPACE = -4
+} cobs_status;
+
+typedef enum { COBS_F32 = 0, COBS_BF16 = 1 } cobs_dtype;
+
+typedef enum { COBS_WS_SELECT = 0, COBS_WS_DECODE = 1, COBS_WS_PREFILL = 2 } cobs_workspace_kind;
+
+/* Problem statement ([COBS] §2.3, [SKILL] "Method"): block size, compression block and
+ * stride, top-k, window and alpha. */
+typedef struct {
+    int32_t B;          /* batch */
+    int32_t Hq;         /* query heads */
+    int32_t Hkv;        /* key/value heads (GQA groups) */
+    int32_t d;          /* head dimension */
+    int32_t T;          /* context length (decode: the query sits at T-1) */
+    int32_t block;      /* selection block L */
+    int32_t cmp_block;  /* compression block l_c */
+    int32_t cmp_stride; /* compression stride s_c */
+    int32_t topk;       /* selected blocks per GQA group */
+    int32_t window;     /* sliding window W */
+    float alpha;        /* weight of the second-order (variance) term */
+    int32_t dtype;      /* cobs_dtype of Q, K, V, Kc, Vc, O */
+} cobs_params;
+
+/*
+ * Block summaries and compressed tokens: one pass over K and V.
+ * [COBS] §2.2/§2.3: per block, the key mean mu_b (kappa_1) and the second-order
+ * statistic, here the per-channel population variance var_b (the diagonal of the
+ * block covariance kappa_2); [NSA-181] compression path: compressed token i is
+ * P · mean(rows cmp_stride*i .. cmp_stride*i + cmp_block - 1), for K with P_k and for V
+ * with P_v ([SKILL] step 4: the compression branch itself is unchanged).
+ *   Pk, Pv     [d, d] float32 device matrices (out = P @ pooled), or NULL for identity.
+ *   t_begin    positions < t_begin are already summarised: only blocks and compressed
+ *              tokens whose last row is >= t_begin are (re)written. 0 = full build;
+ *              T - 1 = the update after appending the token at T - 1.
+ *   summaries, Kc, Vc: outputs (layouts above). Summaries are float32 in a fixed
+ *              summation order (row order), so they are reproducible bit for bit.
+ */
+cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void* V,
+                                 const float* Pk, const float* Pv, int32_t t_begin,
+                                 float* summaries, void* Kc, void* Vc, cobs_stream_t stream);
+
+/*
+ * Block selection ([COBS] §2.3 second-order score; [SKILL] step 3 and "Method": top-k).
+ * For each GQA group g and candidate block b:
+ *   S_{g,b} = (sum_c Qsum_c mu_{b,c}) * RN(1/sqrt(d)) + RN(alpha/(2d)) * (sum_c Q2_c var_{b,c}),
+ *   Qsum = sum_{h in g} q_h, Q2 = sum_{h in g} q_h*q_h   (= sum_h [q_h.mu_b/sqrt(d)
+ *   + alpha/2 * sum_c q_{h,c}^2 var_{b,c}/d]), evaluated in float32 with fused multiply-adds
+ *   in ascending head and channel order. Candidates are the complete blocks
+ *   b < (t + 1) / block at query position t. The topk best by (score descending, block
+ *   ascending) are written in ascending block order, padded with -1.
+ *   prefill = 0: Q [B, Hq, d] at t = T - 1, idx [B, Hkv, topk].
+ *   prefill = 1: Q [B, T, Hq, d] at every t, idx [B, T, Hkv, topk].
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_SELECT) bytes, zero-filled before its
+ *              first use; each call leaves it zero-filled again on completion.
+ */
+cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summaries,
+                        int32_t prefill, int32_t* idx, void* workspace, size_t ws_bytes,
+                        cobs_stream_t stream);
+
+/*
+ * Decode attention at position T - 1 ([NSA-181] three paths; [COBS] §2.3):
+ *   o_h = g_cmp softmax_cmp + g_slc softmax_slc + g_win softmax_win, each branch a
+ *   softmax(q K^T / sqrt(d)) V of its own over the compressed tokens (all nC), the tokens
+ *   of the selected blocks idx (entries -1 skipped) and the tokens max(0, T-W) .. T-1.
+ *   An empty branch contributes zero.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_DECODE) bytes, zero-filled before its
+ *              first use; left zero-filled again on completion. Calls that share one
+ *              workspace must not run concurrently.
+ */
+cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const void* K,
+                                    const void* V, const void* Kc, const void* Vc,
+                                    const int32_t* idx, const float* gates, void* O,
+                                    void* workspace, size_t ws_bytes, cobs_stream_t stream);
+
+/*
+ * Causal prefill attention: the decode computation at every position t = 0 .. T-1, with
+ * the window tokens max(0, t-W+1) .. t, the compressed tokens i with
+ * cmp_stride*i + cmp_block - 1 <= t, and the selected blocks idx[b, t, g, :].
+ *   Q, gates, O, idx in their prefill layouts.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_PREFILL) bytes (may be 0).
+ */
+cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const void* K,
+                                     const void* V, const void* Kc, const void* Vc,
+                                     const int32_t* idx, const float* gates, void* O,
+                                     void* workspace, size_t ws_bytes, cobs_stream_t stream);
+
+/* Bytes of workspace a call needs (0 for an invalid p). */
+size_t cobs_workspace_bytes(const cobs_params* p, int32_t which);
+
+/* Number of float32 elements of the summaries tensor. */
+size_t cobs_summaries_elems(const cobs_params* p);
+
+/* Static text for a status code. */
+const char* cobs_status_string(cobs_status s);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* cobs_last_error(void);
+
+/*
+ * Device error flag of the current device: 0 if no kernel met an out-of-range index or
+ * gave up a bounded wait since the last reset, else a nonzero code. Synchronises the
+ * current device. reset != 0 clears the flag.
+ */
+int32_t cobs_device_error(int32_t reset);
+
+/* Kernel launches this library has issued in this process (all host threads); reset != 0
+ * sets the count back to zero after reading it. */
+int64_t cobs_launch_count(int32_t reset);
+
+/* ABI version (major * 100 + minor). */
+int32_t cobs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COBS_H_ */

@@ -1,0 +1,81 @@
+"""Helpers shared by the GPU parity tests: moving seeded inputs to the device, running the
+library through its C ABI, and reshaping its outputs for comparison with the oracle."""
+import numpy as np
+import torch
+
+import synth
+
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+
+
+def cobs():
+    from block_sparse_long_summary_b200 import build as B
+    B.build()
+    from block_sparse_long_summary_b200 import cobs as C
+    return C
+
+
+def dev(arr, dtype):
+    """Storage-form numpy array (uint16 bf16 bits or float32) -> CUDA tensor."""
+    if arr is None:
+        return None
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32)).cuda()
+
+
+def f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def params_of(w):
+    C = cobs()
+    return C.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
+                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+
+
+def summaries_blocks(flat, p):
+    """Device summaries (channel-interleaved groups of 32 blocks) -> [B, Hkv, nB, 2, d] float32."""
+    nB = p.T // p.block
+    nG = max(1, -(-nB // 32))
+    a = flat[: p.B * p.Hkv * nG * 2 * p.d * 32].cpu().numpy()
+    a = a.reshape(p.B, p.Hkv, nG, 2, p.d // 4, 32, 4).transpose(0, 1, 2, 5, 3, 4, 6)
+    return a.reshape(p.B, p.Hkv, nG * 32, 2, p.d)[:, :, :nB]
+
+
+def run_decode(w, K, V, Q, gates, Pk, Pv):
+    C = cobs()
+    p = params_of(w)
+    buf = C.alloc(p, prefill=False)
+    C.device_error(reset=True)
+    C.decode_step(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),
+                  torch.from_numpy(gates).cuda(), buf, t_begin=0)
+    torch.cuda.synchronize()
+    return p, buf
+
+
+def run_prefill(w, K, V, Q, gates, Pk, Pv):
+    C = cobs()
+    p = params_of(w)
+    buf = C.alloc(p, prefill=True)
+    C.device_error(reset=True)
+    C.prefill(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),
+              torch.from_numpy(gates).cuda(), buf)
+    torch.cuda.synchronize()
+    return p, buf
+
+
+def inputs_decode(w):
+    K, V = synth.kv_cache(w)
+    return K, V, synth.queries_decode(w), synth.gates_decode(w), *synth.projections(w)
+
+
+def kc_close(gpu, ref, dtype):
+    """Compressed tokens: the GPU rounds its float32 result once to the storage type; the oracle
+    rounds the exact value. They differ by at most one unit in the last place of the storage type."""
+    if dtype == "bf16":
+        # one bf16 ulp is at most 2^-7 of the value; 1e-5 covers the float32 sum near zero
+        tol = np.abs(ref) * 2.0 ** -7 + 1e-5
+    else:
+        tol = np.abs(ref) * 1e-5 + 1e-6
+    return np.abs(gpu - ref) <= tol

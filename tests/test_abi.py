@@ -1,0 +1,93 @@
+"""The C ABI library builds, loads, exports every declared entry point and validates
+arguments on the host (no GPU needed: invalid arguments are rejected before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_summary_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = B.build()
+    from block_sparse_long_summary_b200 import cobs
+    return cobs
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(cobs_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert {"cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill"} <= syms
+    so = ctypes.CDLL(B.LIB)
+    for name in sorted(syms):
+        assert hasattr(so, name), name
+    assert set(lib.EXPORTED) <= syms
+
+
+def test_version_and_status_strings(lib):
+    assert lib.version() == 100
+    assert lib._lib.cobs_status_string(0) == b"ok"
+    assert lib._lib.cobs_status_string(-1) == b"invalid argument"
+
+
+def _p(**kw):
+    from block_sparse_long_summary_b200.cobs import Params
+    base = dict(B=1, Hq=4, Hkv=1, d=128, T=4096, topk=16, window=512)
+    base.update(kw)
+    return Params(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), -2),
+    (dict(block=32), -2),
+    (dict(topk=0), -1),
+    (dict(topk=33), -2),
+    (dict(window=32), -1),
+    (dict(Hq=6, Hkv=4), -1),
+    (dict(Hq=64, Hkv=2), -2),
+    (dict(T=0), -1),
+    (dict(cmp_stride=0), -1),
+    (dict(alpha=float("nan")), -1),
+])
+def test_host_validation_rejects_before_launch(lib, kw, status):
+    p = _p(**kw)
+    cp = p.c()
+    fake = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    r = lib._lib.cobs_build_summaries(ctypes.byref(cp), fake, fake, None, None, 0, fake, fake, fake, None)
+    assert r == status, lib._lib.cobs_last_error()
+    assert lib._lib.cobs_last_error() != b""
+    assert lib.workspace_bytes(p, lib.COBS_WS_DECODE) == 0
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _p()
+    cp = p.c()
+    fake = ctypes.c_void_p(256)
+    assert lib._lib.cobs_select(ctypes.byref(cp), None, fake, 0, fake, fake, 1 << 20, None) == -1
+    assert b"Q is NULL" in lib._lib.cobs_last_error()
+    bad = ctypes.c_void_p(258)
+    assert lib._lib.cobs_select(ctypes.byref(cp), bad, fake, 0, fake, fake, 1 << 20, None) == -1
+    assert b"aligned" in lib._lib.cobs_last_error()
+    assert lib._lib.cobs_select(ctypes.byref(cp), fake, fake, 2, fake, fake, 1 << 20, None) == -1
+
+
+def test_workspace_sizes(lib):
+    p = _p(B=8, Hq=32, Hkv=8, T=32768)
+    n_units = 8 * 8
+    # decode partials: units x chunks x G x (d + 4) floats; chunks = 16/2 + 512/128 + ceil(2047/128)
+    assert lib.workspace_bytes(p, lib.COBS_WS_DECODE) == n_units * (8 + 4 + 16) * 4 * 132 * 4
+    assert lib.summaries_elems(p) == n_units * 16 * 2 * 128 * 32
+    assert lib.workspace_bytes(p, lib.COBS_WS_SELECT) > 0
