@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k"])
     ap.add_argument("--copies", type=int, default=6, help="KV-cache copies rotated between steps (L2 defeat)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch size (small profiling cases)")
     return ap.parse_args()
 
 
@@ -248,6 +249,8 @@ def run_ours(args):
     import synth
 
     w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(B=args.batch)
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
     K, V = synth.kv_cache(w)
@@ -306,7 +309,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):   # replay() launches on the current stream
         e0.record(stream)
         for i in range(args.steps):
             graphs[i % R].replay()
@@ -320,19 +323,30 @@ def run_ours(args):
         dist.barrier()
     clocks = clk.summary()
 
-    # ---- per-call durations (same rotation, eager launches with events between the calls) ----
+    # ---- per-call durations: each call captured in its own graph, events recorded between the
+    # replays on the launching stream (same copy rotation as the timed region) ----
+    calls = []
+    for r in range(R):
+        gu, gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gu, stream=stream):
+            cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc, bufs[r].Vc)
+        with torch.cuda.graph(gs, stream=stream):
+            cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select)
+        with torch.cuda.graph(ga, stream=stream):
+            cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg, bufs[r].O,
+                                         bufs[r].ws_attn)
+        calls.append((gu, gs, ga))
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            r = i % R
+            gu, gs, ga = calls[i % R]
             ev[i][0].record(stream)
-            cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc, bufs[r].Vc)
+            gu.replay()
             ev[i][1].record(stream)
-            cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select)
+            gs.replay()
             ev[i][2].record(stream)
-            cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg, bufs[r].O,
-                                         bufs[r].ws_attn)
+            ga.replay()
             ev[i][3].record(stream)
     torch.cuda.synchronize()
     t_upd = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)) / args.steps
@@ -412,8 +426,8 @@ def run_ours(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
-        for gr in graphs:
-            del gr
+        graphs.clear()
+        calls.clear()
         dist.destroy_process_group()
     return 0
 
