@@ -349,6 +349,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         count_launch();
+        count_launch();
         kern<<<dim3(nsplit, m.units()), 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, ws_ctr, m.G, m.nG, ncand, m.k,
                                                      gpc, nsplit, isd, c2, err);
         return cudaGetLastError();
@@ -357,6 +358,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
     auto kern = select_prefill_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     count_launch();
     kern<<<dim3((m.T + kPfPos - 1) / kPfPos, m.units()), 128, smem, s>>>(Q, summ, idx, m.T, m.Hq, m.Hkv, m.G,
                                                                         m.nG, m.L, m.k, isd, c2, err);
