@@ -29,7 +29,7 @@ COBS_WS_PREFILL = 2
 
 EXPORTED = [
     "cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
-    "cobs_workspace_bytes", "cobs_summaries_elems", "cobs_status_string", "cobs_last_error",
+    "cobs_sparse_attn_decode_noalloc", "cobs_workspace_bytes", "cobs_summaries_elems", "cobs_status_string", "cobs_last_error",
     "cobs_device_error", "cobs_launch_count", "cobs_version",
 ]
 
@@ -58,7 +58,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.cobs_select.argtypes = [P, vp, vp, i32, vp, vp, sz, vp]
     lib.cobs_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cobs_sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-    for f in ("cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill"):
+    lib.cobs_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    for f in ("cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
+              "cobs_sparse_attn_decode_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     lib.cobs_workspace_bytes.argtypes = [P, i32]
     lib.cobs_workspace_bytes.restype = sz
@@ -173,6 +175,14 @@ def cobs_sparse_attn_decode(p: Params, Q, K, V, Kc, Vc, idx, gates, O, workspace
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.cobs_sparse_attn_decode(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(Vc), _ptr(idx),
                                         _ptr(gates), _ptr(O), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def cobs_sparse_attn_decode_noalloc(p: Params, Q, K, V, Kc, Vc, idx, gates, O, stream=None):
+    """Decode attention using the library's built-in device scratch instead of a workspace,
+    for callers that cannot provide device memory of their own (see include/cobs.h)."""
+    cp = p.c()
+    _check(_lib.cobs_sparse_attn_decode_noalloc(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(Vc),
+                                                _ptr(idx), _ptr(gates), _ptr(O), _stream(stream)))
 
 
 def cobs_sparse_attn_prefill(p: Params, Q, K, V, Kc, Vc, idx, gates, O, workspace, stream=None):

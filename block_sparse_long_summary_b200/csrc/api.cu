@@ -232,6 +232,25 @@ cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const v
     return COBS_OK;
 }
 
+cobs_status cobs_sparse_attn_decode_noalloc(const cobs_params* p, const void* Q, const void* K, const void* V,
+                                            const void* Kc, const void* Vc, const int32_t* idx, const float* gates,
+                                            void* O, cobs_stream_t stream) {
+    COBS_TRY(attn_common(p, Q, K, V, Kc, Vc, idx, gates, O));
+    const cobs::Dims m = cobs::make_dims(*p);
+    const size_t need = cobs::decode_workspace_bytes(m);
+    const size_t have = cobs::noalloc_scratch_bytes();
+    if (need > have)
+        return fail(COBS_ERR_WORKSPACE,
+                    "this problem needs %zu bytes of decode scratch, more than the %zu bytes built into the library; "
+                    "call cobs_sparse_attn_decode with a workspace instead",
+                    need, have);
+    int* flag = nullptr;
+    COBS_TRY(device_flag(&flag));
+    cudaError_t e = cobs::launch_decode_noalloc(m, Q, K, V, Kc, Vc, idx, gates, O, (cudaStream_t)stream, flag);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_sparse_attn_decode_noalloc launch");
+    return COBS_OK;
+}
+
 cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const void* K, const void* V,
                                      const void* Kc, const void* Vc, const int32_t* idx, const float* gates,
                                      void* O, void* workspace, size_t ws_bytes, cobs_stream_t stream) {

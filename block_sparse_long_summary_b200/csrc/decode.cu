@@ -6,6 +6,7 @@
 // how SLC picks its blocks. Only the selected blocks, the window and the compressed tokens
 // are read from HBM ("Problemstellung": decode is bound by KV-cache reads).
 #include <algorithm>
+#include <mutex>
 
 #include "attn.cuh"
 #include "dims.h"
@@ -441,6 +442,49 @@ cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const voi
     const int CK = m.dtype == COBS_BF16 ? kCK : kCKf;
     AttnArgs a = make_args(m, Q, K, V, Kc, Vc, idx, gates, O, ws, err, 1, CK);
     return m.d == 128 ? launch_decode_d<128>(m, a, s) : launch_decode_d<64>(m, a, s);
+}
+
+// ---------------------------------------------------------------- allocation-free decode variant
+// Scratch of cobs_sparse_attn_decode_noalloc: the split-K partial records live in this fixed
+// array instead of a caller-provided workspace. Every device that loads the library holds it
+// until the process exits. Calls share it, so calls that overlap on the GPU race; nothing in it
+// needs clearing, because a call writes every record before it reads it.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {nullptr};
+
+// The array's name is only a host-side stand-in: its device address is looked up once per
+// device, with that device current.
+cudaError_t noalloc_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_decode_noalloc(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                                  const void* Vc, const int32_t* idx, const float* gates, void* O, cudaStream_t s,
+                                  int* err) {
+    void* scratch = nullptr;
+    cudaError_t e = noalloc_scratch_address(&scratch);
+    if (e != cudaSuccess) return e;
+    return launch_decode(m, Q, K, V, Kc, Vc, idx, gates, O, scratch, s, err);
 }
 
 size_t prefill_workspace_bytes(const Dims&) { return 0; }

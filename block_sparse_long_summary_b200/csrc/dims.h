@@ -52,6 +52,12 @@ cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const voi
                           const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                           cudaStream_t s, int* err);
 
+// Decode with the library's fixed device scratch in place of a workspace (no allocation).
+size_t noalloc_scratch_bytes();
+cudaError_t launch_decode_noalloc(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                                  const void* Vc, const int32_t* idx, const float* gates, void* O, cudaStream_t s,
+                                  int* err);
+
 size_t prefill_workspace_bytes(const Dims& m);
 cudaError_t launch_prefill(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                            const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,

@@ -136,6 +136,28 @@ cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const v
                                     void* workspace, size_t ws_bytes, cobs_stream_t stream);
 
 /*
+ * Decode attention without a workspace. The paper has no counterpart to this call: it exists
+ * for callers that cannot hand the library any device memory of its own, such as a host
+ * program whose allocations all go through a pool it has already carved up, or a plug-in
+ * whose host forbids device allocations after start-up. It computes exactly what
+ * cobs_sparse_attn_decode computes, with the split-K partial results kept in a scratch array
+ * built into the library (8 MiB, one per device that loads the library, held until the
+ * process exits) and no allocation of any kind.
+ *   - Problems whose partials need more than 8 MiB (cobs_workspace_bytes(p, COBS_WS_DECODE))
+ *     are rejected with COBS_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the scratch array's device address (with that
+ *     device current); make that first call before any stream capture begins.
+ *   - Every call on a device shares the one array and it keeps the last call's contents
+ *     (nothing in it needs clearing). Calls whose kernels overlap on the GPU, for example
+ *     on two streams without ordering between them, race on it: order them.
+ * Other arguments, layouts and errors are those of cobs_sparse_attn_decode.
+ */
+cobs_status cobs_sparse_attn_decode_noalloc(const cobs_params* p, const void* Q, const void* K,
+                                            const void* V, const void* Kc, const void* Vc,
+                                            const int32_t* idx, const float* gates, void* O,
+                                            cobs_stream_t stream);
+
+/*
  * Causal prefill attention: the decode computation at every position t = 0 .. T-1, with
  * the window tokens max(0, t-W+1) .. t, the compressed tokens i with
  * cmp_stride*i + cmp_block - 1 <= t, and the selected blocks idx[b, t, g, :].
