@@ -38,7 +38,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k"])
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k"])
+    ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
+    ap.add_argument("--T", type=int, default=None, help="override the context length (small profiling cases)")
     ap.add_argument("--copies", type=int, default=6, help="KV-cache copies rotated between steps (L2 defeat)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the batch size (small profiling cases)")
@@ -47,6 +50,18 @@ def parse():
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group). Every rank
+    must call it at the same point; works with nccl (device tensor) and gloo (host tensor)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def read_peaks():
@@ -228,6 +243,90 @@ def to_dev(a, dtype, dev):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
 
 
+def read_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "measured"
+    return 1590.0, 1400.0, "fallback"
+
+
+def prefill_flops(w, idx):
+    """Algorithmic attention FLOPs of a causal prefill: 4 d per (position, head, attended key),
+    from the selected blocks idx [B, T, Hkv, k] and the window / compressed-token visibility."""
+    import numpy as np
+    t = np.arange(w.T)
+    win = np.minimum(w.window, t + 1).astype(np.int64)
+    vis = np.where(t >= w.cmp_block - 1, np.minimum(w.nC, (t - w.cmp_block + 1) // w.cmp_stride + 1), 0)
+    slc = (idx >= 0).sum(axis=-1).astype(np.int64) * w.block          # [B, T, Hkv]
+    keys_per_group = slc + win[None, :, None] + vis[None, :, None]
+    return float(4 * w.d * w.G * keys_per_group.sum())
+
+
+def bench_prefill(w, steps, warmup, dev, cobs):
+    """One step = full summary build + per-position selection + prefill attention."""
+    import numpy as np
+    import torch
+    import synth
+    p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
+                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+    K, V = synth.kv_cache(w)
+    Q, g = synth.queries_prefill(w), synth.gates_prefill(w)
+    Pk, Pv = synth.projections(w)
+    tQ, tK, tV = to_dev(Q, w.dtype, dev), to_dev(K, w.dtype, dev), to_dev(V, w.dtype, dev)
+    tPk, tPv, tg = to_dev(Pk, "f32", dev), to_dev(Pv, "f32", dev), torch.from_numpy(g).to(dev)
+    buf = cobs.alloc(p, prefill=True, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, warmup)):
+            cobs.prefill(p, tQ, tK, tV, tPk, tPv, tg, buf)
+    stream.synchronize()
+    n0 = cobs.launch_count()
+    times = []
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            e = [ev() for _ in range(4)]
+            e[0].record(stream)
+            cobs.cobs_build_summaries(p, tK, tV, tPk, tPv, 0, buf.summaries, buf.Kc, buf.Vc)
+            e[1].record(stream)
+            cobs.cobs_select(p, tQ, buf.summaries, 1, buf.idx, buf.ws_select)
+            e[2].record(stream)
+            cobs.cobs_sparse_attn_prefill(p, tQ, tK, tV, buf.Kc, buf.Vc, buf.idx, tg, buf.O, buf.ws_attn)
+            e[3].record(stream)
+            times.append(e)
+    torch.cuda.synchronize()
+    launches = cobs.launch_count() - n0
+    t_sum = sum(e[0].elapsed_time(e[1]) for e in times) / steps
+    t_sel = sum(e[1].elapsed_time(e[2]) for e in times) / steps
+    t_att = sum(e[2].elapsed_time(e[3]) for e in times) / steps
+    flops = prefill_flops(w, buf.idx.cpu().numpy())
+    burst, sustained, kind = read_tflops()
+    att_tf = flops / (t_att * 1e-3) / 1e12
+    kv_bytes = 2 * w.B * w.Hkv * w.T * w.d * 2
+    return {
+        "value": flops / ((t_sum + t_sel + t_att) * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "definition": "algorithmic attention FLOPs (4 d per position, head and attended key) / "
+                      "(summary build + selection + attention)",
+        "tflops_select_attn": flops / ((t_sel + t_att) * 1e-3) / 1e12,
+        "ms": {"build_summaries": t_sum, "select": t_sel, "sparse_attn_prefill": t_att},
+        "flops_per_step": flops,
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
+                   "window": w.window, "l2": "inputs larger than L2 (Q 0.5 GB)"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": att_tf, "peak": sustained,
+                     "unit": "TFLOP/s", "frac": att_tf / sustained, "peak_kind": f"{kind} sustained bf16",
+                     "traffic": None},
+        "summary_build_gbs": (kv_bytes + buf.summaries.numel() * 4 + 2 * buf.Kc.numel() * 2) / (t_sum * 1e-3) / 1e9,
+        "gpu_launches": launches,
+        "steps": steps,
+        "device_error": cobs.device_error(),
+    }
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -251,6 +350,10 @@ def run_ours(args):
     w = synth.WORKLOADS[args.workload]
     if args.batch:
         w = w.replace(B=args.batch)
+    if args.T:
+        w = w.replace(T=args.T)
+    if w.mode == "prefill":
+        return run_prefill_line(args, w, dev, cobs, rank, world)
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
     K, V = synth.kv_cache(w)
@@ -315,11 +418,8 @@ def run_ours(args):
             graphs[i % R].replay()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     clocks = clk.summary()
 
@@ -377,11 +477,7 @@ def run_ours(args):
             hO.copy_(bufs[r].O, non_blocking=True)
         a1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = a0.elapsed_time(a1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev)
     dev_err = cobs.device_error()
 
     qheads = w.B * w.Hq * world
@@ -423,11 +519,33 @@ def run_ours(args):
                                   "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
                                             f"full oracle decode incl. summaries ({secs:.1f} s)"}
         del lim
+    if not args.no_prefill and world == 1:
+        wp = synth.WORKLOADS["prefill32k"]
+        del Ks, Vs, bufs, graphs[:], calls[:]
+        torch.cuda.empty_cache()
+        result["prefill"] = bench_prefill(wp, args.prefill_steps, 2, dev, cobs)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         graphs.clear()
         calls.clear()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_prefill_line(args, w, dev, cobs, rank, world):
+    import torch.distributed as dist
+    res = bench_prefill(w, args.steps, max(3, args.warmup), dev, cobs)
+    ms = max_over_ranks(sum(res["ms"].values()), dev)
+    line = {"metric": METRIC, "value": res["flops_per_step"] * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": res["config"], "roofline": res["roofline"], "calls_ms": res["ms"],
+            "tflops_select_attn": res["tflops_select_attn"], "gpu_launches": res["gpu_launches"],
+            "device_error": res["device_error"], "summary_build_gbs": res["summary_build_gbs"]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
         dist.destroy_process_group()
     return 0
 

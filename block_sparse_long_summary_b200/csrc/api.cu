@@ -173,7 +173,9 @@ cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void
         COBS_TRY(check_ptr(Vc, "Vc"));
     }
     if (t_begin < 0 || t_begin > p->T) return fail(COBS_ERR_INVALID_ARG, "t_begin %d outside [0, T]", t_begin);
-    cudaError_t e = cobs::launch_summaries(m, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, (cudaStream_t)stream);
+    int* flag = nullptr;
+    COBS_TRY(device_flag(&flag));
+    cudaError_t e = cobs::launch_summaries(m, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, (cudaStream_t)stream, flag);
     if (e != cudaSuccess) return cuda_fail(e, "cobs_build_summaries launch");
     return COBS_OK;
 }

@@ -1,5 +1,6 @@
-// Decode attention at position T-1: split-K over branch chunks, then a log-sum-exp merge
-// that applies the gates. Also the first prefill path (one CTA per position and group).
+// Decode attention at position T-1 for float32 (split-K over branch chunks, then a
+// log-sum-exp merge that applies the gates; the bf16 path is decode_stream.cu), and the
+// per-position prefill path (one CTA per position and group).
 //
 // NSA's three paths (Janus issue #181) — compression (CMP), selection (SLC), sliding
 // window (WIN) — mixed by per-head gates; COBS (gist.science explainer, §2.3) changes only
@@ -30,50 +31,6 @@ __device__ __forceinline__ void decode_chunk(const AttnArgs& a, int id, int& br,
     } else {
         br = kCMP;
         ch = id - a.nS - a.nW;
-    }
-}
-
-// ---------------------------------------------------------------- bf16 chunk kernel
-template <int D>
-__global__ void __launch_bounds__(kCK) decode_chunk_bf16(AttnArgs a) {
-    constexpr int RS = D + 8;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-    __nv_bfloat16* sV = sK + kCK * RS;
-    // [4][16][D] combine scratch, reused over sK/sV once every warp has finished its MMAs
-    float* scratch = reinterpret_cast<float*>(smem_raw);
-    __shared__ uint32_t vmask[kCK / 32];
-    __shared__ float wm[64], wl[64], sm[16], sl[16];
-    __shared__ float so_buf[16 * D];
-    __shared__ __align__(8) uint64_t bar;
-
-    const int unit = blockIdx.y;
-    const int b = unit / a.Hkv, g = unit % a.Hkv;
-    const int t = a.T - 1;
-    int br, ch;
-    decode_chunk(a, blockIdx.x, br, ch);
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
-        fence_barrier_init();
-    }
-    const int32_t* idx_row = a.idx + (size_t)unit * a.k;
-    bool ok = true;
-    stage_chunk<__nv_bfloat16, D, kCK>(a, unit, idx_row, t, br, ch, sK, sV, vmask, &bar, 0, ok);
-
-    uint32_t qa[D / 16][4];
-    load_q_frags<D>(static_cast<const __nv_bfloat16*>(a.Q) + ((size_t)b * a.Hq + (size_t)g * a.G) * D, a.G, qa);
-    WarpState<D> st;
-    st.init();
-    if (ok) warp_chunk_mma<D>(st, qa, sK, sV, vmask, a.sl2);
-    cta_combine<D>(st, a.G, a.sl2, scratch, wm, wl, sm, sl, so_buf);
-    float* rec = a.part + ((size_t)unit * a.nchunks + blockIdx.x) * a.G * part_stride(D);
-    for (int h = threadIdx.x; h < a.G; h += blockDim.x) {
-        rec[h * part_stride(D) + 0] = sm[h];
-        rec[h * part_stride(D) + 1] = sl[h];
-    }
-    for (int e = threadIdx.x; e < a.G * D; e += blockDim.x) {
-        const int h = e / D, c = e % D;
-        rec[h * part_stride(D) + 4 + c] = so_buf[e];
     }
 }
 
@@ -377,27 +334,13 @@ AttnArgs make_args(const Dims& m, const void* Q, const void* K, const void* V, c
 }
 
 template <int D>
-size_t decode_smem_bf16() { return (size_t)2 * kCK * (D + 8) * 2; }  // >= 4*16*D*4 combine scratch
-template <int D>
 size_t decode_smem_f32() { return (size_t)2 * kCKf * (D + 4) * 4 + (size_t)16 * D * 4 + (size_t)16 * kCKf * 4; }
 
 template <int D>
 cudaError_t launch_decode_d(const Dims& m, AttnArgs a, cudaStream_t s) {
     const dim3 grid(a.nchunks, m.units());
-    cudaError_t e;
-    if (m.dtype == COBS_BF16) {
-        const size_t smem = decode_smem_bf16<D>();
-        e = cudaFuncSetAttribute(decode_chunk_bf16<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        count_launch();
-        decode_chunk_bf16<D><<<grid, kCK, smem, s>>>(a);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        count_launch();
-        decode_merge<__nv_bfloat16, D><<<dim3(m.G, m.units()), 128, 0, s>>>(a, a.sl2);
-        return cudaGetLastError();
-    }
     const size_t smem = decode_smem_f32<D>();
-    e = cudaFuncSetAttribute(decode_chunk_f32<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_chunk_f32<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
     decode_chunk_f32<D><<<grid, kCKf, smem, s>>>(a);
@@ -430,17 +373,17 @@ cudaError_t launch_prefill_d(const Dims& m, AttnArgs a, cudaStream_t s) {
 }  // namespace
 
 size_t decode_workspace_bytes(const Dims& m) {
-    const int CK = m.dtype == COBS_BF16 ? kCK : kCKf;
+    if (m.dtype == COBS_BF16) return decode_stream_workspace_bytes(m);
     AttnArgs a = make_args(m, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                           nullptr, 1, CK);
+                           nullptr, 1, kCKf);
     return (size_t)m.units() * a.nchunks * m.G * part_stride(m.d) * sizeof(float);
 }
 
 cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                           const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                           cudaStream_t s, int* err) {
-    const int CK = m.dtype == COBS_BF16 ? kCK : kCKf;
-    AttnArgs a = make_args(m, Q, K, V, Kc, Vc, idx, gates, O, ws, err, 1, CK);
+    if (m.dtype == COBS_BF16) return launch_decode_stream(m, Q, K, V, Kc, Vc, idx, gates, O, ws, s, err);
+    AttnArgs a = make_args(m, Q, K, V, Kc, Vc, idx, gates, O, ws, err, 1, kCKf);
     return m.d == 128 ? launch_decode_d<128>(m, a, s) : launch_decode_d<64>(m, a, s);
 }
 
@@ -492,6 +435,9 @@ size_t prefill_workspace_bytes(const Dims&) { return 0; }
 cudaError_t launch_prefill(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                            const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                            cudaStream_t s, int* err) {
+    // tensor-core tiles for bf16, d = 128, 16 heads per group; the per-position kernel otherwise
+    const cudaError_t tc = launch_prefill_tc(m, Q, K, V, Kc, Vc, idx, gates, O, s, err);
+    if (tc != cudaErrorNotSupported) return tc;
     const int CK = m.dtype == COBS_BF16 ? kCK : kCKf;
     AttnArgs a = make_args(m, Q, K, V, Kc, Vc, idx, gates, O, ws, err, m.T, CK);
     return m.d == 128 ? launch_prefill_d<128>(m, a, s) : launch_prefill_d<64>(m, a, s);

@@ -1,0 +1,478 @@
+// Decode attention, bf16: stream-K over 32-key tiles with TMA tensor tiles.
+//
+// What is computed is the decode attention of the NSA paths (Janus issue #181: CMP, SLC,
+// WIN) with COBS-selected blocks (gist.science explainer §2.3); only the selected blocks,
+// the window and the compressed tokens are read ("Problemstellung": decode is bound by the
+// KV-cache read). How it is scheduled:
+//
+// * Every (batch, KV-head) unit contributes its tiles in the order SLC (2 tiles per
+//   selected block), WIN (the window rows in 32-row tiles), CMP (compressed tokens in
+//   32-row tiles). The tiles of all units form one sequence that is cut into equal,
+//   contiguous ranges, one per warp, so every SM streams the same number of bytes.
+// * Each warp is its own producer: TMA 2-D loads (128-byte swizzle, no multicast) of the
+//   K and V halves of a tile into a private 3-stage ring, an mbarrier per stage.
+// * The G query heads of the unit are the m16 rows of mma.sync tiles (rows >= G are zero);
+//   the online softmax state lives in registers.
+// * A warp flushes one partial record (m, l, o) per (unit, branch) piece it covers;
+//   decode_stream_merge combines the records of each (unit, branch), applies the gates
+//   and writes O.
+#include <algorithm>
+
+#include "common.cuh"
+#include "dims.h"
+#include "tma.h"
+
+namespace cobs {
+namespace {
+
+#ifndef COBS_DECODE_TK
+#define COBS_DECODE_TK 32
+#endif
+#ifndef COBS_DECODE_STAGES
+#define COBS_DECODE_STAGES 3
+#endif
+#ifndef COBS_DECODE_WARPS
+#define COBS_DECODE_WARPS 4
+#endif
+constexpr int kTK = COBS_DECODE_TK;          // keys per tile (16 or 32)
+constexpr int kStages = COBS_DECODE_STAGES;  // ring depth per warp
+constexpr int kWarps = COBS_DECODE_WARPS;    // independent warps per CTA
+static_assert(kTK == 16 || kTK == 32, "tile of 16 or 32 keys");
+constexpr uint32_t kFull = 0xffffffffu;
+
+struct StreamArgs {
+    const __nv_bfloat16* Q;
+    const int32_t* idx;
+    const float* gates;
+    __nv_bfloat16* O;
+    float* rec;
+    int* err;
+    int Hq, Hkv, G, T, L, k, W, nB, nC;
+    int tS, tW, tC, tpu;  // tiles per unit: SLC, WIN, CMP, total
+    long long total;      // units * tpu
+    int tpw;              // tiles per warp
+    int maxw;             // record slots per (unit, branch)
+    float sl2;            // log2(e) / sqrt(d)
+};
+
+__host__ __device__ __forceinline__ int rec_floats(int D) { return D + 4; }  // m, l, pad, pad, o[D]
+
+__host__ __device__ __forceinline__ int branch_begin(const StreamArgs& a, int br) {
+    return br == 0 ? 0 : (br == 1 ? a.tS : a.tS + a.tW);
+}
+__host__ __device__ __forceinline__ int branch_len(const StreamArgs& a, int br) {
+    return br == 0 ? a.tS : (br == 1 ? a.tW : a.tC);
+}
+
+struct Tile {
+    int unit, br, j;   // branch 0 SLC, 1 WIN, 2 CMP; j = tile within the branch
+    int row;           // first global row in K/V (SLC, WIN) or Kc/Vc (CMP)
+    uint32_t mask;     // valid keys of the tile
+};
+
+// Tile gt of the global sequence. Uniform across the warp.
+__device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt) {
+    Tile tl;
+    tl.unit = (int)(gt / a.tpu);
+    int l = (int)(gt - (long long)tl.unit * a.tpu);
+    const int t = a.T - 1;
+    if (l < a.tS) {
+        tl.br = 0;
+        tl.j = l;
+        const int bi = a.idx[(size_t)tl.unit * a.k + l / (64 / kTK)];
+        tl.mask = 0u;
+        tl.row = 0;
+        if (bi >= 0) {
+            if (bi >= a.nB) {
+                report_error(a.err, kErrBadIndex);
+            } else {
+                tl.row = tl.unit * a.T + bi * a.L + (l % (64 / kTK)) * kTK;
+                tl.mask = kTK == 32 ? kFull : 0xFFFFu;
+            }
+        }
+    } else if (l < a.tS + a.tW) {
+        tl.br = 1;
+        tl.j = l - a.tS;
+        const int r0 = max(0, t - a.W + 1) + tl.j * kTK;
+        tl.row = tl.unit * a.T + r0;
+        const int n = min(kTK, t + 1 - r0);
+        tl.mask = n >= 32 ? kFull : ((1u << n) - 1u);  // n <= kTK
+    } else {
+        tl.br = 2;
+        tl.j = l - a.tS - a.tW;
+        const int c0 = tl.j * kTK;
+        tl.row = tl.unit * a.nC + c0;
+        const int n = min(kTK, a.nC - c0);
+        tl.mask = n >= 32 ? kFull : ((1u << n) - 1u);
+    }
+    return tl;
+}
+
+template <int D>
+struct WState {
+    float m0, m1, l0, l1;
+    float o[D / 8][4];
+    __device__ void init() {
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+    }
+};
+
+template <int D>
+__device__ __forceinline__ void load_q(const __nv_bfloat16* q, int G, uint32_t (&qa)[D / 16][4], int lane) {
+    const int r0 = lane >> 2, r1 = r0 + 8, c = 2 * (lane & 3);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q + (size_t)r0 * D + ks * 16 + c);
+        const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q + (size_t)r1 * D + ks * 16 + c);
+        qa[ks][0] = r0 < G ? q0[0] : 0u;
+        qa[ks][1] = r1 < G ? q1[0] : 0u;
+        qa[ks][2] = r0 < G ? q0[4] : 0u;
+        qa[ks][3] = r1 < G ? q1[4] : 0u;
+    }
+}
+
+// Byte offset of 16-byte chunk `cc` (0..7) of row `r` in a 128-byte-swizzled 32-row box.
+__device__ __forceinline__ uint32_t swz(int r, int cc) { return (uint32_t)(r * 128 + ((cc ^ (r & 7)) << 4)); }
+
+// One tile: S = Q K^T over kTK keys, online softmax update, O += P V.
+template <int D>
+__device__ __forceinline__ void tile_mma(WState<D>& st, const uint32_t (&qa)[D / 16][4], const unsigned char* sK,
+                                         const unsigned char* sV, uint32_t vm, float sl2, int lane) {
+    constexpr int kHalf = kTK * 128;  // bytes of one 64-column box
+    constexpr int NP = kTK / 16;      // 16-key groups
+    const int mi = lane >> 3;
+    float s[2 * NP][4];
+#pragma unroll
+    for (int nt = 0; nt < 2 * NP; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+#pragma unroll
+        for (int np = 0; np < NP; ++np) {
+            const int r = np * 16 + (lane & 7) + ((mi >> 1) << 3);
+            const int cc = (ks & 3) * 2 + (mi & 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(b0, b1, b2, b3, sK + (ks >> 2) * kHalf + swz(r, cc));
+            mma_bf16_16816(s[2 * np], qa[ks], b0, b1);
+            mma_bf16_16816(s[2 * np + 1], qa[ks], b2, b3);
+        }
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2 * NP; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int slot = nt * 8 + 2 * (lane & 3) + j;
+            const bool ok = (vm >> slot) & 1u;
+            s[nt][j] = ok ? s[nt][j] : -INFINITY;
+            s[nt][2 + j] = ok ? s[nt][2 + j] : -INFINITY;
+            mx0 = fmaxf(mx0, s[nt][j]);
+            mx1 = fmaxf(mx1, s[nt][2 + j]);
+        }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
+    const float nm0 = fmaxf(st.m0, mx0), nm1 = fmaxf(st.m1, mx1);
+    const float al0 = exp2f((st.m0 - nm0) * sl2), al1 = exp2f((st.m1 - nm1) * sl2);
+    st.m0 = nm0;
+    st.m1 = nm1;
+    float ps0 = 0.0f, ps1 = 0.0f;
+    uint32_t pa[NP][4];
+#pragma unroll
+    for (int nt = 0; nt < 2 * NP; ++nt) {
+        const float p0 = exp2f((s[nt][0] - nm0) * sl2), p1 = exp2f((s[nt][1] - nm0) * sl2);
+        const float p2 = exp2f((s[nt][2] - nm1) * sl2), p3 = exp2f((s[nt][3] - nm1) * sl2);
+        ps0 += p0 + p1;
+        ps1 += p2 + p3;
+        pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
+        pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
+    }
+    st.l0 = st.l0 * al0 + ps0;
+    st.l1 = st.l1 * al1 + ps1;
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+        st.o[nd][0] *= al0;
+        st.o[nd][1] *= al0;
+        st.o[nd][2] *= al1;
+        st.o[nd][3] *= al1;
+    }
+#pragma unroll
+    for (int kk = 0; kk < NP; ++kk) {
+#pragma unroll
+        for (int np = 0; np < D / 16; ++np) {
+            const int r = kk * 16 + (lane & 7) + ((mi & 1) << 3);
+            const int cc = (np & 3) * 2 + (mi >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4_trans(b0, b1, b2, b3, sV + (np >> 2) * kHalf + swz(r, cc));
+            mma_bf16_16816(st.o[2 * np], pa[kk], b0, b1);
+            mma_bf16_16816(st.o[2 * np + 1], pa[kk], b2, b3);
+        }
+    }
+}
+
+// Partial record of (unit, br) written by warp v.
+template <int D>
+__device__ __forceinline__ void flush(const StreamArgs& a, long long v, int unit, int br, WState<D>& st, int lane) {
+    float l0 = st.l0, l1 = st.l1;
+    l0 += __shfl_xor_sync(kFull, l0, 1);
+    l0 += __shfl_xor_sync(kFull, l0, 2);
+    l1 += __shfl_xor_sync(kFull, l1, 1);
+    l1 += __shfl_xor_sync(kFull, l1, 2);
+    const long long first_v = ((long long)unit * a.tpu + branch_begin(a, br)) / a.tpw;
+    float* rec = a.rec + (((size_t)unit * 3 + br) * a.maxw + (size_t)(v - first_v)) * a.G * rec_floats(D);
+    const int r0 = lane >> 2, r1 = r0 + 8, c = 2 * (lane & 3);
+    if ((lane & 3) == 0) {
+        if (r0 < a.G) {
+            rec[r0 * rec_floats(D) + 0] = st.m0;
+            rec[r0 * rec_floats(D) + 1] = l0;
+        }
+        if (r1 < a.G) {
+            rec[r1 * rec_floats(D) + 0] = st.m1;
+            rec[r1 * rec_floats(D) + 1] = l1;
+        }
+    }
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+        if (r0 < a.G)
+            *reinterpret_cast<float2*>(rec + r0 * rec_floats(D) + 4 + nd * 8 + c) = make_float2(st.o[nd][0], st.o[nd][1]);
+        if (r1 < a.G)
+            *reinterpret_cast<float2*>(rec + r1 * rec_floats(D) + 4 + nd * 8 + c) = make_float2(st.o[nd][2], st.o[nd][3]);
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                     const __grid_constant__ CUtensorMap tmV,
+                                                                     const __grid_constant__ CUtensorMap tmKc,
+                                                                     const __grid_constant__ CUtensorMap tmVc,
+                                                                     StreamArgs a) {
+    constexpr int kBox = kTK * 128;              // one 64-column box
+    constexpr int kMat = (D / 64) * kBox;        // K or V tile
+    constexpr int kStage = 2 * kMat;             // K + V
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t bars[kWarps][kStages];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // 1024-byte aligned ring of this warp
+    unsigned char* base = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    unsigned char* ring = base + (size_t)warp * kStages * kStage;
+    uint64_t* bar = bars[warp];
+
+    // the merge grid may be scheduled now; it still waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const long long v = (long long)blockIdx.x * kWarps + warp;
+    const long long g0 = v * a.tpw;
+    const long long g1 = min(a.total, g0 + a.tpw);
+    if (g0 >= g1) return;
+    const int n = (int)(g1 - g0);
+
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&bar[s], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+
+    auto issue = [&](int i, int s) {  // lane 0 only
+        const Tile tl = tile_at(a, g0 + i);
+        if (tl.mask == 0u) return;
+        const CUtensorMap* mk = tl.br == 2 ? &tmKc : &tmK;
+        const CUtensorMap* mv = tl.br == 2 ? &tmVc : &tmV;
+        unsigned char* dst = ring + (size_t)s * kStage;
+        mbar_arrive_expect_tx(&bar[s], kStage);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+            tma_load_2d(dst + h * kBox, mk, h * 64, tl.row, &bar[s]);
+            tma_load_2d(dst + kMat + h * kBox, mv, h * 64, tl.row, &bar[s]);
+        }
+    };
+    if (lane == 0)
+        for (int i = 0; i < kStages && i < n; ++i) issue(i, i);
+
+    uint32_t phase = 0;  // bit s: parity of the next completion of stage s
+    uint32_t qa[D / 16][4];
+    WState<D> st;
+    st.init();
+    Tile cur = tile_at(a, g0);
+    load_q<D>(a.Q + (size_t)cur.unit * a.G * D, a.G, qa, lane);
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+        const int s = i % kStages;
+        const Tile tl = tile_at(a, g0 + i);
+        if (tl.unit != cur.unit || tl.br != cur.br) {
+            flush<D>(a, v, cur.unit, cur.br, st, lane);
+            st.init();
+            if (tl.unit != cur.unit) load_q<D>(a.Q + (size_t)tl.unit * a.G * D, a.G, qa, lane);
+            cur = tl;
+        }
+        if (tl.mask != 0u) {
+            if (ok) ok = mbar_wait(&bar[s], (phase >> s) & 1u, a.err);
+            ok = __all_sync(kFull, ok);
+            phase ^= 1u << s;
+            if (ok) tile_mma<D>(st, qa, ring + (size_t)s * kStage, ring + (size_t)s * kStage + kMat, tl.mask, a.sl2, lane);
+        }
+        __syncwarp();
+        if (lane == 0 && ok && i + kStages < n) {
+            fence_proxy_async();
+            issue(i + kStages, s);
+        }
+    }
+    flush<D>(a, v, cur.unit, cur.br, st, lane);
+}
+
+// grid (G, units), 4 warps. Warp 0 folds the SLC records of the (unit, head), warp 1 the WIN
+// records, warps 2 and 3 the even and odd CMP records; each warp issues the loads of 4 records
+// at a time. Warp 0 then combines, applies the gates (cmp, slc, win) and writes O. Launched as a
+// programmatic dependent of the decode kernel: it waits for that grid before reading records.
+template <int D>
+__global__ void __launch_bounds__(128) decode_stream_merge(StreamArgs a) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float wM[4], wL[4];
+    __shared__ float wO[4][D];
+    const int h = blockIdx.x, unit = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int hq_row = unit * a.G + h;  // = b * Hq + g * G + h
+    const int c0 = lane * 4;
+    const int br = warp < 2 ? warp : 2;
+    const int len = branch_len(a, br);
+    int nslots = 0;
+    if (len > 0) {
+        const long long s0 = (long long)unit * a.tpu + branch_begin(a, br);
+        nslots = (int)((s0 + len - 1) / a.tpw - s0 / a.tpw) + 1;
+    }
+    const int sl0 = warp < 2 ? 0 : warp - 2, step = warp < 2 ? 1 : 2;
+    const float* base = a.rec + ((size_t)unit * 3 + br) * a.maxw * a.G * rec_floats(D) + (size_t)h * rec_floats(D);
+    const size_t rs = (size_t)a.G * rec_floats(D);
+    float M = -INFINITY, Lsum = 0.0f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sl = sl0; sl < nslots; sl += 4 * step) {
+        float m[4], l[4];
+        float4 o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int s = sl + q * step;
+            m[q] = -INFINITY;
+            l[q] = 0.0f;
+            o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s < nslots) {
+                const float* rec = base + (size_t)s * rs;
+                m[q] = __ldcg(rec);
+                l[q] = __ldcg(rec + 1);
+                if (c0 < D) o[q] = __ldcg(reinterpret_cast<const float4*>(rec + 4 + c0));
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (m[q] == -INFINITY) continue;
+            const float nM = fmaxf(M, m[q]);
+            const float fa = M == -INFINITY ? 0.0f : exp2f((M - nM) * a.sl2);
+            const float fb = exp2f((m[q] - nM) * a.sl2);
+            Lsum = Lsum * fa + l[q] * fb;
+            acc[0] = acc[0] * fa + o[q].x * fb;
+            acc[1] = acc[1] * fa + o[q].y * fb;
+            acc[2] = acc[2] * fa + o[q].z * fb;
+            acc[3] = acc[3] * fa + o[q].w * fb;
+            M = nM;
+        }
+    }
+    if (lane == 0) {
+        wM[warp] = M;
+        wL[warp] = Lsum;
+    }
+    if (c0 < D)
+        for (int j = 0; j < 4; ++j) wO[warp][c0 + j] = acc[j];
+    __syncthreads();
+    if (warp != 0 || c0 >= D) return;
+    const float* gate = a.gates + (size_t)hq_row * 3;
+    float out[4] = {0.f, 0.f, 0.f, 0.f};
+    // branch results: SLC = warp 0, WIN = warp 1, CMP = warps 2 + 3
+    for (int b2 = 0; b2 < 3; ++b2) {
+        const int w0 = b2, w1 = b2 == 2 ? 3 : b2;
+        const float GM = fmaxf(wM[w0], wM[w1]);
+        if (GM == -INFINITY) continue;
+        const float f0 = wM[w0] == -INFINITY ? 0.0f : exp2f((wM[w0] - GM) * a.sl2);
+        const float f1 = (w1 == w0 || wM[w1] == -INFINITY) ? 0.0f : exp2f((wM[w1] - GM) * a.sl2);
+        const float GL = wL[w0] * f0 + (w1 == w0 ? 0.0f : wL[w1] * f1);
+        if (!(GL > 0.0f)) continue;
+        const float gw = gate[b2 == 0 ? 1 : (b2 == 1 ? 2 : 0)] / GL;  // gates are (cmp, slc, win)
+        for (int j = 0; j < 4; ++j)
+            out[j] += gw * (wO[w0][c0 + j] * f0 + (w1 == w0 ? 0.0f : wO[w1][c0 + j] * f1));
+    }
+    __nv_bfloat16* o = a.O + (size_t)hq_row * D + c0;
+    for (int j = 0; j < 4; ++j) o[j] = __float2bfloat16_rn(out[j]);
+}
+
+StreamArgs make_stream_args(const Dims& m) {
+    StreamArgs a{};
+    a.Hq = m.Hq; a.Hkv = m.Hkv; a.G = m.G; a.T = m.T; a.L = m.L; a.k = m.k; a.W = m.W; a.nB = m.nB; a.nC = m.nC;
+    a.tS = m.k * (m.L / kTK);
+    a.tW = (std::min(m.W, m.T) + kTK - 1) / kTK;
+    a.tC = (m.nC + kTK - 1) / kTK;
+    a.tpu = a.tS + a.tW + a.tC;
+    a.total = (long long)m.units() * a.tpu;
+    const long long warps_wanted = (long long)sm_count() * kWarps;
+    a.tpw = (int)std::max<long long>(1, (a.total + warps_wanted - 1) / warps_wanted);
+    a.maxw = std::max(a.tS, std::max(a.tW, a.tC)) / a.tpw + 2;
+    a.sl2 = 1.4426950408889634f / sqrtf((float)m.d);
+    return a;
+}
+
+template <int D>
+size_t stream_smem() { return (size_t)kWarps * kStages * 2 * (D / 64) * kTK * 128 + 1024; }
+
+template <int D>
+cudaError_t launch_stream_d(const Dims& m, StreamArgs a, const void* K, const void* V, const void* Kc, const void* Vc,
+                            cudaStream_t s) {
+    CUtensorMap tk, tv, tkc, tvc;
+    const uint64_t kvrows = (uint64_t)m.units() * m.T;
+    const uint64_t crows = m.nC > 0 ? (uint64_t)m.units() * m.nC : kvrows;
+    if (!encode_tmap_bf16_2d(&tk, K, kvrows, D, kTK) || !encode_tmap_bf16_2d(&tv, V, kvrows, D, kTK) ||
+        !encode_tmap_bf16_2d(&tkc, m.nC > 0 ? Kc : K, crows, D, kTK) ||
+        !encode_tmap_bf16_2d(&tvc, m.nC > 0 ? Vc : V, crows, D, kTK))
+        return cudaErrorInvalidValue;
+    const size_t smem = stream_smem<D>();
+    cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long nwarps = (a.total + a.tpw - 1) / a.tpw;
+    const int grid = (int)((nwarps + kWarps - 1) / kWarps);
+    count_launch();
+    decode_stream_kernel<D><<<grid, kWarps * 32, smem, s>>>(tk, tv, tkc, tvc, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the merge grid may launch while the decode grid drains; it waits for it on the device
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(m.G, m.units());
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    count_launch();
+    return cudaLaunchKernelEx(&cfg, decode_stream_merge<D>, a);
+}
+
+}  // namespace
+
+size_t decode_stream_workspace_bytes(const Dims& m) {
+    const StreamArgs a = make_stream_args(m);
+    return (size_t)m.units() * 3 * a.maxw * m.G * rec_floats(m.d) * sizeof(float);
+}
+
+cudaError_t launch_decode_stream(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                                 const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
+                                 cudaStream_t s, int* err) {
+    StreamArgs a = make_stream_args(m);
+    a.Q = static_cast<const __nv_bfloat16*>(Q);
+    a.idx = idx;
+    a.gates = gates;
+    a.O = static_cast<__nv_bfloat16*>(O);
+    a.rec = static_cast<float*>(ws);
+    a.err = err;
+    return m.d == 128 ? launch_stream_d<128>(m, a, K, V, Kc, Vc, s) : launch_stream_d<64>(m, a, K, V, Kc, Vc, s);
+}
+
+}  // namespace cobs

@@ -41,13 +41,17 @@ void score_constants(int d, float alpha, float* isd, float* c2);
 // ---- launchers (return cudaSuccess or the launch error) ----
 cudaError_t launch_summaries(const Dims& m, const void* K, const void* V, const float* Pk,
                              const float* Pv, int t_begin, float* summ, void* Kc, void* Vc,
-                             cudaStream_t s);
+                             cudaStream_t s, int* err);
 
 size_t select_workspace_bytes(const Dims& m, int prefill);
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx,
                           void* ws, cudaStream_t s, int* err);
 
 size_t decode_workspace_bytes(const Dims& m);
+size_t decode_stream_workspace_bytes(const Dims& m);
+cudaError_t launch_decode_stream(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                                 const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
+                                 cudaStream_t s, int* err);
 cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                           const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                           cudaStream_t s, int* err);
@@ -59,6 +63,10 @@ cudaError_t launch_decode_noalloc(const Dims& m, const void* Q, const void* K, c
                                   int* err);
 
 size_t prefill_workspace_bytes(const Dims& m);
+// tcgen05 prefill (bf16, d = 128, G = 16); cudaErrorNotSupported for other shapes.
+cudaError_t launch_prefill_tc(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
+                              const void* Vc, const int32_t* idx, const float* gates, void* O, cudaStream_t s,
+                              int* err);
 cudaError_t launch_prefill(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                            const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                            cudaStream_t s, int* err);

@@ -14,6 +14,8 @@
 // are reproducible bit for bit. Ties go to the lower block index.
 #include <float.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "dims.h"
 
@@ -136,102 +138,169 @@ __device__ __forceinline__ float block_score(const float* tile, const float* qs,
 }
 
 // ---------------------------------------------------------------------------- decode
-// grid (nsplit, units); one warp; the CTA scores groups [split*gpc, ...) of its unit with
-// a 2-stage bulk-copy pipeline, keeps a top-k list, then either writes the answer (one
-// split) or deposits its list and, if it is the last split of the unit to finish
-// (atomic ticket, no waiting), merges all lists.
+// Warp-wide sorted list helpers: one (score, index) entry per lane, best first.
+__device__ __forceinline__ void cmp_swap(float& s, int& i, int j, bool up, int lane) {
+    const float os = __shfl_xor_sync(kFull, s, j);
+    const int oi = __shfl_xor_sync(kFull, i, j);
+    const bool low = (lane & j) == 0;
+    const bool ob = better(os, oi, s, i);
+    if ((low == up) ? ob : (!ob && !(os == s && oi == i))) {
+        s = os;
+        i = oi;
+    }
+}
+
+// Sort the 32 entries best first (bitonic network).
+__device__ __forceinline__ void warp_sort_best_first(float& s, int& i, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) cmp_swap(s, i, j, (lane & k) == 0, lane);
+    }
+}
+
+// (s, i) and (bs, bi) are both sorted best first; keep the best 32 of their union, sorted.
+__device__ __forceinline__ void warp_merge_best_first(float& s, int& i, float bs, int bi, int lane) {
+    const float rs = __shfl_sync(kFull, bs, 31 - lane);
+    const int ri = __shfl_sync(kFull, bi, 31 - lane);
+    if (better(rs, ri, s, i)) {
+        s = rs;
+        i = ri;
+    }
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) cmp_swap(s, i, j, true, lane);
+}
+
+// Canonical score of block `lane` of a 32-block group read straight from global memory
+// (coalesced: one 512-byte row per warp load). The mean and variance chains are independent,
+// so half of each is loaded, then consumed, then the other half.
+template <int D>
+__device__ __forceinline__ float block_score_global(const float* grp, const float* qs, const float* q2, int lane,
+                                                    float isd, float c2) {
+    const float4* mu4 = reinterpret_cast<const float4*>(grp) + lane;
+    const float4* var4 = reinterpret_cast<const float4*>(grp + D * 32) + lane;
+    constexpr int H = D / 8;  // float4s per half-chain
+    float a = 0.0f, v = 0.0f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float4 m[H], s[H];
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            m[i] = __ldcs(mu4 + (half * H + i) * 32);
+            s[i] = __ldcs(var4 + (half * H + i) * 32);
+        }
+#pragma unroll
+        for (int i = 0; i < H; ++i) {
+            const int c = 4 * (half * H + i);
+            a = __fmaf_rn(qs[c + 0], m[i].x, a);
+            a = __fmaf_rn(qs[c + 1], m[i].y, a);
+            a = __fmaf_rn(qs[c + 2], m[i].z, a);
+            a = __fmaf_rn(qs[c + 3], m[i].w, a);
+            v = __fmaf_rn(q2[c + 0], s[i].x, v);
+            v = __fmaf_rn(q2[c + 1], s[i].y, v);
+            v = __fmaf_rn(q2[c + 2], s[i].z, v);
+            v = __fmaf_rn(q2[c + 3], s[i].w, v);
+        }
+    }
+    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
+}
+
+constexpr int kSelWarps = 4;
+
+// grid (nsplit, units), 4 warps. Warp w of split s scores groups [(s*4 + w)*gpw, +gpw) of its
+// unit and keeps a sorted best-first list; the 4 lists are merged in shared memory. With one
+// split the CTA writes the answer. Otherwise every CTA deposits its list and takes an atomic
+// ticket (nobody waits); the CTA that takes the last ticket merges all lists of the unit with a
+// shared-memory tree and writes the answer. The result is the top-k under a strict total order,
+// so it does not depend on arrival order. The ticket counter returns to zero by itself.
 template <typename T, int D>
-__global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
-                                                           int32_t* __restrict__ idx, float* __restrict__ ws_s,
-                                                           int* __restrict__ ws_i, unsigned* __restrict__ ws_ctr,
-                                                           int G, int nG, int ncand, int k, int gpc, int nsplit,
-                                                           float isd, float c2, int* err) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    float* tiles = reinterpret_cast<float*>(smem_raw);  // [2][2*D*32]
+__global__ void __launch_bounds__(kSelWarps * 32) select_decode_kernel(
+    const T* __restrict__ Q, const float* __restrict__ summ, int32_t* __restrict__ idx, float* __restrict__ ws_s,
+    int* __restrict__ ws_i, unsigned* __restrict__ ws_ctr, int G, int nG, int ncand, int k, int gpw, int nsplit,
+    float isd, float c2) {
     __shared__ float qs[D], q2[D];
-    __shared__ __align__(8) uint64_t bar[2];
-    const int lane = threadIdx.x;
+    __shared__ float ls_sh[16][32];
+    __shared__ int li_sh[16][32];
+    __shared__ unsigned ticket_sh;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.y;
     const int split = blockIdx.x;
     const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
-    const int g0 = split * gpc;
-    const int g1 = min(nGc, g0 + gpc);
     const float* usum = summ + (size_t)unit * nG * 2 * D * 32;
-    constexpr uint32_t kTileBytes = 2 * D * 32 * 4;
-
-    if (lane == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
-    // prologue: first two tiles in flight
-    if (lane == 0) {
-        for (int st = 0; st < 2 && g0 + st < g1; ++st) {
-            mbar_arrive_expect_tx(&bar[st], kTileBytes);
-            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(g0 + st) * 2 * D * 32, kTileBytes, &bar[st]);
-        }
-    }
-    // group query (all lanes), overlapped with the copies
     {
         // unit = b * Hkv + g and Hq = Hkv * G, so the group's first head row is unit * G
         const T* qg = Q + (size_t)unit * G * D;
-        for (int c = lane; c < D; c += 32) group_query(qg, G, D, c, qs[c], q2[c]);
+        for (int c = tid; c < D; c += blockDim.x) group_query(qg, G, D, c, qs[c], q2[c]);
     }
-    __syncwarp();
+    __syncthreads();
 
-    TopK tk;
-    tk.init();
-    bool ok = true;
-    for (int g = g0, it = 0; g < g1; ++g, ++it) {
-        const int st = it & 1;
-        const uint32_t parity = (it >> 1) & 1;
-        if (ok) ok = mbar_wait(&bar[st], parity, err);
-        ok = __all_sync(kFull, ok);
+    float ls = -INFINITY;
+    int li = kInvalid;
+    const int g0 = (split * kSelWarps + warp) * gpw;
+    for (int g = g0; g < min(nGc, g0 + gpw); ++g) {
         const int b = g * kGroupBlocks + lane;
-        float sc = -INFINITY;
-        if (ok) sc = block_score<D>(tiles + st * 2 * D * 32, qs, q2, lane, isd, c2);
-        __syncwarp();
-        // refill this stage with group g + 2
-        if (lane == 0 && ok && g + 2 < g1) {
-            fence_proxy_async();
-            mbar_arrive_expect_tx(&bar[st], kTileBytes);
-            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(g + 2) * 2 * D * 32, kTileBytes, &bar[st]);
+        float sc = block_score_global<D>(usum + (size_t)g * 2 * D * 32, qs, q2, lane, isd, c2);
+        int bi = b;
+        if (b >= ncand) {
+            sc = -INFINITY;
+            bi = kInvalid;
         }
-        tk.offer(sc, b, ok && b < ncand, k, lane);
-    }
-
-    if (nsplit == 1) {
-        emit_sorted(tk, k, lane, idx + (size_t)unit * k);
-        return;
-    }
-    float* my_s = ws_s + ((size_t)unit * nsplit + split) * k;
-    int* my_i = ws_i + ((size_t)unit * nsplit + split) * k;
-    if (lane < k) {
-        my_s[lane] = tk.s;
-        my_i[lane] = tk.i;
-    }
-    __threadfence();
-    __syncwarp();
-    unsigned ticket = 0;
-    if (lane == 0) ticket = atomicInc(ws_ctr + unit, (unsigned)(nsplit - 1));
-    ticket = __shfl_sync(kFull, ticket, 0);
-    if (ticket != (unsigned)(nsplit - 1)) return;
-    __threadfence();
-    TopK all;
-    all.init();
-    for (int sp = 0; sp < nsplit; ++sp) {
-        const float* ps = ws_s + ((size_t)unit * nsplit + sp) * k;
-        const int* pi = ws_i + ((size_t)unit * nsplit + sp) * k;
-        float cs = -INFINITY;
-        int ci = kInvalid;
-        if (lane < k) {
-            cs = __ldcg(ps + lane);
-            ci = __ldcg(pi + lane);
+        warp_sort_best_first(sc, bi, lane);
+        if (g == g0) {
+            ls = sc;
+            li = bi;
+        } else {
+            warp_merge_best_first(ls, li, sc, bi, lane);
         }
-        all.offer(cs, ci, lane < k && ci != kInvalid, k, lane);
     }
-    emit_sorted(all, k, lane, idx + (size_t)unit * k);
+    ls_sh[warp][lane] = ls;
+    li_sh[warp][lane] = li;
+    __syncthreads();
+    if (warp == 0) {
+        for (int w = 1; w < kSelWarps; ++w) warp_merge_best_first(ls, li, ls_sh[w][lane], li_sh[w][lane], lane);
+        if (nsplit == 1) {
+            const int key = warp_sort_asc(lane < k ? li : kInvalid, lane);
+            if (lane < k) idx[(size_t)unit * k + lane] = key == kInvalid ? -1 : key;
+        } else {
+            float* us = ws_s + ((size_t)unit * nsplit + split) * 32;
+            int* ui = ws_i + ((size_t)unit * nsplit + split) * 32;
+            us[lane] = ls;
+            ui[lane] = li;
+            __threadfence();
+            __syncwarp();
+            unsigned t = 0;
+            if (lane == 0) t = atomicInc(ws_ctr + unit, (unsigned)(nsplit - 1));
+            t = __shfl_sync(kFull, t, 0);
+            if (lane == 0) ticket_sh = t;
+        }
+    }
+    if (nsplit == 1) return;
+    __syncthreads();
+    if (ticket_sh != (unsigned)(nsplit - 1)) return;
+    // last CTA of the unit: all lists into shared memory, then a merge tree over 4 warps
+    __threadfence();
+    for (int e = tid; e < nsplit * 32; e += blockDim.x) {
+        ls_sh[e >> 5][e & 31] = __ldcg(ws_s + (size_t)unit * nsplit * 32 + e);
+        li_sh[e >> 5][e & 31] = __ldcg(ws_i + (size_t)unit * nsplit * 32 + e);
+    }
+    __syncthreads();
+    for (int width = 1; width < nsplit; width *= 2) {
+        for (int pair = warp; pair * 2 * width < nsplit; pair += kSelWarps) {
+            const int x = pair * 2 * width, y = x + width;
+            if (y < nsplit) {
+                float s1 = ls_sh[x][lane];
+                int i1 = li_sh[x][lane];
+                warp_merge_best_first(s1, i1, ls_sh[y][lane], li_sh[y][lane], lane);
+                ls_sh[x][lane] = s1;
+                li_sh[x][lane] = i1;
+            }
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+        const int key = warp_sort_asc(lane < k ? li_sh[0][lane] : kInvalid, lane);
+        if (lane < k) idx[(size_t)unit * k + lane] = key == kInvalid ? -1 : key;
+    }
 }
 
 // ---------------------------------------------------------------------------- prefill
@@ -295,16 +364,30 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
         ok = __syncthreads_and(ok) != 0;
         const float* tile = tiles + st * 2 * D * 32;
         const int blk = gi * kGroupBlocks + lane;
+        // scores of this lane's block against the warp's 8 positions: 16 independent chains,
+        // each in the canonical order (ascending channels, one fma per term)
+        float av[kPfPerWarp], vv[kPfPerWarp];
 #pragma unroll
-        for (int j = 0; j < kPfPerWarp; ++j) {
-            const int p = warp * kPfPerWarp + j;
-            const int t = t0 + p;
-            const int nc = (t + 1) / L;
-            float sc = -INFINITY;
-            const bool valid = ok && t < Tctx && blk < nc;
-            if (__any_sync(kFull, valid)) {
-                sc = block_score<D>(tile, sq + (p * 2 + 0) * D, sq + (p * 2 + 1) * D, lane, isd, c2);
-                tk[j].offer(sc, blk, valid, k, lane);
+        for (int j = 0; j < kPfPerWarp; ++j) av[j] = vv[j] = 0.0f;
+        const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
+        const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
+        const float* sqw = sq + (size_t)(warp * kPfPerWarp) * 2 * D;
+#pragma unroll 4
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+            const float4 m = mu4[c4 * 32];
+            const float4 vr = var4[c4 * 32];
+#pragma unroll
+            for (int j = 0; j < kPfPerWarp; ++j) {
+                const float4 qa = reinterpret_cast<const float4*>(sqw + (j * 2 + 0) * D)[c4];
+                const float4 qb = reinterpret_cast<const float4*>(sqw + (j * 2 + 1) * D)[c4];
+                av[j] = __fmaf_rn(qa.x, m.x, av[j]);
+                av[j] = __fmaf_rn(qa.y, m.y, av[j]);
+                av[j] = __fmaf_rn(qa.z, m.z, av[j]);
+                av[j] = __fmaf_rn(qa.w, m.w, av[j]);
+                vv[j] = __fmaf_rn(qb.x, vr.x, vv[j]);
+                vv[j] = __fmaf_rn(qb.y, vr.y, vv[j]);
+                vv[j] = __fmaf_rn(qb.z, vr.z, vv[j]);
+                vv[j] = __fmaf_rn(qb.w, vr.w, vv[j]);
             }
         }
         __syncthreads();  // every warp is done with this stage
@@ -313,12 +396,46 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
             mbar_arrive_expect_tx(&bar[st], kTileBytes);
             bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(gi + 2) * 2 * D * 32, kTileBytes, &bar[st]);
         }
+#pragma unroll
+        for (int j = 0; j < kPfPerWarp; ++j) {
+            const int t = t0 + warp * kPfPerWarp + j;
+            const int nc = (t + 1) / L;
+            const bool valid = ok && t < Tctx && blk < nc;
+            float sc = __fmaf_rn(c2, vv[j], __fmul_rn(av[j], isd));
+            int bi = blk;
+            if (!valid) {
+                sc = -INFINITY;
+                bi = kInvalid;
+            }
+            const int nbetter = __popc(__ballot_sync(kFull, valid && better(sc, bi, tk[j].ts, tk[j].ti)));
+            if (nbetter > 4) {
+                // many newcomers (early groups): sort them and merge with the list
+                warp_sort_best_first(sc, bi, lane);
+                warp_merge_best_first(tk[j].s, tk[j].i, sc, bi, lane);
+                if (lane >= k) {
+                    tk[j].s = -INFINITY;
+                    tk[j].i = kInvalid;
+                }
+                tk[j].ts = __shfl_sync(kFull, tk[j].s, k - 1);
+                tk[j].ti = __shfl_sync(kFull, tk[j].i, k - 1);
+            } else if (nbetter > 0) {
+                tk[j].offer(sc, bi, valid, k, lane);
+            }
+        }
     }
 #pragma unroll
     for (int j = 0; j < kPfPerWarp; ++j) {
         const int t = t0 + warp * kPfPerWarp + j;
         if (t < Tctx) emit_sorted(tk[j], k, lane, idx + (((size_t)b * Tctx + t) * Hkv + g) * k);
     }
+}
+
+// Decode selection split: each warp scores gpw consecutive 32-block groups, a CTA holds 4 warps,
+// and a unit is covered by nsplit <= 16 CTAs.
+void decode_split(const Dims& m, int& gpw, int& nsplit) {
+    const int nGc = (m.T / m.L + 31) / 32;
+    gpw = std::max(1, (nGc + 63) / 64);
+    nsplit = std::max(1, (nGc + kSelWarps * gpw - 1) / (kSelWarps * gpw));
 }
 
 template <typename T, int D>
@@ -329,36 +446,23 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
     const size_t tile_bytes = (size_t)2 * D * 32 * 4;
     if (!prefill) {
         const int ncand = m.T / m.L;
-        const int nGc = (ncand + 31) / 32;
-        int gpc = 1;
-        while ((nGc + gpc - 1) / gpc > 64) gpc *= 2;  // at most 64 lists to merge per unit
-        const int nsplit = nGc == 0 ? 1 : (nGc + gpc - 1) / gpc;
-        float* ws_s = nullptr;
-        int* ws_i = nullptr;
-        unsigned* ws_ctr = nullptr;
-        if (nsplit > 1) {
-            unsigned char* w = static_cast<unsigned char*>(ws);
-            ws_ctr = reinterpret_cast<unsigned*>(w);
-            size_t off = ((size_t)m.units() * sizeof(unsigned) + 255) & ~(size_t)255;
-            ws_s = reinterpret_cast<float*>(w + off);
-            off += (size_t)m.units() * nsplit * m.k * sizeof(float);
-            ws_i = reinterpret_cast<int*>(w + off);
-        }
-        const size_t smem = tile_bytes * (gpc > 1 ? 2 : 1);
-        auto kern = select_decode_kernel<T, D>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
+        int gpw, nsplit;
+        decode_split(m, gpw, nsplit);
+        unsigned char* w = static_cast<unsigned char*>(ws);
+        unsigned* ws_ctr = reinterpret_cast<unsigned*>(w);
+        size_t off = ((size_t)m.units() * sizeof(unsigned) + 255) & ~(size_t)255;
+        float* ws_s = reinterpret_cast<float*>(w + off);
+        off += (size_t)m.units() * nsplit * 32 * sizeof(float);
+        int* ws_i = reinterpret_cast<int*>(w + off);
         count_launch();
-        count_launch();
-        kern<<<dim3(nsplit, m.units()), 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, ws_ctr, m.G, m.nG, ncand, m.k,
-                                                     gpc, nsplit, isd, c2, err);
+        select_decode_kernel<T, D><<<dim3(nsplit, m.units()), kSelWarps * 32, 0, s>>>(
+            Q, summ, idx, ws_s, ws_i, ws_ctr, m.G, m.nG, ncand, m.k, gpw, nsplit, isd, c2);
         return cudaGetLastError();
     }
     const size_t smem = tile_bytes * 2 + (size_t)kPfPos * 2 * D * 4;
     auto kern = select_prefill_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    count_launch();
     count_launch();
     kern<<<dim3((m.T + kPfPos - 1) / kPfPos, m.units()), 128, smem, s>>>(Q, summ, idx, m.T, m.Hq, m.Hkv, m.G,
                                                                         m.nG, m.L, m.k, isd, c2, err);
@@ -369,14 +473,10 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
 
 size_t select_workspace_bytes(const Dims& m, int prefill) {
     if (prefill) return 0;
-    const int ncand = m.T / m.L;
-    const int nGc = (ncand + 31) / 32;
-    int gpc = 1;
-    while ((nGc + gpc - 1) / gpc > 64) gpc *= 2;
-    const int nsplit = nGc == 0 ? 1 : (nGc + gpc - 1) / gpc;
-    if (nsplit <= 1) return 0;
-    size_t off = ((size_t)m.units() * sizeof(unsigned) + 255) & ~(size_t)255;
-    return off + (size_t)m.units() * nsplit * m.k * (sizeof(float) + sizeof(int));
+    int gpw, nsplit;
+    decode_split(m, gpw, nsplit);
+    const size_t off = ((size_t)m.units() * sizeof(unsigned) + 255) & ~(size_t)255;
+    return off + (size_t)m.units() * nsplit * 32 * (sizeof(float) + sizeof(int));
 }
 
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,

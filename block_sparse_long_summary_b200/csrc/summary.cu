@@ -9,8 +9,11 @@
 //
 // Summaries are float32 in a fixed order (rows ascending, one thread per channel),
 // so the selector downstream is reproducible bit for bit.
+#include <algorithm>
+
 #include "common.cuh"
 #include "dims.h"
+#include "tma.h"
 
 namespace cobs {
 namespace {
@@ -54,7 +57,7 @@ __global__ void __launch_bounds__(128) compress_kernel(const T* __restrict__ K, 
                                                        const float* __restrict__ Pv, int Tctx, int d,
                                                        int lc, int sc, int nC, int i_begin,
                                                        T* __restrict__ Kc, T* __restrict__ Vc) {
-    __shared__ float pooled[128];
+    __shared__ __align__(16) float pooled[128];
     const int c = threadIdx.x;
     const int unit = blockIdx.y;
     const int i = i_begin + blockIdx.x;
@@ -64,17 +67,355 @@ __global__ void __launch_bounds__(128) compress_kernel(const T* __restrict__ K, 
     T* out = isv ? Vc : Kc;
     const T* rows = X + ((size_t)unit * Tctx + (size_t)sc * i) * d + c;
     float s = 0.0f;
-    for (int r = 0; r < lc; ++r) s += Elem<T>::load(rows + (size_t)r * d);
+#pragma unroll 16
+    for (int r = 0; r < lc; ++r) s += Elem<T>::load(rows + (size_t)r * d);  // 16 loads in flight
     const float m = s / (float)lc;
     pooled[c] = m;
     __syncthreads();
-    float y = m;
-    if (P != nullptr) {
-        y = 0.0f;
-        const float* prow = P + (size_t)c * d;
-        for (int cc = 0; cc < d; ++cc) y = fmaf(__ldg(prow + cc), pooled[cc], y);
+    T* orow = out + ((size_t)unit * nC + i) * d;
+    if (P == nullptr) {
+        Elem<T>::store(orow + c, m);
+        return;
     }
-    Elem<T>::store(out + ((size_t)unit * nC + i) * d + c, y);
+    // out[j] = P[j, :] . pooled: a warp per output row, lanes over 4-channel slices of the
+    // row (coalesced 512-byte reads of P), shuffle reduction.
+    const int lane = c & 31, warp = c >> 5, nwarps = blockDim.x >> 5;
+    const float4* p4 = reinterpret_cast<const float4*>(P);
+    const float4 q = lane * 4 < d ? reinterpret_cast<const float4*>(pooled)[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int j = warp; j < d; j += nwarps) {
+        float acc = 0.0f;
+        if (lane * 4 < d) {
+            const float4 pv = __ldg(p4 + (size_t)j * (d / 4) + lane);
+            acc = pv.x * q.x + pv.y * q.y + pv.z * q.z + pv.w * q.w;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) Elem<T>::store(orow + j, acc);
+    }
+}
+
+// ---------------------------------------------------------------- fused bf16 build
+// One pass over K and V for bf16, block 64, compression 32 / 16 and a projection. A work item
+// is 2 selection blocks (128 rows) of one unit plus the 16 following rows: it yields the
+// summaries of its 2 blocks and its 8 compressed tokens (token i covers rows 16 i .. 16 i + 31,
+// i.e. 16-row chunks i and i + 1). Persistent CTAs of 8 warps walk the items with a 2-stage
+// bulk-copy ring. Per item:
+//   * threads (block, channel) form the float32 summaries in row order (the canonical order)
+//     and the 16-row chunk sums of K and V;
+//   * the 8 pooled tokens (chunk pair sums / 32) are split into bf16 hi + lo;
+//   * warps 0-3 (K) and 4-7 (V) project them on tensor cores: out = P pooled with P held in
+//     registers as bf16 hi + lo and three products (Phi*hi + Phi*lo + Plo*hi), float32 sums.
+constexpr int kFRows = 144;     // 128 rows + 16 halo rows
+constexpr int kFThreads = 256;
+
+template <int D>
+struct FusedSmem {
+    static constexpr int kRowBytes = D * 2;
+    static constexpr int kStage = 2 * kFRows * kRowBytes;  // K rows then V rows
+    static constexpr int kPooledStride = D + 8;            // bf16 elements per pooled row (bank spread)
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFThreads, 1) summary_fused_kernel(
+    const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, const float* __restrict__ Pk,
+    const float* __restrict__ Pv, int Tctx, int nB, int nG, int nC, int j_begin, int i_begin, int m_begin,
+    int m_count, int units, float* __restrict__ summ, __nv_bfloat16* __restrict__ Kc,
+    __nv_bfloat16* __restrict__ Vc, int* err) {
+    using S = FusedSmem<D>;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* ring = smem_raw;                                             // 2 stages
+    float* cs = reinterpret_cast<float*>(ring + 2 * S::kStage);                 // [2][9][D] chunk sums
+    __nv_bfloat16* pooled = reinterpret_cast<__nv_bfloat16*>(cs + 2 * 9 * D);   // [2 side][2 hi/lo][8][D+8]
+    __nv_bfloat16* outst = pooled + 2 * 2 * 8 * S::kPooledStride;              // [2 side][8][D]
+    __shared__ __align__(8) uint64_t bar[2];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long n_items = (long long)units * m_count;
+
+    // projection rows of this warp as A fragments (bf16 hi and lo): side = warp / 4,
+    // output channels [(warp % 4) * D/4, +D/4) = D/64 m16 tiles
+    constexpr int MT = D / 64, KS = D / 16;
+    const int side = warp >> 2;
+    const float* P = side ? Pv : Pk;
+    uint32_t ahi[MT][KS][4], alo[MT][KS][4];
+    {
+        const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int r0 = (warp & 3) * (D / 4) + mt * 16 + gid, r1 = r0 + 8;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                const int c = ks * 16 + 2 * tig;
+                const float v[4][2] = {{P[r0 * D + c], P[r0 * D + c + 1]},
+                                       {P[r1 * D + c], P[r1 * D + c + 1]},
+                                       {P[r0 * D + c + 8], P[r0 * D + c + 9]},
+                                       {P[r1 * D + c + 8], P[r1 * D + c + 9]}};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const __nv_bfloat16 h0 = __float2bfloat16_rn(v[q][0]), h1 = __float2bfloat16_rn(v[q][1]);
+                    const float l0 = v[q][0] - __bfloat162float(h0), l1 = v[q][1] - __bfloat162float(h1);
+                    __nv_bfloat162 hh; hh.x = h0; hh.y = h1;
+                    ahi[mt][ks][q] = *reinterpret_cast<uint32_t*>(&hh);
+                    alo[mt][ks][q] = pack_bf16(l0, l1);
+                }
+            }
+        }
+    }
+
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    auto rows_of = [&](long long item, int& unit, int& m, int& r0, int& nrows) {
+        unit = (int)(item / m_count);
+        m = m_begin + (int)(item % m_count);
+        r0 = m * 128;
+        nrows = max(0, min(kFRows, Tctx - r0));
+    };
+    auto issue = [&](long long item, int st) {  // tid 0
+        int unit, m, r0, nrows;
+        rows_of(item, unit, m, r0, nrows);
+        if (nrows == 0) return;
+        const uint32_t bytes = (uint32_t)nrows * S::kRowBytes;
+        unsigned char* dst = ring + st * S::kStage;
+        mbar_arrive_expect_tx(&bar[st], 2 * bytes);
+        bulk_g2s(dst, K + ((size_t)unit * Tctx + r0) * D, bytes, &bar[st]);
+        bulk_g2s(dst + kFRows * S::kRowBytes, V + ((size_t)unit * Tctx + r0) * D, bytes, &bar[st]);
+    };
+    const long long first = blockIdx.x, stride = gridDim.x;
+    if (tid == 0) {
+        if (first < n_items) issue(first, 0);
+        if (first + stride < n_items) issue(first + stride, 1);
+    }
+    uint32_t phase = 0;
+    bool ok = true;
+    int it = 0;
+    for (long long item = first; item < n_items; item += stride, ++it) {
+        const int st = it & 1;
+        int unit, m, r0, nrows;
+        rows_of(item, unit, m, r0, nrows);
+        if (nrows > 0 && ok && !mbar_wait(&bar[st], (phase >> st) & 1u, err)) ok = false;
+        ok = __syncthreads_and(ok) != 0;
+        if (nrows > 0) phase ^= 1u << st;
+        const __nv_bfloat16* sK = reinterpret_cast<const __nv_bfloat16*>(ring + st * S::kStage);
+        const __nv_bfloat16* sV = sK + kFRows * D;
+        // ---- summaries and chunk sums (thread = (block, channel))
+        if (tid < 2 * D && ok) {
+            const int blk = tid / D, c = tid % D;
+            const int j = 2 * m + blk;
+            const int rb = blk * 64;
+            const bool have = (rb + 64) <= nrows;
+            float ksum[4] = {0.f, 0.f, 0.f, 0.f};
+            if (have) {
+                float s = 0.0f;
+#pragma unroll 16
+                for (int r = 0; r < 64; ++r) {
+                    const float x = __bfloat162float(sK[(rb + r) * D + c]);
+                    s = __fadd_rn(s, x);
+                    ksum[r >> 4] += x;
+                }
+                const float mu = __fmul_rn(s, 1.0f / 64.0f);
+                float a2 = 0.0f;
+#pragma unroll 16
+                for (int r = 0; r < 64; ++r) {
+                    const float tt = __fsub_rn(__bfloat162float(sK[(rb + r) * D + c]), mu);
+                    a2 = __fmaf_rn(tt, tt, a2);
+                }
+                if (j < nB && j >= j_begin) {
+                    float* base = summ + (size_t)unit * nG * 2 * D * 32;
+                    const int g = j >> 5, ln = j & 31;
+                    base[((size_t)(g * 2 + 0) * (D / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = mu;
+                    base[((size_t)(g * 2 + 1) * (D / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = __fmul_rn(a2, 1.0f / 64.0f);
+                }
+            } else {
+                for (int q = 0; q < 4; ++q) {
+                    float x = 0.0f;
+                    for (int r = rb + 16 * q; r < min(rb + 16 * q + 16, nrows); ++r) x += __bfloat162float(sK[r * D + c]);
+                    ksum[q] = x;
+                }
+            }
+            for (int q = 0; q < 4; ++q) cs[(0 * 9 + blk * 4 + q) * D + c] = ksum[q];
+            // halo chunk of K (rows 128..143) by block-0 threads; V chunks 0-4 / 5-8
+            if (blk == 0) {
+                float x = 0.0f;
+                for (int r = 128; r < min(144, nrows); ++r) x += __bfloat162float(sK[r * D + c]);
+                cs[(0 * 9 + 8) * D + c] = x;
+            }
+            const int q0 = blk == 0 ? 0 : 5, q1 = blk == 0 ? 5 : 9;
+            for (int q = q0; q < q1; ++q) {
+                float x = 0.0f;
+                const int ra = 16 * q, rz = min(16 * q + 16, nrows);
+#pragma unroll 16
+                for (int r = ra; r < rz; ++r) x += __bfloat162float(sV[r * D + c]);
+                cs[(1 * 9 + q) * D + c] = x;
+            }
+        }
+        __syncthreads();
+        // ---- pooled tokens, split into bf16 hi + lo
+        for (int e = tid; e < 2 * 8 * D; e += kFThreads) {
+            const int sd = e / (8 * D), rem = e % (8 * D), p = rem / D, c = rem % D;
+            const float x = (cs[(sd * 9 + p) * D + c] + cs[(sd * 9 + p + 1) * D + c]) * (1.0f / 32.0f);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+            pooled[((sd * 2 + 0) * 8 + p) * S::kPooledStride + c] = hi;
+            pooled[((sd * 2 + 1) * 8 + p) * S::kPooledStride + c] = lo;
+        }
+        __syncthreads();
+        // the stage is free: prefetch the item after next into it
+        if (tid == 0 && ok && item + 2 * stride < n_items) {
+            fence_proxy_async();
+            issue(item + 2 * stride, st);
+        }
+        // ---- projection on tensor cores: out[channel][token] for this warp's channels
+        {
+            const int gid = lane >> 2, tig = lane & 3;
+            const __nv_bfloat16* ph = pooled + (side * 2 + 0) * 8 * S::kPooledStride;
+            const __nv_bfloat16* pl = pooled + (side * 2 + 1) * 8 * S::kPooledStride;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                float c4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int c = ks * 16 + 2 * tig;
+                    const uint32_t bh0 = *reinterpret_cast<const uint32_t*>(ph + gid * S::kPooledStride + c);
+                    const uint32_t bh1 = *reinterpret_cast<const uint32_t*>(ph + gid * S::kPooledStride + c + 8);
+                    const uint32_t bl0 = *reinterpret_cast<const uint32_t*>(pl + gid * S::kPooledStride + c);
+                    const uint32_t bl1 = *reinterpret_cast<const uint32_t*>(pl + gid * S::kPooledStride + c + 8);
+                    mma_bf16_16816(c4, ahi[mt][ks], bh0, bh1);
+                    mma_bf16_16816(c4, ahi[mt][ks], bl0, bl1);
+                    mma_bf16_16816(c4, alo[mt][ks], bh0, bh1);
+                }
+                const int ch = (warp & 3) * (D / 4) + mt * 16 + gid;
+                __nv_bfloat16* o = outst + side * 8 * D;
+                o[(2 * tig) * D + ch] = __float2bfloat16_rn(c4[0]);
+                o[(2 * tig + 1) * D + ch] = __float2bfloat16_rn(c4[1]);
+                o[(2 * tig) * D + ch + 8] = __float2bfloat16_rn(c4[2]);
+                o[(2 * tig + 1) * D + ch + 8] = __float2bfloat16_rn(c4[3]);
+            }
+        }
+        __syncthreads();
+        // ---- compressed tokens out (16-byte stores)
+        for (int e = tid; e < 2 * 8 * (D / 8); e += kFThreads) {
+            const int sd = e / (8 * (D / 8)), rem = e % (8 * (D / 8)), p = rem / (D / 8), c8 = rem % (D / 8);
+            const int i = 8 * m + p;
+            if (ok && i < nC && i >= i_begin) {
+                __nv_bfloat16* dst = (sd ? Vc : Kc) + ((size_t)unit * nC + i) * D + c8 * 8;
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(outst + sd * 8 * D + p * D + c8 * 8);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int D>
+cudaError_t launch_fused(const Dims& m, const __nv_bfloat16* K, const __nv_bfloat16* V, const float* Pk,
+                         const float* Pv, int t_begin, float* summ, __nv_bfloat16* Kc, __nv_bfloat16* Vc,
+                         cudaStream_t s, int* err) {
+    const int j_begin = t_begin <= 0 ? 0 : (t_begin + 1 + m.L - 1) / m.L - 1;
+    int i_begin = 0;
+    if (t_begin > 0) {
+        const int num = t_begin - m.lc + 1;
+        i_begin = num <= 0 ? 0 : (num + m.sc - 1) / m.sc;
+    }
+    const int m_end = std::max((m.nB + 1) / 2, (m.nC + 7) / 8);
+    const int m_begin = std::min(j_begin / 2, i_begin / 8);
+    const int m_count = m_end - m_begin;
+    if (m_count <= 0) return cudaSuccess;
+    using S = FusedSmem<D>;
+    const size_t smem = 2 * (size_t)S::kStage + 2 * 9 * D * 4 + 2 * 2 * 8 * S::kPooledStride * 2 + 2 * 8 * D * 2;
+    cudaError_t e = cudaFuncSetAttribute(summary_fused_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long items = (long long)m.units() * m_count;
+    const int grid = (int)std::min<long long>(items, sm_count());
+    count_launch();
+    summary_fused_kernel<D><<<grid, kFThreads, smem, s>>>(K, V, Pk, Pv, m.T, m.nB, m.nG, m.nC, j_begin, i_begin,
+                                                          m_begin, m_count, m.units(), summ, Kc, Vc, err);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------- decode-step append
+// The update after appending one token: at most one newly complete block (its summary) and one
+// newly complete compressed token (K and V) per unit. One CTA of 256 threads per unit: all row
+// loads in flight at once, then out_j = P[j, :] . pooled with a warp per 8 output rows at a
+// time (coalesced rows of P, interleaved shuffle reductions).
+template <typename T>
+__global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, const T* __restrict__ V,
+                                                     const float* __restrict__ Pk, const float* __restrict__ Pv,
+                                                     int Tctx, int d, int nG, int nC, int lc, int sc, int jb, int ic,
+                                                     float* __restrict__ summ, T* __restrict__ Kc,
+                                                     T* __restrict__ Vc) {
+    __shared__ __align__(16) float pooled[2][128];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int unit = blockIdx.x;
+    // block summary (threads < d): the canonical row-order sums
+    if (jb >= 0 && tid < d) {
+        const int c = tid;
+        const T* rows = K + ((size_t)unit * Tctx + (size_t)jb * kBlock) * d + c;
+        float x[kBlock];
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) x[r] = Elem<T>::load(rows + (size_t)r * d);
+        float sum = 0.0f;
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) sum = __fadd_rn(sum, x[r]);
+        const float mu = __fmul_rn(sum, 1.0f / kBlock);
+        float a2 = 0.0f;
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) {
+            const float t = __fsub_rn(x[r], mu);
+            a2 = __fmaf_rn(t, t, a2);
+        }
+        float* base = summ + (size_t)unit * nG * 2 * d * 32;
+        const int g = jb >> 5, ln = jb & 31;
+        base[((size_t)(g * 2 + 0) * (d / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = mu;
+        base[((size_t)(g * 2 + 1) * (d / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = __fmul_rn(a2, 1.0f / kBlock);
+    }
+    if (ic < 0) return;
+    // pooled compressed token: threads [0, d) for K, [128, 128 + d) for V
+    const int side = tid >> 7, c = tid & 127;
+    if (c < d) {
+        const T* rows = (side ? V : K) + ((size_t)unit * Tctx + (size_t)sc * ic) * d + c;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 32
+        for (int r = 0; r < lc; ++r) acc[r & 3] += Elem<T>::load(rows + (size_t)r * d);
+        pooled[side][c] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) / (float)lc;
+    }
+    __syncthreads();
+    const int ws = warp >> 2;  // warps 0-3: K, 4-7: V
+    const float* P = ws ? Pv : Pk;
+    T* orow = (ws ? Vc : Kc) + ((size_t)unit * nC + ic) * d;
+    if (P == nullptr) {
+        const int cc = tid & 127;
+        if (cc < d) Elem<T>::store(orow + cc, pooled[ws][cc]);
+        return;
+    }
+    const float4 q = lane * 4 < d ? reinterpret_cast<const float4*>(pooled[ws])[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int per_warp = d / 4;  // output rows of this warp
+    const int j0 = (warp & 3) * per_warp;
+    for (int jb8 = 0; jb8 < per_warp; jb8 += 8) {
+        float part[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int j = j0 + jb8 + u;
+            float4 pv = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (jb8 + u < per_warp && lane * 4 < d)
+                pv = __ldg(reinterpret_cast<const float4*>(P + (size_t)j * d) + lane);
+            part[u] = pv.x * q.x + pv.y * q.y + pv.z * q.z + pv.w * q.w;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) part[u] += __shfl_xor_sync(0xffffffffu, part[u], off);
+        if (lane < 8 && jb8 + lane < per_warp) {
+            float v = part[0];
+#pragma unroll
+            for (int u = 1; u < 8; ++u) v = lane == u ? part[u] : v;
+            Elem<T>::store(orow + j0 + jb8 + lane, v);
+        }
+    }
 }
 
 template <typename T>
@@ -109,8 +450,44 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
 
 }  // namespace
 
+template <typename T>
+bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const float* Pv, int t_begin, float* summ,
+                T* Kc, T* Vc, cudaStream_t s, cudaError_t* e) {
+    if (t_begin <= 0 || m.L != kBlock || m.d > 128) return false;
+    const int j_begin = (t_begin + 1 + m.L - 1) / m.L - 1;
+    const int num = t_begin - m.lc + 1;
+    const int i_begin = num <= 0 ? 0 : (num + m.sc - 1) / m.sc;
+    const int nj = m.nB - j_begin, ni = m.nC - i_begin;
+    if (nj > 1 || ni > 1) return false;
+    if (nj <= 0 && ni <= 0) {
+        *e = cudaSuccess;
+        return true;
+    }
+    count_launch();
+    append_kernel<T><<<m.units(), 256, 0, s>>>(K, V, Pk, Pv, m.T, m.d, m.nG, m.nC, m.lc, m.sc, nj > 0 ? j_begin : -1,
+                                               ni > 0 ? i_begin : -1, summ, Kc, Vc);
+    *e = cudaGetLastError();
+    return true;
+}
+
 cudaError_t launch_summaries(const Dims& m, const void* K, const void* V, const float* Pk, const float* Pv,
-                             int t_begin, float* summ, void* Kc, void* Vc, cudaStream_t s) {
+                             int t_begin, float* summ, void* Kc, void* Vc, cudaStream_t s, int* err) {
+    // the decode-step update (one block, one compressed token): a small dedicated kernel
+    cudaError_t ea = cudaSuccess;
+    if (m.dtype == COBS_BF16 ? try_append<__nv_bfloat16>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv,
+                                                         t_begin, summ, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s, &ea)
+                             : try_append<float>(m, (const float*)K, (const float*)V, Pk, Pv, t_begin, summ,
+                                                 (float*)Kc, (float*)Vc, s, &ea))
+        return ea;
+    // fused one-pass kernel for the bf16 layout it is written for; plain kernels otherwise
+    if (m.dtype == COBS_BF16 && m.L == 64 && m.lc == 32 && m.sc == 16 && Pk != nullptr && Pv != nullptr &&
+        (m.d == 128 || m.d == 64) && m.nC > 0) {
+        if (m.d == 128)
+            return launch_fused<128>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv, t_begin, summ,
+                                     (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s, err);
+        return launch_fused<64>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv, t_begin, summ,
+                                (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s, err);
+    }
     if (m.dtype == COBS_BF16)
         return launch_summaries_t<__nv_bfloat16>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv,
                                                  t_begin, summ, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s);

@@ -115,7 +115,11 @@ def test_incremental_update_matches_full_build():
     C.cobs_build_summaries(p, tK, tV, tPk, tPv, w.T - 1, inc.summaries, inc.Kc, inc.Vc)
     torch.cuda.synchronize()
     assert np.array_equal(summaries_blocks(inc.summaries, p), sb)
-    assert torch.equal(inc.Kc, full.Kc) and torch.equal(inc.Vc, full.Vc)
+    # rows before the last compressed token are untouched; the rewritten one matches the full
+    # build within one bf16 ulp (the two paths round their float32 projections separately)
+    assert torch.equal(inc.Kc[:, :, :-1], full.Kc[:, :, :-1]) and torch.equal(inc.Vc[:, :, :-1], full.Vc[:, :, :-1])
+    for a_, b_ in ((inc.Kc, full.Kc), (inc.Vc, full.Vc)):
+        assert kc_close(f64(a_[:, :, -1]), f64(b_[:, :, -1]), "bf16").all()
 
 
 def test_bad_index_sets_device_flag_without_fault():
