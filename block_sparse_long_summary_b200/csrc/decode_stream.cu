@@ -110,7 +110,7 @@ __device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt) {
 
 template <int D>
 struct WState {
-    float m0, m1, l0, l1;
+    float m0, m1, l0, l1;  // reference maxima (scaled log2 units) and row sums
     float o[D / 8][4];
     __device__ void init() {
         m0 = m1 = -INFINITY;
@@ -132,6 +132,13 @@ __device__ __forceinline__ void load_q(const __nv_bfloat16* q, int G, uint32_t (
         qa[ks][2] = r0 < G ? q0[4] : 0u;
         qa[ks][3] = r1 < G ? q1[4] : 0u;
     }
+}
+
+// 2^x on the special-function unit (approximate, flush-to-zero).
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // Byte offset of 16-byte chunk `cc` (0..7) of row `r` in a 128-byte-swizzled 32-row box.
@@ -176,30 +183,47 @@ __device__ __forceinline__ void tile_mma(WState<D>& st, const uint32_t (&qa)[D /
     mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
     mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
     mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
-    const float nm0 = fmaxf(st.m0, mx0), nm1 = fmaxf(st.m1, mx1);
-    const float al0 = exp2f((st.m0 - nm0) * sl2), al1 = exp2f((st.m1 - nm1) * sl2);
-    st.m0 = nm0;
-    st.m1 = nm1;
+    // Lazy rescale: the reference maxima st.m* (scaled log2 units) move only when a row's maximum
+    // exceeds them by more than 8, so p = 2^(s sl2 - m) <= 2^8 and the accumulators are rescaled
+    // rarely. The four threads of a quad hold the same row maxima and decide alike.
+    mx0 *= sl2;
+    mx1 *= sl2;
+    const bool g0 = mx0 != -INFINITY && (st.m0 == -INFINITY || mx0 - st.m0 > 8.0f);
+    const bool g1 = mx1 != -INFINITY && (st.m1 == -INFINITY || mx1 - st.m1 > 8.0f);
+    if (__any_sync(kFull, g0 || g1)) {
+        const float nm0 = g0 ? (st.m0 == -INFINITY ? mx0 : fmaxf(st.m0, mx0)) : st.m0;
+        const float nm1 = g1 ? (st.m1 == -INFINITY ? mx1 : fmaxf(st.m1, mx1)) : st.m1;
+        const float al0 = (g0 && st.m0 != -INFINITY) ? ex2f(st.m0 - nm0) : (g0 ? 0.0f : 1.0f);
+        const float al1 = (g1 && st.m1 != -INFINITY) ? ex2f(st.m1 - nm1) : (g1 ? 0.0f : 1.0f);
+        st.m0 = nm0;
+        st.m1 = nm1;
+        st.l0 *= al0;
+        st.l1 *= al1;
+#pragma unroll
+        for (int nd = 0; nd < D / 8; ++nd) {
+            st.o[nd][0] *= al0;
+            st.o[nd][1] *= al0;
+            st.o[nd][2] *= al1;
+            st.o[nd][3] *= al1;
+        }
+    }
+    const float nm0 = -st.m0, nm1 = -st.m1;
+    const bool z0 = st.m0 == -INFINITY, z1 = st.m1 == -INFINITY;
     float ps0 = 0.0f, ps1 = 0.0f;
     uint32_t pa[NP][4];
 #pragma unroll
     for (int nt = 0; nt < 2 * NP; ++nt) {
-        const float p0 = exp2f((s[nt][0] - nm0) * sl2), p1 = exp2f((s[nt][1] - nm0) * sl2);
-        const float p2 = exp2f((s[nt][2] - nm1) * sl2), p3 = exp2f((s[nt][3] - nm1) * sl2);
+        const float p0 = z0 ? 0.0f : ex2f(fmaf(s[nt][0], sl2, nm0));
+        const float p1 = z0 ? 0.0f : ex2f(fmaf(s[nt][1], sl2, nm0));
+        const float p2 = z1 ? 0.0f : ex2f(fmaf(s[nt][2], sl2, nm1));
+        const float p3 = z1 ? 0.0f : ex2f(fmaf(s[nt][3], sl2, nm1));
         ps0 += p0 + p1;
         ps1 += p2 + p3;
         pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
         pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
     }
-    st.l0 = st.l0 * al0 + ps0;
-    st.l1 = st.l1 * al1 + ps1;
-#pragma unroll
-    for (int nd = 0; nd < D / 8; ++nd) {
-        st.o[nd][0] *= al0;
-        st.o[nd][1] *= al0;
-        st.o[nd][2] *= al1;
-        st.o[nd][3] *= al1;
-    }
+    st.l0 += ps0;
+    st.l1 += ps1;
 #pragma unroll
     for (int kk = 0; kk < NP; ++kk) {
 #pragma unroll
@@ -367,8 +391,8 @@ __global__ void __launch_bounds__(128) decode_stream_merge(StreamArgs a) {
         for (int q = 0; q < 4; ++q) {
             if (m[q] == -INFINITY) continue;
             const float nM = fmaxf(M, m[q]);
-            const float fa = M == -INFINITY ? 0.0f : exp2f((M - nM) * a.sl2);
-            const float fb = exp2f((m[q] - nM) * a.sl2);
+            const float fa = M == -INFINITY ? 0.0f : exp2f(M - nM);  // maxima are in log2 units
+            const float fb = exp2f(m[q] - nM);
             Lsum = Lsum * fa + l[q] * fb;
             acc[0] = acc[0] * fa + o[q].x * fb;
             acc[1] = acc[1] * fa + o[q].y * fb;
@@ -392,8 +416,8 @@ __global__ void __launch_bounds__(128) decode_stream_merge(StreamArgs a) {
         const int w0 = b2, w1 = b2 == 2 ? 3 : b2;
         const float GM = fmaxf(wM[w0], wM[w1]);
         if (GM == -INFINITY) continue;
-        const float f0 = wM[w0] == -INFINITY ? 0.0f : exp2f((wM[w0] - GM) * a.sl2);
-        const float f1 = (w1 == w0 || wM[w1] == -INFINITY) ? 0.0f : exp2f((wM[w1] - GM) * a.sl2);
+        const float f0 = wM[w0] == -INFINITY ? 0.0f : exp2f(wM[w0] - GM);
+        const float f1 = (w1 == w0 || wM[w1] == -INFINITY) ? 0.0f : exp2f(wM[w1] - GM);
         const float GL = wL[w0] * f0 + (w1 == w0 ? 0.0f : wL[w1] * f1);
         if (!(GL > 0.0f)) continue;
         const float gw = gate[b2 == 0 ? 1 : (b2 == 1 ? 2 : 0)] / GL;  // gates are (cmp, slc, win)

@@ -35,9 +35,9 @@ constexpr int kRows = kP * kGH;  // 128 MMA rows
 constexpr int kKB = 64;          // keys per item
 constexpr int kD = 128;          // head dimension handled by this kernel
 constexpr int kStagesKV = 3;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kSoftmaxThreads = 256;            // two threads per row: S / O column halves
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kThreads = kSoftmaxThreads + 64;  // + producer warp + MMA warp
 
 constexpr uint32_t kQBytes = kRows * kD * 2;          // 32 KiB (two 64-column halves)
@@ -60,7 +60,9 @@ struct PfArgs {
     float sl2;  // log2(e) / sqrt(d)
 };
 
-__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void named_sync_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// warps w and w + 4 hold the two halves of the same 32 rows: barrier ids 2..5, 64 threads each
+__device__ __forceinline__ void named_sync_pair(int w4) { asm volatile("bar.sync %0, 64;" ::"r"(2 + w4) : "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                  const __grid_constant__ CUtensorMap tmK,
@@ -72,7 +74,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     __shared__ __align__(8) uint64_t barQ, barKV[kStagesKV], barFree[kStagesKV], barS[2], barP[2], barO[2], barDone;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int n_sh[4];       // item counts: SLC, WIN, CMP, total
-    __shared__ int warp_cnt[8];
+    __shared__ int warp_cnt[kThreads / 32];
+    __shared__ float mx_sh[2][2][kRows];  // [item parity][half][row] row-max exchange
 
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -262,14 +265,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         return;
     }
 
-    // ---------------------------------------------------------------- softmax warpgroup (thread = row)
-    const int row = tid;                 // TMEM lane / MMA row
+    // ---------------------------------------------------------------- softmax warps (two threads per row)
+    const int row = tid & (kRows - 1);   // TMEM lane / MMA row
+    const int half = tid >> 7;           // S columns [32 half, +32), O columns [64 half, +64)
     const int p = row / kGH, h = row % kGH;
     const int t = t0 + p;
     const bool row_ok = t < a.T;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY;  // per-branch reference maxima (scaled log2 units)
-    float l0 = 0.f, l1 = 0.f, l2 = 0.f;                     // per-branch row sums
+    float l0 = 0.f, l1 = 0.f, l2 = 0.f;                     // per-branch partial row sums (this half)
     bool ok = true;
     // Wait until PV_j (and so every earlier MMA) has completed. PV_j completes phase j / 2 of
     // barO[j % 2]; that barrier cannot run a phase ahead of this wait (PV_{j+2} needs this
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         const int fb = br == 0 ? 0 : (br == 1 ? first1 : first2);
         float mref = br == 0 ? m0 : (br == 1 ? m1 : m2);
         float lsum = br == 0 ? l0 : (br == 1 ? l1 : l2);
-        // key range [lo, hi] of this row within the item's 64 keys
+        // key range [lo, hi] of this row within this thread's 32 keys of the item
         int lo = 0, hi = -1;
         const int rowi = item_row[i];
         if (row_ok) {
@@ -300,37 +304,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
                 lo = 0;
                 hi = vis - 1 - cbase;
             }
+            lo = max(lo, 0) - 32 * half;
+            hi = min(hi, kKB - 1) - 32 * half;
             lo = max(lo, 0);
-            hi = min(hi, kKB - 1);
+            hi = min(hi, 31);
         }
         if (ok && !mbar_wait(&barS[i & 1], (i >> 1) & 1, a.err)) ok = false;
         tc::fence_after_sync();
-        float s[64];
-        {
-            float v[32];
-            const uint32_t col = (i & 1) ? kColS1 : kColS0;
-            tc::ld32(tmem + lane_off + col, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = v[j];
-            tc::ld32(tmem + lane_off + col + 32, v);
-            tc::wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[32 + j] = v[j];
-        }
+        float s[32];
+        tc::ld32(tmem + lane_off + ((i & 1) ? kColS1 : kColS0) + 32 * half, s);
+        tc::wait_ld();
         const bool none = hi < lo;
-        const bool full = lo == 0 && hi == kKB - 1;
-        // scaled scores (log2 units) and their maximum; masking only where the row is partial
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (!none) {
+        const bool full = lo == 0 && hi == 31;
+        if (!full) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                float x = s[j] * sl2;
-                if (!full) x = (j >= lo && j <= hi) ? x : -INFINITY;
-                s[j] = x;
-                mx[j & 3] = fmaxf(mx[j & 3], x);
-            }
+            for (int j = 0; j < 32; ++j) s[j] = (j >= lo && j <= hi) ? s[j] : -INFINITY;
         }
-        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        // row maximum of the raw scores over both halves (the scale is positive)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], s[j]);
+        mx_sh[i & 1][half][row] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        named_sync_pair(warp & 3);  // this warp and the one holding the other half of its rows
+        const float mt = fmaxf(mx_sh[i & 1][0][row], mx_sh[i & 1][1][row]) * sl2;
         // lazy rescale: only when the row maximum grows by more than 8 (a factor 2^8)
         float f = 1.0f;
         bool scale = false;
@@ -349,31 +345,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         tc::fence_after_sync();
         if (wscale) {
 #pragma unroll
-            for (int c = 0; c < kD; c += 32) {
+            for (int c = 0; c < 64; c += 32) {
                 float v[32];
-                tc::ld32(tmem + lane_off + br * 128 + c, v);
+                tc::ld32(tmem + lane_off + br * 128 + 64 * half + c, v);
                 tc::wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] *= f;
-                tc::st32(tmem + lane_off + br * 128 + c, v);
+                tc::st32(tmem + lane_off + br * 128 + 64 * half + c, v);
             }
             tc::wait_st();
         }
-        // P row (bf16) into the swizzled tile P[i % 2]
+        // this half of the P row (bf16) into the swizzled tile P[i % 2]: chunks 4 half .. 4 half + 3;
+        // p = 2^(s * scale - m), masked keys are -inf and give 0
         unsigned char* prow = sP + (size_t)(i & 1) * kPBytes + (size_t)row * 128;
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
-        const bool zero = none || mref == -INFINITY;
+        if (none || mref == -INFINITY) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t w4[4];
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (row & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+            const float neg = -mref;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float x0 = zero ? 0.0f : tc::ex2(s[8 * c + 2 * q] - mref);
-                const float x1 = zero ? 0.0f : tc::ex2(s[8 * c + 2 * q + 1] - mref);
-                ps[q] += x0 + x1;
-                w4[q] = pack_bf16(x0, x1);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float x0 = tc::ex2(fmaf(s[8 * c + 2 * q], sl2, neg));
+                    const float x1 = tc::ex2(fmaf(s[8 * c + 2 * q + 1], sl2, neg));
+                    ps[q] += x0 + x1;
+                    w4[q] = pack_bf16(x0, x1);
+                }
+                *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (row & 7)) << 4)) =
+                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         if (br == 0) { m0 = mref; l0 = lsum; } else if (br == 1) { m1 = mref; l1 = lsum; } else { m2 = mref; l2 = lsum; }
@@ -384,7 +388,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
     // all MMAs done
     wait_pv(n - 1);
     tc::fence_after_sync();
-    const float lsum_br[3] = {l0, l1, l2};
+    // full row sums: add the partner half's partial sums
+    __shared__ float lsh[3][2][kRows];
+    lsh[0][half][row] = l0;
+    lsh[1][half][row] = l1;
+    lsh[2][half][row] = l2;
+    named_sync_softmax();
+    const float lsum_br[3] = {lsh[0][0][row] + lsh[0][1][row], lsh[1][0][row] + lsh[1][1][row],
+                              lsh[2][0][row] + lsh[2][1][row]};
     const int cnt[3] = {nS, nW, nCi};
 
     // ---------------------------------------------------------------- epilogue
@@ -397,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             const float gw = row_ok ? a.gates[orow * 3 + gate_slot(br)] : 0.0f;
             wgt[br] = (lsum_br[br] > 0.0f) ? gw / lsum_br[br] : 0.0f;
         }
-        __nv_bfloat16* out = a.O + orow * kD;
+        __nv_bfloat16* out = a.O + orow * kD + 64 * half;
 #pragma unroll
-        for (int c = 0; c < kD; c += 32) {
+        for (int c = 0; c < 64; c += 32) {
             float acc[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
@@ -407,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
             for (int br = 0; br < 3; ++br) {
                 if (cnt[br] == 0) continue;  // uniform: no item of this branch in the tile
                 float v[32];
-                tc::ld32(tmem + lane_off + br * 128 + c, v);
+                tc::ld32(tmem + lane_off + br * 128 + 64 * half + c, v);
                 tc::wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc[j] += wgt[br] * v[j];

@@ -137,6 +137,35 @@ __device__ __forceinline__ float block_score(const float* tile, const float* qs,
     return __fmaf_rn(c2, v, __fmul_rn(a, isd));
 }
 
+// Same canonical score, with the group query held in registers: lane l keeps channels
+// 4l .. 4l + 3 of Qsum and Q2 and the other lanes read them by shuffle (keeps shared memory for
+// the summary tile alone).
+template <int D>
+__device__ __forceinline__ float block_score_regq(const float* tile, float4 qs4, float4 q24, int lane, float isd,
+                                                  float c2) {
+    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
+    const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
+    float a = 0.0f, v = 0.0f;
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 m = mu4[c4 * 32];
+        const float4 s = var4[c4 * 32];
+        const float qa = __shfl_sync(kFull, qs4.x, c4), qb = __shfl_sync(kFull, qs4.y, c4);
+        const float qc = __shfl_sync(kFull, qs4.z, c4), qd = __shfl_sync(kFull, qs4.w, c4);
+        const float ra = __shfl_sync(kFull, q24.x, c4), rb = __shfl_sync(kFull, q24.y, c4);
+        const float rc = __shfl_sync(kFull, q24.z, c4), rd = __shfl_sync(kFull, q24.w, c4);
+        a = __fmaf_rn(qa, m.x, a);
+        a = __fmaf_rn(qb, m.y, a);
+        a = __fmaf_rn(qc, m.z, a);
+        a = __fmaf_rn(qd, m.w, a);
+        v = __fmaf_rn(ra, s.x, v);
+        v = __fmaf_rn(rb, s.y, v);
+        v = __fmaf_rn(rc, s.z, v);
+        v = __fmaf_rn(rd, s.w, v);
+    }
+    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
+}
+
 // ---------------------------------------------------------------------------- decode
 // Warp-wide sorted list helpers: one (score, index) entry per lane, best first.
 __device__ __forceinline__ void cmp_swap(float& s, int& i, int j, bool up, int lane) {
@@ -171,88 +200,97 @@ __device__ __forceinline__ void warp_merge_best_first(float& s, int& i, float bs
     for (int j = 16; j > 0; j >>= 1) cmp_swap(s, i, j, true, lane);
 }
 
-// Canonical score of block `lane` of a 32-block group read straight from global memory
-// (coalesced: one 512-byte row per warp load). The mean and variance chains are independent,
-// so half of each is loaded, then consumed, then the other half.
-template <int D>
-__device__ __forceinline__ float block_score_global(const float* grp, const float* qs, const float* q2, int lane,
-                                                    float isd, float c2) {
-    const float4* mu4 = reinterpret_cast<const float4*>(grp) + lane;
-    const float4* var4 = reinterpret_cast<const float4*>(grp + D * 32) + lane;
-    constexpr int H = D / 8;  // float4s per half-chain
-    float a = 0.0f, v = 0.0f;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        float4 m[H], s[H];
-#pragma unroll
-        for (int i = 0; i < H; ++i) {
-            m[i] = __ldcs(mu4 + (half * H + i) * 32);
-            s[i] = __ldcs(var4 + (half * H + i) * 32);
-        }
-#pragma unroll
-        for (int i = 0; i < H; ++i) {
-            const int c = 4 * (half * H + i);
-            a = __fmaf_rn(qs[c + 0], m[i].x, a);
-            a = __fmaf_rn(qs[c + 1], m[i].y, a);
-            a = __fmaf_rn(qs[c + 2], m[i].z, a);
-            a = __fmaf_rn(qs[c + 3], m[i].w, a);
-            v = __fmaf_rn(q2[c + 0], s[i].x, v);
-            v = __fmaf_rn(q2[c + 1], s[i].y, v);
-            v = __fmaf_rn(q2[c + 2], s[i].z, v);
-            v = __fmaf_rn(q2[c + 3], s[i].w, v);
-        }
-    }
-    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
-}
+#ifndef COBS_SELECT_WARPS
+#define COBS_SELECT_WARPS 1
+#endif
+constexpr int kSelWarps = COBS_SELECT_WARPS;
+constexpr int kMaxSplit = 32;
 
-constexpr int kSelWarps = 4;
-
-// grid (nsplit, units), 4 warps. Warp w of split s scores groups [(s*4 + w)*gpw, +gpw) of its
-// unit and keeps a sorted best-first list; the 4 lists are merged in shared memory. With one
-// split the CTA writes the answer. Otherwise every CTA deposits its list and takes an atomic
-// ticket (nobody waits); the CTA that takes the last ticket merges all lists of the unit with a
-// shared-memory tree and writes the answer. The result is the top-k under a strict total order,
-// so it does not depend on arrival order. The ticket counter returns to zero by itself.
+// grid (nsplit, units), 2 warps. Warp w of split s scores groups [(s*2 + w)*gpw, +gpw) of its
+// unit: each group (32 blocks, 32 KiB) arrives with one bulk (TMA) copy into the warp's own
+// buffer (two buffers when a warp has several groups), lane = block, and the warp keeps a sorted
+// best-first list (bitonic sort + merge). The CTA's two lists are merged in shared memory. With
+// one split the CTA writes the answer; otherwise every CTA deposits its list and takes an atomic
+// ticket (nobody waits), and the CTA that takes the last ticket merges all lists of the unit
+// with a shared-memory tree. The ticket counter returns to zero by itself. The result is the
+// top-k under a strict total order, so it does not depend on arrival order.
 template <typename T, int D>
 __global__ void __launch_bounds__(kSelWarps * 32) select_decode_kernel(
     const T* __restrict__ Q, const float* __restrict__ summ, int32_t* __restrict__ idx, float* __restrict__ ws_s,
     int* __restrict__ ws_i, unsigned* __restrict__ ws_ctr, int G, int nG, int ncand, int k, int gpw, int nsplit,
-    float isd, float c2) {
-    __shared__ float qs[D], q2[D];
-    __shared__ float ls_sh[16][32];
-    __shared__ int li_sh[16][32];
+    float isd, float c2, int* err) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t bar[kSelWarps][2];
     __shared__ unsigned ticket_sh;
+    constexpr uint32_t kTileBytes = 2 * D * 32 * 4;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.y;
     const int split = blockIdx.x;
     const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
     const float* usum = summ + (size_t)unit * nG * 2 * D * 32;
-    {
-        // unit = b * Hkv + g and Hq = Hkv * G, so the group's first head row is unit * G
-        const T* qg = Q + (size_t)unit * G * D;
-        for (int c = tid; c < D; c += blockDim.x) group_query(qg, G, D, c, qs[c], q2[c]);
+    const int stages = gpw > 1 ? 2 : 1;
+    float* tiles = reinterpret_cast<float*>(smem_raw) + (size_t)warp * stages * 2 * D * 32;
+    const int g0 = (split * kSelWarps + warp) * gpw;
+    const int g1 = min(nGc, g0 + gpw);
+    if (lane == 0) {
+        mbar_init(&bar[warp][0], 1);
+        mbar_init(&bar[warp][1], 1);
+        fence_barrier_init();
     }
-    __syncthreads();
+    __syncwarp();
+    if (lane == 0) {
+        for (int st = 0; st < stages && g0 + st < g1; ++st) {
+            mbar_arrive_expect_tx(&bar[warp][st], kTileBytes);
+            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(g0 + st) * 2 * D * 32, kTileBytes, &bar[warp][st]);
+        }
+    }
+    // group query in registers: lane l holds channels 4l .. 4l + 3
+    // (unit = b * Hkv + g and Hq = Hkv * G, so the group's first head row is unit * G)
+    float4 qs4 = make_float4(0.f, 0.f, 0.f, 0.f), q24 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lane * 4 < D) {
+        const T* qg = Q + (size_t)unit * G * D;
+        group_query(qg, G, D, 4 * lane + 0, qs4.x, q24.x);
+        group_query(qg, G, D, 4 * lane + 1, qs4.y, q24.y);
+        group_query(qg, G, D, 4 * lane + 2, qs4.z, q24.z);
+        group_query(qg, G, D, 4 * lane + 3, qs4.w, q24.w);
+    }
 
     float ls = -INFINITY;
     int li = kInvalid;
-    const int g0 = (split * kSelWarps + warp) * gpw;
-    for (int g = g0; g < min(nGc, g0 + gpw); ++g) {
+    bool ok = true;
+    for (int g = g0, it = 0; g < g1; ++g, ++it) {
+        const int st = it % stages;
+        const uint32_t parity = (it / stages) & 1;
+        if (ok) ok = mbar_wait(&bar[warp][st], parity, err);
+        ok = __all_sync(kFull, ok);
         const int b = g * kGroupBlocks + lane;
-        float sc = block_score_global<D>(usum + (size_t)g * 2 * D * 32, qs, q2, lane, isd, c2);
-        int bi = b;
-        if (b >= ncand) {
-            sc = -INFINITY;
-            bi = kInvalid;
+        float sc = -INFINITY;
+        int bi = kInvalid;
+        if (ok) {  // warp-uniform: every lane takes part in the score's shuffles
+            const float s_all = block_score_regq<D>(tiles + st * 2 * D * 32, qs4, q24, lane, isd, c2);
+            if (b < ncand) {
+                sc = s_all;
+                bi = b;
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && ok && g + stages < g1) {
+            fence_proxy_async();
+            mbar_arrive_expect_tx(&bar[warp][st], kTileBytes);
+            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(g + stages) * 2 * D * 32, kTileBytes, &bar[warp][st]);
         }
         warp_sort_best_first(sc, bi, lane);
-        if (g == g0) {
+        if (it == 0) {
             ls = sc;
             li = bi;
         } else {
             warp_merge_best_first(ls, li, sc, bi, lane);
         }
     }
+    // the tile buffers are free once every warp is done: reuse them for the list merges
+    __syncthreads();
+    float (*ls_sh)[32] = reinterpret_cast<float (*)[32]>(smem_raw);
+    int (*li_sh)[32] = reinterpret_cast<int (*)[32]>(smem_raw + kMaxSplit * 32 * sizeof(float));
     ls_sh[warp][lane] = ls;
     li_sh[warp][lane] = li;
     __syncthreads();
@@ -277,7 +315,7 @@ __global__ void __launch_bounds__(kSelWarps * 32) select_decode_kernel(
     if (nsplit == 1) return;
     __syncthreads();
     if (ticket_sh != (unsigned)(nsplit - 1)) return;
-    // last CTA of the unit: all lists into shared memory, then a merge tree over 4 warps
+    // last CTA of the unit: all lists into shared memory, then a merge tree over the warps
     __threadfence();
     for (int e = tid; e < nsplit * 32; e += blockDim.x) {
         ls_sh[e >> 5][e & 31] = __ldcg(ws_s + (size_t)unit * nsplit * 32 + e);
@@ -430,11 +468,11 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     }
 }
 
-// Decode selection split: each warp scores gpw consecutive 32-block groups, a CTA holds 4 warps,
-// and a unit is covered by nsplit <= 16 CTAs.
+// Decode selection split: each warp scores gpw consecutive 32-block groups, a CTA holds 2 warps,
+// and a unit is covered by nsplit <= 32 CTAs.
 void decode_split(const Dims& m, int& gpw, int& nsplit) {
     const int nGc = (m.T / m.L + 31) / 32;
-    gpw = std::max(1, (nGc + 63) / 64);
+    gpw = std::max(1, (nGc + kSelWarps * kMaxSplit - 1) / (kSelWarps * kMaxSplit));
     nsplit = std::max(1, (nGc + kSelWarps * gpw - 1) / (kSelWarps * gpw));
 }
 
@@ -454,9 +492,13 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         float* ws_s = reinterpret_cast<float*>(w + off);
         off += (size_t)m.units() * nsplit * 32 * sizeof(float);
         int* ws_i = reinterpret_cast<int*>(w + off);
+        const size_t smem = (size_t)kSelWarps * (gpw > 1 ? 2 : 1) * tile_bytes;
+        cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
         count_launch();
-        select_decode_kernel<T, D><<<dim3(nsplit, m.units()), kSelWarps * 32, 0, s>>>(
-            Q, summ, idx, ws_s, ws_i, ws_ctr, m.G, m.nG, ncand, m.k, gpw, nsplit, isd, c2);
+        select_decode_kernel<T, D><<<dim3(nsplit, m.units()), kSelWarps * 32, smem, s>>>(
+            Q, summ, idx, ws_s, ws_i, ws_ctr, m.G, m.nG, ncand, m.k, gpw, nsplit, isd, c2, err);
         return cudaGetLastError();
     }
     const size_t smem = tile_bytes * 2 + (size_t)kPfPos * 2 * D * 4;

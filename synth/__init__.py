@@ -317,3 +317,52 @@ def projections(w: Workload):
     pk = (s * normals_f64(key(w.seed, TAG_PK), w.d * w.d)).astype(np.float32).reshape(w.d, w.d)
     pv = (s * normals_f64(key(w.seed, TAG_PV), w.d * w.d)).astype(np.float32).reshape(w.d, w.d)
     return pk, pv
+
+
+# ------------------------------------------------------------------ device-side generation (large workloads)
+
+_CU_SRC = os.path.join(_HERE, "synth_cuda.cu")
+_CU_LIB_PATH = os.path.join(_HERE, "libsynth_cuda.so")
+_cu_lib = None
+
+
+def build_cuda(force: bool = False) -> str:
+    """Compile the device-side generator (nvcc, sm_100a) in place."""
+    if force or not os.path.exists(_CU_LIB_PATH) or os.path.getmtime(_CU_LIB_PATH) < os.path.getmtime(_CU_SRC):
+        tmp = _CU_LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["nvcc", "-O3", "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler", "-fPIC",
+                               "-shared", "-cudart", "static", "-o", tmp, _CU_SRC])
+        os.replace(tmp, _CU_LIB_PATH)
+    return _CU_LIB_PATH
+
+
+def _cu():
+    global _cu_lib
+    if _cu_lib is None:
+        build_cuda()
+        lib = ctypes.CDLL(_CU_LIB_PATH)
+        vp, u64, i64 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64
+        lib.synth_gpu_block_rows_bf16.argtypes = [u64, vp, vp, i64, i64, i64, i64, vp, vp]
+        lib.synth_gpu_block_rows_bf16.restype = ctypes.c_int
+        _cu_lib = lib
+    return _cu_lib
+
+
+def keys_unit_on_device(w: Workload, b: int, h: int, out, T: Optional[int] = None, stream=None) -> None:
+    """Fill a CUDA bf16 tensor out [T, d] with the keys of unit (b, h), drawn on the device.
+
+    Same streams and distribution as keys_unit; the device's double-precision log/cos may put a
+    value on a neighbouring bf16. Use keys_unit where both sides must see identical bytes.
+    """
+    import torch
+    T = w.T if T is None else T
+    assert w.dtype == "bf16" and out.dtype == torch.bfloat16 and out.is_contiguous() and out.numel() == T * w.d
+    mu, sigma = block_params(w, b, h)
+    dmu = torch.from_numpy(mu).to(out.device)
+    dsig = torch.from_numpy(sigma).to(out.device)
+    s = torch.cuda.current_stream(out.device) if stream is None else stream
+    rc = _cu().synth_gpu_block_rows_bf16(key(w.seed, TAG_KZ, b, h), dmu.data_ptr(), dsig.data_ptr(), mu.shape[0],
+                                         T, w.d, w.block, out.data_ptr(), s.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"device generator launch failed ({rc})")
+    s.synchronize()  # dmu / dsig go out of scope
