@@ -38,7 +38,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k"])
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k", "sweep"])
+    ap.add_argument("--contexts", default=None, help="sweep: comma-separated context lengths (default 8k .. 1M)")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
     ap.add_argument("--T", type=int, default=None, help="override the context length (small profiling cases)")
@@ -73,9 +74,17 @@ def read_peaks():
     return 6650.0, "fallback"
 
 
-def source_hash() -> str:
+# the sources a kernel's DRAM traffic depends on (its own file and the headers it includes)
+KERNEL_SOURCES = {
+    "decode_attention": ["decode_stream.cu", "common.cuh", "dims.h", "tma.cu", "tma.h"],
+    "select_decode": ["select.cu", "common.cuh", "dims.h"],
+    "prefill_tc": ["prefill.cu", "tc.cuh", "common.cuh", "dims.h", "tma.cu", "tma.h"],
+}
+
+
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(CSRC)):
+    for fn in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(CSRC, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -90,7 +99,7 @@ def recorded_traffic(kernel: str):
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel)
-    if not ent or ent.get("source_hash") != source_hash():
+    if not ent or ent.get("source_hash") != source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -178,12 +187,13 @@ def decode_bytes(w, idx):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units):
-    """Time the oracle (as it stands) on the listed units; returns (seconds, query heads)."""
+def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False):
+    """Time the oracle (as it stands) on the listed units; returns (seconds, query heads[, result])."""
     from oracle import cobs_oracle as O
     t0 = time.perf_counter()
-    O.decode(w, K, V, Q, g, Pk, Pv, units=units)
-    return time.perf_counter() - t0, len(units) * w.G
+    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units)
+    secs = time.perf_counter() - t0
+    return (secs, len(units) * w.G, res) if with_result else (secs, len(units) * w.G)
 
 
 def limit_threads():
@@ -319,7 +329,7 @@ def bench_prefill(w, steps, warmup, dev, cobs):
                    "window": w.window, "l2": "inputs larger than L2 (Q 0.5 GB)"},
         "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": att_tf, "peak": sustained,
                      "unit": "TFLOP/s", "frac": att_tf / sustained, "peak_kind": f"{kind} sustained bf16",
-                     "traffic": None},
+                     "traffic": recorded_traffic("prefill_tc")},
         "summary_build_gbs": (kv_bytes + buf.summaries.numel() * 4 + 2 * buf.Kc.numel() * 2) / (t_sum * 1e-3) / 1e9,
         "gpu_launches": launches,
         "steps": steps,
@@ -393,19 +403,8 @@ def run_ours(args):
         graphs[r].replay()
     stream.synchronize()
 
-    # parity spot check of what the bench runs: selected blocks of two units vs the oracle
     idx0 = bufs[0].idx.cpu().numpy()
-    parity = None
-    if rank == 0:
-        from oracle import cobs_oracle as O
-        ok = True
-        for (b, h) in [(0, 0), (w.B - 1, w.Hkv - 1)]:
-            Kf = synth.to_f64(K[b, h], w.dtype)
-            summ = O.canonical_summaries(Kf.astype(np.float32), w.block)
-            qs = synth.to_f64(Q[b, h * w.G:(h + 1) * w.G], w.dtype).astype(np.float32)
-            sel, _ = O.select_decode(w, qs, summ)
-            ok &= bool(np.array_equal(sel, idx0[b, h]))
-        parity = "idx bit-exact on 2 sampled units" if ok else "IDX MISMATCH"
+    O0 = bufs[0].O.float().cpu().numpy()
 
     # ---- timed region: K graph replays, cache copies rotated (L2 defeat) ----
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -423,35 +422,38 @@ def run_ours(args):
         dist.barrier()
     clocks = clk.summary()
 
-    # ---- per-call durations: each call captured in its own graph, events recorded between the
-    # replays on the launching stream (same copy rotation as the timed region) ----
-    calls = []
+    # ---- per-call durations inside the step: a second set of step graphs with timing events
+    # captured between the calls (event-record nodes), replayed one at a time on the launching
+    # stream with the same copy rotation; the headline graphs above carry no events ----
+    tgraphs, tevs = [], []
     for r in range(R):
-        gu, gs, ga = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gu, stream=stream):
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            evs[0].record(stream)
             cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc, bufs[r].Vc)
-        with torch.cuda.graph(gs, stream=stream):
+            evs[1].record(stream)
             cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select)
-        with torch.cuda.graph(ga, stream=stream):
+            evs[2].record(stream)
             cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg, bufs[r].O,
                                          bufs[r].ws_attn)
-        calls.append((gu, gs, ga))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+            evs[3].record(stream)
+        tgraphs.append(gr)
+        tevs.append(evs)
+    t_parts = []
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        for i in range(args.steps):
-            gu, gs, ga = calls[i % R]
-            ev[i][0].record(stream)
-            gu.replay()
-            ev[i][1].record(stream)
-            gs.replay()
-            ev[i][2].record(stream)
-            ga.replay()
-            ev[i][3].record(stream)
-    torch.cuda.synchronize()
-    t_upd = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)) / args.steps
-    t_sel = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)) / args.steps
-    t_att = sum(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)) / args.steps
+        for i in range(args.steps + R):
+            r = i % R
+            tgraphs[r].replay()
+            stream.synchronize()
+            if i >= R:   # the first pass over the copies is a warm-up
+                e = tevs[r]
+                t_parts.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])))
+    t_upd = statistics.median(x[0] for x in t_parts)
+    t_sel = statistics.median(x[1] for x in t_parts)
+    t_att = statistics.median(x[2] for x in t_parts)
+    del tgraphs
 
     # ---- end to end through the public API: pinned host inputs in, output back, every step ----
     hQ = torch.from_numpy(np.ascontiguousarray(Q).view(np.int16)).view(torch.bfloat16).pin_memory() \
@@ -495,7 +497,7 @@ def run_ours(args):
                    "parallelism": f"dp{world} (independent decode batches per GPU)"},
         "hbm_gbs": by["total"] / (ms * 1e-3) / 1e9,
         "hbm_bytes_per_step": by["total"],
-        "roofline": {"bound": "hbm", "kernel": "cobs_sparse_attn_decode (chunk + merge)",
+        "roofline": {"bound": "hbm", "kernel": "cobs_sparse_attn_decode (decode_stream_kernel + decode_stream_merge)",
                      "achieved": att_gbs, "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
                      "peak_kind": peak_kind, "algorithmic_bytes_per_launch": by["attn"],
                      "traffic": recorded_traffic("decode_attention")},
@@ -505,7 +507,6 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
-        "parity": parity,
         "device_error": dev_err,
         "kv_tokens_per_unit": by["kv_tokens_per_unit"],
     }
@@ -514,21 +515,26 @@ def run_ours(args):
         os.environ.setdefault("OMP_NUM_THREADS", "1")
         lim = limit_threads()
         units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:24]
-        secs, heads = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units)
+        secs, heads, ref = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=True)
         result["cpu_baseline"] = {"value": heads / secs, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                                   "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
                                             f"full oracle decode incl. summaries ({secs:.1f} s)"}
+        # the same oracle run checks what the bench ran: indices bit for bit, outputs within 2e-2
+        same_idx = all(np.array_equal(ref["idx"][b, h], idx0[b, h]) for (b, h) in units)
+        err = max(float(np.abs(ref["O"][b, h * w.G:(h + 1) * w.G] - O0[b, h * w.G:(h + 1) * w.G]).max())
+                  for (b, h) in units)
+        result["parity"] = {"units": len(units), "idx_bit_exact": same_idx, "out_max_abs_err": err,
+                            "out_tol": 2e-2}
         del lim
     if not args.no_prefill and world == 1:
         wp = synth.WORKLOADS["prefill32k"]
-        del Ks, Vs, bufs, graphs[:], calls[:]
+        del Ks, Vs, bufs, graphs[:]
         torch.cuda.empty_cache()
         result["prefill"] = bench_prefill(wp, args.prefill_steps, 2, dev, cobs)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
         graphs.clear()
-        calls.clear()
         dist.destroy_process_group()
     return 0
 
@@ -550,10 +556,137 @@ def run_prefill_line(args, w, dev, cobs, rank, world):
     return 0
 
 
+# ------------------------------------------------------------------ selector sweep over context length
+
+def osa_top_k(E, k):
+    """Indices of the k largest entries of E (ties to the lower index), ascending."""
+    import numpy as np
+    order = np.lexsort((np.arange(E.shape[0]), -E))
+    return np.sort(order[:k])
+
+
+def run_sweep(args):
+    """Decode selection (cobs_select) on 64 sequences x 8 KV heads (32 query heads, top-16) at
+    each context length: GB/s of the selector, and recall@16 of alpha = 1 and alpha = 0 against
+    the oracle sparse attention (top-16 blocks by exact attention mass, from cobs_block_log_mass)
+    on the first 8 sequences. Keys are drawn on the device; only summaries stay resident."""
+    import numpy as np
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from block_sparse_long_summary_b200 import build as B
+    B.build()
+    from block_sparse_long_summary_b200 import cobs
+    import synth
+    base = synth.WORKLOADS["sweep"]
+    if args.batch:
+        base = base.replace(B=args.batch)
+    contexts = [int(x) for x in args.contexts.split(",")] if args.contexts else list(synth.SWEEP_CONTEXTS)
+    peak, peak_kind = read_peaks()
+    n_rec = min(8, base.B)
+    l2_bytes = 126e6
+    rows, launches = [], 0
+    stream = torch.cuda.Stream(device=dev)
+
+    def params(w, **over):
+        kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
+                  cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+        kw.update(over)
+        return cobs.Params(**kw)
+
+    for T in contexts:
+        w = base.replace(T=T)
+        p, p0, p1 = params(w), params(w, alpha=0.0), params(w, B=1)
+        nB = T // w.block
+        per_b = cobs.summaries_elems(p1)
+        summ = torch.empty(w.B * per_b, dtype=torch.float32, device=dev)
+        Kb = torch.empty((w.Hkv, T, w.d), dtype=torch.bfloat16, device=dev)
+        nC = max(1, (T - w.cmp_block) // w.cmp_stride + 1)
+        Kc = torch.empty((1, w.Hkv, nC, w.d), dtype=torch.bfloat16, device=dev)
+        Vc = torch.empty_like(Kc)
+        Pk, Pv = synth.projections(w)
+        tPk, tPv = to_dev(Pk, "f32", dev), to_dev(Pv, "f32", dev)
+        tQ = to_dev(synth.queries_decode(w), "bf16", dev)
+        mass = torch.empty((n_rec, w.Hq, nB), dtype=torch.float32, device=dev)
+        n0 = cobs.launch_count()
+        with torch.cuda.stream(stream):
+            for b in range(w.B):
+                for h in range(w.Hkv):
+                    synth.keys_unit_on_device(w, b, h, Kb[h], stream=stream)
+                cobs.cobs_build_summaries(p1, Kb, Kb, tPk, tPv, 0, summ[b * per_b:(b + 1) * per_b], Kc, Vc)
+                if b < n_rec:
+                    cobs.cobs_block_log_mass(p1, tQ[b:b + 1], Kb, mass[b:b + 1])
+        stream.synchronize()
+        del Kb, Kc, Vc
+        # L2 defeat: enough summary copies that the rotated working set exceeds 4 x L2
+        sbytes = summ.numel() * 4
+        R = max(1, min(16, int(np.ceil(4 * l2_bytes / sbytes))))
+        copies = [summ] + [summ.clone() for _ in range(R - 1)]
+        idx = torch.empty((w.B, w.Hkv, w.topk), dtype=torch.int32, device=dev)
+        ws = torch.zeros(max(16, cobs.workspace_bytes(p, cobs.COBS_WS_SELECT)), dtype=torch.uint8, device=dev)
+        with torch.cuda.stream(stream):
+            cobs.cobs_select(p0, tQ, summ, 0, idx, ws)
+        stream.synchronize()
+        idx_a0 = idx.cpu().numpy()
+        graphs = []
+        for r in range(R):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                cobs.cobs_select(p, tQ, copies[r], 0, idx, ws)
+            graphs.append(gr)
+        n_rep = max(20, 3 * R)
+        with torch.cuda.stream(stream):
+            for i in range(max(3, args.warmup) * R):
+                graphs[i % R].replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(n_rep):
+                graphs[i % R].replay()
+            e1.record(stream)
+        stream.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / n_rep
+        idx_a1 = idx.cpu().numpy()
+        launches += cobs.launch_count() - n0
+        m = mass.cpu().numpy().astype(np.float64)
+        rec1, rec0 = [], []
+        for b in range(n_rec):
+            for g in range(w.Hkv):
+                osa = osa_top_k(m[b, g * w.G:(g + 1) * w.G].sum(axis=0), w.topk)
+                ref = set(osa.tolist())
+                rec1.append(len(ref & set(int(x) for x in idx_a1[b, g] if x >= 0)) / w.topk)
+                rec0.append(len(ref & set(int(x) for x in idx_a0[b, g] if x >= 0)) / w.topk)
+        by = w.B * w.Hkv * nB * 2 * w.d * 4 + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * w.topk * 4
+        gbs = by / (us * 1e-6) / 1e9
+        rows.append({"T": T, "nB": nB, "bytes": by, "us": us, "gbs": gbs, "frac": gbs / peak,
+                     "recall_alpha1": float(np.mean(rec1)), "recall_alpha0": float(np.mean(rec0)),
+                     "l2": f"{R} summary copies rotated" if R > 1 else "summaries larger than L2"})
+        del graphs, copies, summ, mass
+        torch.cuda.empty_cache()
+    top = rows[-1]
+    line = {"metric": "selector GB/s over context length (decode selection, 64 x 8 units, top-16)",
+            "value": top["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": n_rep, "warmup": max(3, args.warmup),
+            "ms_per_step": top["us"] * 1e-3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (keys drawn on the device)",
+            "config": {"workload": "sweep", "B": base.B, "Hq": base.Hq, "Hkv": base.Hkv, "d": base.d,
+                       "topk": base.topk, "contexts": contexts, "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
+            "roofline": {"bound": "hbm", "kernel": "select_decode_kernel", "achieved": top["gbs"], "peak": peak,
+                         "unit": "GB/s", "frac": top["frac"], "peak_kind": peak_kind,
+                         "traffic": recorded_traffic("select_decode")},
+            "sweep": rows, "gpu_launches": launches, "device_error": cobs.device_error()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
     return run_ours(args)
 
 

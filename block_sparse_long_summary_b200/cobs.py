@@ -30,7 +30,7 @@ COBS_WS_PREFILL = 2
 EXPORTED = [
     "cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
     "cobs_sparse_attn_decode_noalloc", "cobs_workspace_bytes", "cobs_summaries_elems", "cobs_status_string", "cobs_last_error",
-    "cobs_device_error", "cobs_launch_count", "cobs_version",
+    "cobs_device_error", "cobs_launch_count", "cobs_version", "cobs_block_log_mass",
 ]
 
 
@@ -59,8 +59,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.cobs_sparse_attn_decode.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cobs_sparse_attn_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cobs_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.cobs_block_log_mass.argtypes = [P, vp, vp, vp, vp]
     for f in ("cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
-              "cobs_sparse_attn_decode_noalloc"):
+              "cobs_sparse_attn_decode_noalloc", "cobs_block_log_mass"):
         getattr(lib, f).restype = ctypes.c_int
     lib.cobs_workspace_bytes.argtypes = [P, i32]
     lib.cobs_workspace_bytes.restype = sz
@@ -190,6 +191,12 @@ def cobs_sparse_attn_prefill(p: Params, Q, K, V, Kc, Vc, idx, gates, O, workspac
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.cobs_sparse_attn_prefill(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(Kc), _ptr(Vc),
                                          _ptr(idx), _ptr(gates), _ptr(O), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def cobs_block_log_mass(p: Params, Q, K, out, stream=None):
+    """Evaluation only: ln of the exact attention mass of every complete block, out [B, Hq, T // 64]."""
+    cp = p.c()
+    _check(_lib.cobs_block_log_mass(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(out), _stream(stream)))
 
 
 # -------------------------------------------------------------- buffers (allocated by torch, not the library)

@@ -270,4 +270,17 @@ cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const 
     return COBS_OK;
 }
 
+cobs_status cobs_block_log_mass(const cobs_params* p, const void* Q, const void* K, float* out,
+                                cobs_stream_t stream) {
+    COBS_TRY(validate(p));
+    COBS_TRY(check_ptr(Q, "Q"));
+    COBS_TRY(check_ptr(K, "K"));
+    COBS_TRY(check_ptr(out, "out"));
+    const cobs::Dims m = cobs::make_dims(*p);
+    if (m.G > 16) return fail(COBS_ERR_UNSUPPORTED, "cobs_block_log_mass supports at most 16 query heads per group");
+    cudaError_t e = cobs::launch_block_log_mass(m, Q, K, out, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_block_log_mass launch");
+    return COBS_OK;
+}
+
 }  // extern "C"

@@ -13,8 +13,9 @@ enum DeviceError : int {
     kErrWaitTimeout = 2,   // a bounded wait on an mbarrier gave up
 };
 
-// Iterations of a bounded mbarrier wait (each polls once, then sleeps a little):
-// about 0.1 s in total, far above any legitimate wait of these kernels.
+// Iterations of a bounded mbarrier wait (each polls once, or waits in hardware for at most
+// about a microsecond): about 0.1 s (polling) to 1 s (hardware waits) in total, far above any
+// legitimate wait of these kernels.
 constexpr uint32_t kMaxWaitIters = 1u << 20;
 
 __device__ __forceinline__ void report_error(int* flag, int code) {
@@ -74,7 +75,46 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete. Returns false (and
-// records kErrWaitTimeout) if it did not complete within kMaxWaitIters polls.
+// records kErrWaitTimeout) if it did not complete in time.
+#ifndef COBS_WAIT_TRY
+#define COBS_WAIT_TRY 1
+#endif
+#if COBS_WAIT_TRY
+// One hardware wait of at most about kSuspendHintNs: the warp is woken when the phase completes.
+constexpr uint32_t kSuspendHintNs = 1000;
+// Give up after this long (far above any legitimate wait of these kernels), or after
+// kMaxWaitIters hardware waits, whichever comes first.
+constexpr uint64_t kWaitLimitNs = 100000000ull;
+
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kMaxWaitIters; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+    report_error(err, kErrWaitTimeout);
+    return false;
+}
+#else
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
     for (uint32_t i = 0; i < kMaxWaitIters; ++i) {
         if (mbar_test(bar, parity)) return true;
@@ -83,6 +123,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     report_error(err, kErrWaitTimeout);
     return false;
 }
+#endif
 
 // Bulk (TMA) copy of `bytes` (multiple of 16; both addresses 16-byte aligned) from
 // global to this CTA's shared memory, completing on `bar` as transaction bytes.

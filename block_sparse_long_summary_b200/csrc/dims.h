@@ -71,4 +71,8 @@ cudaError_t launch_prefill(const Dims& m, const void* Q, const void* K, const vo
                            const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                            cudaStream_t s, int* err);
 
+// Evaluation only: ln of the exact attention mass of every complete block, out [B, Hq, nB] f32
+// (cudaErrorNotSupported if G > 16).
+cudaError_t launch_block_log_mass(const Dims& m, const void* Q, const void* K, float* out, cudaStream_t s);
+
 }  // namespace cobs

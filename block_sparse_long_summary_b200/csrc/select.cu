@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "dims.h"
+#include "tma.h"
 
 namespace cobs {
 namespace {
@@ -98,14 +99,20 @@ __device__ __forceinline__ float to_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Canonical group query: Qsum_c = sum_h q_{h,c}, Q2_c = fma-sum of q_{h,c}^2, ascending h.
-template <typename T>
-__device__ __forceinline__ void group_query(const T* q, int G, int d, int c, float& qs, float& q2) {
+// Largest GQA group (query heads per KV head) the selectors handle; the host rejects larger.
+constexpr int kMaxGroup = 16;
+
+// Canonical group query: Qsum_c = sum_h q_{h,c} (adds) and Q2_c = fma-sum of q_{h,c}^2, in
+// ascending h, from values already in registers (x[h] = q_{h,c}, ascending h). Callers
+// issue all G loads of a channel at once (independent loads) before reducing in order.
+__device__ __forceinline__ void group_reduce(const float (&x)[kMaxGroup], int G, float& qs, float& q2) {
     float s = 0.0f, s2 = 0.0f;
-    for (int h = 0; h < G; ++h) {
-        const float x = to_f(q[(size_t)h * d + c]);
-        s = __fadd_rn(s, x);
-        s2 = __fmaf_rn(x, x, s2);
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (h < G) {
+            s = __fadd_rn(s, x[h]);
+            s2 = __fmaf_rn(x[h], x[h], s2);
+        }
     }
     qs = s;
     q2 = s2;
@@ -133,35 +140,6 @@ __device__ __forceinline__ float block_score(const float* tile, const float* qs,
         v = __fmaf_rn(q2[4 * c4 + 1], s.y, v);
         v = __fmaf_rn(q2[4 * c4 + 2], s.z, v);
         v = __fmaf_rn(q2[4 * c4 + 3], s.w, v);
-    }
-    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
-}
-
-// Same canonical score, with the group query held in registers: lane l keeps channels
-// 4l .. 4l + 3 of Qsum and Q2 and the other lanes read them by shuffle (keeps shared memory for
-// the summary tile alone).
-template <int D>
-__device__ __forceinline__ float block_score_regq(const float* tile, float4 qs4, float4 q24, int lane, float isd,
-                                                  float c2) {
-    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
-    const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
-    float a = 0.0f, v = 0.0f;
-#pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 m = mu4[c4 * 32];
-        const float4 s = var4[c4 * 32];
-        const float qa = __shfl_sync(kFull, qs4.x, c4), qb = __shfl_sync(kFull, qs4.y, c4);
-        const float qc = __shfl_sync(kFull, qs4.z, c4), qd = __shfl_sync(kFull, qs4.w, c4);
-        const float ra = __shfl_sync(kFull, q24.x, c4), rb = __shfl_sync(kFull, q24.y, c4);
-        const float rc = __shfl_sync(kFull, q24.z, c4), rd = __shfl_sync(kFull, q24.w, c4);
-        a = __fmaf_rn(qa, m.x, a);
-        a = __fmaf_rn(qb, m.y, a);
-        a = __fmaf_rn(qc, m.z, a);
-        a = __fmaf_rn(qd, m.w, a);
-        v = __fmaf_rn(ra, s.x, v);
-        v = __fmaf_rn(rb, s.y, v);
-        v = __fmaf_rn(rc, s.z, v);
-        v = __fmaf_rn(rd, s.w, v);
     }
     return __fmaf_rn(c2, v, __fmul_rn(a, isd));
 }
@@ -200,144 +178,213 @@ __device__ __forceinline__ void warp_merge_best_first(float& s, int& i, float bs
     for (int j = 16; j > 0; j >>= 1) cmp_swap(s, i, j, true, lane);
 }
 
-#ifndef COBS_SELECT_WARPS
-#define COBS_SELECT_WARPS 1
+#ifndef COBS_SELECT_STAGES
+#define COBS_SELECT_STAGES 2
 #endif
-constexpr int kSelWarps = COBS_SELECT_WARPS;
-constexpr int kMaxSplit = 32;
+#ifndef COBS_SELECT_CTAS_PER_SM
+#define COBS_SELECT_CTAS_PER_SM 3
+#endif
+constexpr int kSelStages = COBS_SELECT_STAGES;
+constexpr int kSelCtasPerSm = COBS_SELECT_CTAS_PER_SM;
+// Upper bound of the decode selector's grid (any sm_100 part), fixing the workspace size
+// without a device query.
+constexpr int kSelGridCap = 192 * kSelCtasPerSm;
 
-// grid (nsplit, units), 2 warps. Warp w of split s scores groups [(s*2 + w)*gpw, +gpw) of its
-// unit: each group (32 blocks, 32 KiB) arrives with one bulk (TMA) copy into the warp's own
-// buffer (two buffers when a warp has several groups), lane = block, and the warp keeps a sorted
-// best-first list (bitonic sort + merge). The CTA's two lists are merged in shared memory. With
-// one split the CTA writes the answer; otherwise every CTA deposits its list and takes an atomic
-// ticket (nobody waits), and the CTA that takes the last ticket merges all lists of the unit
-// with a shared-memory tree. The ticket counter returns to zero by itself. The result is the
-// top-k under a strict total order, so it does not depend on arrival order.
+// Stream-K split of the decode selection: the n = units * nGc summary groups, unit-major, are
+// cut into `grid` contiguous ranges [c n / grid, (c + 1) n / grid). CTA of group x:
+__host__ __device__ __forceinline__ int sel_cta_of(long long x, long long n, int grid) {
+    return (int)(((x + 1) * grid + n - 1) / n) - 1;
+}
+
+// Partial lists a unit can be split into (workspace slots per unit). The grid is capped so that
+// a unit's groups meet at most min(nGc, ceil(grid / units) + 1) <= this many CTA ranges.
+constexpr int kSelMaxSeg = 64;
+inline int sel_max_segments(int units, int nGc) {
+    return std::min(std::min(nGc, kSelMaxSeg), kSelGridCap / std::max(1, units) + 2);
+}
+
+// Running best-first list of one warp (lane j = j-th best), with the k-th best as the bar
+// a newcomer must beat. Groups with no lane above the bar cost one ballot.
+struct RunList {
+    float s;
+    int i;
+    float ts;
+    int ti;
+    __device__ void init() {
+        s = -INFINITY;
+        i = kInvalid;
+        ts = -INFINITY;
+        ti = kInvalid;
+    }
+    __device__ void bar(int k) {
+        ts = __shfl_sync(kFull, s, k - 1);
+        ti = __shfl_sync(kFull, i, k - 1);
+    }
+    // one candidate per lane (invalid lanes carry (-inf, kInvalid))
+    __device__ void add(float sc, int bi, int k, int lane) {
+        const unsigned up = __ballot_sync(kFull, bi != kInvalid && better(sc, bi, ts, ti));
+        if (up == 0u) return;
+        warp_sort_best_first(sc, bi, lane);
+        warp_merge_best_first(s, i, sc, bi, lane);
+        bar(k);
+    }
+};
+
+// grid (G_sel), one warp per CTA, persistent. CTA c scores the summary groups of its stream-K
+// range in order: each group (32 blocks, 2 d 32 floats) arrives by one bulk (TMA) copy into a
+// kSelStages-deep ring, lane = block, and the group query of the current unit sits in shared
+// memory (read as broadcasts). When the range leaves a unit, the CTA writes that unit's answer
+// if it held the whole unit, else deposits its segment's exact top-k; select_merge_kernel (a
+// dependent launch) merges the deposits. The result is the top-k under a strict total order,
+// so it does not depend on the split.
 template <typename T, int D>
-__global__ void __launch_bounds__(kSelWarps * 32) select_decode_kernel(
-    const T* __restrict__ Q, const float* __restrict__ summ, int32_t* __restrict__ idx, float* __restrict__ ws_s,
-    int* __restrict__ ws_i, unsigned* __restrict__ ws_ctr, int G, int nG, int ncand, int k, int gpw, int nsplit,
-    float isd, float c2, int* err) {
+__global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
+                                                           int32_t* __restrict__ idx, float* __restrict__ ws_s,
+                                                           int* __restrict__ ws_i, int units, int G, int nG,
+                                                           int ncand, int k, int maxseg,
+                                                           float isd, float c2, int* err) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t bar[kSelWarps][2];
-    __shared__ unsigned ticket_sh;
+    __shared__ __align__(8) uint64_t bar[kSelStages];
+    __shared__ __align__(16) float qsm[2][D];
     constexpr uint32_t kTileBytes = 2 * D * 32 * 4;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int unit = blockIdx.y;
-    const int split = blockIdx.x;
+    constexpr int kTileFloats = 2 * D * 32;
+    // the merge grid may be scheduled now; it still waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int lane = threadIdx.x;
+    const int grid = gridDim.x, c = blockIdx.x;
     const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
-    const float* usum = summ + (size_t)unit * nG * 2 * D * 32;
-    const int stages = gpw > 1 ? 2 : 1;
-    float* tiles = reinterpret_cast<float*>(smem_raw) + (size_t)warp * stages * 2 * D * 32;
-    const int g0 = (split * kSelWarps + warp) * gpw;
-    const int g1 = min(nGc, g0 + gpw);
+    const long long n = (long long)units * nGc;
+    float* tiles = reinterpret_cast<float*>(smem_raw);
+    if (n == 0) {  // no complete block anywhere: every list is empty
+        for (int u = c; u < units; u += grid)
+            if (lane < k) idx[(size_t)u * k + lane] = -1;
+        return;
+    }
+    const long long x0 = (long long)c * n / grid, x1 = (long long)(c + 1) * n / grid;
+    if (x0 >= x1) return;
+    auto group_src = [&](long long x) {
+        const long long u = x / nGc, gl = x % nGc;
+        return summ + ((size_t)u * nG + (size_t)gl) * kTileFloats;
+    };
     if (lane == 0) {
-        mbar_init(&bar[warp][0], 1);
-        mbar_init(&bar[warp][1], 1);
+#pragma unroll
+        for (int st = 0; st < kSelStages; ++st) mbar_init(&bar[st], 1);
         fence_barrier_init();
     }
     __syncwarp();
     if (lane == 0) {
-        for (int st = 0; st < stages && g0 + st < g1; ++st) {
-            mbar_arrive_expect_tx(&bar[warp][st], kTileBytes);
-            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(g0 + st) * 2 * D * 32, kTileBytes, &bar[warp][st]);
+        for (int st = 0; st < kSelStages && x0 + st < x1; ++st) {
+            mbar_arrive_expect_tx(&bar[st], kTileBytes);
+            bulk_g2s(tiles + st * kTileFloats, group_src(x0 + st), kTileBytes, &bar[st]);
         }
     }
-    // group query in registers: lane l holds channels 4l .. 4l + 3
-    // (unit = b * Hkv + g and Hq = Hkv * G, so the group's first head row is unit * G)
-    float4 qs4 = make_float4(0.f, 0.f, 0.f, 0.f), q24 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (lane * 4 < D) {
-        const T* qg = Q + (size_t)unit * G * D;
-        group_query(qg, G, D, 4 * lane + 0, qs4.x, q24.x);
-        group_query(qg, G, D, 4 * lane + 1, qs4.y, q24.y);
-        group_query(qg, G, D, 4 * lane + 2, qs4.z, q24.z);
-        group_query(qg, G, D, 4 * lane + 3, qs4.w, q24.w);
-    }
 
-    float ls = -INFINITY;
-    int li = kInvalid;
+    RunList rl;
+    rl.init();
+    int cur = -1;
     bool ok = true;
-    for (int g = g0, it = 0; g < g1; ++g, ++it) {
-        const int st = it % stages;
-        const uint32_t parity = (it / stages) & 1;
-        if (ok) ok = mbar_wait(&bar[warp][st], parity, err);
+    // Finish unit u: write its answer (this CTA held all of it) or deposit this segment's top-k.
+    auto finish = [&](int u) {
+        const int cf = sel_cta_of((long long)u * nGc, n, grid);
+        const int cl = sel_cta_of((long long)(u + 1) * nGc - 1, n, grid);
+        if (cl == cf) {
+            const int key = warp_sort_asc(lane < k ? rl.i : kInvalid, lane);
+            if (lane < k) idx[(size_t)u * k + lane] = key == kInvalid ? -1 : key;
+            return;
+        }
+        if (lane < k) {
+            ws_s[((size_t)u * maxseg + (c - cf)) * k + lane] = rl.s;
+            ws_i[((size_t)u * maxseg + (c - cf)) * k + lane] = rl.i;
+        }
+    };
+
+    for (long long x = x0; x < x1; ++x) {
+        const int it = (int)(x - x0);
+        const int st = it % kSelStages;
+        const uint32_t parity = (uint32_t)(it / kSelStages) & 1u;
+        const int u = (int)(x / nGc), gl = (int)(x % nGc);
+        if (u != cur) {
+            if (cur >= 0) finish(cur);
+            rl.init();
+            cur = u;
+            // group query of unit u (heads u*G .. u*G+G-1 of Q [B, Hq, d]): Qsum and Q2 of
+            // channels lane + 32 j, every head's value loaded at once
+            __syncwarp();
+            {
+                const T* qg = Q + (size_t)u * G * D;
+                float x[D / 32][kMaxGroup];
+#pragma unroll
+                for (int j = 0; j < D / 32; ++j)
+#pragma unroll
+                    for (int h = 0; h < kMaxGroup; ++h) x[j][h] = h < G ? to_f(qg[(size_t)h * D + lane + 32 * j]) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < D / 32; ++j) group_reduce(x[j], G, qsm[0][lane + 32 * j], qsm[1][lane + 32 * j]);
+            }
+            __syncwarp();
+        }
+        if (ok) ok = mbar_wait(&bar[st], parity, err);
         ok = __all_sync(kFull, ok);
-        const int b = g * kGroupBlocks + lane;
+        const int b = gl * kGroupBlocks + lane;
         float sc = -INFINITY;
         int bi = kInvalid;
-        if (ok) {  // warp-uniform: every lane takes part in the score's shuffles
-            const float s_all = block_score_regq<D>(tiles + st * 2 * D * 32, qs4, q24, lane, isd, c2);
+        if (ok) {
+            const float s_all = block_score<D>(tiles + st * kTileFloats, qsm[0], qsm[1], lane, isd, c2);
             if (b < ncand) {
                 sc = s_all;
                 bi = b;
             }
         }
         __syncwarp();
-        if (lane == 0 && ok && g + stages < g1) {
+        if (lane == 0 && ok && x + kSelStages < x1) {
             fence_proxy_async();
-            mbar_arrive_expect_tx(&bar[warp][st], kTileBytes);
-            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(g + stages) * 2 * D * 32, kTileBytes, &bar[warp][st]);
+            mbar_arrive_expect_tx(&bar[st], kTileBytes);
+            bulk_g2s(tiles + st * kTileFloats, group_src(x + kSelStages), kTileBytes, &bar[st]);
         }
-        warp_sort_best_first(sc, bi, lane);
-        if (it == 0) {
-            ls = sc;
-            li = bi;
-        } else {
-            warp_merge_best_first(ls, li, sc, bi, lane);
-        }
+        rl.add(sc, bi, k, lane);
     }
-    // the tile buffers are free once every warp is done: reuse them for the list merges
-    __syncthreads();
-    float (*ls_sh)[32] = reinterpret_cast<float (*)[32]>(smem_raw);
-    int (*li_sh)[32] = reinterpret_cast<int (*)[32]>(smem_raw + kMaxSplit * 32 * sizeof(float));
-    ls_sh[warp][lane] = ls;
-    li_sh[warp][lane] = li;
-    __syncthreads();
-    if (warp == 0) {
-        for (int w = 1; w < kSelWarps; ++w) warp_merge_best_first(ls, li, ls_sh[w][lane], li_sh[w][lane], lane);
-        if (nsplit == 1) {
-            const int key = warp_sort_asc(lane < k ? li : kInvalid, lane);
-            if (lane < k) idx[(size_t)unit * k + lane] = key == kInvalid ? -1 : key;
-        } else {
-            float* us = ws_s + ((size_t)unit * nsplit + split) * 32;
-            int* ui = ws_i + ((size_t)unit * nsplit + split) * 32;
-            us[lane] = ls;
-            ui[lane] = li;
-            __threadfence();
-            __syncwarp();
-            unsigned t = 0;
-            if (lane == 0) t = atomicInc(ws_ctr + unit, (unsigned)(nsplit - 1));
-            t = __shfl_sync(kFull, t, 0);
-            if (lane == 0) ticket_sh = t;
-        }
-    }
-    if (nsplit == 1) return;
-    __syncthreads();
-    if (ticket_sh != (unsigned)(nsplit - 1)) return;
-    // last CTA of the unit: all lists into shared memory, then a merge tree over the warps
-    __threadfence();
-    for (int e = tid; e < nsplit * 32; e += blockDim.x) {
-        ls_sh[e >> 5][e & 31] = __ldcg(ws_s + (size_t)unit * nsplit * 32 + e);
-        li_sh[e >> 5][e & 31] = __ldcg(ws_i + (size_t)unit * nsplit * 32 + e);
+    finish(cur);
+}
+
+// grid (units), 8 warps: merges the segment lists select_decode_kernel deposited for each unit
+// cut into several ranges (a shared-memory tree of warp merges, log2(segments) levels) and
+// writes the unit's answer in ascending block order. Launched as a programmatic dependent of
+// the selection grid: it waits for that grid to complete before reading the deposits.
+__global__ void __launch_bounds__(256) select_merge_kernel(const float* __restrict__ ws_s,
+                                                           const int* __restrict__ ws_i, int32_t* __restrict__ idx,
+                                                           int nGc, long long n, int grid, int k, int maxseg) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float ls[kSelMaxSeg][32];
+    __shared__ int li[kSelMaxSeg][32];
+    const int u = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (n == 0) return;
+    const int cf = sel_cta_of((long long)u * nGc, n, grid);
+    const int cl = sel_cta_of((long long)(u + 1) * nGc - 1, n, grid);
+    const int nseg = cl - cf + 1;
+    if (nseg == 1) return;  // written by the selection grid
+    for (int e = threadIdx.x; e < nseg * 32; e += blockDim.x) {
+        const int j = e >> 5, p = e & 31;
+        const bool in = p < k;
+        ls[j][p] = in ? ws_s[((size_t)u * maxseg + j) * k + p] : -INFINITY;
+        li[j][p] = in ? ws_i[((size_t)u * maxseg + j) * k + p] : kInvalid;
     }
     __syncthreads();
-    for (int width = 1; width < nsplit; width *= 2) {
-        for (int pair = warp; pair * 2 * width < nsplit; pair += kSelWarps) {
+    for (int width = 1; width < nseg; width *= 2) {
+        for (int pair = warp; pair * 2 * width < nseg; pair += 8) {
             const int x = pair * 2 * width, y = x + width;
-            if (y < nsplit) {
-                float s1 = ls_sh[x][lane];
-                int i1 = li_sh[x][lane];
-                warp_merge_best_first(s1, i1, ls_sh[y][lane], li_sh[y][lane], lane);
-                ls_sh[x][lane] = s1;
-                li_sh[x][lane] = i1;
+            if (y < nseg) {
+                float s1 = ls[x][lane];
+                int i1 = li[x][lane];
+                warp_merge_best_first(s1, i1, ls[y][lane], li[y][lane], lane);
+                ls[x][lane] = s1;
+                li[x][lane] = i1;
             }
         }
         __syncthreads();
     }
     if (warp == 0) {
-        const int key = warp_sort_asc(lane < k ? li_sh[0][lane] : kInvalid, lane);
-        if (lane < k) idx[(size_t)unit * k + lane] = key == kInvalid ? -1 : key;
+        const int key = warp_sort_asc(lane < k ? li[0][lane] : kInvalid, lane);
+        if (lane < k) idx[(size_t)u * k + lane] = key == kInvalid ? -1 : key;
     }
 }
 
@@ -380,14 +427,27 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
             bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)st * 2 * D * 32, kTileBytes, &bar[st]);
         }
     }
-    // group queries of the tile's positions
-    for (int e = tid; e < kPfPos * D; e += blockDim.x) {
-        const int p = e / D, c = e % D;
-        const int t = t0 + p;
-        float a = 0.0f, a2 = 0.0f;
-        if (t < Tctx) group_query(Q + (((size_t)b * Tctx + t) * Hq + (size_t)g * G) * D, G, D, c, a, a2);
-        sq[(p * 2 + 0) * D + c] = a;
-        sq[(p * 2 + 1) * D + c] = a2;
+    // group queries of the tile's positions: thread -> channel c of positions p0, p0 + ppi, ...,
+    // four positions (G head loads each) in flight at a time
+    {
+        constexpr int kPpi = 128 / D;  // positions covered by one pass of the 128 threads
+        const int c = tid % D, p0 = tid / D;
+        for (int pb = p0; pb < kPfPos; pb += 4 * kPpi) {
+            float x[4][kMaxGroup];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int p = pb + j * kPpi, t = t0 + p;
+                const T* qr = Q + (((size_t)b * Tctx + (t < Tctx ? t : 0)) * Hq + (size_t)g * G) * D + c;
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h)
+                    x[j][h] = (h < G && p < kPfPos && t < Tctx) ? to_f(qr[(size_t)h * D]) : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int p = pb + j * kPpi;
+                if (p < kPfPos) group_reduce(x[j], G, sq[(p * 2 + 0) * D + c], sq[(p * 2 + 1) * D + c]);
+            }
+        }
     }
     __syncthreads();
 
@@ -468,14 +528,6 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     }
 }
 
-// Decode selection split: each warp scores gpw consecutive 32-block groups, a CTA holds 2 warps,
-// and a unit is covered by nsplit <= 32 CTAs.
-void decode_split(const Dims& m, int& gpw, int& nsplit) {
-    const int nGc = (m.T / m.L + 31) / 32;
-    gpw = std::max(1, (nGc + kSelWarps * kMaxSplit - 1) / (kSelWarps * kMaxSplit));
-    nsplit = std::max(1, (nGc + kSelWarps * gpw - 1) / (kSelWarps * gpw));
-}
-
 template <typename T, int D>
 cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                             cudaStream_t s, int* err) {
@@ -484,22 +536,41 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
     const size_t tile_bytes = (size_t)2 * D * 32 * 4;
     if (!prefill) {
         const int ncand = m.T / m.L;
-        int gpw, nsplit;
-        decode_split(m, gpw, nsplit);
-        unsigned char* w = static_cast<unsigned char*>(ws);
-        unsigned* ws_ctr = reinterpret_cast<unsigned*>(w);
-        size_t off = ((size_t)m.units() * sizeof(unsigned) + 255) & ~(size_t)255;
-        float* ws_s = reinterpret_cast<float*>(w + off);
-        off += (size_t)m.units() * nsplit * 32 * sizeof(float);
-        int* ws_i = reinterpret_cast<int*>(w + off);
-        const size_t smem = (size_t)kSelWarps * (gpw > 1 ? 2 : 1) * tile_bytes;
+        const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
+        const long long n = (long long)m.units() * nGc;
+        const int maxseg = sel_max_segments(m.units(), std::max(1, nGc));
+        // grid: kSelCtasPerSm CTAs per SM and at least one group each. A unit's groups then meet
+        // at most min(nGc, ceil(grid / units) + 1) <= maxseg ranges (grid <= kSelGridCap).
+        long long grid = std::min<long long>((long long)sm_count() * kSelCtasPerSm, kSelGridCap);
+        grid = std::min<long long>(grid, std::max<long long>(1, n));
+        grid = std::min<long long>(grid, (long long)(kSelMaxSeg - 1) * m.units());
+        if (n == 0) grid = std::min(m.units(), 1024);
+        grid = std::max<long long>(1, grid);
+        float* ws_s = static_cast<float*>(ws);
+        int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
+        const size_t smem = (size_t)kSelStages * tile_bytes;
         cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         count_launch();
-        select_decode_kernel<T, D><<<dim3(nsplit, m.units()), kSelWarps * 32, smem, s>>>(
-            Q, summ, idx, ws_s, ws_i, ws_ctr, m.G, m.nG, ncand, m.k, gpw, nsplit, isd, c2, err);
-        return cudaGetLastError();
+        select_decode_kernel<T, D><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(), m.G, m.nG,
+                                                                    ncand, m.k, maxseg, isd, c2, err);
+        e = cudaGetLastError();
+        // a unit is cut into several ranges only if it has several groups and the grid several CTAs
+        if (e != cudaSuccess || n == 0 || nGc == 1 || grid == 1) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(m.units());
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        count_launch();
+        return cudaLaunchKernelEx(&cfg, select_merge_kernel, (const float*)ws_s, (const int*)ws_i, idx, nGc, n,
+                                  (int)grid, m.k, maxseg);
     }
     const size_t smem = tile_bytes * 2 + (size_t)kPfPos * 2 * D * 4;
     auto kern = select_prefill_kernel<T, D>;
@@ -515,10 +586,9 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
 
 size_t select_workspace_bytes(const Dims& m, int prefill) {
     if (prefill) return 0;
-    int gpw, nsplit;
-    decode_split(m, gpw, nsplit);
-    const size_t off = ((size_t)m.units() * sizeof(unsigned) + 255) & ~(size_t)255;
-    return off + (size_t)m.units() * nsplit * 32 * (sizeof(float) + sizeof(int));
+    const int nGc = (m.T / m.L + kGroupBlocks - 1) / kGroupBlocks;
+    const int maxseg = sel_max_segments(m.units(), std::max(1, nGc));
+    return (size_t)m.units() * maxseg * m.k * (sizeof(float) + sizeof(int));
 }
 
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,

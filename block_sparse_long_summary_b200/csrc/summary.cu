@@ -339,9 +339,11 @@ cudaError_t launch_fused(const Dims& m, const __nv_bfloat16* K, const __nv_bfloa
 
 // ---------------------------------------------------------------- decode-step append
 // The update after appending one token: at most one newly complete block (its summary) and one
-// newly complete compressed token (K and V) per unit. One CTA of 256 threads per unit: all row
-// loads in flight at once, then out_j = P[j, :] . pooled with a warp per 8 output rows at a
-// time (coalesced rows of P, interleaved shuffle reductions).
+// newly complete compressed token (K and V) per unit. Grid (units, 4) of 256 threads: CTA y
+// summarises channels [32 y, 32 y + 32) of the block and projects output rows
+// [y d / 4, (y + 1) d / 4) of both compressed tokens, each warp d / 16 rows at once
+// (out_j = P[j, :] . pooled, coalesced rows of P, interleaved shuffle reductions); every CTA
+// pools the 32 rows itself (all row loads in flight at once).
 template <typename T>
 __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, const T* __restrict__ V,
                                                      const float* __restrict__ Pk, const float* __restrict__ Pv,
@@ -350,10 +352,10 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
                                                      T* __restrict__ Vc) {
     __shared__ __align__(16) float pooled[2][128];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int unit = blockIdx.x;
-    // block summary (threads < d): the canonical row-order sums
-    if (jb >= 0 && tid < d) {
-        const int c = tid;
+    const int unit = blockIdx.x, quarter = blockIdx.y;
+    // block summary (channels 32 quarter + tid): the canonical row-order sums
+    if (jb >= 0 && tid < 32 && quarter * 32 + tid < d) {
+        const int c = quarter * 32 + tid;
         const T* rows = K + ((size_t)unit * Tctx + (size_t)jb * kBlock) * d + c;
         float x[kBlock];
 #pragma unroll
@@ -389,12 +391,12 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
     T* orow = (ws ? Vc : Kc) + ((size_t)unit * nC + ic) * d;
     if (P == nullptr) {
         const int cc = tid & 127;
-        if (cc < d) Elem<T>::store(orow + cc, pooled[ws][cc]);
+        if (cc < d && cc / (d / 4) == quarter) Elem<T>::store(orow + cc, pooled[ws][cc]);
         return;
     }
     const float4 q = lane * 4 < d ? reinterpret_cast<const float4*>(pooled[ws])[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const int per_warp = d / 4;  // output rows of this warp
-    const int j0 = (warp & 3) * per_warp;
+    const int per_warp = d / 16;  // output rows of this warp
+    const int j0 = quarter * (d / 4) + (warp & 3) * per_warp;
     for (int jb8 = 0; jb8 < per_warp; jb8 += 8) {
         float part[8];
 #pragma unroll
@@ -464,7 +466,7 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
         return true;
     }
     count_launch();
-    append_kernel<T><<<m.units(), 256, 0, s>>>(K, V, Pk, Pv, m.T, m.d, m.nG, m.nC, m.lc, m.sc, nj > 0 ? j_begin : -1,
+    append_kernel<T><<<dim3(m.units(), 4), 256, 0, s>>>(K, V, Pk, Pv, m.T, m.d, m.nG, m.nC, m.lc, m.sc, nj > 0 ? j_begin : -1,
                                                ni > 0 ? i_begin : -1, summ, Kc, Vc);
     *e = cudaGetLastError();
     return true;

@@ -113,8 +113,9 @@ cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void
  *   ascending) are written in ascending block order, padded with -1.
  *   prefill = 0: Q [B, Hq, d] at t = T - 1, idx [B, Hkv, topk].
  *   prefill = 1: Q [B, T, Hq, d] at every t, idx [B, T, Hkv, topk].
- *   workspace: >= cobs_workspace_bytes(p, COBS_WS_SELECT) bytes, zero-filled before its
- *              first use; each call leaves it zero-filled again on completion.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_SELECT) bytes of scratch (decode: the
+ *              partial top-k lists of contexts split across CTAs; no initial contents needed).
+ *              Calls that share one workspace must not run concurrently.
  */
 cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summaries,
                         int32_t prefill, int32_t* idx, void* workspace, size_t ws_bytes,
@@ -168,6 +169,20 @@ cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const 
                                      const void* V, const void* Kc, const void* Vc,
                                      const int32_t* idx, const float* gates, void* O,
                                      void* workspace, size_t ws_bytes, cobs_stream_t stream);
+
+/*
+ * Evaluation only (no step of the decode or prefill path calls it): the log of the exact
+ * attention mass of every complete key block for the decode query at T - 1 ([COBS] §2.1,
+ * "attention mass" and the oracle sparse attention OSA that keeps the blocks of largest mass),
+ *   out[b, h, j] = ln sum_{r = 64 j}^{64 j + 63} exp(q_{b,h} . k_{b,h/G,r} / sqrt(d)),
+ * for j < T / 64, in float32 (fused multiply-adds in ascending channel order, then
+ * max + ln(sum exp(s - max)) over the block's 64 keys).
+ *   Q [B, Hq, d] and K [B, Hkv, T, d] in the storage type of p->dtype; out [B, Hq, T / 64]
+ *   float32, caller-owned device memory. Nothing is written when T < 64.
+ *   Errors: the validation of the other calls; COBS_ERR_UNSUPPORTED when Hq / Hkv > 16.
+ */
+cobs_status cobs_block_log_mass(const cobs_params* p, const void* Q, const void* K, float* out,
+                                cobs_stream_t stream);
 
 /* Bytes of workspace a call needs (0 for an invalid p). */
 size_t cobs_workspace_bytes(const cobs_params* p, int32_t which);

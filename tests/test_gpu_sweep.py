@@ -50,3 +50,34 @@ def test_selector_sweep_sampled_units(T):
         for h in range(w.Hkv):
             v = idx[b, h]
             assert np.all(np.diff(v) > 0) and v.min() >= 0 and v.max() < w.nB
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict()),                                   # float32, d = 64, G = 3
+    ("decode32k", dict(B=2, Hkv=2, Hq=8, T=4096 + 50)),  # bf16, d = 128, G = 4, ragged tail
+    ("decode32k", dict(B=1, Hkv=1, Hq=16, T=2048)),      # G = 16
+    ("decode32k", dict(B=1, Hkv=1, Hq=4, T=40)),         # no complete block: nothing written
+])
+def test_block_log_mass_matches_oracle(name, over):
+    """ln of the exact block mass (evaluation call) against the oracle's float64 value."""
+    C = cobs()
+    w = synth.WORKLOADS[name].replace(**over)
+    p = params_of(w)
+    K, _ = synth.kv_cache(w)
+    Q = synth.queries_decode(w)
+    nB = w.T // w.block
+    out = torch.full((w.B, w.Hq, max(1, nB)), 7.0, dtype=torch.float32, device="cuda")
+    C.cobs_block_log_mass(p, dev(Q, w.dtype), dev(K, w.dtype), out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    if nB == 0:
+        assert np.all(got == 7.0)
+        return
+    Qf = synth.to_f64(Q, w.dtype)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            Kf = synth.to_f64(K[b, h], w.dtype)
+            for j in range(w.G):
+                ref = O.exact_log_mass(Qf[b, h * w.G + j], Kf, w.block)
+                # float32 logits (|s| < 40) and exp / log: a few float32 ulps of the logits
+                assert np.abs(got[b, h * w.G + j] - ref).max() <= 1e-4 + 4e-6 * np.abs(ref).max()
