@@ -88,3 +88,48 @@ void cobs_oracle_scores_f32(const float* qsum, const float* q2, const float* sum
         }
     }
 }
+
+/*
+ * Isotropic scalar variant (one second-order scalar per block). COBS §2.2/§2.3 compress the
+ * block covariance Sigma_b; the skill card's "Pitfalls" asks for one or two scalars per block.
+ * Taking Sigma_b ~ sigma2_b I with sigma2_b = tr(Sigma_b) / d (the mean per-channel
+ * variance) gives 1/2 q^T Sigma_b q = 1/2 sigma2_b |q|^2, so per block
+ *   summary   mu_{b,c} (as above) and sigma2_b = (1/d) sum_c var_{b,c}
+ *   score     S_{g,b} = (sum_c Qsum_c mu_{b,c}) * isd + c2 * (Q2tot * sigma2_b),
+ *             Q2tot = sum_c Q2_c  (= sum_{h in g} |q_h|^2).
+ * Canonical order: var_{b,c} as in cobs_oracle_summaries_f32; sigma2_b = (adds over c
+ * ascending from +0) * (1/d) (exact scaling, d a power of two); Q2tot = adds over c
+ * ascending from +0; S = fma(c2, Q2tot * sigma2_b, a * isd) with a as above.
+ */
+
+/* summ: [nb][2][d] (mean, per-channel variance, as written above). out: [nb][d + 1] (mean, sigma2). */
+void cobs_oracle_iso_summaries_f32(const float* summ, int64_t nb, int d, float* out) {
+    const float invd = 1.0f / (float)d; /* exact: d is a power of two */
+    for (int64_t b = 0; b < nb; ++b) {
+        float s = 0.0f;
+        for (int c = 0; c < d; ++c) {
+            out[b * (d + 1) + c] = summ[(b * 2 + 0) * d + c];
+            s = s + summ[(b * 2 + 1) * d + c];
+        }
+        out[b * (d + 1) + d] = s * invd;
+    }
+}
+
+/* qsum, q2: [nq][d]; summ_iso: [nb][d + 1]; S: [nq][nb]. */
+void cobs_oracle_iso_scores_f32(const float* qsum, const float* q2, const float* summ_iso, int64_t nq,
+                                int64_t nb, int d, float isd, float c2, float* S) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nq; ++i) {
+        const float* qs = qsum + i * d;
+        const float* qq = q2 + i * d;
+        float q2tot = 0.0f;
+        for (int c = 0; c < d; ++c) q2tot = q2tot + qq[c];
+        for (int64_t b = 0; b < nb; ++b) {
+            const float* mu = summ_iso + b * (d + 1);
+            float a = 0.0f;
+            for (int c = 0; c < d; ++c) a = fmaf(qs[c], mu[c], a);
+            const float v = q2tot * mu[d];
+            S[i * nb + b] = fmaf(c2, v, a * isd);
+        }
+    }
+}

@@ -65,6 +65,10 @@ def _c():
         lib.cobs_oracle_score_constants.restype = None
         lib.cobs_oracle_scores_f32.argtypes = [vp, vp, vp, i64, i64, i32, f32, f32, vp]
         lib.cobs_oracle_scores_f32.restype = None
+        lib.cobs_oracle_iso_summaries_f32.argtypes = [vp, i64, i32, vp]
+        lib.cobs_oracle_iso_summaries_f32.restype = None
+        lib.cobs_oracle_iso_scores_f32.argtypes = [vp, vp, vp, i64, i64, i32, f32, f32, vp]
+        lib.cobs_oracle_iso_scores_f32.restype = None
         _clib = lib
     return _clib
 
@@ -137,6 +141,38 @@ def canonical_scores(qsum: np.ndarray, q2: np.ndarray, summ: np.ndarray, alpha: 
     return S
 
 
+def canonical_summaries_iso(K32: np.ndarray, L: int) -> np.ndarray:
+    """float32 isotropic block summaries [nB, d + 1]: the block mean, then the mean over channels
+    of the per-channel population variance (one second-order scalar per block).
+
+    [COBS] §2.2/§2.3 (the block covariance kappa_2 = Sigma_b, compressed); [SKILL] "Pitfalls"
+    (one or two scalars per block): Sigma_b taken as sigma2_b I, sigma2_b = tr(Sigma_b) / d.
+    Canonical float32 order: see canonical_fp32.c.
+    """
+    summ = canonical_summaries(K32, L)
+    nB, _, d = summ.shape
+    out = np.zeros((nB, d + 1), np.float32)
+    if nB:
+        _c().cobs_oracle_iso_summaries_f32(summ.ctypes.data, nB, d, out.ctypes.data)
+    return out
+
+
+def canonical_scores_iso(qsum: np.ndarray, q2: np.ndarray, summ_iso: np.ndarray, alpha: float) -> np.ndarray:
+    """float32 group scores S [nq, nB] with isotropic summaries [nB, d + 1]:
+    (sum_c Qsum_c mu_c) isd + c2 (sum_c Q2_c) sigma2_b. Canonical order: see canonical_fp32.c."""
+    d = summ_iso.shape[-1] - 1
+    qsum = _f32c(qsum).reshape(-1, d)
+    q2 = _f32c(q2).reshape(-1, d)
+    summ_iso = _f32c(summ_iso)
+    nq, nb = qsum.shape[0], summ_iso.shape[0]
+    isd, c2 = score_constants(d, alpha)
+    S = np.empty((nq, nb), np.float32)
+    if nq and nb:
+        _c().cobs_oracle_iso_scores_f32(qsum.ctypes.data, q2.ctypes.data, summ_iso.ctypes.data, nq, nb, d,
+                                        float(isd), float(c2), S.ctypes.data)
+    return S
+
+
 # ----------------------------------------------------------------------------------
 # float64 steps
 # ----------------------------------------------------------------------------------
@@ -201,6 +237,21 @@ def group_scores(qs: np.ndarray, mu: np.ndarray, var: np.ndarray, alpha: float) 
     of the heads' log-mass estimates.
     """
     return sum(head_scores(q, mu, var, alpha) for q in qs)
+
+
+def head_scores_iso(q: np.ndarray, mu: np.ndarray, sigma2: np.ndarray, alpha: float) -> np.ndarray:
+    """Isotropic per-head score: q.mu_b/sqrt(d) + alpha * 1/2 * sigma2_b |q|^2 / d.
+
+    The second cumulant 1/2 q^T Sigma_b q / d of [COBS] §2.2 with Sigma_b = sigma2_b I
+    ([SKILL] "Pitfalls": one scalar per block), sigma2_b = mean over channels of var_{b,c}.
+    """
+    d = q.shape[-1]
+    return (mu @ q) / np.sqrt(d) + alpha * 0.5 * sigma2 * float(q @ q) / d
+
+
+def group_scores_iso(qs: np.ndarray, mu: np.ndarray, sigma2: np.ndarray, alpha: float) -> np.ndarray:
+    """Sum of head_scores_iso over the G query heads qs [G, d] (the group-sum reading)."""
+    return sum(head_scores_iso(q, mu, sigma2, alpha) for q in qs)
 
 
 def n_candidates(t: int, L: int) -> int:
@@ -305,9 +356,14 @@ def unit_cache(w, Kst: np.ndarray, Vst: np.ndarray, Pk, Pv):
 
 
 def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
-    """Selected blocks [k] for the decode query at position T-1 of one (batch, group)."""
+    """Selected blocks [k] for the decode query at position T-1 of one (batch, group).
+
+    summ: canonical summaries [nB, 2, d] (per-channel variance) or [nB, d + 1] (isotropic)."""
     qs, q2 = canonical_group_query(q_group32)
-    S = canonical_scores(qs[None], q2[None], summ, w.alpha)[0]
+    if summ.ndim == 2:
+        S = canonical_scores_iso(qs[None], q2[None], summ, w.alpha)[0]
+    else:
+        S = canonical_scores(qs[None], q2[None], summ, w.alpha)[0]
     return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
 
 
@@ -344,12 +400,14 @@ def select_prefill_unit(w, Qst_bh: np.ndarray, summ: np.ndarray, positions=None)
     """Selected blocks [P, k] at every listed position (default all T) of one (batch, group).
 
     Qst_bh: the group's queries [T or P, G, d] in storage form, aligned with ``positions``.
+    summ: canonical summaries [nB, 2, d] (per-channel variance) or [nB, d + 1] (isotropic).
     """
     pos = np.arange(w.T) if positions is None else np.asarray(positions)
     q32 = _to_f64(Qst_bh, w.dtype).astype(np.float32)
     qs, q2 = canonical_group_query(q32)
     nb_max = n_candidates(int(pos.max()), w.block) if len(pos) else 0
-    S = canonical_scores(qs, q2, summ[:nb_max], w.alpha) if nb_max else np.zeros((len(pos), 0), np.float32)
+    scores = canonical_scores_iso if summ.ndim == 2 else canonical_scores
+    S = scores(qs, q2, summ[:nb_max], w.alpha) if nb_max else np.zeros((len(pos), 0), np.float32)
     out = np.empty((len(pos), w.topk), np.int32)
     for i, t in enumerate(pos):
         out[i] = top_k(S[i], n_candidates(int(t), w.block), w.topk)

@@ -425,3 +425,103 @@ def test_gate_order_isolates_each_branch():
         o = O.position_output(q, g, K, V, Kc, Vc, idx, t, L, W, 32, 16)
         np.testing.assert_allclose(o[0], expect[j], rtol=0, atol=1e-12)
     assert not np.allclose(expect[0], expect[1]) and not np.allclose(expect[1], expect[2])
+
+
+# ---------------------------------------------------------------- isotropic scalar variant
+
+def test_iso_summaries_match_library_variance():
+    """sigma2_b = mean over channels of numpy's population variance (ddof=0) of the block."""
+    rng = np.random.default_rng(21)
+    L, d, nB = 64, 64, 6
+    K = synth.bf16_to_f32(synth.f32_to_bf16((rng.standard_normal((nB * L, d)) *
+                                              rng.uniform(0.2, 2.0, (nB * L, 1))).astype(np.float32)))
+    s = O.canonical_summaries_iso(K, L)
+    blocks = K.astype(np.float64).reshape(nB, L, d)
+    assert np.allclose(s[:, :d], blocks.mean(axis=1), rtol=0, atol=1e-6)
+    assert np.allclose(s[:, d], np.var(blocks, axis=1, ddof=0).mean(axis=1), rtol=1e-5, atol=0)
+
+
+def test_iso_score_equals_diagonal_score_for_equal_channel_variances():
+    """When every channel of a block has the same variance, Sigma_b = sigma2 I and the two
+    second-order terms agree: sigma2 |q|^2 = sum_c q_c^2 sigma2 (float64 definitions)."""
+    rng = np.random.default_rng(22)
+    L, d, nB, G = 64, 32, 5, 3
+    centre = rng.standard_normal((nB, 1, d))
+    amp = rng.uniform(0.3, 2.0, size=(nB, 1, 1))
+    signs = np.where(rng.permuted(np.tile((np.arange(L) % 2)[None, :, None], (nB, 1, d)), axis=1) == 0, 1.0, -1.0)
+    K = (centre + amp * signs).reshape(nB * L, d)          # every channel: variance amp^2 exactly
+    mu, var = O.block_summaries(K, L)
+    assert np.allclose(var, np.repeat(amp[:, 0, :] ** 2, d, axis=1))
+    qs = rng.standard_normal((G, d))
+    iso = O.group_scores_iso(qs, mu, var.mean(axis=1), 1.0)
+    diag = O.group_scores(qs, mu, var, 1.0)
+    assert np.allclose(iso, diag, rtol=0, atol=1e-12)
+    # and with unequal channel variances they differ
+    K2 = K * np.linspace(0.5, 1.5, d)
+    mu2, var2 = O.block_summaries(K2, L)
+    assert not np.allclose(O.group_scores_iso(qs, mu2, var2.mean(axis=1), 1.0), O.group_scores(qs, mu2, var2, 1.0))
+
+
+def test_iso_score_exact_for_isotropic_gaussian_keys():
+    """Closed form: keys N(m, s^2 I) give ln E exp(q.k/sqrt(d)) = q.m/sqrt(d) + s^2 |q|^2 / (2 d),
+    which the isotropic score reproduces with the population summaries, and sampled blocks
+    converge to it."""
+    rng = np.random.default_rng(23)
+    d = 16
+    q = rng.standard_normal(d)
+    m = rng.standard_normal(d) * 0.4
+    s = 0.45
+    exact = q @ m / math.sqrt(d) + s * s * (q @ q) / (2 * d)
+    assert abs(O.head_scores_iso(q, m[None], np.array([s * s]), 1.0)[0] - exact) < 1e-12
+    errs = []
+    for logL in (10, 14, 18):
+        L = 1 << logL
+        K = m + s * rng.standard_normal((L, d))
+        errs.append(abs(O.exact_log_mass(q, K, L)[0] - math.log(L) - exact))
+    assert errs[-1] < 0.01 and errs[-1] < errs[0], errs
+
+
+def test_iso_alpha_zero_equals_first_order():
+    """alpha = 0: the isotropic and the per-channel selectors both reduce to mean-pool ranking."""
+    rng = np.random.default_rng(24)
+    L, d, G, nB = 64, 64, 4, 40
+    K = (rng.standard_normal((nB * L, d)) * rng.uniform(0.2, 2.0, size=(nB * L, 1))).astype(np.float32)
+    qs = rng.standard_normal((G, d)).astype(np.float32)
+    a, b = O.canonical_group_query(qs)
+    S_iso = O.canonical_scores_iso(a[None], b[None], O.canonical_summaries_iso(K, L), 0.0)[0]
+    S_diag = O.canonical_scores(a[None], b[None], O.canonical_summaries(K, L), 0.0)[0]
+    assert np.array_equal(S_iso, S_diag)
+    pooled = K.astype(np.float64).reshape(nB, L, d).mean(axis=1)
+    ref = np.sort(np.argsort(-(pooled @ qs.astype(np.float64).sum(axis=0)), kind="stable")[:8])
+    assert list(O.top_k(S_iso, nB, 8)) == list(ref)
+
+
+def test_iso_canonical_matches_exact_rational_emulation():
+    """Brute force: the isotropic canonical steps as exact rationals rounded once to float32."""
+    rng = np.random.default_rng(25)
+    L, d, G, nB = 64, 16, 3, 3
+    K = synth.bf16_to_f32(synth.f32_to_bf16((rng.standard_normal((nB * L, d)) * 1.1).astype(np.float32)))
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    alpha = np.float32(0.77)
+    summ = O.canonical_summaries(K, L)
+    iso = O.canonical_summaries_iso(K, L)
+    qsum, q2 = O.canonical_group_query(q)
+    S = O.canonical_scores_iso(qsum[None], q2[None], iso, float(alpha))[0]
+    F = lambda v: Fraction(float(v))
+    for b in range(nB):
+        acc = Fraction(0)
+        for c in range(d):
+            assert F(iso[b, c]) == F(summ[b, 0, c])
+            acc = _rn32(acc + F(summ[b, 1, c]))
+        assert F(iso[b, d]) == _rn32(acc / d)
+    q2tot = Fraction(0)
+    for c in range(d):
+        q2tot = _rn32(q2tot + F(q2[c]))
+    isd = _rn32(Fraction(1.0 / math.sqrt(d)))
+    c2 = _rn32(F(alpha) / (2 * d))
+    for b in range(nB):
+        a = Fraction(0)
+        for c in range(d):
+            a = _rn32(F(qsum[c]) * F(iso[b, c]) + a)
+        v = _rn32(q2tot * F(iso[b, d]))
+        assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
