@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k", "sweep"])
     ap.add_argument("--contexts", default=None, help="sweep: comma-separated context lengths (default 8k .. 1M)")
+    ap.add_argument("--variance", choices=["channel", "isotropic"], default="channel",
+                    help="second-order statistic of the summaries (per-channel variance or one scalar per block)")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
     ap.add_argument("--T", type=int, default=None, help="override the context length (small profiling cases)")
@@ -158,7 +160,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic bytes
 
-def decode_bytes(w, idx):
+def decode_bytes(w, idx, variance="channel"):
     """Algorithmic HBM bytes of one decode step, from the selected blocks (idx [B, Hkv, k])."""
     import numpy as np
     d, esz = w.d, 2 if w.dtype == "bf16" else 4
@@ -177,21 +179,22 @@ def decode_bytes(w, idx):
     units = w.B * w.Hkv
     attn = kv_tokens * 2 * d * esz + units * ncv * 2 * d * esz          # K/V union + compressed K/V
     attn += w.B * w.Hq * d * esz * 2 + w.B * w.Hq * 3 * 4 + units * w.topk * 4   # Q, O, gates, idx
-    select = units * w.nB * 2 * d * 4 + w.B * w.Hq * d * esz + units * w.topk * 4
+    per_block = (d + 1) * 4 if variance == "isotropic" else 2 * d * 4
+    select = units * w.nB * per_block + w.B * w.Hq * d * esz + units * w.topk * 4
     # summary update for the appended token: the completed block (64 K rows) and the last
     # compressed token (cmp_block K and V rows), plus their outputs
-    update = units * (w.block * d * esz + 2 * d * 4 + 2 * w.cmp_block * d * esz + 2 * d * esz)
+    update = units * (w.block * d * esz + per_block + 2 * w.cmp_block * d * esz + 2 * d * esz)
     return {"attn": attn, "select": select, "update": update, "total": attn + select + update,
             "kv_tokens_per_unit": kv_tokens / units}
 
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False):
+def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False, variance="channel"):
     """Time the oracle (as it stands) on the listed units; returns (seconds, query heads[, result])."""
     from oracle import cobs_oracle as O
     t0 = time.perf_counter()
-    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units)
+    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units, variance=variance)
     secs = time.perf_counter() - t0
     return (secs, len(units) * w.G, res) if with_result else (secs, len(units) * w.G)
 
@@ -365,7 +368,8 @@ def run_ours(args):
     if w.mode == "prefill":
         return run_prefill_line(args, w, dev, cobs, rank, world)
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
-                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
+                    variance=args.variance)
     K, V = synth.kv_cache(w)
     Q, g = synth.queries_decode(w), synth.gates_decode(w)
     Pk, Pv = synth.projections(w)
@@ -483,7 +487,7 @@ def run_ours(args):
     dev_err = cobs.device_error()
 
     qheads = w.B * w.Hq * world
-    by = decode_bytes(w, idx0)
+    by = decode_bytes(w, idx0, args.variance)
     peak, peak_kind = read_peaks()
     att_gbs = by["attn"] / (t_att * 1e-3) / 1e9
     result = {
@@ -492,6 +496,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
                    "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
+                   "variance": args.variance,
                    "step": "summary update at T-1 + select + decode attention, one CUDA graph",
                    "l2": f"{R} KV-cache copies rotated between steps (working set {R} x step bytes > L2)",
                    "parallelism": f"dp{world} (independent decode batches per GPU)"},
@@ -515,7 +520,8 @@ def run_ours(args):
         os.environ.setdefault("OMP_NUM_THREADS", "1")
         lim = limit_threads()
         units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:24]
-        secs, heads, ref = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=True)
+        secs, heads, ref = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=True,
+                                                variance=args.variance)
         result["cpu_baseline"] = {"value": heads / secs, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                                   "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
                                             f"full oracle decode incl. summaries ({secs:.1f} s)"}
@@ -591,7 +597,8 @@ def run_sweep(args):
 
     def params(w, **over):
         kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
-                  cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+                  cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
+                  variance=args.variance)
         kw.update(over)
         return cobs.Params(**kw)
 
@@ -658,7 +665,8 @@ def run_sweep(args):
                 ref = set(osa.tolist())
                 rec1.append(len(ref & set(int(x) for x in idx_a1[b, g] if x >= 0)) / w.topk)
                 rec0.append(len(ref & set(int(x) for x in idx_a0[b, g] if x >= 0)) / w.topk)
-        by = w.B * w.Hkv * nB * 2 * w.d * 4 + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * w.topk * 4
+        per_block = (w.d + 1) * 4 if args.variance == "isotropic" else 2 * w.d * 4
+        by = w.B * w.Hkv * nB * per_block + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * w.topk * 4
         gbs = by / (us * 1e-6) / 1e9
         rows.append({"T": T, "nB": nB, "bytes": by, "us": us, "gbs": gbs, "frac": gbs / peak,
                      "recall_alpha1": float(np.mean(rec1)), "recall_alpha0": float(np.mean(rec0)),
@@ -671,7 +679,7 @@ def run_sweep(args):
             "ms_per_step": top["us"] * 1e-3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic (keys drawn on the device)",
             "config": {"workload": "sweep", "B": base.B, "Hq": base.Hq, "Hkv": base.Hkv, "d": base.d,
-                       "topk": base.topk, "contexts": contexts, "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
+                       "topk": base.topk, "contexts": contexts, "variance": args.variance, "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
             "roofline": {"bound": "hbm", "kernel": "select_decode_kernel", "achieved": top["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": top["frac"], "peak_kind": peak_kind,
                          "traffic": recorded_traffic("select_decode")},

@@ -73,6 +73,8 @@ cobs_status validate(const cobs_params* p) {
         return fail(COBS_ERR_INVALID_ARG, "need 1 <= cmp_stride <= cmp_block (got %d, %d)", p->cmp_stride,
                     p->cmp_block);
     if (p->dtype != COBS_F32 && p->dtype != COBS_BF16) return fail(COBS_ERR_INVALID_ARG, "dtype %d", p->dtype);
+    if (p->variance != COBS_VAR_CHANNEL && p->variance != COBS_VAR_ISOTROPIC)
+        return fail(COBS_ERR_INVALID_ARG, "variance %d (COBS_VAR_CHANNEL or COBS_VAR_ISOTROPIC)", p->variance);
     if (!isfinite(p->alpha)) return fail(COBS_ERR_INVALID_ARG, "alpha is not finite");
     if ((long long)p->B * p->Hkv > 65535) return fail(COBS_ERR_UNSUPPORTED, "B * Hkv > 65535");
     return COBS_OK;

@@ -16,8 +16,12 @@ struct Dims {
     int nC;       // compressed tokens, (T - lc) / sc + 1 (0 if T < lc)
     float alpha;
     int dtype;    // cobs_dtype
+    int iso;      // summaries keep one variance scalar per block (COBS_VAR_ISOTROPIC)
     int units() const { return B * Hkv; }
-    size_t summ_unit_floats() const { return (size_t)nG * 2 * d * 32; }
+    // floats of one 32-block summary group: means and per-channel variances, or means and
+    // one scalar per block
+    size_t group_floats() const { return iso ? (size_t)(d + 1) * 32 : (size_t)2 * d * 32; }
+    size_t summ_unit_floats() const { return (size_t)nG * group_floats(); }
 };
 
 inline Dims make_dims(const cobs_params& p) {
@@ -27,7 +31,7 @@ inline Dims make_dims(const cobs_params& p) {
     m.nB = p.block > 0 ? p.T / p.block : 0;
     m.nG = m.nB > 0 ? (m.nB + 31) / 32 : 1;
     m.nC = (p.cmp_stride > 0 && p.T >= p.cmp_block) ? (p.T - p.cmp_block) / p.cmp_stride + 1 : 0;
-    m.alpha = p.alpha; m.dtype = p.dtype;
+    m.alpha = p.alpha; m.dtype = p.dtype; m.iso = p.variance == COBS_VAR_ISOTROPIC;
     return m;
 }
 

@@ -102,6 +102,72 @@ __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return _
 // Largest GQA group (query heads per KV head) the selectors handle; the host rejects larger.
 constexpr int kMaxGroup = 16;
 
+// NC consecutive elements (16-, 8- or 4-byte aligned vector loads) as float.
+template <typename T, int NC>
+__device__ __forceinline__ void load_chunk(const T* p, float (&x)[NC]) {
+    if constexpr (sizeof(T) == 2) {
+        static_assert(NC == 2 || NC == 4 || NC == 8, "chunk");
+        uint32_t w[NC / 2];
+        if constexpr (NC == 8) {
+            const uint4 u = *reinterpret_cast<const uint4*>(p);
+            w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+        } else if constexpr (NC == 4) {
+            const uint2 u = *reinterpret_cast<const uint2*>(p);
+            w[0] = u.x; w[1] = u.y;
+        } else {
+            w[0] = *reinterpret_cast<const uint32_t*>(p);
+        }
+#pragma unroll
+        for (int i = 0; i < NC / 2; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+        static_assert(NC % 2 == 0, "chunk");
+#pragma unroll
+        for (int i = 0; i < NC; i += (NC % 4 == 0 ? 4 : 2)) {
+            if constexpr (NC % 4 == 0) {
+                const float4 v = *reinterpret_cast<const float4*>(p + i);
+                x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(p + i);
+                x[i] = v.x; x[i + 1] = v.y;
+            }
+        }
+    }
+}
+
+// Canonical group query of channels [c0, c0 + NC) of a group whose G head rows start at q
+// (row stride D): every head's chunk is loaded at once, then Qsum_c = sum_h q_{h,c} (adds)
+// and Q2_c = fma-sum of q_{h,c}^2 in ascending h.
+template <typename T, int NC>
+__device__ __forceinline__ void group_query_chunk(const T* q, int G, int D, int c0, bool valid, float* qs,
+                                                  float* q2) {
+    float x[kMaxGroup][NC];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        if (h < G && valid) {
+            load_chunk<T, NC>(q + (size_t)h * D + c0, x[h]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < NC; ++j) x[h][j] = 0.0f;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+        float s = 0.0f, s2 = 0.0f;
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            if (h < G) {
+                s = __fadd_rn(s, x[h][j]);
+                s2 = __fmaf_rn(x[h][j], x[h][j], s2);
+            }
+        }
+        qs[j] = s;
+        q2[j] = s2;
+    }
+}
+
 // Canonical group query: Qsum_c = sum_h q_{h,c} (adds) and Q2_c = fma-sum of q_{h,c}^2, in
 // ascending h, from values already in registers (x[h] = q_{h,c}, ascending h). Callers
 // issue all G loads of a channel at once (independent loads) before reducing in order.
@@ -143,6 +209,37 @@ __device__ __forceinline__ float block_score(const float* tile, const float* qs,
     }
     return __fmaf_rn(c2, v, __fmul_rn(a, isd));
 }
+
+// Canonical isotropic score: the same mean chain, then v = RN(Q2tot * sigma2_b) with the block's
+// one variance scalar (stored after the group's means) and Q2tot = sum_c Q2_c.
+template <int D>
+__device__ __forceinline__ float block_score_iso(const float* tile, const float* qs, float q2tot, int lane, float isd,
+                                                 float c2) {
+    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
+    float a = 0.0f;
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 m = mu4[c4 * 32];
+        a = __fmaf_rn(qs[4 * c4 + 0], m.x, a);
+        a = __fmaf_rn(qs[4 * c4 + 1], m.y, a);
+        a = __fmaf_rn(qs[4 * c4 + 2], m.z, a);
+        a = __fmaf_rn(qs[4 * c4 + 3], m.w, a);
+    }
+    const float v = __fmul_rn(q2tot, tile[D * 32 + lane]);
+    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
+}
+
+// Q2tot = sum_c Q2_c by adds in ascending channel order from +0 (one thread).
+template <int D>
+__device__ __forceinline__ float q2_total(const float* q2) {
+    float t = 0.0f;
+    for (int c = 0; c < D; ++c) t = __fadd_rn(t, q2[c]);
+    return t;
+}
+
+// Floats of one 32-block summary group: means + per-channel variances, or means + 32 scalars.
+template <int D, bool ISO>
+constexpr int group_floats() { return ISO ? (D + 1) * 32 : 2 * D * 32; }
 
 // ---------------------------------------------------------------------------- decode
 // Warp-wide sorted list helpers: one (score, index) entry per lane, best first.
@@ -237,7 +334,7 @@ struct RunList {
 // if it held the whole unit, else deposits its segment's exact top-k; select_merge_kernel (a
 // dependent launch) merges the deposits. The result is the top-k under a strict total order,
 // so it does not depend on the split.
-template <typename T, int D>
+template <typename T, int D, bool ISO>
 __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
                                                            int32_t* __restrict__ idx, float* __restrict__ ws_s,
                                                            int* __restrict__ ws_i, int units, int G, int nG,
@@ -246,8 +343,9 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bar[kSelStages];
     __shared__ __align__(16) float qsm[2][D];
-    constexpr uint32_t kTileBytes = 2 * D * 32 * 4;
-    constexpr int kTileFloats = 2 * D * 32;
+    __shared__ float q2t_sm;
+    constexpr int kTileFloats = group_floats<D, ISO>();
+    constexpr uint32_t kTileBytes = kTileFloats * 4;
     // the merge grid may be scheduled now; it still waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int lane = threadIdx.x;
@@ -310,17 +408,14 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
             // group query of unit u (heads u*G .. u*G+G-1 of Q [B, Hq, d]): Qsum and Q2 of
             // channels lane + 32 j, every head's value loaded at once
             __syncwarp();
-            {
-                const T* qg = Q + (size_t)u * G * D;
-                float x[D / 32][kMaxGroup];
-#pragma unroll
-                for (int j = 0; j < D / 32; ++j)
-#pragma unroll
-                    for (int h = 0; h < kMaxGroup; ++h) x[j][h] = h < G ? to_f(qg[(size_t)h * D + lane + 32 * j]) : 0.0f;
-#pragma unroll
-                for (int j = 0; j < D / 32; ++j) group_reduce(x[j], G, qsm[0][lane + 32 * j], qsm[1][lane + 32 * j]);
-            }
+            // lane l: channels [l D/32, (l + 1) D/32), one vector load per head
+            group_query_chunk<T, D / 32>(Q + (size_t)u * G * D, G, D, lane * (D / 32), true, &qsm[0][lane * (D / 32)],
+                                         &qsm[1][lane * (D / 32)]);
             __syncwarp();
+            if (ISO) {
+                if (lane == 0) q2t_sm = q2_total<D>(qsm[1]);
+                __syncwarp();
+            }
         }
         if (ok) ok = mbar_wait(&bar[st], parity, err);
         ok = __all_sync(kFull, ok);
@@ -328,7 +423,8 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
         float sc = -INFINITY;
         int bi = kInvalid;
         if (ok) {
-            const float s_all = block_score<D>(tiles + st * kTileFloats, qsm[0], qsm[1], lane, isd, c2);
+            const float s_all = ISO ? block_score_iso<D>(tiles + st * kTileFloats, qsm[0], q2t_sm, lane, isd, c2)
+                                    : block_score<D>(tiles + st * kTileFloats, qsm[0], qsm[1], lane, isd, c2);
             if (b < ncand) {
                 sc = s_all;
                 bi = b;
@@ -396,15 +492,17 @@ constexpr int kPfPos = 32;
 constexpr int kPfWarps = 4;
 constexpr int kPfPerWarp = kPfPos / kPfWarps;
 
-template <typename T, int D>
+template <typename T, int D, bool ISO>
 __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
                                                              int32_t* __restrict__ idx, int Tctx, int Hq, int Hkv,
                                                              int G, int nG, int L, int k, float isd, float c2,
                                                              int* err) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    float* tiles = reinterpret_cast<float*>(smem_raw);           // [2][2*D*32]
-    float* sq = tiles + 2 * 2 * D * 32;                            // [kPfPos][2][D]: Qsum, Q2
+    constexpr int kTileFloats = group_floats<D, ISO>();
+    float* tiles = reinterpret_cast<float*>(smem_raw);           // [2][kTileFloats]
+    float* sq = tiles + 2 * kTileFloats;                           // [kPfPos][2][D]: Qsum, Q2
     __shared__ __align__(8) uint64_t bar[2];
+    __shared__ float q2t[kPfPos];                                  // Q2tot per position (isotropic)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.y;
     const int b = unit / Hkv, g = unit % Hkv;
@@ -412,8 +510,8 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     const int tlast = min(Tctx - 1, t0 + kPfPos - 1);
     const int ncand_max = (tlast + 1) / L;
     const int ngroups = (ncand_max + kGroupBlocks - 1) / kGroupBlocks;
-    const float* usum = summ + (size_t)unit * nG * 2 * D * 32;
-    constexpr uint32_t kTileBytes = 2 * D * 32 * 4;
+    const float* usum = summ + (size_t)unit * nG * kTileFloats;
+    constexpr uint32_t kTileBytes = kTileFloats * 4;
 
     if (tid == 0) {
         mbar_init(&bar[0], 1);
@@ -424,32 +522,22 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     if (tid == 0) {
         for (int st = 0; st < 2 && st < ngroups; ++st) {
             mbar_arrive_expect_tx(&bar[st], kTileBytes);
-            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)st * 2 * D * 32, kTileBytes, &bar[st]);
+            bulk_g2s(tiles + st * kTileFloats, usum + (size_t)st * kTileFloats, kTileBytes, &bar[st]);
         }
     }
-    // group queries of the tile's positions: thread -> channel c of positions p0, p0 + ppi, ...,
-    // four positions (G head loads each) in flight at a time
-    {
-        constexpr int kPpi = 128 / D;  // positions covered by one pass of the 128 threads
-        const int c = tid % D, p0 = tid / D;
-        for (int pb = p0; pb < kPfPos; pb += 4 * kPpi) {
-            float x[4][kMaxGroup];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int p = pb + j * kPpi, t = t0 + p;
-                const T* qr = Q + (((size_t)b * Tctx + (t < Tctx ? t : 0)) * Hq + (size_t)g * G) * D + c;
-#pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h)
-                    x[j][h] = (h < G && p < kPfPos && t < Tctx) ? to_f(qr[(size_t)h * D]) : 0.0f;
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int p = pb + j * kPpi;
-                if (p < kPfPos) group_reduce(x[j], G, sq[(p * 2 + 0) * D + c], sq[(p * 2 + 1) * D + c]);
-            }
-        }
+    // group queries of the tile's positions: thread -> (position, 8-channel chunk), every head's
+    // chunk loaded at once (16-byte loads for bf16)
+    for (int e = tid; e < kPfPos * (D / 8); e += blockDim.x) {
+        const int p = e / (D / 8), c0 = (e % (D / 8)) * 8;
+        const int t = t0 + p;
+        const T* qr = Q + (((size_t)b * Tctx + (t < Tctx ? t : 0)) * Hq + (size_t)g * G) * D;
+        group_query_chunk<T, 8>(qr, G, D, c0, t < Tctx, &sq[(p * 2 + 0) * D + c0], &sq[(p * 2 + 1) * D + c0]);
     }
     __syncthreads();
+    if (ISO) {
+        if (tid < kPfPos) q2t[tid] = q2_total<D>(sq + (tid * 2 + 1) * D);
+        __syncthreads();
+    }
 
     TopK tk[kPfPerWarp];
 #pragma unroll
@@ -460,7 +548,7 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
         const uint32_t parity = (gi >> 1) & 1;
         if (ok) ok = mbar_wait(&bar[st], parity, err);
         ok = __syncthreads_and(ok) != 0;
-        const float* tile = tiles + st * 2 * D * 32;
+        const float* tile = tiles + st * kTileFloats;
         const int blk = gi * kGroupBlocks + lane;
         // scores of this lane's block against the warp's 8 positions: 16 independent chains,
         // each in the canonical order (ascending channels, one fma per term)
@@ -470,29 +558,47 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
         const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
         const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
         const float* sqw = sq + (size_t)(warp * kPfPerWarp) * 2 * D;
+        if (ISO) {
 #pragma unroll 4
-        for (int c4 = 0; c4 < D / 4; ++c4) {
-            const float4 m = mu4[c4 * 32];
-            const float4 vr = var4[c4 * 32];
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 m = mu4[c4 * 32];
 #pragma unroll
-            for (int j = 0; j < kPfPerWarp; ++j) {
-                const float4 qa = reinterpret_cast<const float4*>(sqw + (j * 2 + 0) * D)[c4];
-                const float4 qb = reinterpret_cast<const float4*>(sqw + (j * 2 + 1) * D)[c4];
-                av[j] = __fmaf_rn(qa.x, m.x, av[j]);
-                av[j] = __fmaf_rn(qa.y, m.y, av[j]);
-                av[j] = __fmaf_rn(qa.z, m.z, av[j]);
-                av[j] = __fmaf_rn(qa.w, m.w, av[j]);
-                vv[j] = __fmaf_rn(qb.x, vr.x, vv[j]);
-                vv[j] = __fmaf_rn(qb.y, vr.y, vv[j]);
-                vv[j] = __fmaf_rn(qb.z, vr.z, vv[j]);
-                vv[j] = __fmaf_rn(qb.w, vr.w, vv[j]);
+                for (int j = 0; j < kPfPerWarp; ++j) {
+                    const float4 qa = reinterpret_cast<const float4*>(sqw + (j * 2 + 0) * D)[c4];
+                    av[j] = __fmaf_rn(qa.x, m.x, av[j]);
+                    av[j] = __fmaf_rn(qa.y, m.y, av[j]);
+                    av[j] = __fmaf_rn(qa.z, m.z, av[j]);
+                    av[j] = __fmaf_rn(qa.w, m.w, av[j]);
+                }
+            }
+            const float sig = tile[D * 32 + lane];
+#pragma unroll
+            for (int j = 0; j < kPfPerWarp; ++j) vv[j] = __fmul_rn(q2t[warp * kPfPerWarp + j], sig);
+        } else {
+#pragma unroll 4
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 m = mu4[c4 * 32];
+                const float4 vr = var4[c4 * 32];
+#pragma unroll
+                for (int j = 0; j < kPfPerWarp; ++j) {
+                    const float4 qa = reinterpret_cast<const float4*>(sqw + (j * 2 + 0) * D)[c4];
+                    const float4 qb = reinterpret_cast<const float4*>(sqw + (j * 2 + 1) * D)[c4];
+                    av[j] = __fmaf_rn(qa.x, m.x, av[j]);
+                    av[j] = __fmaf_rn(qa.y, m.y, av[j]);
+                    av[j] = __fmaf_rn(qa.z, m.z, av[j]);
+                    av[j] = __fmaf_rn(qa.w, m.w, av[j]);
+                    vv[j] = __fmaf_rn(qb.x, vr.x, vv[j]);
+                    vv[j] = __fmaf_rn(qb.y, vr.y, vv[j]);
+                    vv[j] = __fmaf_rn(qb.z, vr.z, vv[j]);
+                    vv[j] = __fmaf_rn(qb.w, vr.w, vv[j]);
+                }
             }
         }
         __syncthreads();  // every warp is done with this stage
         if (tid == 0 && ok && gi + 2 < ngroups) {
             fence_proxy_async();
             mbar_arrive_expect_tx(&bar[st], kTileBytes);
-            bulk_g2s(tiles + st * 2 * D * 32, usum + (size_t)(gi + 2) * 2 * D * 32, kTileBytes, &bar[st]);
+            bulk_g2s(tiles + st * kTileFloats, usum + (size_t)(gi + 2) * kTileFloats, kTileBytes, &bar[st]);
         }
 #pragma unroll
         for (int j = 0; j < kPfPerWarp; ++j) {
@@ -528,12 +634,12 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool ISO>
 cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                             cudaStream_t s, int* err) {
     float isd, c2;
     score_constants(m.d, m.alpha, &isd, &c2);
-    const size_t tile_bytes = (size_t)2 * D * 32 * 4;
+    const size_t tile_bytes = (size_t)group_floats<D, ISO>() * 4;
     if (!prefill) {
         const int ncand = m.T / m.L;
         const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
@@ -549,11 +655,11 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         float* ws_s = static_cast<float*>(ws);
         int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
         const size_t smem = (size_t)kSelStages * tile_bytes;
-        cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, ISO>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         count_launch();
-        select_decode_kernel<T, D><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(), m.G, m.nG,
+        select_decode_kernel<T, D, ISO><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(), m.G, m.nG,
                                                                     ncand, m.k, maxseg, isd, c2, err);
         e = cudaGetLastError();
         // a unit is cut into several ranges only if it has several groups and the grid several CTAs
@@ -573,7 +679,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
                                   (int)grid, m.k, maxseg);
     }
     const size_t smem = tile_bytes * 2 + (size_t)kPfPos * 2 * D * 4;
-    auto kern = select_prefill_kernel<T, D>;
+    auto kern = select_prefill_kernel<T, D, ISO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
@@ -591,15 +697,23 @@ size_t select_workspace_bytes(const Dims& m, int prefill) {
     return (size_t)m.units() * maxseg * m.k * (sizeof(float) + sizeof(int));
 }
 
-cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
-                          cudaStream_t s, int* err) {
+template <bool ISO>
+cudaError_t launch_select_v(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
+                            cudaStream_t s, int* err) {
     if (m.dtype == COBS_BF16) {
         if (m.d == 128)
-            return launch_select_t<__nv_bfloat16, 128>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s, err);
-        return launch_select_t<__nv_bfloat16, 64>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s, err);
+            return launch_select_t<__nv_bfloat16, 128, ISO>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s,
+                                                            err);
+        return launch_select_t<__nv_bfloat16, 64, ISO>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s, err);
     }
-    if (m.d == 128) return launch_select_t<float, 128>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
-    return launch_select_t<float, 64>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
+    if (m.d == 128) return launch_select_t<float, 128, ISO>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
+    return launch_select_t<float, 64, ISO>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
+}
+
+cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
+                          cudaStream_t s, int* err) {
+    return m.iso ? launch_select_v<true>(m, Q, summ, prefill, idx, ws, s, err)
+                 : launch_select_v<false>(m, Q, summ, prefill, idx, ws, s, err);
 }
 
 }  // namespace cobs

@@ -20,10 +20,32 @@ namespace {
 
 constexpr int kBlock = 64;  // selection block size (validated by the API)
 
+// Offsets inside a unit's summaries of block j, channel c: the mean, the per-channel variance
+// (channel layout), the block's variance scalar (isotropic layout).
+__host__ __device__ __forceinline__ size_t summ_mu_at(int j, int c, int d, int iso) {
+    const size_t gf = iso ? (size_t)(d + 1) * 32 : (size_t)2 * d * 32;
+    return (size_t)(j >> 5) * gf + ((size_t)(c / 4) * 32 + (j & 31)) * 4 + (c & 3);
+}
+__host__ __device__ __forceinline__ size_t summ_var_at(int j, int c, int d) {
+    return summ_mu_at(j, c, d, 0) + (size_t)d * 32;
+}
+__host__ __device__ __forceinline__ size_t summ_iso_at(int j, int d) {
+    return (size_t)(j >> 5) * (size_t)(d + 1) * 32 + (size_t)d * 32 + (j & 31);
+}
+
+// The isotropic scalar of a block from its per-channel variances v[0..d): adds in ascending
+// channel order from +0, then the exact scaling by 1/d (d a power of two).
+__device__ __forceinline__ float iso_scalar(const float* v, int d) {
+    float s = 0.0f;
+    for (int c = 0; c < d; ++c) s = __fadd_rn(s, v[c]);
+    return __fmul_rn(s, 1.0f / (float)d);
+}
+
 // grid (blocks to build, units), block d threads (one per channel).
 template <typename T>
 __global__ void __launch_bounds__(128) summaries_kernel(const T* __restrict__ K, int Tctx, int d, int nG,
-                                                        int j_begin, float* __restrict__ summ) {
+                                                        int j_begin, int iso, float* __restrict__ summ) {
+    __shared__ float vsm[128];
     const int c = threadIdx.x;
     const int unit = blockIdx.y;
     const int j = j_begin + blockIdx.x;
@@ -42,12 +64,16 @@ __global__ void __launch_bounds__(128) summaries_kernel(const T* __restrict__ K,
         a = __fmaf_rn(t, t, a);
     }
     const float var = __fmul_rn(a, 1.0f / kBlock);
-    float* base = summ + (size_t)unit * nG * 2 * d * 32;
-    const int g = j >> 5, lane = j & 31;
-    const size_t o_mu = ((size_t)(g * 2 + 0) * (d / 4) + c / 4) * 128 + lane * 4 + (c & 3);
-    const size_t o_var = ((size_t)(g * 2 + 1) * (d / 4) + c / 4) * 128 + lane * 4 + (c & 3);
-    base[o_mu] = mu;
-    base[o_var] = var;
+    const size_t gf = iso ? (size_t)(d + 1) * 32 : (size_t)2 * d * 32;
+    float* base = summ + (size_t)unit * nG * gf;
+    base[summ_mu_at(j, c, d, iso)] = mu;
+    if (!iso) {
+        base[summ_var_at(j, c, d)] = var;
+        return;
+    }
+    vsm[c] = var;
+    __syncthreads();
+    if (c == 0) base[summ_iso_at(j, d)] = iso_scalar(vsm, d);
 }
 
 // grid (tokens to build, units, 2 = {K, V}), block d threads. out_i = P @ mean(rows).
@@ -120,9 +146,10 @@ template <int D>
 __global__ void __launch_bounds__(kFThreads, 1) summary_fused_kernel(
     const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, const float* __restrict__ Pk,
     const float* __restrict__ Pv, int Tctx, int nB, int nG, int nC, int j_begin, int i_begin, int m_begin,
-    int m_count, int units, float* __restrict__ summ, __nv_bfloat16* __restrict__ Kc,
+    int m_count, int units, int iso, float* __restrict__ summ, __nv_bfloat16* __restrict__ Kc,
     __nv_bfloat16* __restrict__ Vc, int* err) {
     using S = FusedSmem<D>;
+    __shared__ float vsm[2][D];  // per-channel variances of the item's two blocks (isotropic layout)
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* ring = smem_raw;                                             // 2 stages
     float* cs = reinterpret_cast<float*>(ring + 2 * S::kStage);                 // [2][9][D] chunk sums
@@ -226,10 +253,12 @@ __global__ void __launch_bounds__(kFThreads, 1) summary_fused_kernel(
                     a2 = __fmaf_rn(tt, tt, a2);
                 }
                 if (j < nB && j >= j_begin) {
-                    float* base = summ + (size_t)unit * nG * 2 * D * 32;
-                    const int g = j >> 5, ln = j & 31;
-                    base[((size_t)(g * 2 + 0) * (D / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = mu;
-                    base[((size_t)(g * 2 + 1) * (D / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = __fmul_rn(a2, 1.0f / 64.0f);
+                    float* base = summ + (size_t)unit * nG * (iso ? (D + 1) * 32 : 2 * D * 32);
+                    base[summ_mu_at(j, c, D, iso)] = mu;
+                    if (iso)
+                        vsm[blk][c] = __fmul_rn(a2, 1.0f / 64.0f);
+                    else
+                        base[summ_var_at(j, c, D)] = __fmul_rn(a2, 1.0f / 64.0f);
                 }
             } else {
                 for (int q = 0; q < 4; ++q) {
@@ -255,6 +284,12 @@ __global__ void __launch_bounds__(kFThreads, 1) summary_fused_kernel(
             }
         }
         __syncthreads();
+        // ---- isotropic scalars of the item's two blocks (one thread each, channels ascending)
+        if (iso && ok && tid < 2) {
+            const int j = 2 * m + tid;
+            if ((tid * 64 + 64) <= nrows && j < nB && j >= j_begin)
+                summ[(size_t)unit * nG * (D + 1) * 32 + summ_iso_at(j, D)] = iso_scalar(vsm[tid], D);
+        }
         // ---- pooled tokens, split into bf16 hi + lo
         for (int e = tid; e < 2 * 8 * D; e += kFThreads) {
             const int sd = e / (8 * D), rem = e % (8 * D), p = rem / D, c = rem % D;
@@ -333,7 +368,7 @@ cudaError_t launch_fused(const Dims& m, const __nv_bfloat16* K, const __nv_bfloa
     const int grid = (int)std::min<long long>(items, sm_count());
     count_launch();
     summary_fused_kernel<D><<<grid, kFThreads, smem, s>>>(K, V, Pk, Pv, m.T, m.nB, m.nG, m.nC, j_begin, i_begin,
-                                                          m_begin, m_count, m.units(), summ, Kc, Vc, err);
+                                                          m_begin, m_count, m.units(), m.iso, summ, Kc, Vc, err);
     return cudaGetLastError();
 }
 
@@ -348,14 +383,17 @@ template <typename T>
 __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, const T* __restrict__ V,
                                                      const float* __restrict__ Pk, const float* __restrict__ Pv,
                                                      int Tctx, int d, int nG, int nC, int lc, int sc, int jb, int ic,
-                                                     float* __restrict__ summ, T* __restrict__ Kc,
+                                                     int iso, float* __restrict__ summ, T* __restrict__ Kc,
                                                      T* __restrict__ Vc) {
     __shared__ __align__(16) float pooled[2][128];
+    __shared__ float vsm[128];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.x, quarter = blockIdx.y;
-    // block summary (channels 32 quarter + tid): the canonical row-order sums
-    if (jb >= 0 && tid < 32 && quarter * 32 + tid < d) {
-        const int c = quarter * 32 + tid;
+    // block summary (channels 32 quarter + tid; the isotropic layout needs every channel in
+    // one CTA: quarter 0, thread = channel): the canonical row-order sums
+    const bool sum_here = jb >= 0 && (iso ? (quarter == 0 && tid < d) : (tid < 32 && quarter * 32 + tid < d));
+    if (sum_here) {
+        const int c = iso ? tid : quarter * 32 + tid;
         const T* rows = K + ((size_t)unit * Tctx + (size_t)jb * kBlock) * d + c;
         float x[kBlock];
 #pragma unroll
@@ -370,10 +408,17 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
             const float t = __fsub_rn(x[r], mu);
             a2 = __fmaf_rn(t, t, a2);
         }
-        float* base = summ + (size_t)unit * nG * 2 * d * 32;
-        const int g = jb >> 5, ln = jb & 31;
-        base[((size_t)(g * 2 + 0) * (d / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = mu;
-        base[((size_t)(g * 2 + 1) * (d / 4) + c / 4) * 128 + ln * 4 + (c & 3)] = __fmul_rn(a2, 1.0f / kBlock);
+        float* base = summ + (size_t)unit * nG * (iso ? (size_t)(d + 1) * 32 : (size_t)2 * d * 32);
+        base[summ_mu_at(jb, c, d, iso)] = mu;
+        if (iso)
+            vsm[c] = __fmul_rn(a2, 1.0f / kBlock);
+        else
+            base[summ_var_at(jb, c, d)] = __fmul_rn(a2, 1.0f / kBlock);
+    }
+    if (iso) {
+        __syncthreads();
+        if (jb >= 0 && quarter == 0 && tid == 0)
+            summ[(size_t)unit * nG * (d + 1) * 32 + summ_iso_at(jb, d)] = iso_scalar(vsm, d);
     }
     if (ic < 0) return;
     // pooled compressed token: threads [0, d) for K, [128, 128 + d) for V
@@ -429,7 +474,7 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
     const int nbuild = m.nB - (j_begin < 0 ? 0 : j_begin);
     if (nbuild > 0) {
         count_launch();
-        summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, summ);
+        summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -467,7 +512,7 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
     }
     count_launch();
     append_kernel<T><<<dim3(m.units(), 4), 256, 0, s>>>(K, V, Pk, Pv, m.T, m.d, m.nG, m.nC, m.lc, m.sc, nj > 0 ? j_begin : -1,
-                                               ni > 0 ? i_begin : -1, summ, Kc, Vc);
+                                               ni > 0 ? i_begin : -1, m.iso, summ, Kc, Vc);
     *e = cudaGetLastError();
     return true;
 }

@@ -33,11 +33,14 @@
  *                  already passed through the sigmoid
  *     Kc, Vc       [B, Hkv, nC, d], nC = (T - cmp_block) / cmp_stride + 1 (0 if T < cmp_block)
  *     idx          decode [B, Hkv, topk], prefill [B, T, Hkv, topk]
- *     summaries    [B, Hkv, nG, 2, d/4, 32, 4] float32, nG = ceil(nB / 32), nB = T / block:
- *                  block b of a unit lives in group b/32, lane b%32; entry [..., 0, c/4, b%32, c%4]
- *                  is the key mean mu_{b,c}, [..., 1, ...] the key variance var_{b,c}.
+ *     summaries    variance = COBS_VAR_CHANNEL: [B, Hkv, nG, 2, d/4, 32, 4] float32,
+ *                  nG = ceil(nB / 32), nB = T / block: block b of a unit lives in group b/32,
+ *                  lane b%32; entry [..., 0, c/4, b%32, c%4] is the key mean mu_{b,c},
+ *                  [..., 1, ...] the key variance var_{b,c}.
+ *                  variance = COBS_VAR_ISOTROPIC: [B, Hkv, nG, (d/4 * 32 * 4) + 32] float32:
+ *                  the means as above, then sigma2_b of the group's 32 blocks.
  *                  (32 consecutive blocks are interleaved channel-by-channel so that one
- *                  warp reads one channel of 32 blocks in one 512-byte transaction.)
+ *                  group is one contiguous copy and lane b%32 reads its block's channels.)
  * - GQA: query head h belongs to KV head h / (Hq / Hkv).
  * - Supported: d in {64, 128}; block = 64; 1 <= topk <= 32; window >= block;
  *   Hq % Hkv == 0 and Hq / Hkv <= 16; cmp_block = 32, cmp_stride = 16 for bf16
@@ -67,6 +70,14 @@ typedef enum { COBS_F32 = 0, COBS_BF16 = 1 } cobs_dtype;
 
 typedef enum { COBS_WS_SELECT = 0, COBS_WS_DECODE = 1, COBS_WS_PREFILL = 2 } cobs_workspace_kind;
 
+/* Second-order statistic kept per block ([COBS] §2.2/§2.3: the block covariance Sigma_b, compressed):
+ *   COBS_VAR_CHANNEL    the per-channel population variance var_{b,c} (the diagonal of Sigma_b);
+ *                       score term alpha/2 * sum_c q_c^2 var_{b,c} / d.
+ *   COBS_VAR_ISOTROPIC  one scalar per block ([SKILL] "Pitfalls": one or two scalars per block):
+ *                       Sigma_b ~ sigma2_b I with sigma2_b = (1/d) sum_c var_{b,c};
+ *                       score term alpha/2 * sigma2_b |q|^2 / d. Summaries are about half the bytes. */
+typedef enum { COBS_VAR_CHANNEL = 0, COBS_VAR_ISOTROPIC = 1 } cobs_variance;
+
 /* Problem statement ([COBS] §2.3, [SKILL] "Method"): block size, compression block and
  * stride, top-k, window and alpha. */
 typedef struct {
@@ -82,6 +93,7 @@ typedef struct {
     int32_t window;     /* sliding window W */
     float alpha;        /* weight of the second-order (variance) term */
     int32_t dtype;      /* cobs_dtype of Q, K, V, Kc, Vc, O */
+    int32_t variance;   /* cobs_variance: the second-order statistic of the summaries */
 } cobs_params;
 
 /*
@@ -106,6 +118,8 @@ cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void
  * Block selection ([COBS] §2.3 second-order score; [SKILL] step 3 and "Method": top-k).
  * For each GQA group g and candidate block b:
  *   S_{g,b} = (sum_c Qsum_c mu_{b,c}) * RN(1/sqrt(d)) + RN(alpha/(2d)) * (sum_c Q2_c var_{b,c}),
+ *   or, with COBS_VAR_ISOTROPIC summaries, ... + RN(alpha/(2d)) * RN((sum_c Q2_c) * sigma2_b)
+ *   (sum_c Q2_c by adds in ascending c),
  *   Qsum = sum_{h in g} q_h, Q2 = sum_{h in g} q_h*q_h   (= sum_h [q_h.mu_b/sqrt(d)
  *   + alpha/2 * sum_c q_{h,c}^2 var_{b,c}/d]), evaluated in float32 with fused multiply-adds
  *   in ascending head and channel order. Candidates are the complete blocks

@@ -367,8 +367,10 @@ def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
     return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
 
 
-def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None):
+def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel"):
     """Decode at position T-1 for every (batch, KV head) unit (or the listed units).
+
+    variance: "channel" (per-channel variance summaries) or "isotropic" (one scalar per block).
 
     Returns dict with idx [B, Hkv, k], O [B, Hq, d] (float64; rows of unlisted units are NaN),
     summ, Kc, Vc per computed unit, and near-tie reports (units where the float64 ranking of
@@ -385,10 +387,13 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None):
         K, V, summ, Kc, Vc = unit_cache(w, K_all[b, h], V_all[b, h], Pk, Pv)
         cache[(b, h)] = (summ, Kc, Vc)
         qs = Qf[b, h * G:(h + 1) * G]
-        sel, _ = select_decode(w, qs.astype(np.float32), summ)
+        iso = variance == "isotropic"
+        sel, _ = select_decode(w, qs.astype(np.float32),
+                               canonical_summaries_iso(K.astype(np.float32), w.block) if iso else summ)
         idx[b, h] = sel
         mu, var = block_summaries(K, w.block)
-        sel64 = top_k(group_scores(qs, mu, var, w.alpha), n_candidates(t, w.block), w.topk)
+        S64 = group_scores_iso(qs, mu, var.mean(axis=1), w.alpha) if iso else group_scores(qs, mu, var, w.alpha)
+        sel64 = top_k(S64, n_candidates(t, w.block), w.topk)
         if not np.array_equal(sel, sel64):
             near_ties.append((b, h))
         O[b, h * G:(h + 1) * G] = position_output(qs, gates[b, h * G:(h + 1) * G], K, V, Kc, Vc, sel,

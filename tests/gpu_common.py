@@ -28,24 +28,32 @@ def f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def params_of(w):
+def params_of(w, variance="channel"):
     C = cobs()
     return C.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
-                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype)
+                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype, variance=variance)
 
 
 def summaries_blocks(flat, p):
-    """Device summaries (channel-interleaved groups of 32 blocks) -> [B, Hkv, nB, 2, d] float32."""
+    """Device summaries (channel-interleaved groups of 32 blocks) -> [B, Hkv, nB, 2, d] float32
+    (per-channel variance) or [B, Hkv, nB, d + 1] (isotropic: means, then the block's scalar)."""
     nB = p.T // p.block
     nG = max(1, -(-nB // 32))
+    if p.variance == "isotropic":
+        gf = (p.d + 1) * 32
+        a = flat[: p.B * p.Hkv * nG * gf].cpu().numpy().reshape(p.B, p.Hkv, nG, gf)
+        mu = a[..., :p.d * 32].reshape(p.B, p.Hkv, nG, p.d // 4, 32, 4).transpose(0, 1, 2, 4, 3, 5)
+        mu = mu.reshape(p.B, p.Hkv, nG * 32, p.d)
+        sig = a[..., p.d * 32:].reshape(p.B, p.Hkv, nG * 32, 1)
+        return np.concatenate([mu, sig], axis=-1)[:, :, :nB]
     a = flat[: p.B * p.Hkv * nG * 2 * p.d * 32].cpu().numpy()
     a = a.reshape(p.B, p.Hkv, nG, 2, p.d // 4, 32, 4).transpose(0, 1, 2, 5, 3, 4, 6)
     return a.reshape(p.B, p.Hkv, nG * 32, 2, p.d)[:, :, :nB]
 
 
-def run_decode(w, K, V, Q, gates, Pk, Pv):
+def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel"):
     C = cobs()
-    p = params_of(w)
+    p = params_of(w, variance)
     buf = C.alloc(p, prefill=False)
     C.device_error(reset=True)
     C.decode_step(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),
@@ -54,9 +62,9 @@ def run_decode(w, K, V, Q, gates, Pk, Pv):
     return p, buf
 
 
-def run_prefill(w, K, V, Q, gates, Pk, Pv):
+def run_prefill(w, K, V, Q, gates, Pk, Pv, variance="channel"):
     C = cobs()
-    p = params_of(w)
+    p = params_of(w, variance)
     buf = C.alloc(p, prefill=True)
     C.device_error(reset=True)
     C.prefill(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),
