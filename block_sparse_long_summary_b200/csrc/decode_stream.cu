@@ -300,8 +300,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
     }
     __syncwarp();
 
-    auto issue = [&](int i, int s) {  // lane 0 only
-        const Tile tl = tile_at(a, g0 + i);
+    auto issue = [&](const Tile& tl, int s) {  // lane 0 only
         if (tl.mask == 0u) return;
         const CUtensorMap* mk = tl.br == 2 ? &tmKc : &tmK;
         const CUtensorMap* mv = tl.br == 2 ? &tmVc : &tmV;
@@ -313,19 +312,31 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
             tma_load_2d(dst + kMat + h * kBox, mv, h * 64, tl.row, &bar[s]);
         }
     };
-    if (lane == 0)
-        for (int i = 0; i < kStages && i < n; ++i) issue(i, i);
+    // descriptors of the next kStages tiles, in registers: a selected block's index is read
+    // when its tile is prefetched, not when it is consumed
+    Tile tq[kStages];
+#pragma unroll
+    for (int j = 0; j < kStages; ++j) tq[j] = j < n ? tile_at(a, g0 + j) : Tile{0, 0, 0, 0, 0u};
+    if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < kStages; ++j)
+            if (j < n) issue(tq[j], j);
+    }
 
     uint32_t phase = 0;  // bit s: parity of the next completion of stage s
     uint32_t qa[D / 16][4];
     WState<D> st;
     st.init();
-    Tile cur = tile_at(a, g0);
+    Tile cur = tq[0];
     load_q<D>(a.Q + (size_t)cur.unit * a.G * D, a.G, qa, lane);
     bool ok = true;
     for (int i = 0; i < n; ++i) {
         const int s = i % kStages;
-        const Tile tl = tile_at(a, g0 + i);
+        const Tile tl = tq[0];
+#pragma unroll
+        for (int j = 0; j + 1 < kStages; ++j) tq[j] = tq[j + 1];
+        const bool more = i + kStages < n;
+        tq[kStages - 1] = more ? tile_at(a, g0 + i + kStages) : Tile{0, 0, 0, 0, 0u};
         if (tl.unit != cur.unit || tl.br != cur.br) {
             flush<D>(a, v, cur.unit, cur.br, st, lane);
             st.init();
@@ -339,9 +350,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
             if (ok) tile_mma<D>(st, qa, ring + (size_t)s * kStage, ring + (size_t)s * kStage + kMat, tl.mask, a.sl2, lane);
         }
         __syncwarp();
-        if (lane == 0 && ok && i + kStages < n) {
+        if (lane == 0 && ok && more) {
             fence_proxy_async();
-            issue(i + kStages, s);
+            issue(tq[kStages - 1], s);
         }
     }
     flush<D>(a, v, cur.unit, cur.br, st, lane);

@@ -106,8 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         mbar_init(&barS[0], 1);
         mbar_init(&barS[1], 1);
-        mbar_init(&barP[0], kSoftmaxThreads);
-        mbar_init(&barP[1], kSoftmaxThreads);
+        mbar_init(&barP[0], kSoftmaxThreads / 32);  // one arrival per softmax warp
+        mbar_init(&barP[1], kSoftmaxThreads / 32);
         mbar_init(&barO[0], 1);
         mbar_init(&barO[1], 1);
         mbar_init(&barDone, 1);
@@ -381,9 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tc_kernel(const __grid_co
         }
         lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         if (br == 0) { m0 = mref; l0 = lsum; } else if (br == 1) { m1 = mref; l1 = lsum; } else { m2 = mref; l2 = lsum; }
+        // every lane's P stores and TMEM accesses are ordered before the warp's single arrival
         fence_proxy_async();
         tc::fence_before_sync();
-        mbar_arrive(&barP[i & 1]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&barP[i & 1]);
     }
     // all MMAs done
     wait_pv(n - 1);
