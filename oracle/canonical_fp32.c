@@ -20,10 +20,29 @@
  *              with isd = RN(1/sqrt(d)), c2 = RN(alpha / (2 d)),
  *   which equals sum_{h in g} [ q_h.mu_b / sqrt(d) + alpha/2 * sum_c q_{h,c}^2 var_{b,c} / d ].
  *
- * Order: every sum runs over its index in ascending order starting from +0.
+ * Order: every sum over rows or heads runs over its index in ascending order starting from +0.
+ * The two channel sums of a score (sum_c Qsum_c mu_c and sum_c Q2_c var_c) each run as four
+ * interleaved partial chains, chain j taking the channels c = j (mod 4) in ascending order from
+ * +0 with one fmaf per term, and are combined as (s_0 + s_1) + (s_2 + s_3). (The pages fix no
+ * order; this one keeps the dependency chains short and matches four consecutive channels per
+ * 16-byte load.)
  */
+
+
 #include <math.h>
 #include <stdint.h>
+
+/* sum_c x_c y_c in the canonical four-chain order (d a multiple of 4). */
+static float dot4(const float* x, const float* y, int d) {
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    for (int c = 0; c < d; c += 4) {
+        s0 = fmaf(x[c + 0], y[c + 0], s0);
+        s1 = fmaf(x[c + 1], y[c + 1], s1);
+        s2 = fmaf(x[c + 2], y[c + 2], s2);
+        s3 = fmaf(x[c + 3], y[c + 3], s3);
+    }
+    return (s0 + s1) + (s2 + s3);
+}
 
 /*
  * K: [T][d] float32 rows (exact bf16 or fp32 values). Writes out[j][0][c] = mu,
@@ -81,9 +100,8 @@ void cobs_oracle_scores_f32(const float* qsum, const float* q2, const float* sum
         for (int64_t b = 0; b < nb; ++b) {
             const float* mu = summ + (b * 2 + 0) * d;
             const float* var = summ + (b * 2 + 1) * d;
-            float a = 0.0f, v = 0.0f;
-            for (int c = 0; c < d; ++c) a = fmaf(qs[c], mu[c], a);
-            for (int c = 0; c < d; ++c) v = fmaf(qq[c], var[c], v);
+            const float a = dot4(qs, mu, d);
+            const float v = dot4(qq, var, d);
             S[i * nb + b] = fmaf(c2, v, a * isd);
         }
     }
@@ -99,7 +117,7 @@ void cobs_oracle_scores_f32(const float* qsum, const float* q2, const float* sum
  *             Q2tot = sum_c Q2_c  (= sum_{h in g} |q_h|^2).
  * Canonical order: var_{b,c} as in cobs_oracle_summaries_f32; sigma2_b = (adds over c
  * ascending from +0) * (1/d) (exact scaling, d a power of two); Q2tot = adds over c
- * ascending from +0; S = fma(c2, Q2tot * sigma2_b, a * isd) with a as above.
+ * ascending from +0; S = fma(c2, Q2tot * sigma2_b, a * isd) with a as above (four chains).
  */
 
 /* summ: [nb][2][d] (mean, per-channel variance, as written above). out: [nb][d + 1] (mean, sigma2). */
@@ -126,8 +144,7 @@ void cobs_oracle_iso_scores_f32(const float* qsum, const float* q2, const float*
         for (int c = 0; c < d; ++c) q2tot = q2tot + qq[c];
         for (int64_t b = 0; b < nb; ++b) {
             const float* mu = summ_iso + b * (d + 1);
-            float a = 0.0f;
-            for (int c = 0; c < d; ++c) a = fmaf(qs[c], mu[c], a);
+            const float a = dot4(qs, mu, d);
             const float v = q2tot * mu[d];
             S[i * nb + b] = fmaf(c2, v, a * isd);
         }

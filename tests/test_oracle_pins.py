@@ -170,6 +170,15 @@ def test_group_sum_reading_internal_consistency():
 
 # ---------------------------------------------------------------- canonical float32 arithmetic
 
+def _dot4_exact(F, x, y):
+    """The canonical channel sum: four partial chains (channels c = j mod 4, ascending, one
+    rounded fma per term) combined as (s0 + s1) + (s2 + s3), every step rounded once."""
+    s = [Fraction(0)] * 4
+    for c in range(len(x)):
+        s[c % 4] = _rn32(F(x[c]) * F(y[c]) + s[c % 4])
+    return _rn32(_rn32(s[0] + s[1]) + _rn32(s[2] + s[3]))
+
+
 def _rn32(x: Fraction) -> Fraction:
     """Round an exact rational to the nearest binary32 value, ties to even (normal range)."""
     if x == 0:
@@ -221,11 +230,8 @@ def test_canonical_selector_matches_exact_rational_emulation():
     isd = _rn32(Fraction(1.0 / math.sqrt(d)))
     c2 = _rn32(F(alpha) / (2 * d))
     for b in range(nB):
-        a, v = Fraction(0), Fraction(0)
-        for c in range(d):
-            a = _rn32(F(qsum[c]) * F(summ[b, 0, c]) + a)
-        for c in range(d):
-            v = _rn32(F(q2[c]) * F(summ[b, 1, c]) + v)
+        a = _dot4_exact(F, qsum, summ[b, 0])
+        v = _dot4_exact(F, q2, summ[b, 1])
         assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
 
 
@@ -520,8 +526,6 @@ def test_iso_canonical_matches_exact_rational_emulation():
     isd = _rn32(Fraction(1.0 / math.sqrt(d)))
     c2 = _rn32(F(alpha) / (2 * d))
     for b in range(nB):
-        a = Fraction(0)
-        for c in range(d):
-            a = _rn32(F(qsum[c]) * F(iso[b, c]) + a)
+        a = _dot4_exact(F, qsum, iso[b, :d])
         v = _rn32(q2tot * F(iso[b, d]))
         assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
