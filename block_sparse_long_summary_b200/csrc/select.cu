@@ -184,49 +184,57 @@ __device__ __forceinline__ void group_reduce(const float (&x)[kMaxGroup], int G,
     q2 = s2;
 }
 
+// Canonical channel sums: four interleaved partial chains (chain j takes the channels
+// c = j (mod 4) in ascending order from +0, one rounded fma per term), combined as
+// (s0 + s1) + (s2 + s3). Lane = block; a group tile keeps four consecutive channels of a block
+// in one 16-byte word, so one load feeds the four chains.
+__device__ __forceinline__ float combine4(float s0, float s1, float s2, float s3) {
+    return __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
+}
+
 // Canonical score of the block held by this lane (channel-interleaved group tile in smem).
 template <int D>
 __device__ __forceinline__ float block_score(const float* tile, const float* qs, const float* q2, int lane,
                                              float isd, float c2) {
     const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
     const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
-    float a = 0.0f, v = 0.0f;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
 #pragma unroll 8
     for (int c4 = 0; c4 < D / 4; ++c4) {
         const float4 m = mu4[c4 * 32];
-        a = __fmaf_rn(qs[4 * c4 + 0], m.x, a);
-        a = __fmaf_rn(qs[4 * c4 + 1], m.y, a);
-        a = __fmaf_rn(qs[4 * c4 + 2], m.z, a);
-        a = __fmaf_rn(qs[4 * c4 + 3], m.w, a);
-    }
-#pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
         const float4 s = var4[c4 * 32];
-        v = __fmaf_rn(q2[4 * c4 + 0], s.x, v);
-        v = __fmaf_rn(q2[4 * c4 + 1], s.y, v);
-        v = __fmaf_rn(q2[4 * c4 + 2], s.z, v);
-        v = __fmaf_rn(q2[4 * c4 + 3], s.w, v);
+        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
+        const float4 r = reinterpret_cast<const float4*>(q2)[c4];
+        a0 = __fmaf_rn(q.x, m.x, a0);
+        a1 = __fmaf_rn(q.y, m.y, a1);
+        a2 = __fmaf_rn(q.z, m.z, a2);
+        a3 = __fmaf_rn(q.w, m.w, a3);
+        v0 = __fmaf_rn(r.x, s.x, v0);
+        v1 = __fmaf_rn(r.y, s.y, v1);
+        v2 = __fmaf_rn(r.z, s.z, v2);
+        v3 = __fmaf_rn(r.w, s.w, v3);
     }
-    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
+    return __fmaf_rn(c2, combine4(v0, v1, v2, v3), __fmul_rn(combine4(a0, a1, a2, a3), isd));
 }
 
-// Canonical isotropic score: the same mean chain, then v = RN(Q2tot * sigma2_b) with the block's
+// Canonical isotropic score: the same mean sum, then v = RN(Q2tot * sigma2_b) with the block's
 // one variance scalar (stored after the group's means) and Q2tot = sum_c Q2_c.
 template <int D>
 __device__ __forceinline__ float block_score_iso(const float* tile, const float* qs, float q2tot, int lane, float isd,
                                                  float c2) {
     const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
-    float a = 0.0f;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 8
     for (int c4 = 0; c4 < D / 4; ++c4) {
         const float4 m = mu4[c4 * 32];
-        a = __fmaf_rn(qs[4 * c4 + 0], m.x, a);
-        a = __fmaf_rn(qs[4 * c4 + 1], m.y, a);
-        a = __fmaf_rn(qs[4 * c4 + 2], m.z, a);
-        a = __fmaf_rn(qs[4 * c4 + 3], m.w, a);
+        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
+        a0 = __fmaf_rn(q.x, m.x, a0);
+        a1 = __fmaf_rn(q.y, m.y, a1);
+        a2 = __fmaf_rn(q.z, m.z, a2);
+        a3 = __fmaf_rn(q.w, m.w, a3);
     }
     const float v = __fmul_rn(q2tot, tile[D * 32 + lane]);
-    return __fmaf_rn(c2, v, __fmul_rn(a, isd));
+    return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
 }
 
 // Q2tot = sum_c Q2_c by adds in ascending channel order from +0 (one thread).
@@ -552,9 +560,11 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
         const int blk = gi * kGroupBlocks + lane;
         // scores of this lane's block against the warp's 8 positions: 16 independent chains,
         // each in the canonical order (ascending channels, one fma per term)
-        float av[kPfPerWarp], vv[kPfPerWarp];
+        float av[kPfPerWarp][4], vv[kPfPerWarp][4];
 #pragma unroll
-        for (int j = 0; j < kPfPerWarp; ++j) av[j] = vv[j] = 0.0f;
+        for (int j = 0; j < kPfPerWarp; ++j)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) av[j][q] = vv[j][q] = 0.0f;
         const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
         const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
         const float* sqw = sq + (size_t)(warp * kPfPerWarp) * 2 * D;
@@ -565,15 +575,12 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
 #pragma unroll
                 for (int j = 0; j < kPfPerWarp; ++j) {
                     const float4 qa = reinterpret_cast<const float4*>(sqw + (j * 2 + 0) * D)[c4];
-                    av[j] = __fmaf_rn(qa.x, m.x, av[j]);
-                    av[j] = __fmaf_rn(qa.y, m.y, av[j]);
-                    av[j] = __fmaf_rn(qa.z, m.z, av[j]);
-                    av[j] = __fmaf_rn(qa.w, m.w, av[j]);
+                    av[j][0] = __fmaf_rn(qa.x, m.x, av[j][0]);
+                    av[j][1] = __fmaf_rn(qa.y, m.y, av[j][1]);
+                    av[j][2] = __fmaf_rn(qa.z, m.z, av[j][2]);
+                    av[j][3] = __fmaf_rn(qa.w, m.w, av[j][3]);
                 }
             }
-            const float sig = tile[D * 32 + lane];
-#pragma unroll
-            for (int j = 0; j < kPfPerWarp; ++j) vv[j] = __fmul_rn(q2t[warp * kPfPerWarp + j], sig);
         } else {
 #pragma unroll 4
             for (int c4 = 0; c4 < D / 4; ++c4) {
@@ -583,16 +590,23 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
                 for (int j = 0; j < kPfPerWarp; ++j) {
                     const float4 qa = reinterpret_cast<const float4*>(sqw + (j * 2 + 0) * D)[c4];
                     const float4 qb = reinterpret_cast<const float4*>(sqw + (j * 2 + 1) * D)[c4];
-                    av[j] = __fmaf_rn(qa.x, m.x, av[j]);
-                    av[j] = __fmaf_rn(qa.y, m.y, av[j]);
-                    av[j] = __fmaf_rn(qa.z, m.z, av[j]);
-                    av[j] = __fmaf_rn(qa.w, m.w, av[j]);
-                    vv[j] = __fmaf_rn(qb.x, vr.x, vv[j]);
-                    vv[j] = __fmaf_rn(qb.y, vr.y, vv[j]);
-                    vv[j] = __fmaf_rn(qb.z, vr.z, vv[j]);
-                    vv[j] = __fmaf_rn(qb.w, vr.w, vv[j]);
+                    av[j][0] = __fmaf_rn(qa.x, m.x, av[j][0]);
+                    av[j][1] = __fmaf_rn(qa.y, m.y, av[j][1]);
+                    av[j][2] = __fmaf_rn(qa.z, m.z, av[j][2]);
+                    av[j][3] = __fmaf_rn(qa.w, m.w, av[j][3]);
+                    vv[j][0] = __fmaf_rn(qb.x, vr.x, vv[j][0]);
+                    vv[j][1] = __fmaf_rn(qb.y, vr.y, vv[j][1]);
+                    vv[j][2] = __fmaf_rn(qb.z, vr.z, vv[j][2]);
+                    vv[j][3] = __fmaf_rn(qb.w, vr.w, vv[j][3]);
                 }
             }
+        }
+        float aj[kPfPerWarp], vj[kPfPerWarp];
+        const float sig = ISO ? tile[D * 32 + lane] : 0.0f;
+#pragma unroll
+        for (int j = 0; j < kPfPerWarp; ++j) {
+            aj[j] = combine4(av[j][0], av[j][1], av[j][2], av[j][3]);
+            vj[j] = ISO ? __fmul_rn(q2t[warp * kPfPerWarp + j], sig) : combine4(vv[j][0], vv[j][1], vv[j][2], vv[j][3]);
         }
         __syncthreads();  // every warp is done with this stage
         if (tid == 0 && ok && gi + 2 < ngroups) {
@@ -605,7 +619,7 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
             const int t = t0 + warp * kPfPerWarp + j;
             const int nc = (t + 1) / L;
             const bool valid = ok && t < Tctx && blk < nc;
-            float sc = __fmaf_rn(c2, vv[j], __fmul_rn(av[j], isd));
+            float sc = __fmaf_rn(c2, vj[j], __fmul_rn(aj[j], isd));
             int bi = blk;
             if (!valid) {
                 sc = -INFINITY;

@@ -389,6 +389,18 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
     __shared__ float vsm[128];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int unit = blockIdx.x, quarter = blockIdx.y;
+    // this warp's rows of the projection (d / 16 <= 8 rows, one 16-byte chunk per lane), loaded
+    // first so that their latency overlaps the row loads below
+    const int ws = warp >> 2;  // warps 0-3: K, 4-7: V
+    const float* P = ws ? Pv : Pk;
+    const int per_warp = d / 16;
+    const int j0 = quarter * (d / 4) + (warp & 3) * per_warp;
+    float4 pv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        pv[u] = (ic >= 0 && P != nullptr && u < per_warp && lane * 4 < d)
+                    ? __ldg(reinterpret_cast<const float4*>(P + (size_t)(j0 + u) * d) + lane)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     // block summary (channels 32 quarter + tid; the isotropic layout needs every channel in
     // one CTA: quarter 0, thread = channel): the canonical row-order sums
     const bool sum_here = jb >= 0 && (iso ? (quarter == 0 && tid < d) : (tid < 32 && quarter * 32 + tid < d));
@@ -431,8 +443,6 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
         pooled[side][c] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) / (float)lc;
     }
     __syncthreads();
-    const int ws = warp >> 2;  // warps 0-3: K, 4-7: V
-    const float* P = ws ? Pv : Pk;
     T* orow = (ws ? Vc : Kc) + ((size_t)unit * nC + ic) * d;
     if (P == nullptr) {
         const int cc = tid & 127;
@@ -440,28 +450,18 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
         return;
     }
     const float4 q = lane * 4 < d ? reinterpret_cast<const float4*>(pooled[ws])[lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const int per_warp = d / 16;  // output rows of this warp
-    const int j0 = quarter * (d / 4) + (warp & 3) * per_warp;
-    for (int jb8 = 0; jb8 < per_warp; jb8 += 8) {
-        float part[8];
+    float part[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int j = j0 + jb8 + u;
-            float4 pv = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (jb8 + u < per_warp && lane * 4 < d)
-                pv = __ldg(reinterpret_cast<const float4*>(P + (size_t)j * d) + lane);
-            part[u] = pv.x * q.x + pv.y * q.y + pv.z * q.z + pv.w * q.w;
-        }
+    for (int u = 0; u < 8; ++u) part[u] = pv[u].x * q.x + pv[u].y * q.y + pv[u].z * q.z + pv[u].w * q.w;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
+    for (int off = 16; off > 0; off >>= 1)
 #pragma unroll
-            for (int u = 0; u < 8; ++u) part[u] += __shfl_xor_sync(0xffffffffu, part[u], off);
-        if (lane < 8 && jb8 + lane < per_warp) {
-            float v = part[0];
+        for (int u = 0; u < 8; ++u) part[u] += __shfl_xor_sync(0xffffffffu, part[u], off);
+    if (lane < per_warp) {
+        float v = part[0];
 #pragma unroll
-            for (int u = 1; u < 8; ++u) v = lane == u ? part[u] : v;
-            Elem<T>::store(orow + j0 + jb8 + lane, v);
-        }
+        for (int u = 1; u < 8; ++u) v = lane == u ? part[u] : v;
+        Elem<T>::store(orow + j0 + lane, v);
     }
 }
 
