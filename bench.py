@@ -40,8 +40,10 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k", "sweep"])
     ap.add_argument("--contexts", default=None, help="sweep: comma-separated context lengths (default 8k .. 1M)")
-    ap.add_argument("--variance", choices=["channel", "isotropic"], default="channel",
-                    help="second-order statistic of the summaries (per-channel variance or one scalar per block)")
+    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank"], default="channel",
+                    help="second-order statistic of the summaries (per-channel variance, one scalar per block, "
+                         "or the leading eigenpairs of each block's covariance)")
+    ap.add_argument("--rank", type=int, default=4, help="eigenpairs per block with --variance lowrank")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
     ap.add_argument("--T", type=int, default=None, help="override the context length (small profiling cases)")
@@ -160,7 +162,7 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic bytes
 
-def decode_bytes(w, idx, variance="channel"):
+def decode_bytes(w, idx, variance="channel", rank=4):
     """Algorithmic HBM bytes of one decode step, from the selected blocks (idx [B, Hkv, k])."""
     import numpy as np
     d, esz = w.d, 2 if w.dtype == "bf16" else 4
@@ -179,7 +181,7 @@ def decode_bytes(w, idx, variance="channel"):
     units = w.B * w.Hkv
     attn = kv_tokens * 2 * d * esz + units * ncv * 2 * d * esz          # K/V union + compressed K/V
     attn += w.B * w.Hq * d * esz * 2 + w.B * w.Hq * 3 * 4 + units * w.topk * 4   # Q, O, gates, idx
-    per_block = (d + 1) * 4 if variance == "isotropic" else 2 * d * 4
+    per_block = {"isotropic": (d + 1) * 4, "lowrank": (d + rank * d + rank) * 4}.get(variance, 2 * d * 4)
     select = units * w.nB * per_block + w.B * w.Hq * d * esz + units * w.topk * 4
     # summary update for the appended token: the completed block (64 K rows) and the last
     # compressed token (cmp_block K and V rows), plus their outputs
@@ -190,11 +192,11 @@ def decode_bytes(w, idx, variance="channel"):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False, variance="channel"):
+def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False, variance="channel", rank=4):
     """Time the oracle (as it stands) on the listed units; returns (seconds, query heads[, result])."""
     from oracle import cobs_oracle as O
     t0 = time.perf_counter()
-    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units, variance=variance)
+    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units, variance=variance, rank=rank)
     secs = time.perf_counter() - t0
     return (secs, len(units) * w.G, res) if with_result else (secs, len(units) * w.G)
 
@@ -369,7 +371,7 @@ def run_ours(args):
         return run_prefill_line(args, w, dev, cobs, rank, world)
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
-                    variance=args.variance)
+                    variance=args.variance, rank=args.rank)
     K, V = synth.kv_cache(w)
     Q, g = synth.queries_decode(w), synth.gates_decode(w)
     Pk, Pv = synth.projections(w)
@@ -521,7 +523,7 @@ def run_ours(args):
     dev_err = cobs.device_error()
 
     qheads = w.B * w.Hq * world
-    by = decode_bytes(w, idx0, args.variance)
+    by = decode_bytes(w, idx0, args.variance, args.rank)
     peak, peak_kind = read_peaks()
     att_gbs = by["attn"] / (t_att * 1e-3) / 1e9
     result = {
@@ -530,7 +532,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
                    "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
-                   "variance": args.variance,
+                   "variance": args.variance, **({"rank": args.rank} if args.variance == "lowrank" else {}),
                    "step": "summary update at T-1 + select + decode attention, one CUDA graph",
                    "l2": f"{R} KV-cache copies rotated between steps (working set {R} x step bytes > L2)",
                    "parallelism": f"dp{world} (independent decode batches per GPU)"},
@@ -559,7 +561,7 @@ def run_ours(args):
         lim = limit_threads()
         units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:24]
         secs, heads, ref = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=True,
-                                                variance=args.variance)
+                                                variance=args.variance, rank=args.rank)
         result["cpu_baseline"] = {"value": heads / secs, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                                   "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
                                             f"full oracle decode incl. summaries ({secs:.1f} s)"}
@@ -636,7 +638,7 @@ def run_sweep(args):
     def params(w, **over):
         kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                   cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
-                  variance=args.variance)
+                  variance=args.variance, rank=args.rank)
         kw.update(over)
         return cobs.Params(**kw)
 
@@ -703,7 +705,8 @@ def run_sweep(args):
                 ref = set(osa.tolist())
                 rec1.append(len(ref & set(int(x) for x in idx_a1[b, g] if x >= 0)) / w.topk)
                 rec0.append(len(ref & set(int(x) for x in idx_a0[b, g] if x >= 0)) / w.topk)
-        per_block = (w.d + 1) * 4 if args.variance == "isotropic" else 2 * w.d * 4
+        per_block = {"isotropic": (w.d + 1) * 4,
+                     "lowrank": (w.d + args.rank * w.d + args.rank) * 4}.get(args.variance, 2 * w.d * 4)
         by = w.B * w.Hkv * nB * per_block + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * w.topk * 4
         gbs = by / (us * 1e-6) / 1e9
         rows.append({"T": T, "nB": nB, "bytes": by, "us": us, "gbs": gbs, "frac": gbs / peak,

@@ -23,7 +23,7 @@ COBS_ERR_CUDA = -3
 COBS_ERR_WORKSPACE = -4
 COBS_F32 = 0
 COBS_BF16 = 1
-COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC = 0, 1
+COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC, COBS_VAR_LOWRANK = 0, 1, 2
 COBS_WS_SELECT = 0
 COBS_WS_DECODE = 1
 COBS_WS_PREFILL = 2
@@ -39,7 +39,8 @@ class cobs_params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("T", ctypes.c_int32), ("block", ctypes.c_int32), ("cmp_block", ctypes.c_int32),
                 ("cmp_stride", ctypes.c_int32), ("topk", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32), ("variance", ctypes.c_int32)]
+                ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32), ("variance", ctypes.c_int32),
+                ("rank", ctypes.c_int32)]
 
 
 class CobsError(RuntimeError):
@@ -98,12 +99,14 @@ class Params:
     cmp_stride: int = 16
     alpha: float = 1.0
     dtype: str = "bf16"
-    variance: str = "channel"   # "channel" (per-channel variance) or "isotropic" (one scalar per block)
+    variance: str = "channel"   # "channel", "isotropic" (one scalar per block) or "lowrank"
+    rank: int = 4               # eigenpairs per block for "lowrank"
 
     def c(self) -> cobs_params:
+        var = {"channel": COBS_VAR_CHANNEL, "isotropic": COBS_VAR_ISOTROPIC, "lowrank": COBS_VAR_LOWRANK}[self.variance]
         return cobs_params(self.B, self.Hq, self.Hkv, self.d, self.T, self.block, self.cmp_block, self.cmp_stride,
                            self.topk, self.window, float(self.alpha), COBS_BF16 if self.dtype == "bf16" else COBS_F32,
-                           COBS_VAR_ISOTROPIC if self.variance == "isotropic" else COBS_VAR_CHANNEL)
+                           var, int(self.rank))
 
     @property
     def torch_dtype(self):

@@ -168,22 +168,6 @@ __device__ __forceinline__ void group_query_chunk(const T* q, int G, int D, int 
     }
 }
 
-// Canonical group query: Qsum_c = sum_h q_{h,c} (adds) and Q2_c = fma-sum of q_{h,c}^2, in
-// ascending h, from values already in registers (x[h] = q_{h,c}, ascending h). Callers
-// issue all G loads of a channel at once (independent loads) before reducing in order.
-__device__ __forceinline__ void group_reduce(const float (&x)[kMaxGroup], int G, float& qs, float& q2) {
-    float s = 0.0f, s2 = 0.0f;
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (h < G) {
-            s = __fadd_rn(s, x[h]);
-            s2 = __fmaf_rn(x[h], x[h], s2);
-        }
-    }
-    qs = s;
-    q2 = s2;
-}
-
 // Canonical channel sums: four interleaved partial chains (chain j takes the channels
 // c = j (mod 4) in ascending order from +0, one rounded fma per term), combined as
 // (s0 + s1) + (s2 + s3). Lane = block; a group tile keeps four consecutive channels of a block
@@ -234,6 +218,49 @@ __device__ __forceinline__ float block_score_iso(const float* tile, const float*
         a3 = __fmaf_rn(q.w, m.w, a3);
     }
     const float v = __fmul_rn(q2tot, tile[D * 32 + lane]);
+    return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
+}
+
+// Canonical low-rank score: the same mean sum, then
+//   v = sum over j ascending of fma(lambda_j, e_j, .), e_j = sum over h ascending of fma(p, p, .),
+//   p = four-chain sum_c q_{h,c} u_{j,c};
+// the tile holds the 32 blocks' means, then eigenvector j in the same interleaving for j < R,
+// then the R x 32 eigenvalues. qh: the group's G query heads [G][D] in shared memory.
+template <int D>
+__device__ __forceinline__ float block_score_lr(const float* tile, const float* qs, const float* qh, int G, int R,
+                                                int lane, float isd, float c2) {
+    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 m = mu4[c4 * 32];
+        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
+        a0 = __fmaf_rn(q.x, m.x, a0);
+        a1 = __fmaf_rn(q.y, m.y, a1);
+        a2 = __fmaf_rn(q.z, m.z, a2);
+        a3 = __fmaf_rn(q.w, m.w, a3);
+    }
+    float v = 0.0f;
+    for (int j = 0; j < R; ++j) {
+        const float4* u4 = reinterpret_cast<const float4*>(tile + (size_t)(1 + j) * D * 32) + lane;
+        float e = 0.0f;
+        for (int h = 0; h < G; ++h) {
+            const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)h * D);
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll 8
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 uu = u4[c4 * 32];
+                const float4 q = q4[c4];
+                p0 = __fmaf_rn(q.x, uu.x, p0);
+                p1 = __fmaf_rn(q.y, uu.y, p1);
+                p2 = __fmaf_rn(q.z, uu.z, p2);
+                p3 = __fmaf_rn(q.w, uu.w, p3);
+            }
+            const float pj = combine4(p0, p1, p2, p3);
+            e = __fmaf_rn(pj, pj, e);
+        }
+        v = __fmaf_rn(tile[(size_t)(1 + R) * D * 32 + j * 32 + lane], e, v);
+    }
     return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
 }
 
@@ -342,18 +369,22 @@ struct RunList {
 // if it held the whole unit, else deposits its segment's exact top-k; select_merge_kernel (a
 // dependent launch) merges the deposits. The result is the top-k under a strict total order,
 // so it does not depend on the split.
-template <typename T, int D, bool ISO>
+// MODE 0: per-channel variance summaries, 1: isotropic, 2: low-rank (R eigenpairs, tile_floats
+// floats per group, one ring stage, the group's query heads in shared memory after the ring).
+template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
                                                            int32_t* __restrict__ idx, float* __restrict__ ws_s,
                                                            int* __restrict__ ws_i, int units, int G, int nG,
                                                            int ncand, int k, int maxseg,
-                                                           float isd, float c2, int* err) {
+                                                           float isd, float c2, int R, int tile_floats, int* err) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bar[kSelStages];
     __shared__ __align__(16) float qsm[2][D];
     __shared__ float q2t_sm;
-    constexpr int kTileFloats = group_floats<D, ISO>();
-    constexpr uint32_t kTileBytes = kTileFloats * 4;
+    constexpr bool ISO = MODE == 1;
+    constexpr int kStg = MODE == 2 ? 1 : kSelStages;
+    const int kTileFloats = MODE == 2 ? tile_floats : group_floats<D, ISO>();
+    const uint32_t kTileBytes = (uint32_t)kTileFloats * 4;
     // the merge grid may be scheduled now; it still waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int lane = threadIdx.x;
@@ -374,12 +405,12 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
     };
     if (lane == 0) {
 #pragma unroll
-        for (int st = 0; st < kSelStages; ++st) mbar_init(&bar[st], 1);
+        for (int st = 0; st < kStg; ++st) mbar_init(&bar[st], 1);
         fence_barrier_init();
     }
     __syncwarp();
     if (lane == 0) {
-        for (int st = 0; st < kSelStages && x0 + st < x1; ++st) {
+        for (int st = 0; st < kStg && x0 + st < x1; ++st) {
             mbar_arrive_expect_tx(&bar[st], kTileBytes);
             bulk_g2s(tiles + st * kTileFloats, group_src(x0 + st), kTileBytes, &bar[st]);
         }
@@ -406,8 +437,8 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
 
     for (long long x = x0; x < x1; ++x) {
         const int it = (int)(x - x0);
-        const int st = it % kSelStages;
-        const uint32_t parity = (uint32_t)(it / kSelStages) & 1u;
+        const int st = it % kStg;
+        const uint32_t parity = (uint32_t)(it / kStg) & 1u;
         const int u = (int)(x / nGc), gl = (int)(x % nGc);
         if (u != cur) {
             if (cur >= 0) finish(cur);
@@ -424,6 +455,11 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
                 if (lane == 0) q2t_sm = q2_total<D>(qsm[1]);
                 __syncwarp();
             }
+            if (MODE == 2) {  // the group's heads as float32, after the ring
+                float* qh = tiles + kStg * kTileFloats;
+                for (int e = lane; e < G * D; e += 32) qh[e] = to_f(Q[(size_t)u * G * D + e]);
+                __syncwarp();
+            }
         }
         if (ok) ok = mbar_wait(&bar[st], parity, err);
         ok = __all_sync(kFull, ok);
@@ -431,18 +467,20 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
         float sc = -INFINITY;
         int bi = kInvalid;
         if (ok) {
-            const float s_all = ISO ? block_score_iso<D>(tiles + st * kTileFloats, qsm[0], q2t_sm, lane, isd, c2)
-                                    : block_score<D>(tiles + st * kTileFloats, qsm[0], qsm[1], lane, isd, c2);
+            const float* tl = tiles + st * kTileFloats;
+            const float s_all = MODE == 2 ? block_score_lr<D>(tl, qsm[0], tiles + kStg * kTileFloats, G, R, lane, isd, c2)
+                                : ISO     ? block_score_iso<D>(tl, qsm[0], q2t_sm, lane, isd, c2)
+                                          : block_score<D>(tl, qsm[0], qsm[1], lane, isd, c2);
             if (b < ncand) {
                 sc = s_all;
                 bi = b;
             }
         }
         __syncwarp();
-        if (lane == 0 && ok && x + kSelStages < x1) {
+        if (lane == 0 && ok && x + kStg < x1) {
             fence_proxy_async();
             mbar_arrive_expect_tx(&bar[st], kTileBytes);
-            bulk_g2s(tiles + st * kTileFloats, group_src(x + kSelStages), kTileBytes, &bar[st]);
+            bulk_g2s(tiles + st * kTileFloats, group_src(x + kStg), kTileBytes, &bar[st]);
         }
         rl.add(sc, bi, k, lane);
     }
@@ -648,12 +686,14 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     }
 }
 
-template <typename T, int D, bool ISO>
+template <typename T, int D, int MODE>
 cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                             cudaStream_t s, int* err) {
+    constexpr bool ISO = MODE == 1;
     float isd, c2;
     score_constants(m.d, m.alpha, &isd, &c2);
-    const size_t tile_bytes = (size_t)group_floats<D, ISO>() * 4;
+    const int tile_floats = (int)m.group_floats();
+    const size_t tile_bytes = (size_t)tile_floats * 4;
     if (!prefill) {
         const int ncand = m.T / m.L;
         const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
@@ -668,13 +708,15 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         grid = std::max<long long>(1, grid);
         float* ws_s = static_cast<float*>(ws);
         int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
-        const size_t smem = (size_t)kSelStages * tile_bytes;
-        cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, ISO>,
+        const size_t smem = MODE == 2 ? tile_bytes + (size_t)kMaxGroup * D * 4 : (size_t)kSelStages * tile_bytes;
+        if (smem > 227 * 1024) return cudaErrorNotSupported;
+        cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         count_launch();
-        select_decode_kernel<T, D, ISO><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(), m.G, m.nG,
-                                                                    ncand, m.k, maxseg, isd, c2, err);
+        select_decode_kernel<T, D, MODE><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(), m.G,
+                                                                          m.nG, ncand, m.k, maxseg, isd, c2, m.lr,
+                                                                          tile_floats, err);
         e = cudaGetLastError();
         // a unit is cut into several ranges only if it has several groups and the grid several CTAs
         if (e != cudaSuccess || n == 0 || nGc == 1 || grid == 1) return e;
@@ -693,6 +735,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
                                   (int)grid, m.k, maxseg);
     }
     const size_t smem = tile_bytes * 2 + (size_t)kPfPos * 2 * D * 4;
+    if (MODE == 2) return cudaErrorNotSupported;  // the API rejects it before this point
     auto kern = select_prefill_kernel<T, D, ISO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -711,23 +754,24 @@ size_t select_workspace_bytes(const Dims& m, int prefill) {
     return (size_t)m.units() * maxseg * m.k * (sizeof(float) + sizeof(int));
 }
 
-template <bool ISO>
+template <int MODE>
 cudaError_t launch_select_v(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                             cudaStream_t s, int* err) {
     if (m.dtype == COBS_BF16) {
         if (m.d == 128)
-            return launch_select_t<__nv_bfloat16, 128, ISO>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s,
-                                                            err);
-        return launch_select_t<__nv_bfloat16, 64, ISO>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s, err);
+            return launch_select_t<__nv_bfloat16, 128, MODE>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s,
+                                                             err);
+        return launch_select_t<__nv_bfloat16, 64, MODE>(m, (const __nv_bfloat16*)Q, summ, prefill, idx, ws, s, err);
     }
-    if (m.d == 128) return launch_select_t<float, 128, ISO>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
-    return launch_select_t<float, 64, ISO>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
+    if (m.d == 128) return launch_select_t<float, 128, MODE>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
+    return launch_select_t<float, 64, MODE>(m, (const float*)Q, summ, prefill, idx, ws, s, err);
 }
 
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                           cudaStream_t s, int* err) {
-    return m.iso ? launch_select_v<true>(m, Q, summ, prefill, idx, ws, s, err)
-                 : launch_select_v<false>(m, Q, summ, prefill, idx, ws, s, err);
+    if (m.lr) return launch_select_v<2>(m, Q, summ, prefill, idx, ws, s, err);
+    return m.iso ? launch_select_v<1>(m, Q, summ, prefill, idx, ws, s, err)
+                 : launch_select_v<0>(m, Q, summ, prefill, idx, ws, s, err);
 }
 
 }  // namespace cobs

@@ -76,6 +76,125 @@ __global__ void __launch_bounds__(128) summaries_kernel(const T* __restrict__ K,
     if (c == 0) base[summ_iso_at(j, d)] = iso_scalar(vsm, d);
 }
 
+// ---------------------------------------------------------------- low-rank summaries
+// The block mean and the R leading eigenpairs of the block covariance (COBS explainer §2.2/§2.3:
+// the covariance kept in low-rank form), by a fixed float32 subspace iteration whose every
+// operation is fixed (the same steps as the oracle's solver):
+//   Y = rows - mu; V = V0 (+-1 by a bit of a hash of (c, j));
+//   kLrIters times: T = Y V (four-chain sums over channels), W = Y^T T (four-chain sums over
+//   rows), modified Gram-Schmidt over the columns of W with "32-lane" dot products (lane l sums
+//   channels l, l + 32, ... with fma, then a five-level xor butterfly of adds), V = W;
+//   then T = Y V and lambda_j = (four-chain sum of T[., j]^2) / L, pairs ordered by lambda
+//   descending (ties: lower j).
+// grid (blocks to build, units), D threads (thread = channel).
+constexpr int kLrIters = 24;
+constexpr int kLrMaxR = 8;
+
+__device__ __forceinline__ float lr_v0(int c, int j) {
+    const uint32_t h = (uint32_t)c * 2654435761u + (uint32_t)(j + 1) * 40503u;
+    return ((h >> 11) & 1u) ? 1.0f : -1.0f;
+}
+
+// Four-chain dot over n terms (n a multiple of 4) with strides, (s0 + s1) + (s2 + s3).
+__device__ __forceinline__ float lr_dot4(const float* x, const float* y, int n, int sx, int sy) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    for (int i = 0; i < n; i += 4) {
+        s0 = __fmaf_rn(x[(i + 0) * sx], y[(i + 0) * sy], s0);
+        s1 = __fmaf_rn(x[(i + 1) * sx], y[(i + 1) * sy], s1);
+        s2 = __fmaf_rn(x[(i + 2) * sx], y[(i + 2) * sy], s2);
+        s3 = __fmaf_rn(x[(i + 3) * sx], y[(i + 3) * sy], s3);
+    }
+    return __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
+                                                    float* __restrict__ summ) {
+    __shared__ float Y[kBlock][D];
+    __shared__ float V[D][kLrMaxR], W[D][kLrMaxR];
+    __shared__ float Tm[kBlock][kLrMaxR];
+    __shared__ float bcast;
+    __shared__ int ord_sh[kLrMaxR];
+    __shared__ float lam_sh[kLrMaxR];
+    const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+    const int unit = blockIdx.y;
+    const int j = j_begin + blockIdx.x;
+    // canonical mean of channel c (rows ascending), then the centred rows
+    {
+        const T* rows = K + ((size_t)unit * Tctx + (size_t)j * kBlock) * D + c;
+        float x[kBlock];
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) x[r] = Elem<T>::load(rows + (size_t)r * D);
+        float sum = 0.0f;
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) sum = __fadd_rn(sum, x[r]);
+        const float mu = __fmul_rn(sum, 1.0f / kBlock);
+#pragma unroll
+        for (int r = 0; r < kBlock; ++r) Y[r][c] = __fsub_rn(x[r], mu);
+        const size_t gf = (size_t)32 * (D + R * D + R);
+        float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
+        base[((size_t)(c / 4) * 32 + (j & 31)) * 4 + (c & 3)] = mu;
+        for (int jj = 0; jj < R; ++jj) V[c][jj] = lr_v0(c, jj);
+    }
+    __syncthreads();
+    // "32-lane" dot of columns a and b of W (warp 0 computes, every thread reads the result)
+    auto wdot = [&](int a, int b) -> float {
+        if (warp == 0) {
+            float p = 0.0f;
+            for (int cc = lane; cc < D; cc += 32) p = __fmaf_rn(W[cc][a], W[cc][b], p);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
+            if (lane == 0) bcast = p;
+        }
+        __syncthreads();
+        const float v = bcast;
+        __syncthreads();
+        return v;
+    };
+    for (int it = 0; it <= kLrIters; ++it) {
+        for (int o = c; o < kBlock * R; o += D) {
+            const int r = o / R, jj = o % R;
+            Tm[r][jj] = lr_dot4(&Y[r][0], &V[0][jj], D, 1, kLrMaxR);
+        }
+        __syncthreads();
+        if (it == kLrIters) break;
+        for (int jj = 0; jj < R; ++jj) W[c][jj] = lr_dot4(&Y[0][c], &Tm[0][jj], kBlock, D, kLrMaxR);
+        __syncthreads();
+        for (int jj = 0; jj < R; ++jj) {
+            for (int i = 0; i < jj; ++i) {
+                const float p = wdot(i, jj);
+                W[c][jj] = __fmaf_rn(-p, W[c][i], W[c][jj]);
+                __syncthreads();
+            }
+            const float n = __fsqrt_rn(wdot(jj, jj));
+            W[c][jj] = n > 0.0f ? __fdiv_rn(W[c][jj], n) : 0.0f;
+            __syncthreads();
+        }
+        for (int jj = 0; jj < R; ++jj) V[c][jj] = W[c][jj];
+        __syncthreads();
+    }
+    if (c < R) lam_sh[c] = __fmul_rn(lr_dot4(&Tm[0][c], &Tm[0][c], kBlock, kLrMaxR, kLrMaxR), 1.0f / kBlock);
+    __syncthreads();
+    if (c == 0) {
+        int ord[kLrMaxR];
+        for (int a = 0; a < R; ++a) ord[a] = a;
+        for (int a = 0; a < R; ++a)
+            for (int z = a + 1; z < R; ++z)
+                if (lam_sh[ord[z]] > lam_sh[ord[a]] || (lam_sh[ord[z]] == lam_sh[ord[a]] && ord[z] < ord[a])) {
+                    const int t = ord[a];
+                    ord[a] = ord[z];
+                    ord[z] = t;
+                }
+        for (int a = 0; a < R; ++a) ord_sh[a] = ord[a];
+    }
+    __syncthreads();
+    const size_t gf = (size_t)32 * (D + R * D + R);
+    float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
+    for (int jj = 0; jj < R; ++jj)
+        base[(size_t)(1 + jj) * D * 32 + ((size_t)(c / 4) * 32 + (j & 31)) * 4 + (c & 3)] = V[c][ord_sh[jj]];
+    if (c < R) base[(size_t)(1 + R) * D * 32 + (size_t)c * 32 + (j & 31)] = lam_sh[ord_sh[c]];
+}
+
 // grid (tokens to build, units, 2 = {K, V}), block d threads. out_i = P @ mean(rows).
 template <typename T>
 __global__ void __launch_bounds__(128) compress_kernel(const T* __restrict__ K, const T* __restrict__ V,
@@ -474,7 +593,14 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
     const int nbuild = m.nB - (j_begin < 0 ? 0 : j_begin);
     if (nbuild > 0) {
         count_launch();
-        summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
+        if (m.lr) {
+            if (m.d == 128)
+                lowrank_kernel<T, 128><<<dim3(nbuild, units), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+            else
+                lowrank_kernel<T, 64><<<dim3(nbuild, units), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+        } else {
+            summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
+        }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -521,13 +647,14 @@ cudaError_t launch_summaries(const Dims& m, const void* K, const void* V, const 
                              int t_begin, float* summ, void* Kc, void* Vc, cudaStream_t s, int* err) {
     // the decode-step update (one block, one compressed token): a small dedicated kernel
     cudaError_t ea = cudaSuccess;
-    if (m.dtype == COBS_BF16 ? try_append<__nv_bfloat16>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv,
-                                                         t_begin, summ, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s, &ea)
-                             : try_append<float>(m, (const float*)K, (const float*)V, Pk, Pv, t_begin, summ,
-                                                 (float*)Kc, (float*)Vc, s, &ea))
+    if (!m.lr && (m.dtype == COBS_BF16
+                      ? try_append<__nv_bfloat16>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv, t_begin,
+                                                  summ, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s, &ea)
+                      : try_append<float>(m, (const float*)K, (const float*)V, Pk, Pv, t_begin, summ, (float*)Kc,
+                                          (float*)Vc, s, &ea)))
         return ea;
     // fused one-pass kernel for the bf16 layout it is written for; plain kernels otherwise
-    if (m.dtype == COBS_BF16 && m.L == 64 && m.lc == 32 && m.sc == 16 && Pk != nullptr && Pv != nullptr &&
+    if (!m.lr && m.dtype == COBS_BF16 && m.L == 64 && m.lc == 32 && m.sc == 16 && Pk != nullptr && Pv != nullptr &&
         (m.d == 128 || m.d == 64) && m.nC > 0) {
         if (m.d == 128)
             return launch_fused<128>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv, t_begin, summ,

@@ -39,6 +39,9 @@
  *                  [..., 1, ...] the key variance var_{b,c}.
  *                  variance = COBS_VAR_ISOTROPIC: [B, Hkv, nG, (d/4 * 32 * 4) + 32] float32:
  *                  the means as above, then sigma2_b of the group's 32 blocks.
+ *                  variance = COBS_VAR_LOWRANK (rank R): [B, Hkv, nG, (1 + R) * (d/4 * 32 * 4) + R * 32]
+ *                  float32: the means as above, then eigenvector j < R of the group's blocks in
+ *                  the same [d/4, 32, 4] interleaving, then the R eigenvalues [R, 32].
  *                  (32 consecutive blocks are interleaved channel-by-channel so that one
  *                  group is one contiguous copy and lane b%32 reads its block's channels.)
  * - GQA: query head h belongs to KV head h / (Hq / Hkv).
@@ -75,8 +78,14 @@ typedef enum { COBS_WS_SELECT = 0, COBS_WS_DECODE = 1, COBS_WS_PREFILL = 2 } cob
  *                       score term alpha/2 * sum_c q_c^2 var_{b,c} / d.
  *   COBS_VAR_ISOTROPIC  one scalar per block ([SKILL] "Pitfalls": one or two scalars per block):
  *                       Sigma_b ~ sigma2_b I with sigma2_b = (1/d) sum_c var_{b,c};
- *                       score term alpha/2 * sigma2_b |q|^2 / d. Summaries are about half the bytes. */
-typedef enum { COBS_VAR_CHANNEL = 0, COBS_VAR_ISOTROPIC = 1 } cobs_variance;
+ *                       score term alpha/2 * sigma2_b |q|^2 / d. Summaries are about half the bytes.
+ *   COBS_VAR_LOWRANK    the `rank` leading eigenpairs (lambda_j, u_j) of Sigma_b ([COBS] §2.2/§2.3,
+ *                       low-rank compression of the covariance); score term
+ *                       alpha/2 * sum_j lambda_j (q . u_j)^2 / d. The eigenpairs come from a fixed
+ *                       float32 subspace iteration (24 steps, modified Gram-Schmidt), so they are
+ *                       reproducible bit for bit. Decode selection only (prefill selection with
+ *                       these summaries returns COBS_ERR_UNSUPPORTED). */
+typedef enum { COBS_VAR_CHANNEL = 0, COBS_VAR_ISOTROPIC = 1, COBS_VAR_LOWRANK = 2 } cobs_variance;
 
 /* Problem statement ([COBS] §2.3, [SKILL] "Method"): block size, compression block and
  * stride, top-k, window and alpha. */
@@ -94,6 +103,7 @@ typedef struct {
     float alpha;        /* weight of the second-order (variance) term */
     int32_t dtype;      /* cobs_dtype of Q, K, V, Kc, Vc, O */
     int32_t variance;   /* cobs_variance: the second-order statistic of the summaries */
+    int32_t rank;       /* eigenpairs per block for COBS_VAR_LOWRANK (1 .. 8); ignored otherwise */
 } cobs_params;
 
 /*
@@ -119,7 +129,10 @@ cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void
  * For each GQA group g and candidate block b:
  *   S_{g,b} = (sum_c Qsum_c mu_{b,c}) * RN(1/sqrt(d)) + RN(alpha/(2d)) * (sum_c Q2_c var_{b,c}),
  *   or, with COBS_VAR_ISOTROPIC summaries, ... + RN(alpha/(2d)) * RN((sum_c Q2_c) * sigma2_b)
- *   (sum_c Q2_c by adds in ascending c),
+ *   (sum_c Q2_c by adds in ascending c), or, with COBS_VAR_LOWRANK summaries,
+ *   ... + RN(alpha/(2d)) * sum_j lambda_j * (sum_{h in g} (q_h . u_j)^2) (fma, ascending j and h);
+ *   every channel sum runs as four partial chains (channels c = j mod 4) combined as
+ *   (s0 + s1) + (s2 + s3),
  *   Qsum = sum_{h in g} q_h, Q2 = sum_{h in g} q_h*q_h   (= sum_h [q_h.mu_b/sqrt(d)
  *   + alpha/2 * sum_c q_{h,c}^2 var_{b,c}/d]), evaluated in float32 with fused multiply-adds
  *   in ascending head and channel order. Candidates are the complete blocks

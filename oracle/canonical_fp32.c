@@ -30,6 +30,7 @@
 
 
 #include <math.h>
+#include <stddef.h>
 #include <stdint.h>
 
 /* sum_c x_c y_c in the canonical four-chain order (d a multiple of 4). */
@@ -148,5 +149,136 @@ void cobs_oracle_iso_scores_f32(const float* qsum, const float* q2, const float*
             const float v = q2tot * mu[d];
             S[i * nb + b] = fmaf(c2, v, a * isd);
         }
+    }
+}
+
+/*
+ * Low-rank variant. COBS §2.2/§2.3 keep the block covariance Sigma_b in compressed form, first
+ * of all as its leading eigenpairs (lambda_j, u_j), j < r: 1/2 q^T Sigma_b q ~ 1/2 sum_j
+ * lambda_j (q . u_j)^2. Per block the summary holds the mean mu_b, the r unit vectors u_j and
+ * the r values lambda_j; the score of a GQA group (the sum of its heads' scores) is
+ *   S_{g,b} = (sum_c Qsum_c mu_c) * isd + c2 * sum_j lambda_j * (sum_{h in g} (q_h . u_j)^2).
+ *
+ * The eigenpairs come from a fixed, deterministic float32 solver whose every operation this
+ * file fixes (the GPU runs the same steps in the same order, so both produce the same bits):
+ *   Y[r][c] = k_{r,c} - mu_c                       (rows r < L of the block, channels c < d)
+ *   V = V0 (d x R), V0[c][j] = +-1 by a fixed bit pattern of (c, j)
+ *   repeat LR_ITERS times:
+ *     T[r][j] = dot4_c(Y[r][.], V[.][j])            (four-chain order over c, as the scores)
+ *     W[c][j] = dot4_r(Y[.][c], T[.][j])            (four-chain order over r)
+ *     modified Gram-Schmidt over j ascending:
+ *       for i < j: p = wdot(W[.][i], W[.][j]); W[c][j] = fmaf(-p, W[c][i], W[c][j])
+ *       n = sqrtf(wdot(W[.][j], W[.][j])); W[c][j] = W[c][j] / n   (n == 0: the column is 0)
+ *     V = W
+ *   T = Y V; lambda_j = dot4_r(T[.][j], T[.][j]) * (1/L)
+ *   order the pairs by lambda descending (ties: lower j first)
+ * wdot is the "32-lane" order: partial p_l = sum over c = l, l + 32, ... (ascending, fmaf),
+ * l < 32, then five butterfly levels p_l = p_l + p_{l xor o}, o = 16, 8, 4, 2, 1; the result
+ * is p_0. sqrtf and the division are correctly rounded (IEEE).
+ * The fixed iteration count makes the result a deterministic function of the block; for
+ * well-separated leading eigenvalues it converges to the leading eigenpairs.
+ */
+#define LR_ITERS 24
+#define LR_MAXR 8
+
+static float wdot32(const float* x, const float* y, int d, int stride_x, int stride_y) {
+    float p[32];
+    for (int l = 0; l < 32; ++l) {
+        float s = 0.0f;
+        for (int c = l; c < d; c += 32) s = fmaf(x[(size_t)c * stride_x], y[(size_t)c * stride_y], s);
+        p[l] = s;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        float q[32];
+        for (int l = 0; l < 32; ++l) q[l] = p[l] + p[l ^ o];
+        for (int l = 0; l < 32; ++l) p[l] = q[l];
+    }
+    return p[0];
+}
+
+/* four-chain dot with strides (n a multiple of 4) */
+static float dot4s(const float* x, const float* y, int n, int sx, int sy) {
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+    for (int i = 0; i < n; i += 4) {
+        s0 = fmaf(x[(size_t)(i + 0) * sx], y[(size_t)(i + 0) * sy], s0);
+        s1 = fmaf(x[(size_t)(i + 1) * sx], y[(size_t)(i + 1) * sy], s1);
+        s2 = fmaf(x[(size_t)(i + 2) * sx], y[(size_t)(i + 2) * sy], s2);
+        s3 = fmaf(x[(size_t)(i + 3) * sx], y[(size_t)(i + 3) * sy], s3);
+    }
+    return (s0 + s1) + (s2 + s3);
+}
+
+/* The fixed start V0[c][j]: +1 or -1 by bit 11 of (c * 2654435761 + (j + 1) * 40503) (32-bit). */
+static float lr_v0(int c, int j) {
+    const uint32_t h = (uint32_t)c * 2654435761u + (uint32_t)(j + 1) * 40503u;
+    return ((h >> 11) & 1u) ? 1.0f : -1.0f;
+}
+
+/*
+ * K: [T][d] float32 rows; mu: [nb][d] canonical block means (cobs_oracle_summaries_f32);
+ * out_u: [nb][R][d] eigenvectors, out_l: [nb][R] eigenvalues (descending).
+ */
+void cobs_oracle_lowrank_f32(const float* K, const float* mu, int64_t nb, int d, int L, int R, float* out_u,
+                             float* out_l) {
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; ++b) {
+        float Y[64 * 128], V[128 * LR_MAXR], W[128 * LR_MAXR], T[64 * LR_MAXR], lam[LR_MAXR];
+        const float* m = mu + b * d;
+        for (int r = 0; r < L; ++r)
+            for (int c = 0; c < d; ++c) Y[r * d + c] = K[(b * L + r) * (int64_t)d + c] - m[c];
+        for (int c = 0; c < d; ++c)
+            for (int j = 0; j < R; ++j) V[c * R + j] = lr_v0(c, j);
+        for (int it = 0; it <= LR_ITERS; ++it) {
+            for (int r = 0; r < L; ++r)
+                for (int j = 0; j < R; ++j) T[r * R + j] = dot4s(Y + r * d, V + j, d, 1, R);
+            if (it == LR_ITERS) break;
+            for (int c = 0; c < d; ++c)
+                for (int j = 0; j < R; ++j) W[c * R + j] = dot4s(Y + c, T + j, L, d, R);
+            for (int j = 0; j < R; ++j) {
+                for (int i = 0; i < j; ++i) {
+                    const float p = wdot32(W + i, W + j, d, R, R);
+                    for (int c = 0; c < d; ++c) W[c * R + j] = fmaf(-p, W[c * R + i], W[c * R + j]);
+                }
+                const float n = sqrtf(wdot32(W + j, W + j, d, R, R));
+                for (int c = 0; c < d; ++c) W[c * R + j] = n > 0.0f ? W[c * R + j] / n : 0.0f;
+            }
+            for (int e = 0; e < d * R; ++e) V[e] = W[e];
+        }
+        for (int j = 0; j < R; ++j) lam[j] = dot4s(T + j, T + j, L, R, R) * (1.0f / (float)L);
+        /* order by lambda descending, ties by j (stable selection) */
+        int ord[LR_MAXR];
+        for (int j = 0; j < R; ++j) ord[j] = j;
+        for (int a = 0; a < R; ++a)
+            for (int z = a + 1; z < R; ++z)
+                if (lam[ord[z]] > lam[ord[a]] || (lam[ord[z]] == lam[ord[a]] && ord[z] < ord[a])) {
+                    const int t = ord[a]; ord[a] = ord[z]; ord[z] = t;
+                }
+        for (int j = 0; j < R; ++j) {
+            out_l[b * R + j] = lam[ord[j]];
+            for (int c = 0; c < d; ++c) out_u[(b * R + j) * d + c] = V[c * R + ord[j]];
+        }
+    }
+}
+
+/*
+ * Low-rank group scores. q: [G][d] the group's query heads (exact float32 values); qsum: [d]
+ * (cobs_oracle_group_query_f32); mu: [nb][d]; u: [nb][R][d]; lam: [nb][R]; S: [nb].
+ *   a = dot4(qsum, mu_b); for j: e_j = sum over h ascending of fmaf(p, p, .) with p = dot4(q_h, u_j);
+ *   v = sum over j ascending of fmaf(lam_j, e_j, .); S = fmaf(c2, v, a * isd).
+ */
+void cobs_oracle_lowrank_scores_f32(const float* q, const float* qsum, int G, const float* mu, const float* u,
+                                    const float* lam, int64_t nb, int d, int R, float isd, float c2, float* S) {
+    for (int64_t b = 0; b < nb; ++b) {
+        const float a = dot4s(qsum, mu + b * d, d, 1, 1);
+        float v = 0.0f;
+        for (int j = 0; j < R; ++j) {
+            float e = 0.0f;
+            for (int h = 0; h < G; ++h) {
+                const float p = dot4s(q + h * d, u + (b * R + j) * d, d, 1, 1);
+                e = fmaf(p, p, e);
+            }
+            v = fmaf(lam[b * R + j], e, v);
+        }
+        S[b] = fmaf(c2, v, a * isd);
     }
 }

@@ -69,6 +69,10 @@ def _c():
         lib.cobs_oracle_iso_summaries_f32.restype = None
         lib.cobs_oracle_iso_scores_f32.argtypes = [vp, vp, vp, i64, i64, i32, f32, f32, vp]
         lib.cobs_oracle_iso_scores_f32.restype = None
+        lib.cobs_oracle_lowrank_f32.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp]
+        lib.cobs_oracle_lowrank_f32.restype = None
+        lib.cobs_oracle_lowrank_scores_f32.argtypes = [vp, vp, i32, vp, vp, vp, i64, i32, i32, f32, f32, vp]
+        lib.cobs_oracle_lowrank_scores_f32.restype = None
         _clib = lib
     return _clib
 
@@ -173,6 +177,45 @@ def canonical_scores_iso(qsum: np.ndarray, q2: np.ndarray, summ_iso: np.ndarray,
     return S
 
 
+class LowRank(tuple):
+    """Low-rank block summaries: (mu [nB, d], u [nB, R, d], lam [nB, R]), float32."""
+
+
+def canonical_summaries_lowrank(K32: np.ndarray, L: int, R: int) -> LowRank:
+    """float32 low-rank summaries: the block mean and the R leading eigenpairs of the block
+    covariance from the fixed float32 solver of canonical_fp32.c.
+
+    [COBS] §2.2/§2.3: the second cumulant kappa_2 = Sigma_b kept as its leading eigenpairs
+    (the low-rank compression of the block covariance).
+    """
+    K32 = _f32c(K32)
+    T, d = K32.shape
+    nB = T // L
+    mu = np.ascontiguousarray(canonical_summaries(K32, L)[:, 0, :])
+    u = np.zeros((nB, R, d), np.float32)
+    lam = np.zeros((nB, R), np.float32)
+    if nB:
+        _c().cobs_oracle_lowrank_f32(K32.ctypes.data, mu.ctypes.data, nB, d, L, R, u.ctypes.data, lam.ctypes.data)
+    return LowRank((mu, u, lam))
+
+
+def canonical_scores_lowrank(q_group32: np.ndarray, summ: LowRank, alpha: float) -> np.ndarray:
+    """float32 group scores [nB] of one group's query heads [G, d] against low-rank summaries:
+    (sum_c Qsum_c mu_c) isd + c2 sum_j lam_j sum_h (q_h . u_j)^2. Canonical order: canonical_fp32.c."""
+    mu, u, lam = summ
+    q = _f32c(q_group32)
+    G, d = q.shape
+    qs, _ = canonical_group_query(q)
+    qs = _f32c(qs)
+    isd, c2 = score_constants(d, alpha)
+    S = np.empty(mu.shape[0], np.float32)
+    if mu.shape[0]:
+        _c().cobs_oracle_lowrank_scores_f32(q.ctypes.data, qs.ctypes.data, G, _f32c(mu).ctypes.data,
+                                            _f32c(u).ctypes.data, _f32c(lam).ctypes.data, mu.shape[0], d,
+                                            u.shape[1], float(isd), float(c2), S.ctypes.data)
+    return S
+
+
 # ----------------------------------------------------------------------------------
 # float64 steps
 # ----------------------------------------------------------------------------------
@@ -252,6 +295,40 @@ def head_scores_iso(q: np.ndarray, mu: np.ndarray, sigma2: np.ndarray, alpha: fl
 def group_scores_iso(qs: np.ndarray, mu: np.ndarray, sigma2: np.ndarray, alpha: float) -> np.ndarray:
     """Sum of head_scores_iso over the G query heads qs [G, d] (the group-sum reading)."""
     return sum(head_scores_iso(q, mu, sigma2, alpha) for q in qs)
+
+
+def block_eigenpairs(K: np.ndarray, L: int, R: int):
+    """Block mean mu [nB, d] and the R leading eigenpairs (u [nB, R, d], lam [nB, R]) of the
+    population covariance Sigma_b = (1/L) sum_r (k_r - mu_b)(k_r - mu_b)^T, float64 (numpy eigh).
+
+    [COBS] §2.2/§2.3: kappa_2 = Sigma_b, compressed to its leading eigenpairs.
+    """
+    T, d = K.shape
+    nB = T // L
+    mu = np.zeros((nB, d))
+    u = np.zeros((nB, R, d))
+    lam = np.zeros((nB, R))
+    for b in range(nB):
+        rows = K[b * L:(b + 1) * L]
+        mu[b] = rows.sum(axis=0) / L
+        Y = rows - mu[b]
+        w, vecs = np.linalg.eigh(Y.T @ Y / L)
+        order = np.argsort(-w, kind="stable")[:R]
+        lam[b] = w[order]
+        u[b] = vecs[:, order].T
+    return mu, u, lam
+
+
+def head_scores_lowrank(q: np.ndarray, mu: np.ndarray, u: np.ndarray, lam: np.ndarray, alpha: float) -> np.ndarray:
+    """Low-rank per-head score: q.mu_b/sqrt(d) + alpha * 1/2 * sum_j lam_j (q . u_j)^2 / d
+    (the second cumulant 1/2 q^T Sigma_b q / d with Sigma_b ~ sum_j lam_j u_j u_j^T)."""
+    d = q.shape[-1]
+    return (mu @ q) / np.sqrt(d) + alpha * 0.5 * ((u @ q) ** 2 * lam).sum(axis=-1) / d
+
+
+def group_scores_lowrank(qs: np.ndarray, mu, u, lam, alpha: float) -> np.ndarray:
+    """Sum of head_scores_lowrank over the G query heads qs [G, d] (the group-sum reading)."""
+    return sum(head_scores_lowrank(q, mu, u, lam, alpha) for q in qs)
 
 
 def n_candidates(t: int, L: int) -> int:
@@ -358,7 +435,11 @@ def unit_cache(w, Kst: np.ndarray, Vst: np.ndarray, Pk, Pv):
 def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
     """Selected blocks [k] for the decode query at position T-1 of one (batch, group).
 
-    summ: canonical summaries [nB, 2, d] (per-channel variance) or [nB, d + 1] (isotropic)."""
+    summ: canonical summaries [nB, 2, d] (per-channel variance), [nB, d + 1] (isotropic) or a
+    LowRank triple (mean, eigenvectors, eigenvalues)."""
+    if isinstance(summ, LowRank):
+        S = canonical_scores_lowrank(q_group32, summ, w.alpha)
+        return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
     qs, q2 = canonical_group_query(q_group32)
     if summ.ndim == 2:
         S = canonical_scores_iso(qs[None], q2[None], summ, w.alpha)[0]
@@ -367,10 +448,11 @@ def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
     return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
 
 
-def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel"):
+def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", rank=4):
     """Decode at position T-1 for every (batch, KV head) unit (or the listed units).
 
-    variance: "channel" (per-channel variance summaries) or "isotropic" (one scalar per block).
+    variance: "channel" (per-channel variance summaries), "isotropic" (one scalar per block) or
+    "lowrank" (the rank leading eigenpairs of each block's covariance).
 
     Returns dict with idx [B, Hkv, k], O [B, Hq, d] (float64; rows of unlisted units are NaN),
     summ, Kc, Vc per computed unit, and near-tie reports (units where the float64 ranking of
@@ -387,12 +469,21 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel"):
         K, V, summ, Kc, Vc = unit_cache(w, K_all[b, h], V_all[b, h], Pk, Pv)
         cache[(b, h)] = (summ, Kc, Vc)
         qs = Qf[b, h * G:(h + 1) * G]
-        iso = variance == "isotropic"
-        sel, _ = select_decode(w, qs.astype(np.float32),
-                               canonical_summaries_iso(K.astype(np.float32), w.block) if iso else summ)
+        if variance == "isotropic":
+            sel_summ = canonical_summaries_iso(K.astype(np.float32), w.block)
+        elif variance == "lowrank":
+            sel_summ = canonical_summaries_lowrank(K.astype(np.float32), w.block, rank)
+        else:
+            sel_summ = summ
+        sel, _ = select_decode(w, qs.astype(np.float32), sel_summ)
         idx[b, h] = sel
         mu, var = block_summaries(K, w.block)
-        S64 = group_scores_iso(qs, mu, var.mean(axis=1), w.alpha) if iso else group_scores(qs, mu, var, w.alpha)
+        if variance == "isotropic":
+            S64 = group_scores_iso(qs, mu, var.mean(axis=1), w.alpha)
+        elif variance == "lowrank":
+            S64 = group_scores_lowrank(qs, *block_eigenpairs(K, w.block, rank), w.alpha)
+        else:
+            S64 = group_scores(qs, mu, var, w.alpha)
         sel64 = top_k(S64, n_candidates(t, w.block), w.topk)
         if not np.array_equal(sel, sel64):
             near_ties.append((b, h))

@@ -28,10 +28,11 @@ def f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def params_of(w, variance="channel"):
+def params_of(w, variance="channel", rank=4):
     C = cobs()
     return C.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
-                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype, variance=variance)
+                    cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype, variance=variance,
+                    rank=rank)
 
 
 def summaries_blocks(flat, p):
@@ -39,6 +40,19 @@ def summaries_blocks(flat, p):
     (per-channel variance) or [B, Hkv, nB, d + 1] (isotropic: means, then the block's scalar)."""
     nB = p.T // p.block
     nG = max(1, -(-nB // 32))
+    if p.variance == "lowrank":
+        R, d = p.rank, p.d
+        gf = 32 * (d + R * d + R)
+        a = flat[: p.B * p.Hkv * nG * gf].cpu().numpy().reshape(p.B, p.Hkv, nG, gf)
+
+        def planes(x, n):   # [B, Hkv, nG, n, d/4, 32, 4] -> [B, Hkv, nG*32, n, d]
+            x = x.reshape(p.B, p.Hkv, nG, n, d // 4, 32, 4).transpose(0, 1, 2, 5, 3, 4, 6)
+            return x.reshape(p.B, p.Hkv, nG * 32, n, d)
+        mu = planes(a[..., :d * 32], 1)[:, :, :nB, 0]
+        u = planes(a[..., d * 32:(1 + R) * d * 32], R)[:, :, :nB]
+        lam = a[..., (1 + R) * d * 32:].reshape(p.B, p.Hkv, nG, R, 32).transpose(0, 1, 2, 4, 3)
+        lam = lam.reshape(p.B, p.Hkv, nG * 32, R)[:, :, :nB]
+        return mu, u, lam
     if p.variance == "isotropic":
         gf = (p.d + 1) * 32
         a = flat[: p.B * p.Hkv * nG * gf].cpu().numpy().reshape(p.B, p.Hkv, nG, gf)
@@ -51,9 +65,9 @@ def summaries_blocks(flat, p):
     return a.reshape(p.B, p.Hkv, nG * 32, 2, p.d)[:, :, :nB]
 
 
-def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel"):
+def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel", rank=4):
     C = cobs()
-    p = params_of(w, variance)
+    p = params_of(w, variance, rank)
     buf = C.alloc(p, prefill=False)
     C.device_error(reset=True)
     C.decode_step(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),

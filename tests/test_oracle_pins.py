@@ -529,3 +529,107 @@ def test_iso_canonical_matches_exact_rational_emulation():
         a = _dot4_exact(F, qsum, iso[b, :d])
         v = _rn32(q2tot * F(iso[b, d]))
         assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
+
+
+# ---------------------------------------------------------------- low-rank covariance variant
+
+def _aniso_blocks(rng, nB, L, d, spectrum, noise):
+    U, _ = np.linalg.qr(rng.standard_normal((d, len(spectrum))))
+    mu = rng.standard_normal((nB, 1, d)) * 0.5
+    Z = rng.standard_normal((nB, L, len(spectrum))) * np.asarray(spectrum)
+    return (mu + Z @ U.T + noise * rng.standard_normal((nB, L, d))).reshape(nB * L, d)
+
+
+def test_lowrank_solver_matches_library_eigh():
+    """The fixed float32 subspace iteration reaches numpy's eigh on well-separated spectra."""
+    rng = np.random.default_rng(31)
+    L, d, R, nB = 64, 128, 4, 8
+    K = _aniso_blocks(rng, nB, L, d, [3.0, 2.2, 1.6, 1.2, 0.5, 0.3], 0.05).astype(np.float32)
+    mu32, u32, lam32 = O.canonical_summaries_lowrank(K, L, R)
+    mu, u, lam = O.block_eigenpairs(K.astype(np.float64), L, R)
+    assert np.allclose(mu32, mu, atol=1e-6)
+    assert np.abs(lam32 / lam - 1).max() < 1e-4
+    cos = np.abs(np.einsum("brd,brd->br", u32.astype(np.float64), u))
+    assert cos.min() > 0.9999
+    assert np.all(np.diff(lam32, axis=1) <= 0)   # descending
+
+
+def test_lowrank_score_is_the_covariance_quadratic_form_for_low_rank_blocks():
+    """Blocks whose keys span an R-dimensional affine subspace: sum_j lam_j (q.u_j)^2 = q^T Sigma q,
+    so the low-rank score equals the full second-order score (float64 definitions)."""
+    rng = np.random.default_rng(32)
+    L, d, R, nB, G = 64, 32, 3, 5, 4
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.0, 0.5], 0.0)
+    mu, u, lam = O.block_eigenpairs(K, L, R)
+    qs = rng.standard_normal((G, d))
+    full = np.zeros(nB)
+    for b in range(nB):
+        Y = K[b * L:(b + 1) * L] - mu[b]
+        S = Y.T @ Y / L
+        full[b] = sum(q @ mu[b] / math.sqrt(d) + 0.5 * (q @ S @ q) / d for q in qs)
+    assert np.allclose(O.group_scores_lowrank(qs, mu, u, lam, 1.0), full, rtol=0, atol=1e-10)
+    # a rank-R truncation of a rank-(R+2) block loses the smallest directions
+    K2 = _aniso_blocks(rng, nB, L, d, [2.0, 1.0, 0.5, 0.4, 0.3], 0.0)
+    mu2, u2, lam2 = O.block_eigenpairs(K2, L, R)
+    mu5, u5, lam5 = O.block_eigenpairs(K2, L, R + 2)
+    assert np.all(O.group_scores_lowrank(qs, mu2, u2, lam2, 1.0) <= O.group_scores_lowrank(qs, mu5, u5, lam5, 1.0) + 1e-12)
+
+
+def test_lowrank_axis_aligned_block_equals_per_channel_score():
+    """Variance in R channels only (a diagonal covariance): the eigenvectors are those axes and
+    the low-rank score equals the per-channel-variance score."""
+    rng = np.random.default_rng(33)
+    L, d, R, nB, G = 64, 16, 3, 4, 3
+    # deviations along R channels by mutually orthogonal, zero-mean +-1 patterns (rows of a
+    # Sylvester-Hadamard matrix other than the first): the block covariance is exactly diagonal
+    H = np.array([[1.0]])
+    while H.shape[0] < L:
+        H = np.block([[H, H], [H, -H]])
+    K = np.repeat(rng.standard_normal((nB, 1, d)), L, axis=1)
+    for b in range(nB):
+        chans = rng.choice(d, size=R, replace=False)
+        amps = np.sort(rng.uniform(0.5, 2.0, size=R))[::-1] + np.arange(R)[::-1] * 0.3  # distinct
+        for i, c in enumerate(chans):
+            K[b][:, c] += amps[i] * H[1 + 3 * i]
+    K = K.reshape(nB * L, d)
+    mu, var = O.block_summaries(K, L)
+    mu2, u, lam = O.block_eigenpairs(K, L, R)
+    qs = rng.standard_normal((G, d))
+    assert np.allclose(O.group_scores_lowrank(qs, mu2, u, lam, 1.0), O.group_scores(qs, mu, var, 1.0), atol=1e-10)
+
+
+def test_lowrank_alpha_zero_is_first_order():
+    rng = np.random.default_rng(34)
+    L, d, R, nB, G = 64, 64, 4, 24, 4
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.5, 1.0, 0.7, 0.4], 0.1).astype(np.float32)
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    S = O.canonical_scores_lowrank(q, O.canonical_summaries_lowrank(K, L, R), 0.0)
+    pooled = K.astype(np.float64).reshape(nB, L, d).mean(axis=1)
+    ref = np.sort(np.argsort(-(pooled @ q.astype(np.float64).sum(axis=0)), kind="stable")[:8])
+    assert list(O.top_k(S, nB, 8)) == list(ref)
+
+
+def test_lowrank_scores_match_exact_rational_emulation():
+    """Brute force: the low-rank score's float32 steps as exact rationals rounded once each."""
+    rng = np.random.default_rng(35)
+    L, d, R, nB, G = 64, 16, 2, 3, 3
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.0, 0.4], 0.05).astype(np.float32)
+    summ = O.canonical_summaries_lowrank(K, L, R)
+    mu, u, lam = summ
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    alpha = np.float32(0.9)
+    S = O.canonical_scores_lowrank(q, summ, float(alpha))
+    qsum, _ = O.canonical_group_query(q)
+    F = lambda v: Fraction(float(v))
+    isd = _rn32(Fraction(1.0 / math.sqrt(d)))
+    c2 = _rn32(F(alpha) / (2 * d))
+    for b in range(nB):
+        a = _dot4_exact(F, qsum, mu[b])
+        v = Fraction(0)
+        for j in range(R):
+            e = Fraction(0)
+            for h in range(G):
+                pj = _dot4_exact(F, q[h], u[b, j])
+                e = _rn32(pj * pj + e)
+            v = _rn32(F(lam[b, j]) * e + v)
+        assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
