@@ -110,7 +110,7 @@ __device__ __forceinline__ float lr_dot4(const float* x, const float* y, int n, 
 template <typename T, int D>
 __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
                                                     float* __restrict__ summ) {
-    __shared__ float Y[kBlock][D];
+    __shared__ float Y[kBlock][D + 1];  // +1: rows on different banks
     __shared__ float V[D][kLrMaxR], W[D][kLrMaxR];
     __shared__ float Tm[kBlock][kLrMaxR];
     __shared__ float bcast;
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
         }
         __syncthreads();
         if (it == kLrIters) break;
-        for (int jj = 0; jj < R; ++jj) W[c][jj] = lr_dot4(&Y[0][c], &Tm[0][jj], kBlock, D, kLrMaxR);
+        for (int jj = 0; jj < R; ++jj) W[c][jj] = lr_dot4(&Y[0][c], &Tm[0][jj], kBlock, D + 1, kLrMaxR);
         __syncthreads();
         for (int jj = 0; jj < R; ++jj) {
             for (int i = 0; i < jj; ++i) {
@@ -632,14 +632,25 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
     const int i_begin = num <= 0 ? 0 : (num + m.sc - 1) / m.sc;
     const int nj = m.nB - j_begin, ni = m.nC - i_begin;
     if (nj > 1 || ni > 1) return false;
-    if (nj <= 0 && ni <= 0) {
-        *e = cudaSuccess;
-        return true;
+    *e = cudaSuccess;
+    // low-rank summaries: the block goes to the eigen-solver, the token to the append kernel
+    const bool block_here = nj > 0 && !m.lr;
+    if (block_here || ni > 0) {
+        count_launch();
+        append_kernel<T><<<dim3(m.units(), 4), 256, 0, s>>>(K, V, Pk, Pv, m.T, m.d, m.nG, m.nC, m.lc, m.sc,
+                                                            block_here ? j_begin : -1, ni > 0 ? i_begin : -1, m.iso,
+                                                            summ, Kc, Vc);
+        *e = cudaGetLastError();
+        if (*e != cudaSuccess) return true;
     }
-    count_launch();
-    append_kernel<T><<<dim3(m.units(), 4), 256, 0, s>>>(K, V, Pk, Pv, m.T, m.d, m.nG, m.nC, m.lc, m.sc, nj > 0 ? j_begin : -1,
-                                               ni > 0 ? i_begin : -1, m.iso, summ, Kc, Vc);
-    *e = cudaGetLastError();
+    if (nj > 0 && m.lr) {
+        count_launch();
+        if (m.d == 128)
+            lowrank_kernel<T, 128><<<dim3(1, m.units()), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+        else
+            lowrank_kernel<T, 64><<<dim3(1, m.units()), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+        *e = cudaGetLastError();
+    }
     return true;
 }
 
@@ -647,7 +658,7 @@ cudaError_t launch_summaries(const Dims& m, const void* K, const void* V, const 
                              int t_begin, float* summ, void* Kc, void* Vc, cudaStream_t s, int* err) {
     // the decode-step update (one block, one compressed token): a small dedicated kernel
     cudaError_t ea = cudaSuccess;
-    if (!m.lr && (m.dtype == COBS_BF16
+    if ((m.dtype == COBS_BF16
                       ? try_append<__nv_bfloat16>(m, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, Pk, Pv, t_begin,
                                                   summ, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, s, &ea)
                       : try_append<float>(m, (const float*)K, (const float*)V, Pk, Pv, t_begin, summ, (float*)Kc,

@@ -47,7 +47,8 @@ def test_lowrank_decode_matches_oracle(name, over, R):
             assert np.abs(O_g[b, h * G:(h + 1) * G] - out).max() <= TOL[w.dtype]
 
 
-def test_lowrank_incremental_update_matches_full_build():
+@pytest.mark.parametrize("back", [1, 64])   # t_begin = T - 1 (the decode-step path) and T - 64
+def test_lowrank_incremental_update_matches_full_build(back):
     C = cobs()
     w = synth.WORKLOADS["decode32k"].replace(B=1, Hkv=2, Hq=8, T=4096)
     K, V, Q, g, Pk, Pv = inputs_decode(w)
@@ -64,15 +65,18 @@ def test_lowrank_incremental_update_matches_full_build():
     view = inc.summaries.view(p.B, p.Hkv, -1, gf)
     grp = (nb - 1) // 32
     view[:, :, grp] = float("nan")  # the whole group of the last block
-    C.cobs_build_summaries(p, tK, tV, tPk, tPv, w.T - 1 - 63, inc.summaries, inc.Kc, inc.Vc)
+    C.cobs_build_summaries(p, tK, tV, tPk, tPv, w.T - back, inc.summaries, inc.Kc, inc.Vc)
     torch.cuda.synchronize()
-    # rows T-64 .. T-1 rewrite exactly the last block; the poisoned lanes of earlier blocks in
-    # the group stay poisoned, so compare the last block only, bit for bit
+    # the update rewrites exactly the last block; the poisoned lanes of earlier blocks in the
+    # group stay poisoned, so compare the last block only, bit for bit (and the compressed
+    # tokens the update rewrote within one bf16 ulp of the full build)
     mu_f, u_f, lam_f = summaries_blocks(full.summaries, p)
     mu_i, u_i, lam_i = summaries_blocks(inc.summaries, p)
     assert np.array_equal(mu_i[:, :, nb - 1], mu_f[:, :, nb - 1])
     assert np.array_equal(u_i[:, :, nb - 1], u_f[:, :, nb - 1])
     assert np.array_equal(lam_i[:, :, nb - 1], lam_f[:, :, nb - 1])
+    from gpu_common import kc_close
+    assert kc_close(f64(inc.Kc[:, :, -1]), f64(full.Kc[:, :, -1]), "bf16").all()
 
 
 def test_lowrank_prefill_selection_is_rejected():
