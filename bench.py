@@ -44,6 +44,8 @@ def parse():
                     help="second-order statistic of the summaries (per-channel variance, one scalar per block, "
                          "or the leading eigenpairs of each block's covariance)")
     ap.add_argument("--rank", type=int, default=4, help="eigenpairs per block with --variance lowrank")
+    ap.add_argument("--aniso", type=int, default=0,
+                    help="sweep: draw anisotropic key blocks (spread on this many directions) instead of isotropic")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
     ap.add_argument("--T", type=int, default=None, help="override the context length (small profiling cases)")
@@ -660,7 +662,7 @@ def run_sweep(args):
         with torch.cuda.stream(stream):
             for b in range(w.B):
                 for h in range(w.Hkv):
-                    synth.keys_unit_on_device(w, b, h, Kb[h], stream=stream)
+                    synth.keys_unit_on_device(w, b, h, Kb[h], stream=stream, aniso_rank=args.aniso)
                 cobs.cobs_build_summaries(p1, Kb, Kb, tPk, tPv, 0, summ[b * per_b:(b + 1) * per_b], Kc, Vc)
                 if b < n_rec:
                     cobs.cobs_block_log_mass(p1, tQ[b:b + 1], Kb, mass[b:b + 1])
@@ -718,7 +720,8 @@ def run_sweep(args):
     line = {"metric": "selector GB/s over context length (decode selection, 64 x 8 units, top-16)",
             "value": top["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": n_rep, "warmup": max(3, args.warmup),
             "ms_per_step": top["us"] * 1e-3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic (keys drawn on the device)",
+            "dtype": "f32", "data": "synthetic (keys drawn on the device" +
+                                    (f", anisotropic blocks of rank {args.aniso})" if args.aniso else ")"),
             "config": {"workload": "sweep", "B": base.B, "Hq": base.Hq, "Hkv": base.Hkv, "d": base.d,
                        "topk": base.topk, "contexts": contexts, "variance": args.variance, "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
             "roofline": {"bound": "hbm", "kernel": "select_decode_kernel", "achieved": top["gbs"], "peak": peak,

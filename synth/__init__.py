@@ -41,6 +41,7 @@ _lib = None
 
 # stream tags
 TAG_KMU, TAG_KSIG, TAG_KZ, TAG_V, TAG_Q, TAG_GATE, TAG_PK, TAG_PV, TAG_NEEDLE, TAG_NMU = range(1, 11)
+TAG_KU = 11  # per-block direction bases of the anisotropic key model
 
 
 def build(force: bool = False) -> str:
@@ -344,15 +345,21 @@ def _cu():
         vp, u64, i64 = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int64
         lib.synth_gpu_block_rows_bf16.argtypes = [u64, vp, vp, i64, i64, i64, i64, vp, vp]
         lib.synth_gpu_block_rows_bf16.restype = ctypes.c_int
+        lib.synth_gpu_aniso_rows_bf16.argtypes = [u64, u64, vp, vp, i64, i64, i64, i64, ctypes.c_int, vp, vp]
+        lib.synth_gpu_aniso_rows_bf16.restype = ctypes.c_int
         _cu_lib = lib
     return _cu_lib
 
 
-def keys_unit_on_device(w: Workload, b: int, h: int, out, T: Optional[int] = None, stream=None) -> None:
+def keys_unit_on_device(w: Workload, b: int, h: int, out, T: Optional[int] = None, stream=None,
+                        aniso_rank: int = 0) -> None:
     """Fill a CUDA bf16 tensor out [T, d] with the keys of unit (b, h), drawn on the device.
 
     Same streams and distribution as keys_unit; the device's double-precision log/cos may put a
     value on a neighbouring bf16. Use keys_unit where both sides must see identical bytes.
+    aniso_rank > 0 draws the anisotropic model instead: each block's spread sigma_j concentrated
+    on aniso_rank seeded directions with variances decaying by halves, plus 10% isotropic noise
+    (device only; for measurements that compare selectors, not for bit-exact parity).
     """
     import torch
     T = w.T if T is None else T
@@ -361,8 +368,13 @@ def keys_unit_on_device(w: Workload, b: int, h: int, out, T: Optional[int] = Non
     dmu = torch.from_numpy(mu).to(out.device)
     dsig = torch.from_numpy(sigma).to(out.device)
     s = torch.cuda.current_stream(out.device) if stream is None else stream
-    rc = _cu().synth_gpu_block_rows_bf16(key(w.seed, TAG_KZ, b, h), dmu.data_ptr(), dsig.data_ptr(), mu.shape[0],
-                                         T, w.d, w.block, out.data_ptr(), s.cuda_stream)
+    if aniso_rank > 0:
+        rc = _cu().synth_gpu_aniso_rows_bf16(key(w.seed, TAG_KZ, b, h), key(w.seed, TAG_KU, b, h), dmu.data_ptr(),
+                                             dsig.data_ptr(), mu.shape[0], T, w.d, w.block, int(aniso_rank),
+                                             out.data_ptr(), s.cuda_stream)
+    else:
+        rc = _cu().synth_gpu_block_rows_bf16(key(w.seed, TAG_KZ, b, h), dmu.data_ptr(), dsig.data_ptr(),
+                                             mu.shape[0], T, w.d, w.block, out.data_ptr(), s.cuda_stream)
     if rc != 0:
         raise RuntimeError(f"device generator launch failed ({rc})")
     s.synchronize()  # dmu / dsig go out of scope
