@@ -282,3 +282,59 @@ void cobs_oracle_lowrank_scores_f32(const float* q, const float* qsum, int G, co
         S[b] = fmaf(c2, v, a * isd);
     }
 }
+
+/*
+ * FP4 variant of the low-rank summaries (COBS §2.3: the eigenvectors stored in FP4, E2M1, and
+ * the mean in BF16). From the canonical float32 mean and eigenvectors above:
+ *   mean:  mu'_c = RN_bf16(mu_c)  (round to nearest, ties to even, as a float32 value)
+ *   vector j: a = max_c |u_c|; s = a / 6 (float32 division); code_c = E2M1(u_c / s), u'_c = (+-m) * s
+ *     where E2M1 rounds |x| to the nearest of the magnitudes m = 0, 0.5, 1, 1.5, 2, 3, 4, 6 (ties to
+ *     the even magnitude index, |x| > 6 saturates to 6) and keeps the sign (a zero magnitude has
+ *     code 0); s = 0 gives code 0 everywhere.
+ * The eigenvalues stay float32; the score is the low-rank score of (mu', u', lambda).
+ */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+int cobs_oracle_e2m1_code(float x) {
+    const float a = fabsf(x);
+    int best = 0;
+    float bd = a;  /* distance to magnitude 0 */
+    for (int i = 1; i < 8; ++i) {
+        const float dist = fabsf(a - kE2M1[i]);
+        if (dist < bd || (dist == bd && (i & 1) == 0)) {
+            best = i;
+            bd = dist;
+        }
+    }
+    if (a > 6.0f) best = 7;
+    if (best == 0) return 0;
+    return (x < 0.0f ? 8 : 0) | best;
+}
+
+float cobs_oracle_bf16_rn(float x) {
+    union { float f; uint32_t u; } v;
+    v.f = x;
+    v.u = (v.u + 0x7FFFu + ((v.u >> 16) & 1u)) & 0xFFFF0000u;
+    return v.f;
+}
+
+/* mu: [nb][d] -> mu_q [nb][d]; u: [nb][R][d] -> codes [nb][R][d] (0..15), scales [nb][R], u_q [nb][R][d]. */
+void cobs_oracle_lowrank_fp4_f32(const float* mu, const float* u, int64_t nb, int d, int R, float* mu_q,
+                                 uint8_t* codes, float* scales, float* u_q) {
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int c = 0; c < d; ++c) mu_q[b * d + c] = cobs_oracle_bf16_rn(mu[b * d + c]);
+        for (int j = 0; j < R; ++j) {
+            const float* x = u + (b * R + j) * (int64_t)d;
+            float a = 0.0f;
+            for (int c = 0; c < d; ++c) a = fmaxf(a, fabsf(x[c]));
+            const float s = a / 6.0f;
+            scales[b * R + j] = s;
+            for (int c = 0; c < d; ++c) {
+                const int code = s > 0.0f ? cobs_oracle_e2m1_code(x[c] / s) : 0;
+                codes[(b * R + j) * (int64_t)d + c] = (uint8_t)code;
+                const float m = (code & 8) ? -kE2M1[code & 7] : kE2M1[code & 7];
+                u_q[(b * R + j) * (int64_t)d + c] = m * s;
+            }
+        }
+    }
+}

@@ -73,6 +73,12 @@ def _c():
         lib.cobs_oracle_lowrank_f32.restype = None
         lib.cobs_oracle_lowrank_scores_f32.argtypes = [vp, vp, i32, vp, vp, vp, i64, i32, i32, f32, f32, vp]
         lib.cobs_oracle_lowrank_scores_f32.restype = None
+        lib.cobs_oracle_lowrank_fp4_f32.argtypes = [vp, vp, i64, i32, i32, vp, vp, vp, vp]
+        lib.cobs_oracle_lowrank_fp4_f32.restype = None
+        lib.cobs_oracle_e2m1_code.argtypes = [f32]
+        lib.cobs_oracle_e2m1_code.restype = i32
+        lib.cobs_oracle_bf16_rn.argtypes = [f32]
+        lib.cobs_oracle_bf16_rn.restype = f32
         _clib = lib
     return _clib
 
@@ -197,6 +203,36 @@ def canonical_summaries_lowrank(K32: np.ndarray, L: int, R: int) -> LowRank:
     if nB:
         _c().cobs_oracle_lowrank_f32(K32.ctypes.data, mu.ctypes.data, nB, d, L, R, u.ctypes.data, lam.ctypes.data)
     return LowRank((mu, u, lam))
+
+
+class LowRankFP4(tuple):
+    """FP4 low-rank summaries: (mu_q [nB, d] bf16 values as float32, codes [nB, R, d] uint8,
+    scales [nB, R] float32, lam [nB, R] float32, u_q [nB, R, d] the dequantized vectors)."""
+
+    def dequantized(self) -> LowRank:
+        mu_q, _, _, lam, u_q = self
+        return LowRank((mu_q, u_q, lam))
+
+
+def e2m1_code(x: float) -> int:
+    """E2M1 (FP4) code of x: nearest magnitude of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even
+    index, saturating; sign in bit 3 (canonical_fp32.c)."""
+    return int(_c().cobs_oracle_e2m1_code(float(x)))
+
+
+def canonical_summaries_lowrank_fp4(K32: np.ndarray, L: int, R: int) -> LowRankFP4:
+    """The low-rank summaries with the mean rounded to bf16 and each eigenvector stored in E2M1
+    with one float32 scale (max |u| / 6) ([COBS] §2.3: FP4 eigenvectors, BF16 mean)."""
+    mu, u, lam = canonical_summaries_lowrank(K32, L, R)
+    nB, d = mu.shape
+    mu_q = np.zeros_like(mu)
+    codes = np.zeros((nB, R, d), np.uint8)
+    scales = np.zeros((nB, R), np.float32)
+    u_q = np.zeros_like(u)
+    if nB:
+        _c().cobs_oracle_lowrank_fp4_f32(mu.ctypes.data, np.ascontiguousarray(u).ctypes.data, nB, d, R,
+                                         mu_q.ctypes.data, codes.ctypes.data, scales.ctypes.data, u_q.ctypes.data)
+    return LowRankFP4((mu_q, codes, scales, lam, u_q))
 
 
 def canonical_scores_lowrank(q_group32: np.ndarray, summ: LowRank, alpha: float) -> np.ndarray:
@@ -437,6 +473,8 @@ def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
 
     summ: canonical summaries [nB, 2, d] (per-channel variance), [nB, d + 1] (isotropic) or a
     LowRank triple (mean, eigenvectors, eigenvalues)."""
+    if isinstance(summ, LowRankFP4):
+        summ = summ.dequantized()
     if isinstance(summ, LowRank):
         S = canonical_scores_lowrank(q_group32, summ, w.alpha)
         return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
@@ -473,6 +511,8 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
             sel_summ = canonical_summaries_iso(K.astype(np.float32), w.block)
         elif variance == "lowrank":
             sel_summ = canonical_summaries_lowrank(K.astype(np.float32), w.block, rank)
+        elif variance == "lowrank_fp4":
+            sel_summ = canonical_summaries_lowrank_fp4(K.astype(np.float32), w.block, rank)
         else:
             sel_summ = summ
         sel, _ = select_decode(w, qs.astype(np.float32), sel_summ)
@@ -480,7 +520,7 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
         mu, var = block_summaries(K, w.block)
         if variance == "isotropic":
             S64 = group_scores_iso(qs, mu, var.mean(axis=1), w.alpha)
-        elif variance == "lowrank":
+        elif variance in ("lowrank", "lowrank_fp4"):
             S64 = group_scores_lowrank(qs, *block_eigenpairs(K, w.block, rank), w.alpha)
         else:
             S64 = group_scores(qs, mu, var, w.alpha)

@@ -633,3 +633,61 @@ def test_lowrank_scores_match_exact_rational_emulation():
                 e = _rn32(pj * pj + e)
             v = _rn32(F(lam[b, j]) * e + v)
         assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
+
+
+# ---------------------------------------------------------------- FP4 (E2M1) low-rank variant
+
+_E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_rounding_is_nearest_with_ties_to_even_and_saturation():
+    """Brute force over a fine grid (and every tie point): the code's magnitude is the nearest
+    of the eight E2M1 magnitudes, ties go to the even index, |x| > 6 saturates, the sign is bit 3."""
+    grid = list(np.linspace(-8, 8, 3201)) + [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -1.75, -5.0]
+    for x in grid:
+        code = O.e2m1_code(x)
+        a = abs(x)
+        d = [abs(a - m) for m in _E2M1]
+        best = min(range(8), key=lambda i: (d[i], i % 2))
+        if a > 6:
+            best = 7
+        assert code & 7 == best, (x, code)
+        assert (code >> 3) == (1 if (x < 0 and best > 0) else 0), (x, code)
+
+
+def test_fp4_mean_is_bf16_round_to_nearest_even():
+    rng = np.random.default_rng(41)
+    K = (rng.standard_normal((4 * 64, 32)) * 3).astype(np.float32)
+    fp4 = O.canonical_summaries_lowrank_fp4(K, 64, 2)
+    mu = O.canonical_summaries(K, 64)[:, 0, :]
+    ref = torch.from_numpy(mu).to(torch.bfloat16).to(torch.float32).numpy()
+    assert np.array_equal(fp4[0], ref)
+
+
+def test_fp4_vectors_within_the_e2m1_grid_bound():
+    """Dequantized eigenvectors: u'_c = code * s with s = max|u| / 6; the error is at most half
+    the E2M1 gap at that magnitude (at most s), and the largest entry is exact up to rounding of s."""
+    rng = np.random.default_rng(42)
+    L, d, R, nB = 64, 128, 4, 6
+    K = _aniso_blocks(rng, nB, L, d, [3.0, 2.0, 1.4, 1.0, 0.5], 0.05).astype(np.float32)
+    mu, u, lam = O.canonical_summaries_lowrank(K, L, R)
+    mu_q, codes, scales, lam_q, u_q = O.canonical_summaries_lowrank_fp4(K, L, R)
+    assert np.array_equal(lam_q, lam)
+    s = scales[..., None].astype(np.float64)
+    err = np.abs(u_q.astype(np.float64) - u.astype(np.float64))
+    half_gap = np.where(np.abs(u) / s > 4, 1.0, np.where(np.abs(u) / s > 2, 0.5, 0.25))
+    assert np.all(err <= half_gap * s * (1 + 1e-6) + 1e-12)
+    assert np.allclose(scales, np.abs(u).max(axis=-1) / 6, rtol=1e-7)
+
+
+def test_fp4_selection_tracks_float32_low_rank_selection():
+    """On anisotropic blocks the FP4 summaries select nearly the same blocks as float32 ones."""
+    rng = np.random.default_rng(43)
+    L, d, R, nB, G, k = 64, 128, 4, 96, 4, 16
+    K = _aniso_blocks(rng, nB, L, d, [3.0, 2.0, 1.4, 1.0, 0.6, 0.4], 0.05).astype(np.float32)
+    K += (rng.standard_normal((nB, 1, d)) * rng.uniform(0.2, 1.5, (nB, 1, 1))).repeat(L, axis=1).reshape(nB * L, d).astype(np.float32)
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    s32 = O.canonical_scores_lowrank(q, O.canonical_summaries_lowrank(K, L, R), 1.0)
+    s4 = O.canonical_scores_lowrank(q, O.canonical_summaries_lowrank_fp4(K, L, R).dequantized(), 1.0)
+    a, b = set(O.top_k(s32, nB, k).tolist()), set(O.top_k(s4, nB, k).tolist())
+    assert len(a & b) >= 13
