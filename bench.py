@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k", "sweep"])
     ap.add_argument("--contexts", default=None, help="sweep: comma-separated context lengths (default 8k .. 1M)")
-    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank"], default="channel",
+    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank", "lowrank_fp4"], default="channel",
                     help="second-order statistic of the summaries (per-channel variance, one scalar per block, "
                          "or the leading eigenpairs of each block's covariance)")
     ap.add_argument("--rank", type=int, default=4, help="eigenpairs per block with --variance lowrank")
@@ -183,7 +183,8 @@ def decode_bytes(w, idx, variance="channel", rank=4):
     units = w.B * w.Hkv
     attn = kv_tokens * 2 * d * esz + units * ncv * 2 * d * esz          # K/V union + compressed K/V
     attn += w.B * w.Hq * d * esz * 2 + w.B * w.Hq * 3 * 4 + units * w.topk * 4   # Q, O, gates, idx
-    per_block = {"isotropic": (d + 1) * 4, "lowrank": (d + rank * d + rank) * 4}.get(variance, 2 * d * 4)
+    per_block = {"isotropic": (d + 1) * 4, "lowrank": (d + rank * d + rank) * 4,
+                 "lowrank_fp4": 2 * d + rank * d // 2 + 8 * rank}.get(variance, 2 * d * 4)
     select = units * w.nB * per_block + w.B * w.Hq * d * esz + units * w.topk * 4
     # summary update for the appended token: the completed block (64 K rows) and the last
     # compressed token (cmp_block K and V rows), plus their outputs
@@ -534,7 +535,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
                    "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
-                   "variance": args.variance, **({"rank": args.rank} if args.variance == "lowrank" else {}),
+                   "variance": args.variance, **({"rank": args.rank} if args.variance.startswith("lowrank") else {}),
                    "step": "summary update at T-1 + select + decode attention, one CUDA graph",
                    "l2": f"{R} KV-cache copies rotated between steps (working set {R} x step bytes > L2)",
                    "parallelism": f"dp{world} (independent decode batches per GPU)"},
@@ -707,8 +708,8 @@ def run_sweep(args):
                 ref = set(osa.tolist())
                 rec1.append(len(ref & set(int(x) for x in idx_a1[b, g] if x >= 0)) / w.topk)
                 rec0.append(len(ref & set(int(x) for x in idx_a0[b, g] if x >= 0)) / w.topk)
-        per_block = {"isotropic": (w.d + 1) * 4,
-                     "lowrank": (w.d + args.rank * w.d + args.rank) * 4}.get(args.variance, 2 * w.d * 4)
+        per_block = {"isotropic": (w.d + 1) * 4, "lowrank": (w.d + args.rank * w.d + args.rank) * 4,
+                     "lowrank_fp4": 2 * w.d + args.rank * w.d // 2 + 8 * args.rank}.get(args.variance, 2 * w.d * 4)
         by = w.B * w.Hkv * nB * per_block + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * w.topk * 4
         gbs = by / (us * 1e-6) / 1e9
         rows.append({"T": T, "nB": nB, "bytes": by, "us": us, "gbs": gbs, "frac": gbs / peak,

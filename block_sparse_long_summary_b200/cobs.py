@@ -23,7 +23,7 @@ COBS_ERR_CUDA = -3
 COBS_ERR_WORKSPACE = -4
 COBS_F32 = 0
 COBS_BF16 = 1
-COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC, COBS_VAR_LOWRANK = 0, 1, 2
+COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC, COBS_VAR_LOWRANK, COBS_VAR_LOWRANK_FP4 = 0, 1, 2, 3
 COBS_WS_SELECT = 0
 COBS_WS_DECODE = 1
 COBS_WS_PREFILL = 2
@@ -99,11 +99,12 @@ class Params:
     cmp_stride: int = 16
     alpha: float = 1.0
     dtype: str = "bf16"
-    variance: str = "channel"   # "channel", "isotropic" (one scalar per block) or "lowrank"
+    variance: str = "channel"   # "channel", "isotropic" (one scalar per block), "lowrank" or "lowrank_fp4"
     rank: int = 4               # eigenpairs per block for "lowrank"
 
     def c(self) -> cobs_params:
-        var = {"channel": COBS_VAR_CHANNEL, "isotropic": COBS_VAR_ISOTROPIC, "lowrank": COBS_VAR_LOWRANK}[self.variance]
+        var = {"channel": COBS_VAR_CHANNEL, "isotropic": COBS_VAR_ISOTROPIC, "lowrank": COBS_VAR_LOWRANK,
+               "lowrank_fp4": COBS_VAR_LOWRANK_FP4}[self.variance]
         return cobs_params(self.B, self.Hq, self.Hkv, self.d, self.T, self.block, self.cmp_block, self.cmp_stride,
                            self.topk, self.window, float(self.alpha), COBS_BF16 if self.dtype == "bf16" else COBS_F32,
                            var, int(self.rank))

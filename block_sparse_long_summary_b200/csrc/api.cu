@@ -73,10 +73,9 @@ cobs_status validate(const cobs_params* p) {
         return fail(COBS_ERR_INVALID_ARG, "need 1 <= cmp_stride <= cmp_block (got %d, %d)", p->cmp_stride,
                     p->cmp_block);
     if (p->dtype != COBS_F32 && p->dtype != COBS_BF16) return fail(COBS_ERR_INVALID_ARG, "dtype %d", p->dtype);
-    if (p->variance != COBS_VAR_CHANNEL && p->variance != COBS_VAR_ISOTROPIC && p->variance != COBS_VAR_LOWRANK)
-        return fail(COBS_ERR_INVALID_ARG, "variance %d (COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC or COBS_VAR_LOWRANK)",
-                    p->variance);
-    if (p->variance == COBS_VAR_LOWRANK && (p->rank < 1 || p->rank > 8))
+    if (p->variance < COBS_VAR_CHANNEL || p->variance > COBS_VAR_LOWRANK_FP4)
+        return fail(COBS_ERR_INVALID_ARG, "variance %d (a cobs_variance value)", p->variance);
+    if ((p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4) && (p->rank < 1 || p->rank > 8))
         return fail(COBS_ERR_UNSUPPORTED, "rank %d (supported: 1 .. 8)", p->rank);
     if (!isfinite(p->alpha)) return fail(COBS_ERR_INVALID_ARG, "alpha is not finite");
     if ((long long)p->B * p->Hkv > 65535) return fail(COBS_ERR_UNSUPPORTED, "B * Hkv > 65535");
@@ -192,7 +191,7 @@ cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summar
     COBS_TRY(check_ptr(summaries, "summaries"));
     COBS_TRY(check_ptr(idx, "idx"));
     if (prefill != 0 && prefill != 1) return fail(COBS_ERR_INVALID_ARG, "prefill must be 0 or 1");
-    if (prefill && p->variance == COBS_VAR_LOWRANK)
+    if (prefill && (p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4))
         return fail(COBS_ERR_UNSUPPORTED, "prefill selection with low-rank summaries");
     const cobs::Dims m = cobs::make_dims(*p);
     const size_t need = cobs::select_workspace_bytes(m, prefill);

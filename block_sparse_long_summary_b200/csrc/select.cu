@@ -16,6 +16,8 @@
 
 #include <algorithm>
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "dims.h"
 #include "tma.h"
@@ -243,25 +245,122 @@ __device__ __forceinline__ float block_score_lr(const float* tile, const float* 
     float v = 0.0f;
     for (int j = 0; j < R; ++j) {
         const float4* u4 = reinterpret_cast<const float4*>(tile + (size_t)(1 + j) * D * 32) + lane;
+        // heads in fours: each 32-channel chunk of u_j is read once per four heads, and every
+        // per-head chain keeps its canonical order (channel c to chain c mod 4, ascending c)
         float e = 0.0f;
-        for (int h = 0; h < G; ++h) {
-            const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)h * D);
-            float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll 8
-            for (int c4 = 0; c4 < D / 4; ++c4) {
-                const float4 uu = u4[c4 * 32];
-                const float4 q = q4[c4];
-                p0 = __fmaf_rn(q.x, uu.x, p0);
-                p1 = __fmaf_rn(q.y, uu.y, p1);
-                p2 = __fmaf_rn(q.z, uu.z, p2);
-                p3 = __fmaf_rn(q.w, uu.w, p3);
+        for (int hb = 0; hb < G; hb += 4) {
+            float p[4][4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) p[h][0] = p[h][1] = p[h][2] = p[h][3] = 0.0f;
+            for (int w = 0; w < D / 32; ++w) {
+                float4 uu[8];
+#pragma unroll
+                for (int t4 = 0; t4 < 8; ++t4) uu[t4] = u4[(w * 8 + t4) * 32];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    if (hb + h < G) {
+                        const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)(hb + h) * D) + w * 8;
+#pragma unroll
+                        for (int t4 = 0; t4 < 8; ++t4) {
+                            const float4 q = q4[t4];
+                            p[h][0] = __fmaf_rn(q.x, uu[t4].x, p[h][0]);
+                            p[h][1] = __fmaf_rn(q.y, uu[t4].y, p[h][1]);
+                            p[h][2] = __fmaf_rn(q.z, uu[t4].z, p[h][2]);
+                            p[h][3] = __fmaf_rn(q.w, uu[t4].w, p[h][3]);
+                        }
+                    }
+                }
             }
-            const float pj = combine4(p0, p1, p2, p3);
-            e = __fmaf_rn(pj, pj, e);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                if (hb + h < G) {
+                    const float pj = combine4(p[h][0], p[h][1], p[h][2], p[h][3]);
+                    e = __fmaf_rn(pj, pj, e);
+                }
+            }
         }
         v = __fmaf_rn(tile[(size_t)(1 + R) * D * 32 + j * 32 + lane], e, v);
     }
     return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
+}
+
+// Two E2M1 codes (one byte: the first channel in the low nibble) to two exact half values with
+// sm_100a's FP4 conversion.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(out) : "r"(byte));
+    return out;
+}
+
+// Canonical low-rank score from FP4 summaries: the bf16 means and the dequantized eigenvectors
+// u'_c = value(code_c) * scale_j (one rounded multiply), then the low-rank score's sums. Tile
+// bytes: bf16 means [D/8][32][8], codes of vector j [D/32][32][16] (channel 2i in the low nibble
+// of byte i), scales [R][32] f32, eigenvalues [R][32] f32.
+template <int D>
+__device__ __forceinline__ float block_score_lr_fp4(const float* tile, const float* qs, const float* qh, int G, int R,
+                                                    int lane, float isd, float c2) {
+    const unsigned char* t8 = reinterpret_cast<const unsigned char*>(tile);
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(t8 + ((size_t)c8 * 32 + lane) * 16);
+        const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const uint32_t hw = (w4[t >> 1] >> ((t & 1) * 16)) & 0xFFFFu;
+            const float mu = __uint_as_float(hw << 16);
+            a[t & 3] = __fmaf_rn(qs[8 * c8 + t], mu, a[t & 3]);
+        }
+    }
+    const float* scl = reinterpret_cast<const float*>(t8 + (size_t)64 * D + (size_t)R * 16 * D);
+    const float* lam = scl + R * 32;
+    float v = 0.0f;
+    for (int j = 0; j < R; ++j) {
+        const float sj = scl[j * 32 + lane];
+        const unsigned char* cj = t8 + (size_t)64 * D + (size_t)j * 16 * D;
+        // heads in fours: each 32-channel chunk is decoded once per four heads
+        // (u'_c = value * scale, one rounded multiply)
+        float e = 0.0f;
+        for (int hb = 0; hb < G; hb += 4) {
+            float p[4][4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) p[h][0] = p[h][1] = p[h][2] = p[h][3] = 0.0f;
+            for (int w = 0; w < D / 32; ++w) {
+                const uint4 wv = *reinterpret_cast<const uint4*>(cj + ((size_t)w * 32 + lane) * 16);
+                const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+                float u[32];
+#pragma unroll
+                for (int bi = 0; bi < 16; ++bi) {
+                    const uint32_t h2 = e2m1x2_to_f16x2((w4[bi >> 2] >> ((bi & 3) * 8)) & 0xFFu);
+                    u[2 * bi] = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))), sj);
+                    u[2 * bi + 1] = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(h2 >> 16))), sj);
+                }
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    if (hb + h < G) {
+                        const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)(hb + h) * D) + w * 8;
+#pragma unroll
+                        for (int t4 = 0; t4 < 8; ++t4) {
+                            const float4 q = q4[t4];
+                            p[h][0] = __fmaf_rn(q.x, u[4 * t4 + 0], p[h][0]);
+                            p[h][1] = __fmaf_rn(q.y, u[4 * t4 + 1], p[h][1]);
+                            p[h][2] = __fmaf_rn(q.z, u[4 * t4 + 2], p[h][2]);
+                            p[h][3] = __fmaf_rn(q.w, u[4 * t4 + 3], p[h][3]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                if (hb + h < G) {
+                    const float pj = combine4(p[h][0], p[h][1], p[h][2], p[h][3]);
+                    e = __fmaf_rn(pj, pj, e);
+                }
+            }
+        }
+        v = __fmaf_rn(lam[j * 32 + lane], e, v);
+    }
+    return __fmaf_rn(c2, v, __fmul_rn(combine4(a[0], a[1], a[2], a[3]), isd));
 }
 
 // Q2tot = sum_c Q2_c by adds in ascending channel order from +0 (one thread).
@@ -370,7 +469,8 @@ struct RunList {
 // dependent launch) merges the deposits. The result is the top-k under a strict total order,
 // so it does not depend on the split.
 // MODE 0: per-channel variance summaries, 1: isotropic, 2: low-rank (R eigenpairs, tile_floats
-// floats per group, one ring stage, the group's query heads in shared memory after the ring).
+// floats per group, one ring stage, the group's query heads in shared memory after the ring),
+// 3: low-rank with FP4 eigenvectors and bf16 means (as 2, with the ring of the other modes).
 template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
                                                            int32_t* __restrict__ idx, float* __restrict__ ws_s,
@@ -383,7 +483,7 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
     __shared__ float q2t_sm;
     constexpr bool ISO = MODE == 1;
     constexpr int kStg = MODE == 2 ? 1 : kSelStages;
-    const int kTileFloats = MODE == 2 ? tile_floats : group_floats<D, ISO>();
+    const int kTileFloats = MODE >= 2 ? tile_floats : group_floats<D, ISO>();
     const uint32_t kTileBytes = (uint32_t)kTileFloats * 4;
     // the merge grid may be scheduled now; it still waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -455,7 +555,7 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
                 if (lane == 0) q2t_sm = q2_total<D>(qsm[1]);
                 __syncwarp();
             }
-            if (MODE == 2) {  // the group's heads as float32, after the ring
+            if (MODE >= 2) {  // the group's heads as float32, after the ring
                 float* qh = tiles + kStg * kTileFloats;
                 for (int e = lane; e < G * D; e += 32) qh[e] = to_f(Q[(size_t)u * G * D + e]);
                 __syncwarp();
@@ -468,9 +568,11 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
         int bi = kInvalid;
         if (ok) {
             const float* tl = tiles + st * kTileFloats;
-            const float s_all = MODE == 2 ? block_score_lr<D>(tl, qsm[0], tiles + kStg * kTileFloats, G, R, lane, isd, c2)
-                                : ISO     ? block_score_iso<D>(tl, qsm[0], q2t_sm, lane, isd, c2)
-                                          : block_score<D>(tl, qsm[0], qsm[1], lane, isd, c2);
+            const float* qh = tiles + kStg * kTileFloats;
+            const float s_all = MODE == 3 ? block_score_lr_fp4<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
+                                : MODE == 2 ? block_score_lr<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
+                                : ISO       ? block_score_iso<D>(tl, qsm[0], q2t_sm, lane, isd, c2)
+                                            : block_score<D>(tl, qsm[0], qsm[1], lane, isd, c2);
             if (b < ncand) {
                 sc = s_all;
                 bi = b;
@@ -708,7 +810,9 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         grid = std::max<long long>(1, grid);
         float* ws_s = static_cast<float*>(ws);
         int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
-        const size_t smem = MODE == 2 ? tile_bytes + (size_t)kMaxGroup * D * 4 : (size_t)kSelStages * tile_bytes;
+        const size_t smem = MODE == 2   ? tile_bytes + (size_t)kMaxGroup * D * 4
+                            : MODE == 3 ? (size_t)kSelStages * tile_bytes + (size_t)kMaxGroup * D * 4
+                                        : (size_t)kSelStages * tile_bytes;
         if (smem > 227 * 1024) return cudaErrorNotSupported;
         cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -735,7 +839,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
                                   (int)grid, m.k, maxseg);
     }
     const size_t smem = tile_bytes * 2 + (size_t)kPfPos * 2 * D * 4;
-    if (MODE == 2) return cudaErrorNotSupported;  // the API rejects it before this point
+    if (MODE >= 2) return cudaErrorNotSupported;  // the API rejects it before this point
     auto kern = select_prefill_kernel<T, D, ISO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -769,7 +873,8 @@ cudaError_t launch_select_v(const Dims& m, const void* Q, const float* summ, int
 
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                           cudaStream_t s, int* err) {
-    if (m.lr) return launch_select_v<2>(m, Q, summ, prefill, idx, ws, s, err);
+    if (m.lr) return m.fp4 ? launch_select_v<3>(m, Q, summ, prefill, idx, ws, s, err)
+                           : launch_select_v<2>(m, Q, summ, prefill, idx, ws, s, err);
     return m.iso ? launch_select_v<1>(m, Q, summ, prefill, idx, ws, s, err)
                  : launch_select_v<0>(m, Q, summ, prefill, idx, ws, s, err);
 }

@@ -107,18 +107,40 @@ __device__ __forceinline__ float lr_dot4(const float* x, const float* y, int n, 
     return __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
 }
 
+// E2M1 (FP4) code of x: the nearest of the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (ties to the even
+// magnitude index), saturating above 6; the sign in bit 3 (a zero magnitude has code 0).
+__device__ __forceinline__ int e2m1_code(float x) {
+    const float mags[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    const float a = fabsf(x);
+    int best = 0;
+    float bd = a;
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        const float dist = fabsf(__fsub_rn(a, mags[i]));
+        if (dist < bd || (dist == bd && (i & 1) == 0)) {
+            best = i;
+            bd = dist;
+        }
+    }
+    if (a > 6.0f) best = 7;
+    return best == 0 ? 0 : ((x < 0.0f ? 8 : 0) | best);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
-                                                    float* __restrict__ summ) {
+                                                    int fp4, float* __restrict__ summ) {
     __shared__ float Y[kBlock][D + 1];  // +1: rows on different banks
     __shared__ float V[D][kLrMaxR], W[D][kLrMaxR];
     __shared__ float Tm[kBlock][kLrMaxR];
     __shared__ float bcast;
     __shared__ int ord_sh[kLrMaxR];
     __shared__ float lam_sh[kLrMaxR];
+    __shared__ float red[D];
+    __shared__ int code_sh[D];
     const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
     const int unit = blockIdx.y;
     const int j = j_begin + blockIdx.x;
+    float mu_c;
     // canonical mean of channel c (rows ascending), then the centred rows
     {
         const T* rows = K + ((size_t)unit * Tctx + (size_t)j * kBlock) * D + c;
@@ -131,9 +153,7 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
         const float mu = __fmul_rn(sum, 1.0f / kBlock);
 #pragma unroll
         for (int r = 0; r < kBlock; ++r) Y[r][c] = __fsub_rn(x[r], mu);
-        const size_t gf = (size_t)32 * (D + R * D + R);
-        float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
-        base[((size_t)(c / 4) * 32 + (j & 31)) * 4 + (c & 3)] = mu;
+        mu_c = mu;
         for (int jj = 0; jj < R; ++jj) V[c][jj] = lr_v0(c, jj);
     }
     __syncthreads();
@@ -188,11 +208,44 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
         for (int a = 0; a < R; ++a) ord_sh[a] = ord[a];
     }
     __syncthreads();
-    const size_t gf = (size_t)32 * (D + R * D + R);
-    float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
-    for (int jj = 0; jj < R; ++jj)
-        base[(size_t)(1 + jj) * D * 32 + ((size_t)(c / 4) * 32 + (j & 31)) * 4 + (c & 3)] = V[c][ord_sh[jj]];
-    if (c < R) base[(size_t)(1 + R) * D * 32 + (size_t)c * 32 + (j & 31)] = lam_sh[ord_sh[c]];
+    const int ln = j & 31;
+    if (!fp4) {
+        const size_t gf = (size_t)32 * (D + R * D + R);
+        float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
+        base[((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = mu_c;
+        for (int jj = 0; jj < R; ++jj)
+            base[(size_t)(1 + jj) * D * 32 + ((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = V[c][ord_sh[jj]];
+        if (c < R) base[(size_t)(1 + R) * D * 32 + (size_t)c * 32 + ln] = lam_sh[ord_sh[c]];
+        return;
+    }
+    // FP4 layout (bytes): bf16 means [D/8][32][8], E2M1 codes of vector jj [D/32][32][16]
+    // (channel 2i in the low nibble of byte i), scales [R][32] f32, eigenvalues [R][32] f32
+    const size_t gbytes = (size_t)32 * (2 * D + R * D / 2 + 8 * R);
+    unsigned char* g8 = reinterpret_cast<unsigned char*>(summ) + ((size_t)unit * nG + (size_t)(j >> 5)) * gbytes;
+    const __nv_bfloat16 mb = __float2bfloat16_rn(mu_c);
+    *reinterpret_cast<__nv_bfloat16*>(g8 + ((size_t)(c / 8) * 32 + ln) * 16 + (c % 8) * 2) = mb;
+    float* scl = reinterpret_cast<float*>(g8 + (size_t)64 * D + (size_t)R * 16 * D);
+    float* lamo = scl + R * 32;
+    for (int jj = 0; jj < R; ++jj) {
+        const float x = V[c][ord_sh[jj]];
+        red[c] = fabsf(x);
+        __syncthreads();
+        for (int o = D / 2; o > 0; o >>= 1) {  // max is exact in any order
+            if (c < o) red[c] = fmaxf(red[c], red[c + o]);
+            __syncthreads();
+        }
+        const float sc = __fdiv_rn(red[0], 6.0f);
+        code_sh[c] = sc > 0.0f ? e2m1_code(__fdiv_rn(x, sc)) : 0;
+        __syncthreads();
+        if ((c & 1) == 0)
+            g8[(size_t)64 * D + (size_t)jj * 16 * D + ((size_t)(c / 32) * 32 + ln) * 16 + (c % 32) / 2] =
+                (unsigned char)(code_sh[c] | (code_sh[c + 1] << 4));
+        if (c == 0) {
+            scl[jj * 32 + ln] = sc;
+            lamo[jj * 32 + ln] = lam_sh[ord_sh[jj]];
+        }
+        __syncthreads();
+    }
 }
 
 // grid (tokens to build, units, 2 = {K, V}), block d threads. out_i = P @ mean(rows).
@@ -595,9 +648,9 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
         count_launch();
         if (m.lr) {
             if (m.d == 128)
-                lowrank_kernel<T, 128><<<dim3(nbuild, units), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+                lowrank_kernel<T, 128><<<dim3(nbuild, units), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
             else
-                lowrank_kernel<T, 64><<<dim3(nbuild, units), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+                lowrank_kernel<T, 64><<<dim3(nbuild, units), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
         } else {
             summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
         }
@@ -646,9 +699,9 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
     if (nj > 0 && m.lr) {
         count_launch();
         if (m.d == 128)
-            lowrank_kernel<T, 128><<<dim3(1, m.units()), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+            lowrank_kernel<T, 128><<<dim3(1, m.units()), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
         else
-            lowrank_kernel<T, 64><<<dim3(1, m.units()), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, summ);
+            lowrank_kernel<T, 64><<<dim3(1, m.units()), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
         *e = cudaGetLastError();
     }
     return true;

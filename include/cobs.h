@@ -42,6 +42,11 @@
  *                  variance = COBS_VAR_LOWRANK (rank R): [B, Hkv, nG, (1 + R) * (d/4 * 32 * 4) + R * 32]
  *                  float32: the means as above, then eigenvector j < R of the group's blocks in
  *                  the same [d/4, 32, 4] interleaving, then the R eigenvalues [R, 32].
+ *                  variance = COBS_VAR_LOWRANK_FP4 (rank R): per group of 32 blocks, bytes
+ *                  [d/8, 32, 8] bf16 means, then for j < R [d/32, 32, 16] bytes of E2M1 codes
+ *                  (byte i of a lane's 16-byte word: channel 2i in the low nibble, 2i + 1 in the
+ *                  high one), then [R, 32] float32 scales, then [R, 32] float32 eigenvalues
+ *                  (8 (2d + R d / 2 + 8 R) float32 elements per group).
  *                  (32 consecutive blocks are interleaved channel-by-channel so that one
  *                  group is one contiguous copy and lane b%32 reads its block's channels.)
  * - GQA: query head h belongs to KV head h / (Hq / Hkv).
@@ -84,8 +89,17 @@ typedef enum { COBS_WS_SELECT = 0, COBS_WS_DECODE = 1, COBS_WS_PREFILL = 2 } cob
  *                       alpha/2 * sum_j lambda_j (q . u_j)^2 / d. The eigenpairs come from a fixed
  *                       float32 subspace iteration (24 steps, modified Gram-Schmidt), so they are
  *                       reproducible bit for bit. Decode selection only (prefill selection with
- *                       these summaries returns COBS_ERR_UNSUPPORTED). */
-typedef enum { COBS_VAR_CHANNEL = 0, COBS_VAR_ISOTROPIC = 1, COBS_VAR_LOWRANK = 2 } cobs_variance;
+ *                       these summaries returns COBS_ERR_UNSUPPORTED).
+ *   COBS_VAR_LOWRANK_FP4  the same eigenpairs with each eigenvector in FP4 (E2M1, one float32
+ *                       scale max|u|/6 per vector, round to nearest with ties to even, saturating)
+ *                       and the mean in bf16 ([COBS] §2.3); the score uses the dequantized values.
+ *                       About a fifth of the float32 low-rank bytes. Decode selection only. */
+typedef enum {
+    COBS_VAR_CHANNEL = 0,
+    COBS_VAR_ISOTROPIC = 1,
+    COBS_VAR_LOWRANK = 2,
+    COBS_VAR_LOWRANK_FP4 = 3
+} cobs_variance;
 
 /* Problem statement ([COBS] §2.3, [SKILL] "Method"): block size, compression block and
  * stride, top-k, window and alpha. */

@@ -79,6 +79,41 @@ def test_lowrank_incremental_update_matches_full_build(back):
     assert kc_close(f64(inc.Kc[:, :, -1]), f64(full.Kc[:, :, -1]), "bf16").all()
 
 
+@pytest.mark.parametrize("name,over,R", [
+    ("tiny", dict(), 4),                                              # float32, d = 64
+    ("decode32k", dict(B=2, Hkv=2, Hq=8, T=4096), 4),                  # bf16, d = 128, G = 4
+    ("decode32k", dict(B=1, Hkv=1, Hq=16, T=2048 + 37), 3),            # G = 16, odd rank, ragged tail
+    ("decode32k", dict(B=1, Hkv=2, Hq=2, d=64, T=3000, topk=32), 8),  # d = 64, G = 1, rank 8
+])
+def test_lowrank_fp4_decode_matches_oracle(name, over, R):
+    """FP4 eigenvectors and bf16 means: codes, scales, eigenvalues, means and selected blocks bit
+    for bit against the oracle's quantisation of its canonical eigenpairs."""
+    w = synth.WORKLOADS[name].replace(**over)
+    K, V, Q, g, Pk, Pv = inputs_decode(w)
+    p, buf = run_decode(w, K, V, Q, g, Pk, Pv, variance="lowrank_fp4", rank=R)
+    assert cobs().device_error() == 0
+    mu_g, codes_g, sc_g, lam_g = summaries_blocks(buf.summaries, p)
+    idx_g = buf.idx.cpu().numpy()
+    O_g = f64(buf.O)
+    Qf = synth.to_f64(Q, w.dtype)
+    G = w.G
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            ref = O.canonical_summaries_lowrank_fp4(synth.to_f64(K[b, h], w.dtype).astype(np.float32), w.block, R)
+            mu_q, codes, scales, lam, _ = ref
+            assert np.array_equal(mu_g[b, h], mu_q), f"bf16 means differ at {(b, h)}"
+            assert np.array_equal(codes_g[b, h], codes), f"E2M1 codes differ at {(b, h)}"
+            assert np.array_equal(sc_g[b, h], scales), f"scales differ at {(b, h)}"
+            assert np.array_equal(lam_g[b, h], lam), f"eigenvalues differ at {(b, h)}"
+            qs = Qf[b, h * G:(h + 1) * G]
+            sel, _ = O.select_decode(w, qs.astype(np.float32), ref)
+            assert np.array_equal(idx_g[b, h], sel), f"idx {(b, h)}: {idx_g[b, h]} vs {sel}"
+            Kf, Vf, _, Kc, Vc = O.unit_cache(w, K[b, h], V[b, h], Pk, Pv)
+            out = O.position_output(qs, g[b, h * G:(h + 1) * G], Kf, Vf, Kc, Vc, sel, w.T - 1, w.block, w.window,
+                                    w.cmp_block, w.cmp_stride)
+            assert np.abs(O_g[b, h * G:(h + 1) * G] - out).max() <= TOL[w.dtype]
+
+
 def test_lowrank_prefill_selection_is_rejected():
     C = cobs()
     w = synth.WORKLOADS["prefill32k"].replace(B=1, Hq=16, Hkv=1, T=512)
