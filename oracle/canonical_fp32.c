@@ -338,3 +338,40 @@ void cobs_oracle_lowrank_fp4_f32(const float* mu, const float* u, int64_t nb, in
         }
     }
 }
+
+/*
+ * Query-subspace variant (COBS §2.3: the eigenvectors kept as coordinates in a query subspace of
+ * dimension s < d, r d -> r s numbers per block). P: [d][s] with orthonormal columns, the
+ * caller's estimate of the subspace the queries live in (from their second moment). Per block the
+ * summary keeps mu (d), u~_j = P^T u_j (s numbers) and lambda_j; a query head is projected the
+ * same way, q~ = P^T q, and the covariance term uses (q~ . u~_j) in place of (q . u_j):
+ *   x~_i = four-chain sum over c of P[c][i] x_c            (i < s)
+ *   S = fmaf(c2, sum_j fmaf(lambda_j, e_j, .), a * isd), e_j = sum_h fmaf(p, p, .),
+ *   p = four-chain sum over i of q~_{h,i} u~_{j,i},  a = four-chain sum over c of Qsum_c mu_c.
+ */
+/* out[n][s] = P^T x_n for n rows x [n][d] */
+void cobs_oracle_subspace_project(const float* P, const float* x, int64_t n, int d, int s, float* out) {
+    for (int64_t r = 0; r < n; ++r)
+        for (int i = 0; i < s; ++i) out[r * s + i] = dot4s(P + i, x + r * d, d, s, 1);
+}
+
+/* q: [G][d]; qsum: [d]; mu: [nb][d]; ut: [nb][R][s]; lam: [nb][R]; P: [d][s]; S: [nb] */
+void cobs_oracle_subspace_scores(const float* q, const float* qsum, int G, const float* mu, const float* ut,
+                                 const float* lam, int64_t nb, int d, int s, int R, const float* P, float isd,
+                                 float c2, float* S) {
+    float qt[16 * 128];
+    cobs_oracle_subspace_project(P, q, G, d, s, qt);
+    for (int64_t b = 0; b < nb; ++b) {
+        const float a = dot4s(qsum, mu + b * d, d, 1, 1);
+        float v = 0.0f;
+        for (int j = 0; j < R; ++j) {
+            float e = 0.0f;
+            for (int h = 0; h < G; ++h) {
+                const float p = dot4s(qt + h * s, ut + (b * R + j) * (int64_t)s, s, 1, 1);
+                e = fmaf(p, p, e);
+            }
+            v = fmaf(lam[b * R + j], e, v);
+        }
+        S[b] = fmaf(c2, v, a * isd);
+    }
+}

@@ -79,6 +79,10 @@ def _c():
         lib.cobs_oracle_e2m1_code.restype = i32
         lib.cobs_oracle_bf16_rn.argtypes = [f32]
         lib.cobs_oracle_bf16_rn.restype = f32
+        lib.cobs_oracle_subspace_project.argtypes = [vp, vp, i64, i32, i32, vp]
+        lib.cobs_oracle_subspace_project.restype = None
+        lib.cobs_oracle_subspace_scores.argtypes = [vp, vp, i32, vp, vp, vp, i64, i32, i32, i32, vp, f32, f32, vp]
+        lib.cobs_oracle_subspace_scores.restype = None
         _clib = lib
     return _clib
 
@@ -235,6 +239,41 @@ def canonical_summaries_lowrank_fp4(K32: np.ndarray, L: int, R: int) -> LowRankF
     return LowRankFP4((mu_q, codes, scales, lam, u_q))
 
 
+class Subspace(tuple):
+    """Query-subspace low-rank summaries: (mu [nB, d], ut [nB, R, s] = P^T u_j, lam [nB, R], P [d, s])."""
+
+
+def canonical_summaries_subspace(K32: np.ndarray, L: int, R: int, P: np.ndarray) -> Subspace:
+    """The low-rank summaries with each eigenvector kept as its s coordinates in the query
+    subspace spanned by the orthonormal columns of P ([COBS] §2.3: query-subspace projection,
+    r d -> r s numbers per block). Canonical float32 order: canonical_fp32.c."""
+    mu, u, lam = canonical_summaries_lowrank(K32, L, R)
+    P = _f32c(P)
+    d, sdim = P.shape
+    nB = mu.shape[0]
+    ut = np.zeros((nB, R, sdim), np.float32)
+    if nB:
+        _c().cobs_oracle_subspace_project(P.ctypes.data, np.ascontiguousarray(u).ctypes.data, nB * R, d, sdim,
+                                          ut.ctypes.data)
+    return Subspace((mu, ut, lam, P))
+
+
+def canonical_scores_subspace(q_group32: np.ndarray, summ: Subspace, alpha: float) -> np.ndarray:
+    """float32 group scores [nB] with query-subspace summaries (canonical_fp32.c)."""
+    mu, ut, lam, P = summ
+    q = _f32c(q_group32)
+    G, d = q.shape
+    qs, _ = canonical_group_query(q)
+    isd, c2 = score_constants(d, alpha)
+    S = np.empty(mu.shape[0], np.float32)
+    if mu.shape[0]:
+        _c().cobs_oracle_subspace_scores(q.ctypes.data, _f32c(qs).ctypes.data, G, _f32c(mu).ctypes.data,
+                                         _f32c(ut).ctypes.data, _f32c(lam).ctypes.data, mu.shape[0], d,
+                                         ut.shape[2], ut.shape[1], _f32c(P).ctypes.data, float(isd), float(c2),
+                                         S.ctypes.data)
+    return S
+
+
 def canonical_scores_lowrank(q_group32: np.ndarray, summ: LowRank, alpha: float) -> np.ndarray:
     """float32 group scores [nB] of one group's query heads [G, d] against low-rank summaries:
     (sum_c Qsum_c mu_c) isd + c2 sum_j lam_j sum_h (q_h . u_j)^2. Canonical order: canonical_fp32.c."""
@@ -362,6 +401,17 @@ def head_scores_lowrank(q: np.ndarray, mu: np.ndarray, u: np.ndarray, lam: np.nd
     return (mu @ q) / np.sqrt(d) + alpha * 0.5 * ((u @ q) ** 2 * lam).sum(axis=-1) / d
 
 
+def group_scores_subspace(qs: np.ndarray, mu, u, lam, P, alpha: float) -> np.ndarray:
+    """Query-subspace per-group score: sum_h [q_h.mu/sqrt(d) + alpha/2 sum_j lam_j ((P^T q_h).(P^T u_j))^2 / d]."""
+    d = qs.shape[-1]
+    up = u @ P                      # [nB, R, s]
+    out = 0.0
+    for q in qs:
+        qp = P.T @ q
+        out = out + (mu @ q) / np.sqrt(d) + alpha * 0.5 * ((up @ qp) ** 2 * lam).sum(axis=-1) / d
+    return out
+
+
 def group_scores_lowrank(qs: np.ndarray, mu, u, lam, alpha: float) -> np.ndarray:
     """Sum of head_scores_lowrank over the G query heads qs [G, d] (the group-sum reading)."""
     return sum(head_scores_lowrank(q, mu, u, lam, alpha) for q in qs)
@@ -473,6 +523,9 @@ def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
 
     summ: canonical summaries [nB, 2, d] (per-channel variance), [nB, d + 1] (isotropic) or a
     LowRank triple (mean, eigenvectors, eigenvalues)."""
+    if isinstance(summ, Subspace):
+        S = canonical_scores_subspace(q_group32, summ, w.alpha)
+        return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
     if isinstance(summ, LowRankFP4):
         summ = summ.dequantized()
     if isinstance(summ, LowRank):

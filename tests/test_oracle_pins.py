@@ -691,3 +691,70 @@ def test_fp4_selection_tracks_float32_low_rank_selection():
     s4 = O.canonical_scores_lowrank(q, O.canonical_summaries_lowrank_fp4(K, L, R).dequantized(), 1.0)
     a, b = set(O.top_k(s32, nB, k).tolist()), set(O.top_k(s4, nB, k).tolist())
     assert len(a & b) >= 13
+
+
+# ---------------------------------------------------------------- query-subspace variant
+
+def _orthonormal(rng, d, s):
+    Pm, _ = np.linalg.qr(rng.standard_normal((d, s)))
+    return Pm
+
+
+def test_subspace_with_the_identity_basis_is_the_low_rank_selector():
+    """P = I (s = d): every projection is exact, so the subspace scores equal the low-rank scores
+    bit for bit in float32."""
+    rng = np.random.default_rng(51)
+    L, d, R, nB, G = 64, 32, 3, 10, 4
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.2, 0.7, 0.4], 0.05).astype(np.float32)
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    I = np.eye(d, dtype=np.float32)
+    S_sub = O.canonical_scores_subspace(q, O.canonical_summaries_subspace(K, L, R, I), 1.0)
+    S_lr = O.canonical_scores_lowrank(q, O.canonical_summaries_lowrank(K, L, R), 1.0)
+    assert np.array_equal(S_sub, S_lr)
+
+
+def test_subspace_score_is_exact_for_queries_in_the_subspace():
+    """Queries in span(P): (P^T q).(P^T u) = q^T P P^T u = q.u, so the float64 subspace score equals
+    the low-rank score; queries outside it lose their out-of-subspace part."""
+    rng = np.random.default_rng(52)
+    L, d, R, nB, G, s = 64, 32, 3, 6, 3, 12
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.2, 0.7, 0.4], 0.05)
+    mu, u, lam = O.block_eigenpairs(K, L, R)
+    P = _orthonormal(rng, d, s)
+    qs = (P @ rng.standard_normal((s, G))).T
+    assert np.allclose(O.group_scores_subspace(qs, mu, u, lam, P, 1.0), O.group_scores_lowrank(qs, mu, u, lam, 1.0),
+                       atol=1e-10)
+    q_out = rng.standard_normal((G, d))
+    assert not np.allclose(O.group_scores_subspace(q_out, mu, u, lam, P, 1.0),
+                           O.group_scores_lowrank(q_out, mu, u, lam, 1.0))
+
+
+def test_subspace_canonical_matches_exact_rational_emulation():
+    rng = np.random.default_rng(53)
+    L, d, R, nB, G, s = 64, 16, 2, 3, 2, 8
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.0, 0.4], 0.05).astype(np.float32)
+    P = _orthonormal(rng, d, s).astype(np.float32)
+    summ = O.canonical_summaries_subspace(K, L, R, P)
+    mu, ut, lam, _ = summ
+    _, u, _ = O.canonical_summaries_lowrank(K, L, R)
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    S = O.canonical_scores_subspace(q, summ, 0.8)
+    F = lambda v: Fraction(float(v))
+    for b in range(nB):
+        for j in range(R):
+            for i in range(s):
+                assert F(ut[b, j, i]) == _dot4_exact(F, P[:, i], u[b, j])
+    qsum, _ = O.canonical_group_query(q)
+    qt = [[_dot4_exact(F, P[:, i], q[h]) for i in range(s)] for h in range(G)]
+    isd = _rn32(Fraction(1.0 / math.sqrt(d)))
+    c2 = _rn32(F(np.float32(0.8)) / (2 * d))
+    for b in range(nB):
+        a = _dot4_exact(F, qsum, mu[b])
+        v = Fraction(0)
+        for j in range(R):
+            e = Fraction(0)
+            for h in range(G):
+                pj = _dot4_exact(lambda x: x, qt[h], [F(x) for x in ut[b, j]])
+                e = _rn32(pj * pj + e)
+            v = _rn32(F(lam[b, j]) * e + v)
+        assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
