@@ -40,10 +40,14 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k", "sweep"])
     ap.add_argument("--contexts", default=None, help="sweep: comma-separated context lengths (default 8k .. 1M)")
-    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank", "lowrank_fp4"], default="channel",
+    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank", "lowrank_fp4", "subspace"],
+                    default="channel",
                     help="second-order statistic of the summaries (per-channel variance, one scalar per block, "
                          "or the leading eigenpairs of each block's covariance)")
-    ap.add_argument("--rank", type=int, default=4, help="eigenpairs per block with --variance lowrank")
+    ap.add_argument("--rank", type=int, default=4, help="eigenpairs per block with the low-rank variances")
+    ap.add_argument("--sub", type=int, default=84,
+                    help="query-subspace dimension with --variance subspace (seeded orthonormal basis; the "
+                         "queries are drawn concentrated in its span)")
     ap.add_argument("--aniso", type=int, default=0,
                     help="sweep: draw anisotropic key blocks (spread on this many directions) instead of isotropic")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
@@ -164,7 +168,14 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ algorithmic bytes
 
-def decode_bytes(w, idx, variance="channel", rank=4):
+def summary_block_bytes(d, variance, rank, sub):
+    """Summary bytes per selection block for each second-order form."""
+    return {"isotropic": (d + 1) * 4, "lowrank": (d + rank * d + rank) * 4,
+            "lowrank_fp4": 2 * d + rank * d // 2 + 8 * rank,
+            "subspace": (d + rank * sub + rank) * 4}.get(variance, 2 * d * 4)
+
+
+def decode_bytes(w, idx, variance="channel", rank=4, sub=84):
     """Algorithmic HBM bytes of one decode step, from the selected blocks (idx [B, Hkv, k])."""
     import numpy as np
     d, esz = w.d, 2 if w.dtype == "bf16" else 4
@@ -183,9 +194,10 @@ def decode_bytes(w, idx, variance="channel", rank=4):
     units = w.B * w.Hkv
     attn = kv_tokens * 2 * d * esz + units * ncv * 2 * d * esz          # K/V union + compressed K/V
     attn += w.B * w.Hq * d * esz * 2 + w.B * w.Hq * 3 * 4 + units * w.topk * 4   # Q, O, gates, idx
-    per_block = {"isotropic": (d + 1) * 4, "lowrank": (d + rank * d + rank) * 4,
-                 "lowrank_fp4": 2 * d + rank * d // 2 + 8 * rank}.get(variance, 2 * d * 4)
+    per_block = summary_block_bytes(d, variance, rank, sub)
     select = units * w.nB * per_block + w.B * w.Hq * d * esz + units * w.topk * 4
+    if variance == "subspace":
+        select += d * sub * 4   # the basis
     # summary update for the appended token: the completed block (64 K rows) and the last
     # compressed token (cmp_block K and V rows), plus their outputs
     update = units * (w.block * d * esz + per_block + 2 * w.cmp_block * d * esz + 2 * d * esz)
@@ -195,11 +207,12 @@ def decode_bytes(w, idx, variance="channel", rank=4):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False, variance="channel", rank=4):
+def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False, variance="channel", rank=4,
+                         basis=None):
     """Time the oracle (as it stands) on the listed units; returns (seconds, query heads[, result])."""
     from oracle import cobs_oracle as O
     t0 = time.perf_counter()
-    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units, variance=variance, rank=rank)
+    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units, variance=variance, rank=rank, basis=basis)
     secs = time.perf_counter() - t0
     return (secs, len(units) * w.G, res) if with_result else (secs, len(units) * w.G)
 
@@ -372,11 +385,14 @@ def run_ours(args):
         w = w.replace(T=args.T)
     if w.mode == "prefill":
         return run_prefill_line(args, w, dev, cobs, rank, world)
+    basis = synth.subspace_basis(w, args.sub) if args.variance == "subspace" else None
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
-                    variance=args.variance, rank=args.rank)
+                    variance=args.variance, rank=args.rank,
+                    **(dict(sub=args.sub, basis=torch.from_numpy(basis).to(dev)) if basis is not None else {}))
     K, V = synth.kv_cache(w)
-    Q, g = synth.queries_decode(w), synth.gates_decode(w)
+    Q = synth.queries_decode(w) if basis is None else synth.queries_decode_subspace(w, basis)
+    g = synth.gates_decode(w)
     Pk, Pv = synth.projections(w)
 
     R = max(1, args.copies)
@@ -526,7 +542,7 @@ def run_ours(args):
     dev_err = cobs.device_error()
 
     qheads = w.B * w.Hq * world
-    by = decode_bytes(w, idx0, args.variance, args.rank)
+    by = decode_bytes(w, idx0, args.variance, args.rank, args.sub)
     peak, peak_kind = read_peaks()
     att_gbs = by["attn"] / (t_att * 1e-3) / 1e9
     result = {
@@ -535,7 +551,10 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
                    "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
-                   "variance": args.variance, **({"rank": args.rank} if args.variance.startswith("lowrank") else {}),
+                   "variance": args.variance,
+                   **({"rank": args.rank} if args.variance in ("lowrank", "lowrank_fp4", "subspace") else {}),
+                   **({"sub": args.sub, "queries": "concentrated in the subspace (leak 0.1)"}
+                      if args.variance == "subspace" else {}),
                    "step": "summary update at T-1 + select + decode attention, one CUDA graph",
                    "l2": f"{R} KV-cache copies rotated between steps (working set {R} x step bytes > L2)",
                    "parallelism": f"dp{world} (independent decode batches per GPU)"},
@@ -564,7 +583,7 @@ def run_ours(args):
         lim = limit_threads()
         units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:24]
         secs, heads, ref = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=True,
-                                                variance=args.variance, rank=args.rank)
+                                                variance=args.variance, rank=args.rank, basis=basis)
         result["cpu_baseline"] = {"value": heads / secs, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                                   "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
                                             f"full oracle decode incl. summaries ({secs:.1f} s)"}
@@ -638,10 +657,16 @@ def run_sweep(args):
     rows, launches = [], 0
     stream = torch.cuda.Stream(device=dev)
 
+    basis = synth.subspace_basis(base, args.sub) if args.variance == "subspace" else None
+    tbasis = torch.from_numpy(basis).to(dev) if basis is not None else None
+    qbasis = synth.subspace_basis(base, args.sub) if (basis is not None or args.subspace_queries) else None
+
     def params(w, **over):
         kw = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                   cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
                   variance=args.variance, rank=args.rank)
+        if basis is not None:
+            kw.update(sub=args.sub, basis=tbasis)
         kw.update(over)
         return cobs.Params(**kw)
 
@@ -657,7 +682,8 @@ def run_sweep(args):
         Vc = torch.empty_like(Kc)
         Pk, Pv = synth.projections(w)
         tPk, tPv = to_dev(Pk, "f32", dev), to_dev(Pv, "f32", dev)
-        tQ = to_dev(synth.queries_decode(w), "bf16", dev)
+        tQ = to_dev(synth.queries_decode(w) if qbasis is None else synth.queries_decode_subspace(w, qbasis), "bf16",
+                    dev)
         mass = torch.empty((n_rec, w.Hq, nB), dtype=torch.float32, device=dev)
         n0 = cobs.launch_count()
         with torch.cuda.stream(stream):
@@ -708,8 +734,7 @@ def run_sweep(args):
                 ref = set(osa.tolist())
                 rec1.append(len(ref & set(int(x) for x in idx_a1[b, g] if x >= 0)) / w.topk)
                 rec0.append(len(ref & set(int(x) for x in idx_a0[b, g] if x >= 0)) / w.topk)
-        per_block = {"isotropic": (w.d + 1) * 4, "lowrank": (w.d + args.rank * w.d + args.rank) * 4,
-                     "lowrank_fp4": 2 * w.d + args.rank * w.d // 2 + 8 * args.rank}.get(args.variance, 2 * w.d * 4)
+        per_block = summary_block_bytes(w.d, args.variance, args.rank, args.sub)
         by = w.B * w.Hkv * nB * per_block + w.B * w.Hq * w.d * 2 + w.B * w.Hkv * w.topk * 4
         gbs = by / (us * 1e-6) / 1e9
         rows.append({"T": T, "nB": nB, "bytes": by, "us": us, "gbs": gbs, "frac": gbs / peak,
@@ -724,7 +749,10 @@ def run_sweep(args):
             "dtype": "f32", "data": "synthetic (keys drawn on the device" +
                                     (f", anisotropic blocks of rank {args.aniso})" if args.aniso else ")"),
             "config": {"workload": "sweep", "B": base.B, "Hq": base.Hq, "Hkv": base.Hkv, "d": base.d,
-                       "topk": base.topk, "contexts": contexts, "variance": args.variance, "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
+                       "topk": base.topk, "contexts": contexts, "variance": args.variance,
+                       **({"sub": args.sub, "queries": "concentrated in the subspace (leak 0.1)"}
+                          if qbasis is not None else {}),
+                       "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
             "roofline": {"bound": "hbm", "kernel": "select_decode_kernel", "achieved": top["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": top["frac"], "peak_kind": peak_kind,
                          "traffic": recorded_traffic("select_decode")},

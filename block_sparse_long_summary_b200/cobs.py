@@ -23,7 +23,7 @@ COBS_ERR_CUDA = -3
 COBS_ERR_WORKSPACE = -4
 COBS_F32 = 0
 COBS_BF16 = 1
-COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC, COBS_VAR_LOWRANK, COBS_VAR_LOWRANK_FP4 = 0, 1, 2, 3
+COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC, COBS_VAR_LOWRANK, COBS_VAR_LOWRANK_FP4, COBS_VAR_SUBSPACE = 0, 1, 2, 3, 4
 COBS_WS_SELECT = 0
 COBS_WS_DECODE = 1
 COBS_WS_PREFILL = 2
@@ -40,7 +40,7 @@ class cobs_params(ctypes.Structure):
                 ("T", ctypes.c_int32), ("block", ctypes.c_int32), ("cmp_block", ctypes.c_int32),
                 ("cmp_stride", ctypes.c_int32), ("topk", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32), ("variance", ctypes.c_int32),
-                ("rank", ctypes.c_int32)]
+                ("rank", ctypes.c_int32), ("sub", ctypes.c_int32), ("basis", ctypes.c_void_p)]
 
 
 class CobsError(RuntimeError):
@@ -99,15 +99,22 @@ class Params:
     cmp_stride: int = 16
     alpha: float = 1.0
     dtype: str = "bf16"
-    variance: str = "channel"   # "channel", "isotropic" (one scalar per block), "lowrank" or "lowrank_fp4"
-    rank: int = 4               # eigenpairs per block for "lowrank"
+    variance: str = "channel"   # "channel", "isotropic", "lowrank", "lowrank_fp4" or "subspace"
+    rank: int = 4               # eigenpairs per block for the low-rank forms
+    sub: int = 84               # "subspace": coordinates kept per eigenvector
+    basis: object = dataclasses.field(default=None, compare=False, repr=False)  # "subspace": [d, sub] f32 CUDA
 
     def c(self) -> cobs_params:
         var = {"channel": COBS_VAR_CHANNEL, "isotropic": COBS_VAR_ISOTROPIC, "lowrank": COBS_VAR_LOWRANK,
-               "lowrank_fp4": COBS_VAR_LOWRANK_FP4}[self.variance]
+               "lowrank_fp4": COBS_VAR_LOWRANK_FP4, "subspace": COBS_VAR_SUBSPACE}[self.variance]
+        sub = var == COBS_VAR_SUBSPACE
+        if sub and self.basis is not None and (self.basis.dtype != torch.float32 or
+                                                tuple(self.basis.shape) != (self.d, self.sub)):
+            raise ValueError("basis must be a float32 [d, sub] tensor")
         return cobs_params(self.B, self.Hq, self.Hkv, self.d, self.T, self.block, self.cmp_block, self.cmp_stride,
                            self.topk, self.window, float(self.alpha), COBS_BF16 if self.dtype == "bf16" else COBS_F32,
-                           var, int(self.rank))
+                           var, int(self.rank), int(self.sub) if sub else 0,
+                           _ptr(self.basis) if sub and self.basis is not None else None)
 
     @property
     def torch_dtype(self):

@@ -73,10 +73,16 @@ cobs_status validate(const cobs_params* p) {
         return fail(COBS_ERR_INVALID_ARG, "need 1 <= cmp_stride <= cmp_block (got %d, %d)", p->cmp_stride,
                     p->cmp_block);
     if (p->dtype != COBS_F32 && p->dtype != COBS_BF16) return fail(COBS_ERR_INVALID_ARG, "dtype %d", p->dtype);
-    if (p->variance < COBS_VAR_CHANNEL || p->variance > COBS_VAR_LOWRANK_FP4)
+    if (p->variance < COBS_VAR_CHANNEL || p->variance > COBS_VAR_SUBSPACE)
         return fail(COBS_ERR_INVALID_ARG, "variance %d (a cobs_variance value)", p->variance);
-    if ((p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4) && (p->rank < 1 || p->rank > 8))
+    if ((p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4 ||
+         p->variance == COBS_VAR_SUBSPACE) &&
+        (p->rank < 1 || p->rank > 8))
         return fail(COBS_ERR_UNSUPPORTED, "rank %d (supported: 1 .. 8)", p->rank);
+    if (p->variance == COBS_VAR_SUBSPACE) {
+        if (p->sub < 4 || p->sub > p->d || p->sub % 4 != 0)
+            return fail(COBS_ERR_UNSUPPORTED, "subspace dimension %d (a multiple of 4 in 4 .. d)", p->sub);
+    }
     if (!isfinite(p->alpha)) return fail(COBS_ERR_INVALID_ARG, "alpha is not finite");
     if ((long long)p->B * p->Hkv > 65535) return fail(COBS_ERR_UNSUPPORTED, "B * Hkv > 65535");
     return COBS_OK;
@@ -171,6 +177,7 @@ cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void
     COBS_TRY(check_ptr(Pk, "Pk", true));
     COBS_TRY(check_ptr(Pv, "Pv", true));
     COBS_TRY(check_ptr(summaries, "summaries"));
+    if (p->variance == COBS_VAR_SUBSPACE) COBS_TRY(check_ptr(p->basis, "basis"));
     const cobs::Dims m = cobs::make_dims(*p);
     if (m.nC > 0) {
         COBS_TRY(check_ptr(Kc, "Kc"));
@@ -191,7 +198,9 @@ cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summar
     COBS_TRY(check_ptr(summaries, "summaries"));
     COBS_TRY(check_ptr(idx, "idx"));
     if (prefill != 0 && prefill != 1) return fail(COBS_ERR_INVALID_ARG, "prefill must be 0 or 1");
-    if (prefill && (p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4))
+    if (p->variance == COBS_VAR_SUBSPACE && !prefill) COBS_TRY(check_ptr(p->basis, "basis"));
+    if (prefill && (p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4 ||
+                    p->variance == COBS_VAR_SUBSPACE))
         return fail(COBS_ERR_UNSUPPORTED, "prefill selection with low-rank summaries");
     const cobs::Dims m = cobs::make_dims(*p);
     const size_t need = cobs::select_workspace_bytes(m, prefill);

@@ -284,6 +284,92 @@ __device__ __forceinline__ float block_score_lr(const float* tile, const float* 
     return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
 }
 
+// Canonical query-subspace score: the mean sum as above, then
+//   v = sum over j ascending of fma(lambda_j, e_j, .), e_j = sum over h ascending of fma(p, p, .),
+//   p = four-chain sum over i < S of q~_{h,i} u~_{j,i} (coordinate i to chain i mod 4);
+// the tile holds the 32 blocks' means, then the S coordinates of eigenvector j < R in an
+// [S/4][32][4] interleaving, then the R x 32 eigenvalues. qt: the group's projected heads [G][S].
+template <int D>
+__device__ __forceinline__ float block_score_sub(const float* tile, const float* qs, const float* qt, int G, int R,
+                                                 int S, int lane, float isd, float c2) {
+    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 m = mu4[c4 * 32];
+        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
+        a0 = __fmaf_rn(q.x, m.x, a0);
+        a1 = __fmaf_rn(q.y, m.y, a1);
+        a2 = __fmaf_rn(q.z, m.z, a2);
+        a3 = __fmaf_rn(q.w, m.w, a3);
+    }
+    const int S4 = S / 4;
+    float v = 0.0f;
+    for (int j = 0; j < R; ++j) {
+        const float4* u4 = reinterpret_cast<const float4*>(tile + (size_t)32 * D + (size_t)j * S * 32) + lane;
+        float e = 0.0f;
+        for (int hb = 0; hb < G; hb += 4) {  // each coordinate of u~_j read once per four heads
+            float p[4][4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) p[h][0] = p[h][1] = p[h][2] = p[h][3] = 0.0f;
+#pragma unroll 3
+            for (int i4 = 0; i4 < S4; ++i4) {
+                const float4 uu = u4[i4 * 32];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    if (hb + h < G) {
+                        const float4 q = reinterpret_cast<const float4*>(qt + (size_t)(hb + h) * S)[i4];
+                        p[h][0] = __fmaf_rn(q.x, uu.x, p[h][0]);
+                        p[h][1] = __fmaf_rn(q.y, uu.y, p[h][1]);
+                        p[h][2] = __fmaf_rn(q.z, uu.z, p[h][2]);
+                        p[h][3] = __fmaf_rn(q.w, uu.w, p[h][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                if (hb + h < G) {
+                    const float pj = combine4(p[h][0], p[h][1], p[h][2], p[h][3]);
+                    e = __fmaf_rn(pj, pj, e);
+                }
+            }
+        }
+        v = __fmaf_rn(tile[(size_t)32 * (D + R * S) + j * 32 + lane], e, v);
+    }
+    return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
+}
+
+// Query heads projected on the subspace basis, q~_{h,i} = four-chain sum over c of P[c][i] q_{h,c}
+// (channel c to chain c mod 4, ascending c; chains combined as (s0 + s1) + (s2 + s3)).
+// grid (units, ceil(G S / 64)), 256 threads: four threads per output, thread k of the four runs
+// chain k (D/4 independent loads of P, then its fused multiply-adds), and two shuffles combine
+// the chains. Out: qt [units][G][S] float32. The selection grid that follows is launched as its
+// programmatic dependent and waits for this grid before reading qt.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) project_queries_kernel(const T* __restrict__ Q, const float* __restrict__ P,
+                                                              int G, int S, float* __restrict__ qt) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ __align__(16) float qh[kMaxGroup * D];
+    const int u = blockIdx.x;
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) qh[e] = to_f(Q[(size_t)u * G * D + e]);
+    __syncthreads();
+    const int o = blockIdx.y * 64 + (threadIdx.x >> 2), k = threadIdx.x & 3;
+    const bool live = o < G * S;
+    const int h = live ? o / S : 0, i = live ? o % S : 0;
+    float acc = 0.0f;
+    if (live) {
+        float pv[D / 4];
+#pragma unroll
+        for (int n = 0; n < D / 4; ++n) pv[n] = __ldg(P + (size_t)(4 * n + k) * S + i);
+#pragma unroll
+        for (int n = 0; n < D / 4; ++n) acc = __fmaf_rn(pv[n], qh[h * D + 4 * n + k], acc);
+    }
+    // lanes 4m..4m+3 hold chains 0..3 of one output
+    const float pair = __fadd_rn(acc, __shfl_xor_sync(kFull, acc, 1));    // s0 + s1 at k = 0, s2 + s3 at k = 2
+    const float all = __fadd_rn(pair, __shfl_xor_sync(kFull, pair, 2));   // (s0 + s1) + (s2 + s3) at k = 0
+    if (live && k == 0) qt[(size_t)u * G * S + o] = all;
+}
+
 // Two E2M1 codes (one byte: the first channel in the low nibble) to two exact half values with
 // sm_100a's FP4 conversion.
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
@@ -470,19 +556,22 @@ struct RunList {
 // so it does not depend on the split.
 // MODE 0: per-channel variance summaries, 1: isotropic, 2: low-rank (R eigenpairs, tile_floats
 // floats per group, one ring stage, the group's query heads in shared memory after the ring),
-// 3: low-rank with FP4 eigenvectors and bf16 means (as 2, with the ring of the other modes).
+// 3: low-rank with FP4 eigenvectors and bf16 means (as 2, with the ring of the other modes),
+// 4: query subspace (as 2, with the projected heads qt_ws [units][G][S] written by
+// project_queries_kernel, which this grid waits for, in place of the heads).
 template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
                                                            int32_t* __restrict__ idx, float* __restrict__ ws_s,
                                                            int* __restrict__ ws_i, int units, int G, int nG,
                                                            int ncand, int k, int maxseg,
-                                                           float isd, float c2, int R, int tile_floats, int* err) {
+                                                           float isd, float c2, int R, int tile_floats,
+                                                           const float* qt_ws, int S, int* err) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bar[kSelStages];
     __shared__ __align__(16) float qsm[2][D];
     __shared__ float q2t_sm;
     constexpr bool ISO = MODE == 1;
-    constexpr int kStg = MODE == 2 ? 1 : kSelStages;
+    constexpr int kStg = (MODE == 2 || MODE == 4) ? 1 : kSelStages;
     const int kTileFloats = MODE >= 2 ? tile_floats : group_floats<D, ISO>();
     const uint32_t kTileBytes = (uint32_t)kTileFloats * 4;
     // the merge grid may be scheduled now; it still waits for this grid to complete
@@ -555,7 +644,12 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
                 if (lane == 0) q2t_sm = q2_total<D>(qsm[1]);
                 __syncwarp();
             }
-            if (MODE >= 2) {  // the group's heads as float32, after the ring
+            if (MODE == 4) {  // the group's projected heads, after the ring
+                float* qh = tiles + kStg * kTileFloats;
+                if (x == x0) asm volatile("griddepcontrol.wait;" ::: "memory");  // qt_ws is complete
+                for (int e = lane; e < G * S; e += 32) qh[e] = __ldcg(qt_ws + (size_t)u * G * S + e);
+                __syncwarp();
+            } else if (MODE >= 2) {  // the group's heads as float32, after the ring
                 float* qh = tiles + kStg * kTileFloats;
                 for (int e = lane; e < G * D; e += 32) qh[e] = to_f(Q[(size_t)u * G * D + e]);
                 __syncwarp();
@@ -569,7 +663,8 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
         if (ok) {
             const float* tl = tiles + st * kTileFloats;
             const float* qh = tiles + kStg * kTileFloats;
-            const float s_all = MODE == 3 ? block_score_lr_fp4<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
+            const float s_all = MODE == 4 ? block_score_sub<D>(tl, qsm[0], qh, G, R, S, lane, isd, c2)
+                                : MODE == 3 ? block_score_lr_fp4<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
                                 : MODE == 2 ? block_score_lr<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
                                 : ISO       ? block_score_iso<D>(tl, qsm[0], q2t_sm, lane, isd, c2)
                                             : block_score<D>(tl, qsm[0], qsm[1], lane, isd, c2);
@@ -788,6 +883,15 @@ __global__ void __launch_bounds__(128) select_prefill_kernel(const T* __restrict
     }
 }
 
+// The projected query heads of the query-subspace form: the 16-byte aligned region that follows
+// the segment lists in the decode selection workspace.
+float* select_qt_region(const Dims& m, void* ws) {
+    const int nGc = (m.T / m.L + kGroupBlocks - 1) / kGroupBlocks;
+    const int maxseg = sel_max_segments(m.units(), std::max(1, nGc));
+    const size_t lists = (size_t)m.units() * maxseg * m.k * (sizeof(float) + sizeof(int));
+    return reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + (lists + 15) / 16 * 16);
+}
+
 template <typename T, int D, int MODE>
 cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                             cudaStream_t s, int* err) {
@@ -812,16 +916,40 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
         const size_t smem = MODE == 2   ? tile_bytes + (size_t)kMaxGroup * D * 4
                             : MODE == 3 ? (size_t)kSelStages * tile_bytes + (size_t)kMaxGroup * D * 4
+                            : MODE == 4 ? tile_bytes + (size_t)m.G * m.sub * 4
                                         : (size_t)kSelStages * tile_bytes;
         if (smem > 227 * 1024) return cudaErrorNotSupported;
         cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        count_launch();
-        select_decode_kernel<T, D, MODE><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(), m.G,
-                                                                          m.nG, ncand, m.k, maxseg, isd, c2, m.lr,
-                                                                          tile_floats, err);
-        e = cudaGetLastError();
+        float* qt_ws = MODE == 4 ? select_qt_region(m, ws) : nullptr;
+        if (MODE == 4 && n > 0) {  // the projected heads, then the selection grid as their dependent
+            count_launch();
+            project_queries_kernel<T, D><<<dim3(m.units(), (m.G * m.sub + 63) / 64), 256, 0, s>>>(Q, m.basis, m.G,
+                                                                                                   m.sub, qt_ws);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)grid);
+            cfg.blockDim = dim3(32);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = s;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            count_launch();
+            e = cudaLaunchKernelEx(&cfg, select_decode_kernel<T, D, MODE>, Q, summ, idx, ws_s, ws_i, m.units(), m.G,
+                                   m.nG, ncand, m.k, maxseg, isd, c2, m.lr, tile_floats, (const float*)qt_ws, m.sub,
+                                   err);
+        } else {
+            count_launch();
+            select_decode_kernel<T, D, MODE><<<(unsigned)grid, 32, smem, s>>>(Q, summ, idx, ws_s, ws_i, m.units(),
+                                                                              m.G, m.nG, ncand, m.k, maxseg, isd, c2,
+                                                                              m.lr, tile_floats, qt_ws, m.sub, err);
+            e = cudaGetLastError();
+        }
         // a unit is cut into several ranges only if it has several groups and the grid several CTAs
         if (e != cudaSuccess || n == 0 || nGc == 1 || grid == 1) return e;
         cudaLaunchConfig_t cfg = {};
@@ -855,7 +983,10 @@ size_t select_workspace_bytes(const Dims& m, int prefill) {
     if (prefill) return 0;
     const int nGc = (m.T / m.L + kGroupBlocks - 1) / kGroupBlocks;
     const int maxseg = sel_max_segments(m.units(), std::max(1, nGc));
-    return (size_t)m.units() * maxseg * m.k * (sizeof(float) + sizeof(int));
+    const size_t lists = (size_t)m.units() * maxseg * m.k * (sizeof(float) + sizeof(int));
+    if (!m.sub) return lists;
+    // query-subspace summaries: the projected heads [units][G][sub] float32 after the lists
+    return (lists + 15) / 16 * 16 + (size_t)m.units() * m.G * m.sub * sizeof(float);
 }
 
 template <int MODE>
@@ -873,6 +1004,7 @@ cudaError_t launch_select_v(const Dims& m, const void* Q, const float* summ, int
 
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                           cudaStream_t s, int* err) {
+    if (m.sub) return launch_select_v<4>(m, Q, summ, prefill, idx, ws, s, err);
     if (m.lr) return m.fp4 ? launch_select_v<3>(m, Q, summ, prefill, idx, ws, s, err)
                            : launch_select_v<2>(m, Q, summ, prefill, idx, ws, s, err);
     return m.iso ? launch_select_v<1>(m, Q, summ, prefill, idx, ws, s, err)

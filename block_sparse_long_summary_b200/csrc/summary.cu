@@ -128,7 +128,8 @@ __device__ __forceinline__ int e2m1_code(float x) {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
-                                                    int fp4, float* __restrict__ summ) {
+                                                    int fp4, const float* __restrict__ Pb, int S,
+                                                    float* __restrict__ summ) {
     __shared__ float Y[kBlock][D + 1];  // +1: rows on different banks
     __shared__ float V[D][kLrMaxR], W[D][kLrMaxR];
     __shared__ float Tm[kBlock][kLrMaxR];
@@ -209,6 +210,20 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
     }
     __syncthreads();
     const int ln = j & 31;
+    if (S > 0) {
+        // query-subspace form: eigenvector jj kept as u~_i = four-chain sum over c of P[c][i] u_c
+        // (i < S), in the [S/4][32][4] interleaving
+        const size_t gf = (size_t)32 * (D + R * S + R);
+        float* base = summ + ((size_t)unit * nG + (size_t)(j >> 5)) * gf;
+        base[((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = mu_c;
+        for (int o = c; o < R * S; o += D) {
+            const int jj = o / S, i = o % S;
+            base[(size_t)32 * D + (size_t)jj * S * 32 + ((size_t)(i / 4) * 32 + ln) * 4 + (i & 3)] =
+                lr_dot4(Pb + i, &V[0][ord_sh[jj]], D, S, kLrMaxR);
+        }
+        if (c < R) base[(size_t)32 * (D + R * S) + (size_t)c * 32 + ln] = lam_sh[ord_sh[c]];
+        return;
+    }
     if (!fp4) {
         const size_t gf = (size_t)32 * (D + R * D + R);
         float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
@@ -648,9 +663,11 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
         count_launch();
         if (m.lr) {
             if (m.d == 128)
-                lowrank_kernel<T, 128><<<dim3(nbuild, units), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
+                lowrank_kernel<T, 128><<<dim3(nbuild, units), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                    m.basis, m.sub, summ);
             else
-                lowrank_kernel<T, 64><<<dim3(nbuild, units), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
+                lowrank_kernel<T, 64><<<dim3(nbuild, units), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                    m.basis, m.sub, summ);
         } else {
             summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
         }
@@ -699,9 +716,11 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
     if (nj > 0 && m.lr) {
         count_launch();
         if (m.d == 128)
-            lowrank_kernel<T, 128><<<dim3(1, m.units()), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
+            lowrank_kernel<T, 128><<<dim3(1, m.units()), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                m.basis, m.sub, summ);
         else
-            lowrank_kernel<T, 64><<<dim3(1, m.units()), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4, summ);
+            lowrank_kernel<T, 64><<<dim3(1, m.units()), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                m.basis, m.sub, summ);
         *e = cudaGetLastError();
     }
     return true;

@@ -47,6 +47,9 @@
  *                  (byte i of a lane's 16-byte word: channel 2i in the low nibble, 2i + 1 in the
  *                  high one), then [R, 32] float32 scales, then [R, 32] float32 eigenvalues
  *                  (8 (2d + R d / 2 + 8 R) float32 elements per group).
+ *                  variance = COBS_VAR_SUBSPACE (rank R, sub s): [B, Hkv, nG, 32 (d + R s + R)]
+ *                  float32: the means as above, then the s coordinates of eigenvector j < R in a
+ *                  [s/4, 32, 4] interleaving, then the R eigenvalues [R, 32].
  *                  (32 consecutive blocks are interleaved channel-by-channel so that one
  *                  group is one contiguous copy and lane b%32 reads its block's channels.)
  * - GQA: query head h belongs to KV head h / (Hq / Hkv).
@@ -93,12 +96,20 @@ typedef enum { COBS_WS_SELECT = 0, COBS_WS_DECODE = 1, COBS_WS_PREFILL = 2 } cob
  *   COBS_VAR_LOWRANK_FP4  the same eigenpairs with each eigenvector in FP4 (E2M1, one float32
  *                       scale max|u|/6 per vector, round to nearest with ties to even, saturating)
  *                       and the mean in bf16 ([COBS] §2.3); the score uses the dequantized values.
- *                       About a fifth of the float32 low-rank bytes. Decode selection only. */
+ *                       About a fifth of the float32 low-rank bytes. Decode selection only.
+ *   COBS_VAR_SUBSPACE   the COBS_VAR_LOWRANK eigenpairs with each eigenvector kept as its `sub`
+ *                       coordinates u~_j = P^T u_j in the query subspace spanned by the columns of
+ *                       `basis` ([COBS] §2.3, projection onto the query subspace: r d -> r s numbers
+ *                       per block); the query heads are projected the same way, q~ = P^T q (float32,
+ *                       four-chain sums over the d channels), and the score term is
+ *                       alpha/2 * sum_j lambda_j (q~ . u~_j)^2 / d. Exact for queries inside span(P)
+ *                       when P has orthonormal columns. Decode selection only. */
 typedef enum {
     COBS_VAR_CHANNEL = 0,
     COBS_VAR_ISOTROPIC = 1,
     COBS_VAR_LOWRANK = 2,
-    COBS_VAR_LOWRANK_FP4 = 3
+    COBS_VAR_LOWRANK_FP4 = 3,
+    COBS_VAR_SUBSPACE = 4
 } cobs_variance;
 
 /* Problem statement ([COBS] §2.3, [SKILL] "Method"): block size, compression block and
@@ -117,7 +128,11 @@ typedef struct {
     float alpha;        /* weight of the second-order (variance) term */
     int32_t dtype;      /* cobs_dtype of Q, K, V, Kc, Vc, O */
     int32_t variance;   /* cobs_variance: the second-order statistic of the summaries */
-    int32_t rank;       /* eigenpairs per block for COBS_VAR_LOWRANK (1 .. 8); ignored otherwise */
+    int32_t rank;       /* eigenpairs per block for the low-rank forms (1 .. 8); ignored otherwise */
+    int32_t sub;        /* COBS_VAR_SUBSPACE: subspace dimension s (a multiple of 4, 4 .. d); else ignored */
+    const float* basis; /* COBS_VAR_SUBSPACE: device array [d][sub] float32, the basis P of the query
+                           subspace (orthonormal columns expected, not checked), read by
+                           cobs_build_summaries and cobs_select and owned by the caller; else ignored */
 } cobs_params;
 
 /*

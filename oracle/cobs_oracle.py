@@ -539,11 +539,12 @@ def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
     return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
 
 
-def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", rank=4):
+def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", rank=4, basis=None):
     """Decode at position T-1 for every (batch, KV head) unit (or the listed units).
 
-    variance: "channel" (per-channel variance summaries), "isotropic" (one scalar per block) or
-    "lowrank" (the rank leading eigenpairs of each block's covariance).
+    variance: "channel" (per-channel variance summaries), "isotropic" (one scalar per block),
+    "lowrank" / "lowrank_fp4" (the rank leading eigenpairs of each block's covariance) or
+    "subspace" (those eigenpairs with the eigenvectors as coordinates in basis [d, s]).
 
     Returns dict with idx [B, Hkv, k], O [B, Hq, d] (float64; rows of unlisted units are NaN),
     summ, Kc, Vc per computed unit, and near-tie reports (units where the float64 ranking of
@@ -566,6 +567,8 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
             sel_summ = canonical_summaries_lowrank(K.astype(np.float32), w.block, rank)
         elif variance == "lowrank_fp4":
             sel_summ = canonical_summaries_lowrank_fp4(K.astype(np.float32), w.block, rank)
+        elif variance == "subspace":
+            sel_summ = canonical_summaries_subspace(K.astype(np.float32), w.block, rank, basis)
         else:
             sel_summ = summ
         sel, _ = select_decode(w, qs.astype(np.float32), sel_summ)
@@ -575,6 +578,9 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
             S64 = group_scores_iso(qs, mu, var.mean(axis=1), w.alpha)
         elif variance in ("lowrank", "lowrank_fp4"):
             S64 = group_scores_lowrank(qs, *block_eigenpairs(K, w.block, rank), w.alpha)
+        elif variance == "subspace":
+            S64 = group_scores_subspace(qs, *block_eigenpairs(K, w.block, rank), np.asarray(basis, np.float64),
+                                        w.alpha)
         else:
             S64 = group_scores(qs, mu, var, w.alpha)
         sel64 = top_k(S64, n_candidates(t, w.block), w.topk)

@@ -42,6 +42,7 @@ _lib = None
 # stream tags
 TAG_KMU, TAG_KSIG, TAG_KZ, TAG_V, TAG_Q, TAG_GATE, TAG_PK, TAG_PV, TAG_NEEDLE, TAG_NMU = range(1, 11)
 TAG_KU = 11  # per-block direction bases of the anisotropic key model
+TAG_QB, TAG_QZ = 12, 13  # query-subspace basis and the queries drawn in it
 
 
 def build(force: bool = False) -> str:
@@ -275,6 +276,30 @@ def queries_prefill(w: Workload, positions: Optional[np.ndarray] = None) -> np.n
                 k = key(w.seed, TAG_Q, b, hq)
                 for i, t in enumerate(positions):
                     q[b, i, hq] = normals_f32(k, w.d, offset=int(t) * w.d)
+    return _store(q, w.dtype)
+
+
+def subspace_basis(w: Workload, s: int) -> np.ndarray:
+    """P [d, s] float32 with orthonormal columns: the QR factor of a seeded Gaussian d x s matrix
+    (column signs fixed by a positive diagonal of R). It stands for the leading eigenvectors of the
+    queries' second moment, the subspace the query-subspace summaries are kept in."""
+    a = normals_f64(key(w.seed, TAG_QB), w.d * s).reshape(w.d, s)
+    q, r = np.linalg.qr(a)
+    q = q * np.where(np.diag(r) < 0, -1.0, 1.0)
+    return np.ascontiguousarray(q.astype(np.float32))
+
+
+def queries_decode_subspace(w: Workload, P: np.ndarray, leak: float = 0.1) -> np.ndarray:
+    """Q [B, Hq, d] concentrated in span(P): q = sqrt(1 - leak^2) sqrt(d/s) P z + leak n with
+    z ~ N(0, I_s) and n ~ N(0, I_d), so E|q|^2 = d as for the plain N(0, I) queries and a share
+    leak^2 of it lies (mostly) outside the subspace."""
+    d, s = P.shape
+    q = np.empty((w.B, w.Hq, d), np.float32)
+    a = np.sqrt(1.0 - leak * leak) * np.sqrt(d / s)
+    for b in range(w.B):
+        for hq in range(w.Hq):
+            z = normals_f64(key(w.seed, TAG_QZ, b, hq), s + d)
+            q[b, hq] = (a * (P.astype(np.float64) @ z[:s]) + leak * z[s:]).astype(np.float32)
     return _store(q, w.dtype)
 
 

@@ -28,11 +28,15 @@ def f64(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def params_of(w, variance="channel", rank=4):
+def params_of(w, variance="channel", rank=4, basis=None):
+    """basis: the query-subspace basis [d, s] (numpy float32) for variance "subspace"."""
     C = cobs()
+    extra = {}
+    if basis is not None:
+        extra = dict(sub=basis.shape[1], basis=torch.from_numpy(np.ascontiguousarray(basis)).cuda())
     return C.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype, variance=variance,
-                    rank=rank)
+                    rank=rank, **extra)
 
 
 def summaries_blocks(flat, p):
@@ -53,6 +57,17 @@ def summaries_blocks(flat, p):
         scales = tail[..., 0, :, :].transpose(0, 1, 2, 4, 3).reshape(p.B, p.Hkv, nG * 32, R)
         lam = tail[..., 1, :, :].transpose(0, 1, 2, 4, 3).reshape(p.B, p.Hkv, nG * 32, R)
         return mu[:, :, :nB], codes[:, :, :nB].astype(np.uint8), scales[:, :, :nB], lam[:, :, :nB]
+    if p.variance == "subspace":
+        R, d, S = p.rank, p.d, p.sub
+        gf = 32 * (d + R * S + R)
+        a = flat[: p.B * p.Hkv * nG * gf].cpu().numpy().reshape(p.B, p.Hkv, nG, gf)
+        mu = a[..., :d * 32].reshape(p.B, p.Hkv, nG, d // 4, 32, 4).transpose(0, 1, 2, 4, 3, 5)
+        mu = mu.reshape(p.B, p.Hkv, nG * 32, d)[:, :, :nB]
+        ut = a[..., d * 32:(d + R * S) * 32].reshape(p.B, p.Hkv, nG, R, S // 4, 32, 4).transpose(0, 1, 2, 5, 3, 4, 6)
+        ut = ut.reshape(p.B, p.Hkv, nG * 32, R, S)[:, :, :nB]
+        lam = a[..., (d + R * S) * 32:].reshape(p.B, p.Hkv, nG, R, 32).transpose(0, 1, 2, 4, 3)
+        lam = lam.reshape(p.B, p.Hkv, nG * 32, R)[:, :, :nB]
+        return mu, ut, lam
     if p.variance == "lowrank":
         R, d = p.rank, p.d
         gf = 32 * (d + R * d + R)
@@ -78,9 +93,9 @@ def summaries_blocks(flat, p):
     return a.reshape(p.B, p.Hkv, nG * 32, 2, p.d)[:, :, :nB]
 
 
-def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel", rank=4):
+def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel", rank=4, basis=None):
     C = cobs()
-    p = params_of(w, variance, rank)
+    p = params_of(w, variance, rank, basis)
     buf = C.alloc(p, prefill=False)
     C.device_error(reset=True)
     C.decode_step(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),

@@ -758,3 +758,17 @@ def test_subspace_canonical_matches_exact_rational_emulation():
                 e = _rn32(pj * pj + e)
             v = _rn32(F(lam[b, j]) * e + v)
         assert F(S[b]) == _rn32(c2 * v + _rn32(a * isd)), b
+
+
+def test_subspace_decode_with_identity_basis_is_low_rank_decode():
+    """The oracle's decode driver: with P = I the query-subspace selection and output are the
+    low-rank ones."""
+    import synth
+    w = synth.WORKLOADS["tiny"]
+    K, V = synth.kv_cache(w)
+    Q, g = synth.queries_decode(w), synth.gates_decode(w)
+    Pk, Pv = synth.projections(w)
+    a = O.decode(w, K, V, Q, g, Pk, Pv, variance="lowrank", rank=4)
+    b = O.decode(w, K, V, Q, g, Pk, Pv, variance="subspace", rank=4, basis=np.eye(w.d, dtype=np.float32))
+    assert np.array_equal(a["idx"], b["idx"])
+    assert np.array_equal(a["O"], b["O"])
