@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--sub", type=int, default=84,
                     help="query-subspace dimension with --variance subspace (seeded orthonormal basis; the "
                          "queries are drawn concentrated in its span)")
+    ap.add_argument("--subspace-queries", action="store_true",
+                    help="draw the queries concentrated in the seeded --sub basis with any --variance (to "
+                         "compare the summary forms on the queries the query-subspace form is built for)")
     ap.add_argument("--aniso", type=int, default=0,
                     help="sweep: draw anisotropic key blocks (spread on this many directions) instead of isotropic")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")

@@ -223,72 +223,13 @@ __device__ __forceinline__ float block_score_iso(const float* tile, const float*
     return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
 }
 
-// Canonical low-rank score: the same mean sum, then
-//   v = sum over j ascending of fma(lambda_j, e_j, .), e_j = sum over h ascending of fma(p, p, .),
-//   p = four-chain sum_c q_{h,c} u_{j,c};
-// the tile holds the 32 blocks' means, then eigenvector j in the same interleaving for j < R,
-// then the R x 32 eigenvalues. qh: the group's G query heads [G][D] in shared memory.
-template <int D>
-__device__ __forceinline__ float block_score_lr(const float* tile, const float* qs, const float* qh, int G, int R,
-                                                int lane, float isd, float c2) {
-    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 m = mu4[c4 * 32];
-        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
-        a0 = __fmaf_rn(q.x, m.x, a0);
-        a1 = __fmaf_rn(q.y, m.y, a1);
-        a2 = __fmaf_rn(q.z, m.z, a2);
-        a3 = __fmaf_rn(q.w, m.w, a3);
-    }
-    float v = 0.0f;
-    for (int j = 0; j < R; ++j) {
-        const float4* u4 = reinterpret_cast<const float4*>(tile + (size_t)(1 + j) * D * 32) + lane;
-        // heads in fours: each 32-channel chunk of u_j is read once per four heads, and every
-        // per-head chain keeps its canonical order (channel c to chain c mod 4, ascending c)
-        float e = 0.0f;
-        for (int hb = 0; hb < G; hb += 4) {
-            float p[4][4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) p[h][0] = p[h][1] = p[h][2] = p[h][3] = 0.0f;
-            for (int w = 0; w < D / 32; ++w) {
-                float4 uu[8];
-#pragma unroll
-                for (int t4 = 0; t4 < 8; ++t4) uu[t4] = u4[(w * 8 + t4) * 32];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    if (hb + h < G) {
-                        const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)(hb + h) * D) + w * 8;
-#pragma unroll
-                        for (int t4 = 0; t4 < 8; ++t4) {
-                            const float4 q = q4[t4];
-                            p[h][0] = __fmaf_rn(q.x, uu[t4].x, p[h][0]);
-                            p[h][1] = __fmaf_rn(q.y, uu[t4].y, p[h][1]);
-                            p[h][2] = __fmaf_rn(q.z, uu[t4].z, p[h][2]);
-                            p[h][3] = __fmaf_rn(q.w, uu[t4].w, p[h][3]);
-                        }
-                    }
-                }
-            }
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                if (hb + h < G) {
-                    const float pj = combine4(p[h][0], p[h][1], p[h][2], p[h][3]);
-                    e = __fmaf_rn(pj, pj, e);
-                }
-            }
-        }
-        v = __fmaf_rn(tile[(size_t)(1 + R) * D * 32 + j * 32 + lane], e, v);
-    }
-    return __fmaf_rn(c2, v, __fmul_rn(combine4(a0, a1, a2, a3), isd));
-}
-
-// Canonical query-subspace score: the mean sum as above, then
+// Canonical low-rank score on S-coordinate eigenvectors: a = four-chain sum over c of Qsum_c mu_c, then
 //   v = sum over j ascending of fma(lambda_j, e_j, .), e_j = sum over h ascending of fma(p, p, .),
 //   p = four-chain sum over i < S of q~_{h,i} u~_{j,i} (coordinate i to chain i mod 4);
 // the tile holds the 32 blocks' means, then the S coordinates of eigenvector j < R in an
-// [S/4][32][4] interleaving, then the R x 32 eigenvalues. qt: the group's projected heads [G][S].
+// [S/4][32][4] interleaving, then the R x 32 eigenvalues. qt: the group's heads [G][S], projected
+// on the subspace basis (query-subspace summaries) or as they are with S = D (low-rank summaries,
+// whose layout is this one with S = D).
 template <int D>
 __device__ __forceinline__ float block_score_sub(const float* tile, const float* qs, const float* qt, int G, int R,
                                                  int S, int lane, float isd, float c2) {
@@ -502,10 +443,14 @@ __device__ __forceinline__ void warp_merge_best_first(float& s, int& i, float bs
 #define COBS_SELECT_CTAS_PER_SM 3
 #endif
 constexpr int kSelStages = COBS_SELECT_STAGES;
+// At most this many one-warp selection CTAs per SM (twice as many for the FP4 low-rank
+// summaries, whose scoring is bound by arithmetic and whose tiles are small); the grid takes the
+// smaller of this and the number that fit an SM with the mode's shared memory (2 for the float32
+// low-rank summaries), so that every CTA is resident from the start.
 constexpr int kSelCtasPerSm = COBS_SELECT_CTAS_PER_SM;
 // Upper bound of the decode selector's grid (any sm_100 part), fixing the workspace size
 // without a device query.
-constexpr int kSelGridCap = 192 * kSelCtasPerSm;
+constexpr int kSelGridCap = 192 * 2 * kSelCtasPerSm;
 
 // Stream-K split of the decode selection: the n = units * nGc summary groups, unit-major, are
 // cut into `grid` contiguous ranges [c n / grid, (c + 1) n / grid). CTA of group x:
@@ -665,7 +610,7 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
             const float* qh = tiles + kStg * kTileFloats;
             const float s_all = MODE == 4 ? block_score_sub<D>(tl, qsm[0], qh, G, R, S, lane, isd, c2)
                                 : MODE == 3 ? block_score_lr_fp4<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
-                                : MODE == 2 ? block_score_lr<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
+                                : MODE == 2 ? block_score_sub<D>(tl, qsm[0], qh, G, R, D, lane, isd, c2)
                                 : ISO       ? block_score_iso<D>(tl, qsm[0], q2t_sm, lane, isd, c2)
                                             : block_score<D>(tl, qsm[0], qsm[1], lane, isd, c2);
             if (b < ncand) {
@@ -905,15 +850,6 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         const int nGc = (ncand + kGroupBlocks - 1) / kGroupBlocks;
         const long long n = (long long)m.units() * nGc;
         const int maxseg = sel_max_segments(m.units(), std::max(1, nGc));
-        // grid: kSelCtasPerSm CTAs per SM and at least one group each. A unit's groups then meet
-        // at most min(nGc, ceil(grid / units) + 1) <= maxseg ranges (grid <= kSelGridCap).
-        long long grid = std::min<long long>((long long)sm_count() * kSelCtasPerSm, kSelGridCap);
-        grid = std::min<long long>(grid, std::max<long long>(1, n));
-        grid = std::min<long long>(grid, (long long)(kSelMaxSeg - 1) * m.units());
-        if (n == 0) grid = std::min(m.units(), 1024);
-        grid = std::max<long long>(1, grid);
-        float* ws_s = static_cast<float*>(ws);
-        int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
         const size_t smem = MODE == 2   ? tile_bytes + (size_t)kMaxGroup * D * 4
                             : MODE == 3 ? (size_t)kSelStages * tile_bytes + (size_t)kMaxGroup * D * 4
                             : MODE == 4 ? tile_bytes + (size_t)m.G * m.sub * 4
@@ -922,6 +858,19 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_decode_kernel<T, D, MODE>, 32, smem);
+        if (e != cudaSuccess) return e;
+        per_sm = std::max(1, std::min(per_sm, MODE == 3 ? 2 * kSelCtasPerSm : kSelCtasPerSm));
+        // grid: the resident CTAs of every SM and at least one group each. A unit's groups then
+        // meet at most min(nGc, ceil(grid / units) + 1) <= maxseg ranges (grid <= kSelGridCap).
+        long long grid = std::min<long long>((long long)sm_count() * per_sm, kSelGridCap);
+        grid = std::min<long long>(grid, std::max<long long>(1, n));
+        grid = std::min<long long>(grid, (long long)(kSelMaxSeg - 1) * m.units());
+        if (n == 0) grid = std::min(m.units(), 1024);
+        grid = std::max<long long>(1, grid);
+        float* ws_s = static_cast<float*>(ws);
+        int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
         float* qt_ws = MODE == 4 ? select_qt_region(m, ws) : nullptr;
         if (MODE == 4 && n > 0) {  // the projected heads, then the selection grid as their dependent
             count_launch();
