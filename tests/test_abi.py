@@ -93,3 +93,58 @@ def test_workspace_sizes(lib):
     assert ws <= (8 << 20)
     assert lib.summaries_elems(p) == n_units * 16 * 2 * 128 * 32
     assert lib.workspace_bytes(p, lib.COBS_WS_SELECT) > 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(variance="lowrank", rank=0), -2),
+    (dict(variance="lowrank", rank=9), -2),
+    (dict(variance="lowrank_fp4", rank=9), -2),
+    (dict(variance="subspace", rank=4, sub=82), -2),   # not a multiple of 4
+    (dict(variance="subspace", rank=4, sub=0), -2),
+    (dict(variance="subspace", rank=4, sub=132), -2),  # more than d
+])
+def test_summary_form_validation(lib, kw, status):
+    p = _p(**kw)
+    cp = p.c()
+    fake = ctypes.c_void_p(256)
+    r = lib._lib.cobs_build_summaries(ctypes.byref(cp), fake, fake, None, None, 0, fake, fake, fake, None)
+    assert r == status, lib._lib.cobs_last_error()
+    assert lib.summaries_elems(p) == 0
+
+
+def test_unknown_variance_rejected(lib):
+    cp = _p().c()
+    cp.variance = 5
+    fake = ctypes.c_void_p(256)
+    assert lib._lib.cobs_build_summaries(ctypes.byref(cp), fake, fake, None, None, 0, fake, fake, fake, None) == -1
+    assert b"variance" in lib._lib.cobs_last_error()
+
+
+def test_subspace_needs_a_basis(lib):
+    p = _p(variance="subspace", rank=4, sub=84)   # no basis: sizing works, compute calls refuse
+    assert lib.summaries_elems(p) > 0
+    cp = p.c()
+    fake = ctypes.c_void_p(256)
+    assert lib._lib.cobs_select(ctypes.byref(cp), fake, fake, 0, fake, fake, 1 << 30, None) == -1
+    assert b"basis is NULL" in lib._lib.cobs_last_error()
+    assert lib._lib.cobs_build_summaries(ctypes.byref(cp), fake, fake, None, None, 0, fake, fake, fake, None) == -1
+    assert b"basis is NULL" in lib._lib.cobs_last_error()
+    cp.basis = ctypes.c_void_p(264)   # misaligned
+    assert lib._lib.cobs_select(ctypes.byref(cp), fake, fake, 0, fake, fake, 1 << 30, None) == -1
+    assert b"aligned" in lib._lib.cobs_last_error()
+
+
+def test_summary_sizes_of_every_form(lib):
+    """Floats per unit: nG groups of 32 blocks, each group in the layout of its form."""
+    B_, Hkv, d, T = 2, 8, 128, 32768 + 64 * 5      # nB = 517 -> nG = 17
+    units, nG = B_ * Hkv, 17
+    kw = dict(B=B_, Hq=32, Hkv=Hkv, d=d, T=T)
+    assert lib.summaries_elems(_p(**kw)) == units * nG * 2 * d * 32
+    assert lib.summaries_elems(_p(variance="isotropic", **kw)) == units * nG * (d + 1) * 32
+    assert lib.summaries_elems(_p(variance="lowrank", rank=4, **kw)) == units * nG * 32 * (d + 4 * d + 4)
+    assert lib.summaries_elems(_p(variance="lowrank_fp4", rank=3, **kw)) == units * nG * 8 * (2 * d + 3 * d // 2 + 24)
+    assert lib.summaries_elems(_p(variance="subspace", rank=4, sub=84, **kw)) == units * nG * 32 * (d + 4 * 84 + 4)
+    # the query-subspace form's selection workspace adds the projected heads [units, G, s] float32
+    ws_lr = lib.workspace_bytes(_p(variance="lowrank", rank=4, **kw), lib.COBS_WS_SELECT)
+    ws_sub = lib.workspace_bytes(_p(variance="subspace", rank=4, sub=84, **kw), lib.COBS_WS_SELECT)
+    assert ws_sub >= ws_lr + units * 4 * 84 * 4
