@@ -131,7 +131,9 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
                                                     int fp4, const float* __restrict__ Pb, int S,
                                                     float* __restrict__ summ) {
     __shared__ float Y[kBlock][D + 1];  // +1: rows on different banks
-    __shared__ float V[D][kLrMaxR], W[D][kLrMaxR];
+    // rows of kLrMaxR + 1 floats: thread c's row starts on bank 9c mod 32, so the per-thread row
+    // accesses of a warp are free of bank conflicts
+    __shared__ float V[D][kLrMaxR + 1], W[D][kLrMaxR + 1];
     __shared__ float Tm[kBlock][kLrMaxR];
     __shared__ float bcast;
     __shared__ int ord_sh[kLrMaxR];
@@ -175,7 +177,7 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
     for (int it = 0; it <= kLrIters; ++it) {
         for (int o = c; o < kBlock * R; o += D) {
             const int r = o / R, jj = o % R;
-            Tm[r][jj] = lr_dot4(&Y[r][0], &V[0][jj], D, 1, kLrMaxR);
+            Tm[r][jj] = lr_dot4(&Y[r][0], &V[0][jj], D, 1, kLrMaxR + 1);
         }
         __syncthreads();
         if (it == kLrIters) break;
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
         for (int o = c; o < R * S; o += D) {
             const int jj = o / S, i = o % S;
             base[(size_t)32 * D + (size_t)jj * S * 32 + ((size_t)(i / 4) * 32 + ln) * 4 + (i & 3)] =
-                lr_dot4(Pb + i, &V[0][ord_sh[jj]], D, S, kLrMaxR);
+                lr_dot4(Pb + i, &V[0][ord_sh[jj]], D, S, kLrMaxR + 1);
         }
         if (c < R) base[(size_t)32 * (D + R * S) + (size_t)c * 32 + ln] = lam_sh[ord_sh[c]];
         return;
