@@ -18,7 +18,11 @@ the per-channel population variance of the keys (the diagonal of the block covar
 the constant ln L is dropped (it is the same for every complete block); the group score
 is the sum of its heads' scores; candidates are the complete blocks at or before the
 query position; an empty branch contributes zero; gates arrive post-sigmoid in the
-order (compressed, selected, window).
+order (compressed, selected, window). For the compressed covariance forms of [COBS] §2.3:
+the low-rank eigenpairs come from a fixed float32 subspace iteration (pinned against
+numpy's eigh); FP4 keeps one float32 scale max|u|/6 per eigenvector; the query-subspace
+basis is given by the caller, and both the eigenvectors and the query heads are projected
+on it.
 
 Nothing here is blocked, fused or reordered: each function follows the definition it
 cites, with numpy's matmul, sum and sort as the only library steps.
