@@ -148,3 +148,21 @@ def test_summary_sizes_of_every_form(lib):
     ws_lr = lib.workspace_bytes(_p(variance="lowrank", rank=4, **kw), lib.COBS_WS_SELECT)
     ws_sub = lib.workspace_bytes(_p(variance="subspace", rank=4, sub=84, **kw), lib.COBS_WS_SELECT)
     assert ws_sub >= ws_lr + units * 4 * 84 * 4
+
+
+def test_header_compiles_as_c99_and_links_from_c(lib, tmp_path):
+    """The public header is plain C: a C99 program includes it with all warnings as errors,
+    links against the library and runs the host-side part of the ABI."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = str(tmp_path / "abi_from_c")
+    lib_dir = os.path.dirname(B.LIB)
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                           "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "abi_from_c.c"),
+                           "-L", lib_dir, "-lcobs", f"-Wl,-rpath,{lib_dir}", "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip() == "ok"
