@@ -594,8 +594,10 @@ def run_ours(args):
         same_idx = all(np.array_equal(ref["idx"][b, h], idx0[b, h]) for (b, h) in units)
         err = max(float(np.abs(ref["O"][b, h * w.G:(h + 1) * w.G] - O0[b, h * w.G:(h + 1) * w.G]).max())
                   for (b, h) in units)
+        gaps = [gp for (_, _, gp) in ref["near_ties"]]
         result["parity"] = {"units": len(units), "idx_bit_exact": same_idx, "out_max_abs_err": err,
-                            "out_tol": 2e-2}
+                            "out_tol": 2e-2,
+                            "fp64_near_ties": len(gaps), "fp64_near_tie_max_rel_gap": max(gaps) if gaps else None}
         del lim
     if not args.no_prefill and world == 1:
         wp = synth.WORKLOADS["prefill32k"]

@@ -227,7 +227,7 @@ class Buffers:
 
 
 def alloc(p: Params, prefill: bool, device="cuda") -> Buffers:
-    """Output and workspace tensors for one problem (workspaces zero-filled, as the ABI requires)."""
+    """Output and workspace tensors for one problem (workspaces zero-filled)."""
     dt = p.torch_dtype
     nq = p.T if prefill else 1
     summ = torch.empty(max(1, summaries_elems(p)), dtype=torch.float32, device=device)

@@ -85,6 +85,19 @@ cobs_status validate(const cobs_params* p) {
     }
     if (!isfinite(p->alpha)) return fail(COBS_ERR_INVALID_ARG, "alpha is not finite");
     if ((long long)p->B * p->Hkv > 65535) return fail(COBS_ERR_UNSUPPORTED, "B * Hkv > 65535");
+    // K / V rows (and the compressed rows, fewer) are addressed by int32 row coordinates in the
+    // TMA tensor maps and tile descriptors
+    if ((long long)p->B * p->Hkv * p->T > INT32_MAX)
+        return fail(COBS_ERR_UNSUPPORTED, "B * Hkv * T = %lld rows exceeds 2^31 - 1",
+                    (long long)p->B * p->Hkv * p->T);
+    return COBS_OK;
+}
+
+// Prefill calls address query rows [B, T, Hq] with int32 coordinates as well.
+cobs_status validate_prefill_rows(const cobs_params* p) {
+    if ((long long)p->B * p->Hq * p->T > INT32_MAX)
+        return fail(COBS_ERR_UNSUPPORTED, "B * Hq * T = %lld query rows exceeds 2^31 - 1",
+                    (long long)p->B * p->Hq * p->T);
     return COBS_OK;
 }
 
@@ -198,6 +211,7 @@ cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summar
     COBS_TRY(check_ptr(summaries, "summaries"));
     COBS_TRY(check_ptr(idx, "idx"));
     if (prefill != 0 && prefill != 1) return fail(COBS_ERR_INVALID_ARG, "prefill must be 0 or 1");
+    if (prefill) COBS_TRY(validate_prefill_rows(p));
     if (p->variance == COBS_VAR_SUBSPACE && !prefill) COBS_TRY(check_ptr(p->basis, "basis"));
     if (prefill && (p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4 ||
                     p->variance == COBS_VAR_SUBSPACE))
@@ -272,6 +286,7 @@ cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const 
                                      const void* Kc, const void* Vc, const int32_t* idx, const float* gates,
                                      void* O, void* workspace, size_t ws_bytes, cobs_stream_t stream) {
     COBS_TRY(attn_common(p, Q, K, V, Kc, Vc, idx, gates, O));
+    COBS_TRY(validate_prefill_rows(p));
     const cobs::Dims m = cobs::make_dims(*p);
     const size_t need = cobs::prefill_workspace_bytes(m);
     if (need > 0) {

@@ -183,9 +183,9 @@ cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summar
  *   softmax(q K^T / sqrt(d)) V of its own over the compressed tokens (all nC), the tokens
  *   of the selected blocks idx (entries -1 skipped) and the tokens max(0, T-W) .. T-1.
  *   An empty branch contributes zero.
- *   workspace: >= cobs_workspace_bytes(p, COBS_WS_DECODE) bytes, zero-filled before its
- *              first use; left zero-filled again on completion. Calls that share one
- *              workspace must not run concurrently.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_DECODE) bytes of scratch for the split-K
+ *              partial results; no initial contents are needed (every partial is written
+ *              before it is read). Calls that share one workspace must not run concurrently.
  */
 cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const void* K,
                                     const void* V, const void* Kc, const void* Vc,

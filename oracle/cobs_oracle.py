@@ -499,6 +499,29 @@ def osa_top_k(qs, K, L, ncand, k) -> np.ndarray:
     return top_k(exact_group_score(qs, K, L), ncand, k)
 
 
+def near_tie_gap(S64: np.ndarray, sel32: np.ndarray, ncand: int, k: int):
+    """How far apart, in float64, the blocks are on which the float32 selection differs from
+    the float64 one: None when both pick the same set, else the relative gap
+    (max S64 over the float64-only picks - min S64 over the float32-only picks) / max(1, max |S64|).
+
+    The float32 decision and the float64 ranking of the same definition ([COBS] §2.3 score,
+    [SKILL] "Method" top-k) can differ only where float64 scores lie within float32 rounding of
+    each other, so this gap is of the order of the float32 unit roundoff (about 1e-7) times the
+    magnitude of the summed terms.
+    """
+    sel64 = top_k(S64, ncand, k)
+    a = set(int(x) for x in sel64 if x >= 0)
+    b = set(int(x) for x in sel32 if x >= 0)
+    if a == b:
+        return None
+    S = np.asarray(S64[:ncand], np.float64)
+    only64, only32 = sorted(a - b), sorted(b - a)
+    hi = max(S[i] for i in only64) if only64 else -np.inf
+    lo = min(S[i] for i in only32) if only32 else np.inf
+    gap = max(0.0, hi - lo) if only64 and only32 else np.inf
+    return float(gap / max(1.0, float(np.abs(S).max())))
+
+
 def recall(sel: np.ndarray, ref: np.ndarray) -> float:
     a = set(int(x) for x in sel if x >= 0)
     b = set(int(x) for x in ref if x >= 0)
@@ -551,8 +574,8 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
     "subspace" (those eigenpairs with the eigenvectors as coordinates in basis [d, s]).
 
     Returns dict with idx [B, Hkv, k], O [B, Hq, d] (float64; rows of unlisted units are NaN),
-    summ, Kc, Vc per computed unit, and near-tie reports (units where the float64 ranking of
-    the group score disagrees with the float32 canonical one).
+    summ, Kc, Vc per computed unit, and near-tie reports (b, h, relative gap) for the units where
+    the float64 ranking of the group score disagrees with the float32 canonical one (near_tie_gap).
     """
     G, t = w.G, w.T - 1
     units = [(b, h) for b in range(w.B) for h in range(w.Hkv)] if units is None else units
@@ -587,9 +610,9 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
                                         w.alpha)
         else:
             S64 = group_scores(qs, mu, var, w.alpha)
-        sel64 = top_k(S64, n_candidates(t, w.block), w.topk)
-        if not np.array_equal(sel, sel64):
-            near_ties.append((b, h))
+        gap = near_tie_gap(S64, sel, n_candidates(t, w.block), w.topk)
+        if gap is not None:
+            near_ties.append((b, h, gap))
         O[b, h * G:(h + 1) * G] = position_output(qs, gates[b, h * G:(h + 1) * G], K, V, Kc, Vc, sel,
                                                   t, w.block, w.window, w.cmp_block, w.cmp_stride)
     return {"idx": idx, "O": O, "cache": cache, "near_ties": near_ties}

@@ -61,6 +61,7 @@ def _p(**kw):
     (dict(T=0), -1),
     (dict(cmp_stride=0), -1),
     (dict(alpha=float("nan")), -1),
+    (dict(B=65535, Hkv=1, Hq=1, T=65536), -2),          # B * Hkv * T rows beyond int32 coordinates
 ])
 def test_host_validation_rejects_before_launch(lib, kw, status):
     p = _p(**kw)
@@ -70,6 +71,19 @@ def test_host_validation_rejects_before_launch(lib, kw, status):
     assert r == status, lib._lib.cobs_last_error()
     assert lib._lib.cobs_last_error() != b""
     assert lib.workspace_bytes(p, lib.COBS_WS_DECODE) == 0
+
+
+def test_prefill_query_rows_bounded_by_int32(lib):
+    """B * Hq * T query rows beyond int32 coordinates: prefill calls refuse on the host; the decode
+    selection of the same shape (queries [B, Hq, d] only) is accepted by validation."""
+    p = _p(B=1024, Hkv=1, Hq=16, T=1 << 18)
+    cp = p.c()
+    fake = ctypes.c_void_p(256)
+    assert lib._lib.cobs_select(ctypes.byref(cp), fake, fake, 1, fake, fake, 1 << 40, None) == -2
+    assert b"query rows" in lib._lib.cobs_last_error()
+    assert lib._lib.cobs_sparse_attn_prefill(ctypes.byref(cp), fake, fake, fake, fake, fake, fake, fake, fake,
+                                             fake, 1 << 40, None) == -2
+    assert lib.summaries_elems(p) > 0
 
 
 def test_null_and_misaligned_pointers_rejected(lib):

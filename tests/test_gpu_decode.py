@@ -31,6 +31,10 @@ def _check_units(w, K, V, Q, gates, Pk, Pv, p, buf, units, check_out=True):
         qs = Qf[b, h * G:(h + 1) * G]
         sel, _ = O.select_decode(w, qs.astype(np.float32), summ_o)
         assert np.array_equal(idx_g[b, h], sel), f"idx unit {(b, h)}: {idx_g[b, h]} vs {sel}"
+        # the float32 decision against the float64 ranking of the same score
+        mu, var = O.block_summaries(Kf, w.block)
+        gap = O.near_tie_gap(O.group_scores(qs, mu, var, w.alpha), sel, O.n_candidates(w.T - 1, w.block), w.topk)
+        assert gap is None or gap < 1e-5, f"unit {(b, h)}: float32 and float64 selections differ by {gap}"
         if check_out:
             ref = O.position_output(qs, gates[b, h * G:(h + 1) * G], Kf, Vf, Kc_o, Vc_o, sel, w.T - 1, w.block,
                                     w.window, w.cmp_block, w.cmp_stride)

@@ -33,6 +33,14 @@ def _check(w, K, V, Q, gates, Pk, Pv, buf, positions, b=0, check_idx_all=True):
     pos = np.asarray(positions)
     Oref, idx_ref = O.prefill_positions(w, K, V, Q[b, pos], gates[b, pos], Pk, Pv, pos, b=b)
     assert np.array_equal(idx_g[b, pos], idx_ref)
+    # the float32 decisions against the float64 ranking of the same score at the checked positions
+    Qf = synth.to_f64(Q[b], w.dtype)
+    for h in range(w.Hkv):
+        mu, var = O.block_summaries(synth.to_f64(K[b, h], w.dtype), w.block)
+        for i, t in enumerate(pos):
+            S64 = O.group_scores(Qf[t, h * G:(h + 1) * G], mu, var, w.alpha)
+            gap = O.near_tie_gap(S64, idx_ref[i, h], O.n_candidates(int(t), w.block), w.topk)
+            assert gap is None or gap < 1e-5, f"position {t} group {h}: float32/float64 gap {gap}"
     err = np.abs(O_g[b, pos] - Oref).max()
     assert err <= TOL[w.dtype], f"max-abs {err}"
     return err

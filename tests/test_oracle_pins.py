@@ -157,6 +157,77 @@ def test_alpha_zero_is_first_order_mean_pool():
     assert list(O.top_k(S, nB, 8)) == list(ref)
 
 
+@pytest.mark.parametrize("G", [2, 4, 16])
+def test_group_score_identical_key_blocks_equal_exact_group_mass(G):
+    """Zero spread, several heads: every form's group score equals the exact group log-mass
+    sum_h (ln m_{h,b} - ln L) (COBS §2.1 mass, §2.2 series ending at kappa_1). A group score
+    that averaged, took the max, or dropped a head would miss it."""
+    rng = np.random.default_rng(11 + G)
+    L, d, nB = 64, 32, 6
+    rows = rng.standard_normal((nB, d)) * 0.7
+    K = np.repeat(rows, L, axis=0)
+    qs = rng.standard_normal((G, d))
+    exact = O.exact_group_score(qs, K, L)
+    mu, var = O.block_summaries(K, L)
+    tol = 1e-12 * G
+    np.testing.assert_allclose(O.group_scores(qs, mu, var, 1.0), exact, rtol=0, atol=tol)
+    np.testing.assert_allclose(O.group_scores_iso(qs, mu, var.mean(axis=1), 1.0), exact, rtol=0, atol=tol)
+    m2, u, lam = O.block_eigenpairs(K, L, 2)
+    np.testing.assert_allclose(O.group_scores_lowrank(qs, m2, u, lam, 1.0), exact, rtol=0, atol=1e-10 * G)
+    # the same blocks ranked by the exact group mass and by the group score
+    assert list(O.top_k(O.group_scores(qs, mu, var, 1.0), nB, 3)) == list(O.osa_top_k(qs, K, L, nB, 3))
+
+
+def test_group_score_gaussian_blocks_converge_to_exact_group_mass():
+    """Gaussian keys N(m, diag s^2), G = 4: the exact group log-mass of sampled blocks converges
+    (error ~ L^-1/2) to sum_h [q_h.m/sqrt(d) + 1/2 sum_c q_{h,c}^2 s_c^2 / d] (lognormal mean per
+    head, COBS §2.2), which is the group score of the population summaries; the first-order
+    group score keeps the bias sum_h 1/2 sum_c q_{h,c}^2 s_c^2 / d."""
+    rng = np.random.default_rng(21)
+    d, G = 8, 4
+    qs = rng.standard_normal((G, d)) * 0.8
+    m = rng.standard_normal(d) * 0.3
+    s = np.linspace(0.1, 0.45, d)
+    closed = sum(q @ m / np.sqrt(d) + 0.5 * (q * q) @ (s * s) / d for q in qs)
+    got = O.group_scores(qs, m[None], (s * s)[None], 1.0)[0]
+    assert abs(got - closed) < 1e-12
+    bias = sum(0.5 * (q * q) @ (s * s) / d for q in qs)
+    assert abs(O.group_scores(qs, m[None], (s * s)[None], 0.0)[0] - closed) == pytest.approx(bias, abs=1e-12)
+    errs, errs_emp = [], []
+    for logL in (10, 14, 18):
+        L = 1 << logL
+        K = m + s * rng.standard_normal((L, d))
+        exact = O.exact_group_score(qs, K, L)[0]
+        errs.append(abs(exact - closed))
+        mu, var = O.block_summaries(K, L)
+        errs_emp.append(abs(exact - O.group_scores(qs, mu, var, 1.0)[0]))
+    assert errs[2] < errs[0], errs
+    assert errs[2] < 0.01 and errs_emp[2] < 5e-3, (errs, errs_emp)
+    assert bias > 0.05 and errs_emp[2] < bias / 10
+
+
+def test_near_tie_gap_reports_only_float_level_disagreements():
+    """near_tie_gap: None when the float32 and float64 choices agree; otherwise the float64 gap
+    between the swapped blocks, relative to the largest score."""
+    S64 = np.array([3.0, 1.0, 2.0, 2.0 + 1e-9, 0.5])
+    assert O.near_tie_gap(S64, np.array([0, 3], np.int32), 5, 2) is None
+    gap = O.near_tie_gap(S64, np.array([0, 2], np.int32), 5, 2)   # float32 took 2 over 3
+    assert gap == pytest.approx(1e-9 / 3.0, rel=1e-6)
+    assert O.near_tie_gap(S64, np.array([0, 1], np.int32), 5, 2) == pytest.approx((2.0 + 1e-9 - 1.0) / 3.0)
+
+
+def test_float32_selection_agrees_with_float64_ranking_on_the_decode_workload():
+    """On seeded decode-workload units the float32 canonical choice equals the float64 top-k of
+    the same definition, or differs only at a float64 gap below 1e-5 relative."""
+    w = synth.WORKLOADS["decode32k"].replace(B=1, Hkv=2, Hq=8, T=8192)
+    K, V = synth.kv_cache(w)
+    Q, g = synth.queries_decode(w), synth.gates_decode(w)
+    Pk, Pv = synth.projections(w)
+    res = O.decode(w, K, V, Q, g, Pk, Pv)
+    for (_, _, gap) in res["near_ties"]:
+        assert gap < 1e-5
+
+
 def test_group_sum_reading_internal_consistency():
     """Group score = sum of head scores = collapsed form (reading; parity unpinned by the pages)."""
     rng = np.random.default_rng(5)

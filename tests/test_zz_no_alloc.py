@@ -21,8 +21,15 @@ from gpu_common import TOL, cobs, dev, params_of
 pytestmark = pytest.mark.gpu
 
 
-def _problem(seed):
-    w = synth.WORKLOADS["decode32k"].replace(B=2, Hkv=2, Hq=8, T=8192 + 64, seed=seed)
+# the bf16 stream kernel at d = 128 and d = 64, and the float32 chunk kernel (a different record
+# layout in the scratch array)
+CASES = [("decode32k", dict(B=2, Hkv=2, Hq=8, T=8192 + 64)),
+         ("decode32k", dict(B=2, Hkv=1, Hq=8, d=64, T=3000)),
+         ("tiny", dict(T=2048 + 17, Hq=4, Hkv=2))]
+
+
+def _problem(name, over, seed):
+    w = synth.WORKLOADS[name].replace(seed=seed, **over)
     K, V = synth.kv_cache(w)
     Q, g = synth.queries_decode(w), synth.gates_decode(w)
     Pk, Pv = synth.projections(w)
@@ -35,11 +42,12 @@ def _problem(seed):
     return p, buf, t
 
 
-def test_noalloc_decode_matches_workspace_call_on_consecutive_calls():
+@pytest.mark.parametrize("name,over", CASES)
+def test_noalloc_decode_matches_workspace_call_on_consecutive_calls(name, over):
     C = cobs()
     lib = C._lib
     for seed in (4242, 4343):   # two calls in a row, on different inputs
-        p, buf, t = _problem(seed)
+        p, buf, t = _problem(name, over, seed)
         ref = torch.empty_like(buf.O)
         C.cobs_sparse_attn_decode(p, t["Q"], t["K"], t["V"], buf.Kc, buf.Vc, buf.idx, t["g"], ref, buf.ws_attn)
         out = torch.full_like(buf.O, float("nan"))
@@ -52,7 +60,9 @@ def test_noalloc_decode_matches_workspace_call_on_consecutive_calls():
         torch.cuda.synchronize()
         assert C.device_error() == 0
         err = (out.float() - ref.float()).abs().max().item()
-        assert err <= TOL["bf16"], err
+        assert err <= TOL[p.dtype], err
+        # the same kernels on the same inputs: the results agree bit for bit
+        assert torch.equal(out, ref)
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
