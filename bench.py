@@ -16,6 +16,8 @@ batches, no collective on the data path: weak scaling); the step time is the max
 from __future__ import annotations
 
 import argparse
+import contextlib
+import dataclasses
 import hashlib
 import json
 import os
@@ -55,6 +57,8 @@ def parse():
                     help="sweep: draw anisotropic key blocks (spread on this many directions) instead of isotropic")
     ap.add_argument("--prefill-steps", type=int, default=5, help="timed prefill steps in the default run")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill sub-measurement")
+    ap.add_argument("--no-subrecords", action="store_true",
+                    help="skip the decode128k and selector-sweep sub-measurements of the default run")
     ap.add_argument("--T", type=int, default=None, help="override the context length (small profiling cases)")
     ap.add_argument("--copies", type=int, default=6, help="KV-cache copies rotated between steps (L2 defeat)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -89,8 +93,10 @@ def read_peaks():
 
 # the sources a kernel's DRAM traffic depends on (its own file and the headers it includes)
 KERNEL_SOURCES = {
-    "decode_attention": ["decode_stream.cu", "common.cuh", "dims.h", "tma.cu", "tma.h"],
-    "select_decode": ["select.cu", "common.cuh", "dims.h"],
+    "decode_step": ["decode_step.cu", "select_core.cuh", "stream_tile.cuh", "common.cuh", "dims.h", "tma.cu",
+                    "tma.h"],
+    "decode_attention": ["decode_stream.cu", "stream_tile.cuh", "common.cuh", "dims.h", "tma.cu", "tma.h"],
+    "select_decode": ["select.cu", "select_core.cuh", "common.cuh", "dims.h"],
     "prefill_tc": ["prefill.cu", "tc.cuh", "common.cuh", "dims.h", "tma.cu", "tma.h"],
 }
 
@@ -210,58 +216,134 @@ def decode_bytes(w, idx, variance="channel", rank=4, sub=84):
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=False, variance="channel", rank=4,
-                         basis=None):
-    """Time the oracle (as it stands) on the listed units; returns (seconds, query heads[, result])."""
-    from oracle import cobs_oracle as O
-    t0 = time.perf_counter()
-    res = O.decode(w, K, V, Q, g, Pk, Pv, units=units, variance=variance, rank=rank, basis=basis)
-    secs = time.perf_counter() - t0
-    return (secs, len(units) * w.G, res) if with_result else (secs, len(units) * w.G)
-
-
-def limit_threads():
+def host_cores() -> int:
     try:
-        from threadpoolctl import threadpool_limits
-        return threadpool_limits(limits=1)
-    except Exception:  # pragma: no cover
-        return None
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+_ORACLE_STATE = {}
+
+
+def _oracle_worker_init(w, shm_names, shapes, dtypes, Q, g, Pk, Pv, variance, rank, basis):
+    """Pool worker: attach the shared K / V cache (no copy) and keep the small inputs."""
+    import numpy as np
+    from multiprocessing import shared_memory
+    os.environ["OMP_NUM_THREADS"] = "1"
+    shms = [shared_memory.SharedMemory(name=n) for n in shm_names]
+    arrs = [np.ndarray(sh, dtype=dt, buffer=m.buf) for m, sh, dt in zip(shms, shapes, dtypes)]
+    _ORACLE_STATE.update(w=w, shms=shms, K=arrs[0], V=arrs[1], Q=Q, g=g, Pk=Pk, Pv=Pv, variance=variance,
+                         rank=rank, basis=basis)
+
+
+def _oracle_worker_unit(unit):
+    """The oracle (as it stands, float64) on one (batch, KV-head) unit: its idx row, its output
+    rows and its near-tie report."""
+    from oracle import cobs_oracle as O
+    st = _ORACLE_STATE
+    w = st["w"]
+    b, h = unit
+    res = O.decode(w, st["K"], st["V"], st["Q"], st["g"], st["Pk"], st["Pv"], units=[unit],
+                   variance=st["variance"], rank=st["rank"], basis=st["basis"])
+    return unit, res["idx"][b, h], res["O"][b, h * w.G:(h + 1) * w.G], res["near_ties"]
+
+
+class OraclePool:
+    """The oracle on all host cores: one process per core (spawned, so safe after CUDA is up),
+    each taking whole (batch, KV-head) units; K and V are shared, not copied."""
+
+    def __init__(self, w, K, V, Q, g, Pk, Pv, variance="channel", rank=4, basis=None, procs=None):
+        import numpy as np
+        from multiprocessing import get_context, shared_memory
+        self.procs = procs or host_cores()
+        self.shms = []
+        names, shapes, dtypes = [], [], []
+        for a in (K, V):
+            a = np.ascontiguousarray(a)
+            m = shared_memory.SharedMemory(create=True, size=max(1, a.nbytes))
+            np.ndarray(a.shape, dtype=a.dtype, buffer=m.buf)[...] = a
+            self.shms.append(m)
+            names.append(m.name)
+            shapes.append(a.shape)
+            dtypes.append(a.dtype)
+        os.environ.setdefault("OMP_NUM_THREADS", "1")
+        self.pool = get_context("spawn").Pool(self.procs, initializer=_oracle_worker_init,
+                                              initargs=(w, names, shapes, dtypes, Q, g, Pk, Pv, variance, rank,
+                                                        basis))
+        # every worker started before any timing (bounded: a worker that cannot start fails the run)
+        self.pool.map_async(int, range(self.procs)).get(timeout=300)
+
+    def run(self, units):
+        """(seconds of wall time, results per unit)."""
+        t0 = time.perf_counter()
+        out = self.pool.map_async(_oracle_worker_unit, units, chunksize=1).get(timeout=3600)
+        return time.perf_counter() - t0, out
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+        for m in self.shms:
+            m.close()
+            m.unlink()
+
+
+def decode_config(w, args, R=None, world=1):
+    """The `config` object of a decode line (identical for both arms)."""
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
+           "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
+           "variance": args.variance}
+    if args.variance in ("lowrank", "lowrank_fp4", "subspace"):
+        cfg["rank"] = args.rank
+    if args.variance == "subspace":
+        cfg.update(sub=args.sub, queries="concentrated in the subspace (leak 0.1)")
+    cfg["step"] = ("cobs_decode_step: summary update at T-1, then selection + decode attention in one kernel; "
+                   "one CUDA graph")
+    cfg["l2"] = f"{R or max(1, args.copies)} KV-cache copies rotated between steps (working set > L2)"
+    cfg["parallelism"] = f"dp{world} (independent decode batches per GPU)"
+    return cfg
 
 
 def run_reference(args):
-    """Reference arm: the CPU oracle on host cores, bounded sample per step."""
+    """Reference arm: the CPU oracle on the host cores, every step all units of the workload
+    spread over one process per core (rank 0 only)."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     import synth
     w = synth.WORKLOADS[args.workload]
-    os.environ.setdefault("OMP_NUM_THREADS", "1")
-    lim = limit_threads()
+    if args.batch:
+        w = w.replace(B=args.batch)
     units_all = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     K, V = synth.kv_cache(w)
     Q, g = synth.queries_decode(w), synth.gates_decode(w)
     Pk, Pv = synth.projections(w)
-    per_step = 1
-    for i in range(args.warmup):
-        oracle_decode_sample(w, K, V, Q, g, Pk, Pv, [units_all[i % len(units_all)]])
-    secs, heads = 0.0, 0
-    for i in range(args.steps):
-        s, hh = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, [units_all[i % len(units_all)]])
-        secs += s
-        heads += hh
+    pool = OraclePool(w, K, V, Q, g, Pk, Pv)
+    # a bounded sample per step: as many units as there are worker processes
+    per_step = min(len(units_all), pool.procs)
+    try:
+        for i in range(args.warmup):
+            pool.run([units_all[(i * per_step + j) % len(units_all)] for j in range(per_step)])
+        secs, heads = 0.0, 0
+        for i in range(args.steps):
+            sec, _ = pool.run([units_all[(i * per_step + j) % len(units_all)] for j in range(per_step)])
+            secs += sec
+            heads += per_step * w.G
+    finally:
+        pool.close()
     value = heads / secs
-    sample = f"{per_step} (batch, KV-head) unit of {w.name} per step ({w.G} query heads), full oracle decode"
+    sample = (f"{per_step} (batch, KV-head) units of {w.name} per step ({per_step * w.G} query heads, "
+              f"one process per unit), full oracle decode incl. summaries")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "query-heads/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
-                   "window": w.window},
-        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "config": decode_config(w, args, world=world),
+        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": pool.procs, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "query-heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
-    del lim
     return 0
 
 
@@ -361,33 +443,34 @@ def bench_prefill(w, steps, warmup, dev, cobs):
     }
 
 
-def run_ours(args):
+def traffic_ratios(w, idx, idx_a0, variance="channel", rank=4, sub=84):
+    """KV-cache read traffic of one decode step ([COBS] §4.1 "Verkehrseffizienz"): dense attention
+    (every K and V row of the context), COBS (its summaries, the compressed K/V and the K/V of the
+    selected blocks and the window, from idx) and first-order mean-pool selection (alpha = 0: the
+    means alone, the compressed K/V and the K/V of its own selected blocks and the window)."""
+    d, esz = w.d, 2 if w.dtype == "bf16" else 4
+    units = w.B * w.Hkv
+    dense = units * w.T * 2 * d * esz
+    cobs_b = decode_bytes(w, idx, variance, rank, sub)
+    first = decode_bytes(w, idx_a0, "isotropic")
+    # first order keeps only the block means: drop the isotropic scalar from the summary bytes
+    first_sel = first["select"] - units * w.nB * 4
+    cobs_read = cobs_b["select"] + cobs_b["attn"]
+    first_read = first_sel + first["attn"]
+    return {"dense_bytes": dense, "cobs_bytes": cobs_read, "first_order_bytes": first_read,
+            "dense_over_cobs": dense / cobs_read, "cobs_over_first_order": cobs_read / first_read,
+            "definition": "bytes read per decode step from idx: dense = all K/V rows; COBS = summaries + "
+                          "compressed K/V + K/V of (selected blocks U window) + Q, gates, O; first order = "
+                          "block means + the same with its own alpha = 0 selection"}
+
+
+def measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=True, clocks=True):
+    """Time the decode step of workload w on this GPU (see the module docstring); returns the
+    measurements, the selected blocks and outputs of copy 0, and the host inputs."""
     import numpy as np
     import torch
     import torch.distributed as dist
-
-    rank, world, local = dist_env()
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-
-    from block_sparse_long_summary_b200 import build as B
-    if rank == 0:
-        B.build()
-    if world > 1:
-        dist.barrier()
-    from block_sparse_long_summary_b200 import cobs
     import synth
-
-    w = synth.WORKLOADS[args.workload]
-    if args.batch:
-        w = w.replace(B=args.batch)
-    if args.T:
-        w = w.replace(T=args.T)
-    if w.mode == "prefill":
-        return run_prefill_line(args, w, dev, cobs, rank, world)
     basis = synth.subspace_basis(w, args.sub) if args.variance == "subspace" else None
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
@@ -398,7 +481,6 @@ def run_ours(args):
     g = synth.gates_decode(w)
     Pk, Pv = synth.projections(w)
 
-    R = max(1, args.copies)
     tQ, tg = to_dev(Q, w.dtype, dev), torch.from_numpy(g).to(dev)
     tPk, tPv = to_dev(Pk, "f32", dev), to_dev(Pv, "f32", dev)
     Ks = [to_dev(K, w.dtype, dev) for _ in range(R)]
@@ -416,7 +498,7 @@ def run_ours(args):
 
     # warm-up, then one CUDA graph per cache copy
     with torch.cuda.stream(stream):
-        for i in range(max(3, args.warmup)):
+        for i in range(max(3, warmup)):
             step(i % R)
     stream.synchronize()
     launches0 = cobs.launch_count()
@@ -430,64 +512,114 @@ def run_ours(args):
     for r in range(R):
         graphs[r].replay()
     stream.synchronize()
-
     idx0 = bufs[0].idx.cpu().numpy()
     O0 = bufs[0].O.float().cpu().numpy()
+    # first-order (alpha = 0) selection on the same summaries, for the traffic comparison
+    p0 = dataclasses.replace(p, alpha=0.0)
+    idx_a0_t = torch.empty_like(bufs[0].idx)
+    with torch.cuda.stream(stream):
+        cobs.cobs_select(p0, tQ, bufs[0].summaries, 0, idx_a0_t, bufs[0].ws_select)
+    stream.synchronize()
+    idx_a0 = idx_a0_t.cpu().numpy()
 
     # ---- timed region: K graph replays, cache copies rotated (L2 defeat) ----
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk, torch.cuda.stream(stream):   # replay() launches on the current stream
+    gpu = dev.index if dev.index is not None else 0
+    with (ClockSampler(gpu) if clocks else contextlib.nullcontext()) as clk, torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             graphs[i % R].replay()
         e1.record(stream)
         torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
     if world > 1:
         dist.barrier()
-    clocks = clk.summary()
+    clk_summary = clk.summary() if clocks else None
 
-    # ---- per-call durations inside the step: a second set of step graphs with timing events
-    # captured between the calls (event-record nodes), replayed one at a time on the launching
-    # stream with the same copy rotation; the headline graphs above carry no events ----
-    tgraphs, tevs = [], []
+    # ---- per-call durations: graphs of one part of the step each, replayed one at a time on the
+    # launching stream with the same copy rotation (cold, isolated figures: no overlap with the
+    # neighbouring kernels): the summary update alone; the fused selection + attention kernel alone
+    # (cobs_decode_step with nothing to update); and the three separate calls of the unfused step ----
+    def timed_parts(build_parts, nparts):
+        graphs_, evs_ = [], []
+        for r in range(R):
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nparts + 1)]
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                evs[0].record(stream)
+                for j, part in enumerate(build_parts(r)):
+                    part()
+                    evs[j + 1].record(stream)
+            graphs_.append(gr)
+            evs_.append(evs)
+        out = []
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(steps + R):
+                r = i % R
+                graphs_[r].replay()
+                stream.synchronize()
+                if i >= R:   # the first pass over the copies is a warm-up
+                    e = evs_[r]
+                    out.append([e[j].elapsed_time(e[j + 1]) for j in range(nparts)])
+        del graphs_
+        return [statistics.median(x[j] for x in out) for j in range(nparts)]
+
+    def upd(r):
+        return lambda: cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc,
+                                                 bufs[r].Vc)
+
+    def fused_only(r):
+        return lambda: cobs.cobs_decode_step(p, tQ, Ks[r], Vs[r], tPk, tPv, w.T, bufs[r].summaries, bufs[r].Kc,
+                                             bufs[r].Vc, bufs[r].idx, tg, bufs[r].O, bufs[r].ws_step)
+
+    t_upd, t_fused = timed_parts(lambda r: [upd(r), fused_only(r)], 2)
+    t_upd2, t_sel, t_att = timed_parts(lambda r: [
+        upd(r),
+        lambda: cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select),
+        lambda: cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg,
+                                             bufs[r].O, bufs[r].ws_attn)], 3)
+    # the unfused step (three calls, five kernels) as one graph, for comparison with the headline
+    ugraphs = []
     for r in range(R):
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
         gr = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gr, stream=stream):
-            evs[0].record(stream)
-            cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc, bufs[r].Vc)
-            evs[1].record(stream)
-            cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select)
-            evs[2].record(stream)
-            cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg, bufs[r].O,
-                                         bufs[r].ws_attn)
-            evs[3].record(stream)
-        tgraphs.append(gr)
-        tevs.append(evs)
-    t_parts = []
+            cobs.decode_step(p, tQ, Ks[r], Vs[r], tPk, tPv, tg, bufs[r], t_begin=w.T - 1, fused=False)
+        ugraphs.append(gr)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        for i in range(args.steps + R):
-            r = i % R
-            tgraphs[r].replay()
-            stream.synchronize()
-            if i >= R:   # the first pass over the copies is a warm-up
-                e = tevs[r]
-                t_parts.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])))
-    t_upd = statistics.median(x[0] for x in t_parts)
-    t_sel = statistics.median(x[1] for x in t_parts)
-    t_att = statistics.median(x[2] for x in t_parts)
-    del tgraphs
+        for i in range(R):
+            ugraphs[i].replay()
+        e0.record(stream)
+        for i in range(steps):
+            ugraphs[i % R].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms_unfused = e0.elapsed_time(e1) / steps
+    del ugraphs
 
-    # ---- end to end through the public API: pinned host inputs in, output back, every step ----
-    # The step's inputs travel in one pinned host buffer: Q | gates | the appended token's K rows
-    # | its V rows (byte offsets 16-aligned), copied to a device staging buffer with one
-    # host-to-device copy; Q and gates are used in place, the K / V rows are scattered into
-    # the cache at T-1. O comes back with one device-to-host copy.
+    e2e = None
+    if with_e2e:
+        e2e = measure_e2e(w, p, Q, g, Ks, Vs, bufs, tPk, tPv, tQ, tg, stream, dev, cobs, R, steps)
+    out = {"ms": ms, "clocks": clk_summary, "t_upd": t_upd, "t_fused": t_fused, "t_upd2": t_upd2, "t_sel": t_sel,
+           "t_att": t_att, "ms_unfused": ms_unfused, "e2e": e2e, "launches_per_step": launches_per_step,
+           "device_error": cobs.device_error(), "idx0": idx0, "O0": O0, "idx_a0": idx_a0,
+           "host": (K, V, Q, g, Pk, Pv, basis)}
+    del graphs[:], Ks, Vs, bufs
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_e2e(w, p, Q, g, Ks, Vs, bufs, tPk, tPv, tQ, tg, stream, dev, cobs, R, steps):
+    """The step end to end through the public API: the step's inputs in one pinned host buffer
+    (Q | gates | the appended token's K rows | its V rows, byte offsets 16-aligned), copied to the
+    device with one host-to-device copy (Q and gates used in place, the K / V rows scattered into
+    the cache at T-1), cobs_decode_step, and O back with one device-to-host copy."""
+    import numpy as np
+    import torch
     esz = 2 if w.dtype == "bf16" else 4
     nq, ng, nkv = Q.size * esz, g.size * 4, w.B * w.Hkv * w.d * esz
     offs = [0, nq, nq + ng, nq + ng + nkv]
@@ -518,13 +650,13 @@ def run_ours(args):
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         a0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             e2e_step(i % R)
         a1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e_eager = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev)
-    # the same step (copies in from pinned memory, the three calls, the copy out) captured once
-    # in a CUDA graph per cache copy and replayed: how a serving loop would issue it
+    ms_eager = max_over_ranks(a0.elapsed_time(a1) / steps, dev)
+    # the same step (copies in from pinned memory, the call, the copy out) captured once in a CUDA
+    # graph per cache copy and replayed: how a serving loop would issue it
     e2e_graphs = []
     for r in range(R):
         gr = torch.cuda.CUDAGraph()
@@ -536,78 +668,161 @@ def run_ours(args):
         for i in range(R):
             e2e_graphs[i].replay()
         a0.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             e2e_graphs[i % R].replay()
         a1.record(stream)
     torch.cuda.synchronize()
     e2e_graphs.clear()
-    ms_e2e = max_over_ranks(a0.elapsed_time(a1) / args.steps, dev)
-    dev_err = cobs.device_error()
+    ms_graph = max_over_ranks(a0.elapsed_time(a1) / steps, dev)
+    return {"ms": ms_graph, "ms_eager": ms_eager, "h2d": h2d, "d2h": d2h}
 
+
+def oracle_parity(w, idx_g, O_g, res_units, tol):
+    """Compare the GPU's idx and outputs of copy 0 with the oracle results of the listed units."""
+    import numpy as np
+    same_idx, err, gaps = True, 0.0, []
+    for (unit, idx_u, O_u, near) in res_units:
+        b, h = unit
+        same_idx &= bool(np.array_equal(idx_u, idx_g[b, h]))
+        err = max(err, float(np.abs(O_u - O_g[b, h * w.G:(h + 1) * w.G]).max()))
+        gaps += [gp for (_, _, gp) in near]
+    return {"units": len(res_units), "idx_bit_exact": same_idx, "out_max_abs_err": err, "out_tol": tol,
+            "fp64_near_ties": len(gaps), "fp64_near_tie_max_rel_gap": max(gaps) if gaps else None}
+
+
+def decode_subrecord(name, args, dev, cobs, world, steps=50, warmup=5, R=4):
+    """A decode workload other than the headline one, measured the same way (no end-to-end
+    pass): step time, the fused kernel's roofline, traffic ratios, oracle parity on two units."""
+    import synth
+    w = synth.WORKLOADS[name]
+    m = measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=False, clocks=False)
+    by = decode_bytes(w, m["idx0"], args.variance, args.rank, args.sub)
+    peak, peak_kind = read_peaks()
+    fused_gbs = (by["select"] + by["attn"]) / (m["t_fused"] * 1e-3) / 1e9
+    rec = {"workload": name, "config": decode_config(w, args, R, world), "ms_per_step": m["ms"],
+           "value": w.B * w.Hq * world / (m["ms"] * 1e-3), "unit": "query-heads/s",
+           "hbm_gbs": by["total"] / (m["ms"] * 1e-3) / 1e9, "hbm_bytes_per_step": by["total"],
+           "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": fused_gbs, "peak": peak,
+                        "unit": "GB/s", "frac": fused_gbs / peak, "peak_kind": peak_kind,
+                        "algorithmic_bytes_per_launch": by["select"] + by["attn"]},
+           "calls_ms": {"build_summaries_update": m["t_upd"], "decode_step_kernel": m["t_fused"],
+                        "unfused_ms_per_step": m["ms_unfused"], "select": m["t_sel"], "sparse_attn_decode": m["t_att"]},
+           "traffic": traffic_ratios(w, m["idx0"], m["idx_a0"], args.variance, args.rank, args.sub),
+           "gpu_launches": m["launches_per_step"] * steps, "steps": steps, "device_error": m["device_error"]}
+    if not args.no_cpu_baseline:
+        K, V, Q, g, Pk, Pv, basis = m["host"]
+        pool = OraclePool(w, K, V, Q, g, Pk, Pv, args.variance, args.rank, basis, procs=min(2, host_cores()))
+        try:
+            _, res = pool.run([(0, 0), (w.B - 1, w.Hkv - 1)])
+        finally:
+            pool.close()
+        rec["parity"] = oracle_parity(w, m["idx0"], m["O0"], res, 2e-2)
+    return rec
+
+
+def sweep_subrecord(args, dev, cobs, contexts):
+    """The selector sweep at a few context lengths (GB/s and recall), as run_sweep measures it."""
+    rows = sweep_rows(args, dev, cobs, contexts)
+    return {"workload": "sweep", "contexts": contexts, "rows": rows,
+            "definition": "cobs_select on 64 sequences x 8 KV heads (32 query heads, top-16); GB/s of the "
+                          "summaries read; recall@16 of alpha = 1 and alpha = 0 against the exact-mass top-16 "
+                          "on the first 8 sequences"}
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from block_sparse_long_summary_b200 import build as B
+    if rank == 0:
+        B.build()
+    if world > 1:
+        dist.barrier()
+    from block_sparse_long_summary_b200 import cobs
+    import synth
+
+    w = synth.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(B=args.batch)
+    if args.T:
+        w = w.replace(T=args.T)
+    if w.mode == "prefill":
+        return run_prefill_line(args, w, dev, cobs, rank, world)
+    R = max(1, args.copies)
+    m = measure_decode(w, args, dev, cobs, world, R, args.steps, args.warmup)
+    ms, e2e = m["ms"], m["e2e"]
+    idx0, O0 = m["idx0"], m["O0"]
     qheads = w.B * w.Hq * world
     by = decode_bytes(w, idx0, args.variance, args.rank, args.sub)
     peak, peak_kind = read_peaks()
-    att_gbs = by["attn"] / (t_att * 1e-3) / 1e9
+    fused_gbs = (by["select"] + by["attn"]) / (m["t_fused"] * 1e-3) / 1e9
+    att_gbs = by["attn"] / (m["t_att"] * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": qheads / (ms * 1e-3), "unit": "query-heads/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
-                   "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
-                   "variance": args.variance,
-                   **({"rank": args.rank} if args.variance in ("lowrank", "lowrank_fp4", "subspace") else {}),
-                   **({"sub": args.sub, "queries": "concentrated in the subspace (leak 0.1)"}
-                      if args.variance == "subspace" else {}),
-                   "step": "summary update at T-1 + select + decode attention, one CUDA graph",
-                   "l2": f"{R} KV-cache copies rotated between steps (working set {R} x step bytes > L2)",
-                   "parallelism": f"dp{world} (independent decode batches per GPU)"},
+        "config": decode_config(w, args, R, world),
         "hbm_gbs": by["total"] / (ms * 1e-3) / 1e9,
         "hbm_bytes_per_step": by["total"],
-        "roofline": {"bound": "hbm", "kernel": "cobs_sparse_attn_decode (decode_stream_kernel + decode_stream_merge)",
-                     "achieved": att_gbs, "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
-                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": by["attn"],
-                     "traffic": recorded_traffic("decode_attention")},
-        "calls_ms": {"build_summaries_update": t_upd, "select": t_sel, "sparse_attn_decode": t_att,
-                     "select_gbs": by["select"] / (t_sel * 1e-3) / 1e9},
-        "e2e": {"value": qheads / (ms_e2e * 1e-3), "unit": "query-heads/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel (selection + three-branch attention, one launch)",
+                     "achieved": fused_gbs, "peak": peak, "unit": "GB/s", "frac": fused_gbs / peak,
+                     "peak_kind": f"{peak_kind} (copy, read + write)",
+                     "algorithmic_bytes_per_launch": by["select"] + by["attn"],
+                     "timing": "CUDA events around the kernel alone (graph per copy, replayed on the launching "
+                               "stream, median)",
+                     "traffic": recorded_traffic("decode_step")},
+        "calls_ms": {"build_summaries_update": m["t_upd"], "decode_step_kernel": m["t_fused"],
+                     "unfused": {"ms_per_step": m["ms_unfused"], "build_summaries_update": m["t_upd2"],
+                                 "select": m["t_sel"], "sparse_attn_decode": m["t_att"],
+                                 "select_gbs": by["select"] / (m["t_sel"] * 1e-3) / 1e9,
+                                 "attn_gbs": att_gbs, "attn_frac": att_gbs / peak}},
+        "traffic": traffic_ratios(w, idx0, m["idx_a0"], args.variance, args.rank, args.sub),
+        "e2e": {"value": qheads / (e2e["ms"] * 1e-3), "unit": "query-heads/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms"],
                 "issue": "one CUDA graph per step: one H2D copy of Q, gates and the appended K/V rows "
-                         "from pinned memory, the rows scattered into the cache, cobs_build_summaries + "
-                         "cobs_select + cobs_sparse_attn_decode, one D2H copy of O",
-                "eager_value": qheads / (ms_e2e_eager * 1e-3), "eager_ms_per_step": ms_e2e_eager},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks,
-        "device_error": dev_err,
+                         "from pinned memory, the rows scattered into the cache, cobs_decode_step, one D2H "
+                         "copy of O",
+                "eager_value": qheads / (e2e["ms_eager"] * 1e-3), "eager_ms_per_step": e2e["ms_eager"]},
+        "gpu_launches": m["launches_per_step"] * args.steps,
+        "clocks": m["clocks"],
+        "device_error": m["device_error"],
         "kv_tokens_per_unit": by["kv_tokens_per_unit"],
     }
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        os.environ.setdefault("OMP_NUM_THREADS", "1")
-        lim = limit_threads()
-        units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:24]
-        secs, heads, ref = oracle_decode_sample(w, K, V, Q, g, Pk, Pv, units, with_result=True,
-                                                variance=args.variance, rank=args.rank, basis=basis)
-        result["cpu_baseline"] = {"value": heads / secs, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
-                                  "sample": f"{len(units)} of {w.B * w.Hkv} (batch, KV-head) units of {w.name}, "
-                                            f"full oracle decode incl. summaries ({secs:.1f} s)"}
+        # the oracle as it stands on every host core: all units of the workload, one process per core
+        K, V, Q, g, Pk, Pv, basis = m["host"]
+        units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+        pool = OraclePool(w, K, V, Q, g, Pk, Pv, args.variance, args.rank, basis)
+        try:
+            secs, res = pool.run(units)
+        finally:
+            pool.close()
+        result["cpu_baseline"] = {"value": len(units) * w.G / secs, "unit": "query-heads/s", "cores": pool.procs,
+                                  "kind": "oracle",
+                                  "sample": f"all {len(units)} (batch, KV-head) units of {w.name} over "
+                                            f"{pool.procs} processes, full oracle decode incl. summaries "
+                                            f"({secs:.1f} s)"}
         # the same oracle run checks what the bench ran: indices bit for bit, outputs within 2e-2
-        same_idx = all(np.array_equal(ref["idx"][b, h], idx0[b, h]) for (b, h) in units)
-        err = max(float(np.abs(ref["O"][b, h * w.G:(h + 1) * w.G] - O0[b, h * w.G:(h + 1) * w.G]).max())
-                  for (b, h) in units)
-        gaps = [gp for (_, _, gp) in ref["near_ties"]]
-        result["parity"] = {"units": len(units), "idx_bit_exact": same_idx, "out_max_abs_err": err,
-                            "out_tol": 2e-2,
-                            "fp64_near_ties": len(gaps), "fp64_near_tie_max_rel_gap": max(gaps) if gaps else None}
-        del lim
+        result["parity"] = oracle_parity(w, idx0, O0, res, 2e-2)
+    if world == 1 and args.workload == "decode32k" and not args.no_subrecords:
+        result["decode128k"] = decode_subrecord("decode128k", args, dev, cobs, world)
+        result["sweep"] = sweep_subrecord(args, dev, cobs, [8192, 131072, 1048576])
     if not args.no_prefill and world == 1:
         wp = synth.WORKLOADS["prefill32k"]
-        del Ks, Vs, bufs, graphs[:]
         torch.cuda.empty_cache()
         result["prefill"] = bench_prefill(wp, args.prefill_steps, 2, dev, cobs)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
-        graphs.clear()
         dist.destroy_process_group()
     return 0
 
@@ -638,28 +853,21 @@ def osa_top_k(E, k):
     return np.sort(order[:k])
 
 
-def run_sweep(args):
+def sweep_rows(args, dev, cobs, contexts):
     """Decode selection (cobs_select) on 64 sequences x 8 KV heads (32 query heads, top-16) at
     each context length: GB/s of the selector, and recall@16 of alpha = 1 and alpha = 0 against
     the oracle sparse attention (top-16 blocks by exact attention mass, from cobs_block_log_mass)
     on the first 8 sequences. Keys are drawn on the device; only summaries stay resident."""
     import numpy as np
     import torch
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    from block_sparse_long_summary_b200 import build as B
-    B.build()
-    from block_sparse_long_summary_b200 import cobs
     import synth
     base = synth.WORKLOADS["sweep"]
     if args.batch:
         base = base.replace(B=args.batch)
-    contexts = [int(x) for x in args.contexts.split(",")] if args.contexts else list(synth.SWEEP_CONTEXTS)
     peak, peak_kind = read_peaks()
     n_rec = min(8, base.B)
     l2_bytes = 126e6
-    rows, launches = [], 0
+    rows = []
     stream = torch.cuda.Stream(device=dev)
 
     basis = synth.subspace_basis(base, args.sub) if args.variance == "subspace" else None
@@ -730,7 +938,7 @@ def run_sweep(args):
         stream.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / n_rep
         idx_a1 = idx.cpu().numpy()
-        launches += cobs.launch_count() - n0
+        launches = cobs.launch_count() - n0
         m = mass.cpu().numpy().astype(np.float64)
         rec1, rec0 = [], []
         for b in range(n_rec):
@@ -744,24 +952,46 @@ def run_sweep(args):
         gbs = by / (us * 1e-6) / 1e9
         rows.append({"T": T, "nB": nB, "bytes": by, "us": us, "gbs": gbs, "frac": gbs / peak,
                      "recall_alpha1": float(np.mean(rec1)), "recall_alpha0": float(np.mean(rec0)),
-                     "l2": f"{R} summary copies rotated" if R > 1 else "summaries larger than L2"})
+                     "l2": f"{R} summary copies rotated" if R > 1 else "summaries larger than L2",
+                     "gpu_launches": launches, "steps": n_rep})
         del graphs, copies, summ, mass
         torch.cuda.empty_cache()
+    return rows
+
+
+def run_sweep(args):
+    """The selector sweep as its own line (sweep_rows over the listed or all context lengths)."""
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from block_sparse_long_summary_b200 import build as B
+    B.build()
+    from block_sparse_long_summary_b200 import cobs
+    import synth
+    base = synth.WORKLOADS["sweep"]
+    if args.batch:
+        base = base.replace(B=args.batch)
+    contexts = [int(x) for x in args.contexts.split(",")] if args.contexts else list(synth.SWEEP_CONTEXTS)
+    peak, peak_kind = read_peaks()
+    n_rec = min(8, base.B)
+    rows = sweep_rows(args, dev, cobs, contexts)
+    basis_used = args.variance == "subspace" or args.subspace_queries
     top = rows[-1]
     line = {"metric": "selector GB/s over context length (decode selection, 64 x 8 units, top-16)",
-            "value": top["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": n_rep, "warmup": max(3, args.warmup),
+            "value": top["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": top["steps"], "warmup": max(3, args.warmup),
             "ms_per_step": top["us"] * 1e-3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic (keys drawn on the device" +
                                     (f", anisotropic blocks of rank {args.aniso})" if args.aniso else ")"),
             "config": {"workload": "sweep", "B": base.B, "Hq": base.Hq, "Hkv": base.Hkv, "d": base.d,
                        "topk": base.topk, "contexts": contexts, "variance": args.variance,
                        **({"sub": args.sub, "queries": "concentrated in the subspace (leak 0.1)"}
-                          if qbasis is not None else {}),
+                          if basis_used else {}),
                        "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
             "roofline": {"bound": "hbm", "kernel": "select_decode_kernel", "achieved": top["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": top["frac"], "peak_kind": peak_kind,
                          "traffic": recorded_traffic("select_decode")},
-            "sweep": rows, "gpu_launches": launches, "device_error": cobs.device_error()}
+            "sweep": rows, "gpu_launches": sum(r["gpu_launches"] for r in rows), "device_error": cobs.device_error()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0

@@ -7,6 +7,8 @@
 
 namespace cobs {
 
+constexpr unsigned kFull = 0xffffffffu;  // all lanes of a warp
+
 // Error codes written to the device error flag (first error wins).
 enum DeviceError : int {
     kErrBadIndex = 1,      // a selected block index outside [0, nB)

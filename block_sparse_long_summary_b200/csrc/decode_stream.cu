@@ -20,25 +20,20 @@
 
 #include "common.cuh"
 #include "dims.h"
+#include "stream_tile.cuh"
 #include "tma.h"
 
 namespace cobs {
 namespace {
 
-#ifndef COBS_DECODE_TK
-#define COBS_DECODE_TK 32
-#endif
 #ifndef COBS_DECODE_STAGES
 #define COBS_DECODE_STAGES 3
 #endif
 #ifndef COBS_DECODE_WARPS
 #define COBS_DECODE_WARPS 4
 #endif
-constexpr int kTK = COBS_DECODE_TK;          // keys per tile (16 or 32)
 constexpr int kStages = COBS_DECODE_STAGES;  // ring depth per warp
 constexpr int kWarps = COBS_DECODE_WARPS;    // independent warps per CTA
-static_assert(kTK == 16 || kTK == 32, "tile of 16 or 32 keys");
-constexpr uint32_t kFull = 0xffffffffu;
 
 struct StreamArgs {
     const __nv_bfloat16* Q;
@@ -106,136 +101,6 @@ __device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt) {
         tl.mask = n >= 32 ? kFull : ((1u << n) - 1u);
     }
     return tl;
-}
-
-template <int D>
-struct WState {
-    float m0, m1, l0, l1;  // reference maxima (scaled log2 units) and row sums
-    float o[D / 8][4];
-    __device__ void init() {
-        m0 = m1 = -INFINITY;
-        l0 = l1 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-    }
-};
-
-template <int D>
-__device__ __forceinline__ void load_q(const __nv_bfloat16* q, int G, uint32_t (&qa)[D / 16][4], int lane) {
-    const int r0 = lane >> 2, r1 = r0 + 8, c = 2 * (lane & 3);
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t* q0 = reinterpret_cast<const uint32_t*>(q + (size_t)r0 * D + ks * 16 + c);
-        const uint32_t* q1 = reinterpret_cast<const uint32_t*>(q + (size_t)r1 * D + ks * 16 + c);
-        qa[ks][0] = r0 < G ? q0[0] : 0u;
-        qa[ks][1] = r1 < G ? q1[0] : 0u;
-        qa[ks][2] = r0 < G ? q0[4] : 0u;
-        qa[ks][3] = r1 < G ? q1[4] : 0u;
-    }
-}
-
-// 2^x on the special-function unit (approximate, flush-to-zero).
-__device__ __forceinline__ float ex2f(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// Byte offset of 16-byte chunk `cc` (0..7) of row `r` in a 128-byte-swizzled 32-row box.
-__device__ __forceinline__ uint32_t swz(int r, int cc) { return (uint32_t)(r * 128 + ((cc ^ (r & 7)) << 4)); }
-
-// One tile: S = Q K^T over kTK keys, online softmax update, O += P V.
-template <int D>
-__device__ __forceinline__ void tile_mma(WState<D>& st, const uint32_t (&qa)[D / 16][4], const unsigned char* sK,
-                                         const unsigned char* sV, uint32_t vm, float sl2, int lane) {
-    constexpr int kHalf = kTK * 128;  // bytes of one 64-column box
-    constexpr int NP = kTK / 16;      // 16-key groups
-    const int mi = lane >> 3;
-    float s[2 * NP][4];
-#pragma unroll
-    for (int nt = 0; nt < 2 * NP; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.0f;
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-#pragma unroll
-        for (int np = 0; np < NP; ++np) {
-            const int r = np * 16 + (lane & 7) + ((mi >> 1) << 3);
-            const int cc = (ks & 3) * 2 + (mi & 1);
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4(b0, b1, b2, b3, sK + (ks >> 2) * kHalf + swz(r, cc));
-            mma_bf16_16816(s[2 * np], qa[ks], b0, b1);
-            mma_bf16_16816(s[2 * np + 1], qa[ks], b2, b3);
-        }
-    }
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 2 * NP; ++nt) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int slot = nt * 8 + 2 * (lane & 3) + j;
-            const bool ok = (vm >> slot) & 1u;
-            s[nt][j] = ok ? s[nt][j] : -INFINITY;
-            s[nt][2 + j] = ok ? s[nt][2 + j] : -INFINITY;
-            mx0 = fmaxf(mx0, s[nt][j]);
-            mx1 = fmaxf(mx1, s[nt][2 + j]);
-        }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, 2));
-    // Lazy rescale: the reference maxima st.m* (scaled log2 units) move only when a row's maximum
-    // exceeds them by more than 8, so p = 2^(s sl2 - m) <= 2^8 and the accumulators are rescaled
-    // rarely. The four threads of a quad hold the same row maxima and decide alike.
-    mx0 *= sl2;
-    mx1 *= sl2;
-    const bool g0 = mx0 != -INFINITY && (st.m0 == -INFINITY || mx0 - st.m0 > 8.0f);
-    const bool g1 = mx1 != -INFINITY && (st.m1 == -INFINITY || mx1 - st.m1 > 8.0f);
-    if (__any_sync(kFull, g0 || g1)) {
-        const float nm0 = g0 ? (st.m0 == -INFINITY ? mx0 : fmaxf(st.m0, mx0)) : st.m0;
-        const float nm1 = g1 ? (st.m1 == -INFINITY ? mx1 : fmaxf(st.m1, mx1)) : st.m1;
-        const float al0 = (g0 && st.m0 != -INFINITY) ? ex2f(st.m0 - nm0) : (g0 ? 0.0f : 1.0f);
-        const float al1 = (g1 && st.m1 != -INFINITY) ? ex2f(st.m1 - nm1) : (g1 ? 0.0f : 1.0f);
-        st.m0 = nm0;
-        st.m1 = nm1;
-        st.l0 *= al0;
-        st.l1 *= al1;
-#pragma unroll
-        for (int nd = 0; nd < D / 8; ++nd) {
-            st.o[nd][0] *= al0;
-            st.o[nd][1] *= al0;
-            st.o[nd][2] *= al1;
-            st.o[nd][3] *= al1;
-        }
-    }
-    const float nm0 = -st.m0, nm1 = -st.m1;
-    const bool z0 = st.m0 == -INFINITY, z1 = st.m1 == -INFINITY;
-    float ps0 = 0.0f, ps1 = 0.0f;
-    uint32_t pa[NP][4];
-#pragma unroll
-    for (int nt = 0; nt < 2 * NP; ++nt) {
-        const float p0 = z0 ? 0.0f : ex2f(fmaf(s[nt][0], sl2, nm0));
-        const float p1 = z0 ? 0.0f : ex2f(fmaf(s[nt][1], sl2, nm0));
-        const float p2 = z1 ? 0.0f : ex2f(fmaf(s[nt][2], sl2, nm1));
-        const float p3 = z1 ? 0.0f : ex2f(fmaf(s[nt][3], sl2, nm1));
-        ps0 += p0 + p1;
-        ps1 += p2 + p3;
-        pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
-        pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
-    }
-    st.l0 += ps0;
-    st.l1 += ps1;
-#pragma unroll
-    for (int kk = 0; kk < NP; ++kk) {
-#pragma unroll
-        for (int np = 0; np < D / 16; ++np) {
-            const int r = kk * 16 + (lane & 7) + ((mi & 1) << 3);
-            const int cc = (np & 3) * 2 + (mi >> 1);
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4_trans(b0, b1, b2, b3, sV + (np >> 2) * kHalf + swz(r, cc));
-            mma_bf16_16816(st.o[2 * np], pa[kk], b0, b1);
-            mma_bf16_16816(st.o[2 * np + 1], pa[kk], b2, b3);
-        }
-    }
 }
 
 // Partial record of (unit, br) written by warp v.

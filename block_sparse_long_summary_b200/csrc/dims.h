@@ -82,6 +82,14 @@ cudaError_t launch_decode_noalloc(const Dims& m, const void* Q, const void* K, c
                                   const void* Vc, const int32_t* idx, const float* gates, void* O, cudaStream_t s,
                                   int* err);
 
+// Fused decode step (selection + decode attention in one persistent kernel): bf16, d in {64, 128},
+// the per-channel or isotropic summaries.
+bool decode_step_supported(const Dims& m);
+size_t decode_step_workspace_bytes(const Dims& m);
+cudaError_t launch_decode_step(const Dims& m, const void* Q, const float* summ, const void* K, const void* V,
+                               const void* Kc, const void* Vc, int32_t* idx, const float* gates, void* O, void* ws,
+                               cudaStream_t s, int* err);
+
 size_t prefill_workspace_bytes(const Dims& m);
 // tcgen05 prefill (bf16, d = 128, G = 16); cudaErrorNotSupported for other shapes.
 cudaError_t launch_prefill_tc(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,

@@ -20,18 +20,11 @@
 
 #include "common.cuh"
 #include "dims.h"
+#include "select_core.cuh"
 #include "tma.h"
 
 namespace cobs {
 namespace {
-
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kInvalid = 0x7fffffff;
-constexpr int kGroupBlocks = 32;
-
-__device__ __forceinline__ bool better(float s1, int i1, float s2, int i2) {
-    return s1 > s2 || (s1 == s2 && i1 < i2);
-}
 
 // Warp-wide top-k list: lane j < k holds the j-th best (score desc, index asc);
 // lanes >= k hold (-inf, kInvalid).
@@ -73,20 +66,6 @@ struct TopK {
     }
 };
 
-// Ascending bitonic sort of one int key per lane.
-__device__ __forceinline__ int warp_sort_asc(int key, int lane) {
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const int other = __shfl_xor_sync(kFull, key, stride);
-            const bool up = (lane & size) == 0;
-            const bool low = (lane & stride) == 0;
-            key = (low == up) ? min(key, other) : max(key, other);
-        }
-    }
-    return key;
-}
 
 // Write the list (lanes < k) in ascending block order, -1 for empty slots.
 __device__ __forceinline__ void emit_sorted(const TopK& tk, int k, int lane, int32_t* out) {
@@ -94,113 +73,13 @@ __device__ __forceinline__ void emit_sorted(const TopK& tk, int k, int lane, int
     if (lane < k) out[lane] = key == kInvalid ? -1 : key;
 }
 
-template <typename T>
-__device__ __forceinline__ float to_f(T x);
-template <>
-__device__ __forceinline__ float to_f<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Largest GQA group (query heads per KV head) the selectors handle; the host rejects larger.
-constexpr int kMaxGroup = 16;
-
-// NC consecutive elements (16-, 8- or 4-byte aligned vector loads) as float.
-template <typename T, int NC>
-__device__ __forceinline__ void load_chunk(const T* p, float (&x)[NC]) {
-    if constexpr (sizeof(T) == 2) {
-        static_assert(NC == 2 || NC == 4 || NC == 8, "chunk");
-        uint32_t w[NC / 2];
-        if constexpr (NC == 8) {
-            const uint4 u = *reinterpret_cast<const uint4*>(p);
-            w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
-        } else if constexpr (NC == 4) {
-            const uint2 u = *reinterpret_cast<const uint2*>(p);
-            w[0] = u.x; w[1] = u.y;
-        } else {
-            w[0] = *reinterpret_cast<const uint32_t*>(p);
-        }
-#pragma unroll
-        for (int i = 0; i < NC / 2; ++i) {
-            x[2 * i] = __uint_as_float(w[i] << 16);
-            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-    } else {
-        static_assert(NC % 2 == 0, "chunk");
-#pragma unroll
-        for (int i = 0; i < NC; i += (NC % 4 == 0 ? 4 : 2)) {
-            if constexpr (NC % 4 == 0) {
-                const float4 v = *reinterpret_cast<const float4*>(p + i);
-                x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
-            } else {
-                const float2 v = *reinterpret_cast<const float2*>(p + i);
-                x[i] = v.x; x[i + 1] = v.y;
-            }
-        }
-    }
-}
-
-// Canonical group query of channels [c0, c0 + NC) of a group whose G head rows start at q
-// (row stride D): every head's chunk is loaded at once, then Qsum_c = sum_h q_{h,c} (adds)
-// and Q2_c = fma-sum of q_{h,c}^2 in ascending h.
-template <typename T, int NC>
-__device__ __forceinline__ void group_query_chunk(const T* q, int G, int D, int c0, bool valid, float* qs,
-                                                  float* q2) {
-    float x[kMaxGroup][NC];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-        if (h < G && valid) {
-            load_chunk<T, NC>(q + (size_t)h * D + c0, x[h]);
-        } else {
-#pragma unroll
-            for (int j = 0; j < NC; ++j) x[h][j] = 0.0f;
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < NC; ++j) {
-        float s = 0.0f, s2 = 0.0f;
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h < G) {
-                s = __fadd_rn(s, x[h][j]);
-                s2 = __fmaf_rn(x[h][j], x[h][j], s2);
-            }
-        }
-        qs[j] = s;
-        q2[j] = s2;
-    }
-}
-
-// Canonical channel sums: four interleaved partial chains (chain j takes the channels
-// c = j (mod 4) in ascending order from +0, one rounded fma per term), combined as
-// (s0 + s1) + (s2 + s3). Lane = block; a group tile keeps four consecutive channels of a block
-// in one 16-byte word, so one load feeds the four chains.
-__device__ __forceinline__ float combine4(float s0, float s1, float s2, float s3) {
-    return __fadd_rn(__fadd_rn(s0, s1), __fadd_rn(s2, s3));
-}
-
-// Canonical score of the block held by this lane (channel-interleaved group tile in smem).
+// Canonical score of the block held by this lane (channel-interleaved group tile in smem): the
+// mean half and the variance half are independent chains, combined once.
 template <int D>
 __device__ __forceinline__ float block_score(const float* tile, const float* qs, const float* q2, int lane,
                                              float isd, float c2) {
-    const float4* mu4 = reinterpret_cast<const float4*>(tile) + lane;
-    const float4* var4 = reinterpret_cast<const float4*>(tile + D * 32) + lane;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
-#pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 m = mu4[c4 * 32];
-        const float4 s = var4[c4 * 32];
-        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
-        const float4 r = reinterpret_cast<const float4*>(q2)[c4];
-        a0 = __fmaf_rn(q.x, m.x, a0);
-        a1 = __fmaf_rn(q.y, m.y, a1);
-        a2 = __fmaf_rn(q.z, m.z, a2);
-        a3 = __fmaf_rn(q.w, m.w, a3);
-        v0 = __fmaf_rn(r.x, s.x, v0);
-        v1 = __fmaf_rn(r.y, s.y, v1);
-        v2 = __fmaf_rn(r.z, s.z, v2);
-        v3 = __fmaf_rn(r.w, s.w, v3);
-    }
-    return __fmaf_rn(c2, combine4(v0, v1, v2, v3), __fmul_rn(combine4(a0, a1, a2, a3), isd));
+    return score_combine(score_mean_part<D>(tile, qs, lane), score_var_part<D>(tile + D * 32, q2, lane), isd, c2);
 }
 
 // Canonical isotropic score: the same mean sum, then v = RN(Q2tot * sigma2_b) with the block's
@@ -390,52 +269,12 @@ __device__ __forceinline__ float block_score_lr_fp4(const float* tile, const flo
     return __fmaf_rn(c2, v, __fmul_rn(combine4(a[0], a[1], a[2], a[3]), isd));
 }
 
-// Q2tot = sum_c Q2_c by adds in ascending channel order from +0 (one thread).
-template <int D>
-__device__ __forceinline__ float q2_total(const float* q2) {
-    float t = 0.0f;
-    for (int c = 0; c < D; ++c) t = __fadd_rn(t, q2[c]);
-    return t;
-}
 
 // Floats of one 32-block summary group: means + per-channel variances, or means + 32 scalars.
 template <int D, bool ISO>
 constexpr int group_floats() { return ISO ? (D + 1) * 32 : 2 * D * 32; }
 
 // ---------------------------------------------------------------------------- decode
-// Warp-wide sorted list helpers: one (score, index) entry per lane, best first.
-__device__ __forceinline__ void cmp_swap(float& s, int& i, int j, bool up, int lane) {
-    const float os = __shfl_xor_sync(kFull, s, j);
-    const int oi = __shfl_xor_sync(kFull, i, j);
-    const bool low = (lane & j) == 0;
-    const bool ob = better(os, oi, s, i);
-    if ((low == up) ? ob : (!ob && !(os == s && oi == i))) {
-        s = os;
-        i = oi;
-    }
-}
-
-// Sort the 32 entries best first (bitonic network).
-__device__ __forceinline__ void warp_sort_best_first(float& s, int& i, int lane) {
-#pragma unroll
-    for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) cmp_swap(s, i, j, (lane & k) == 0, lane);
-    }
-}
-
-// (s, i) and (bs, bi) are both sorted best first; keep the best 32 of their union, sorted.
-__device__ __forceinline__ void warp_merge_best_first(float& s, int& i, float bs, int bi, int lane) {
-    const float rs = __shfl_sync(kFull, bs, 31 - lane);
-    const int ri = __shfl_sync(kFull, bi, 31 - lane);
-    if (better(rs, ri, s, i)) {
-        s = rs;
-        i = ri;
-    }
-#pragma unroll
-    for (int j = 16; j > 0; j >>= 1) cmp_swap(s, i, j, true, lane);
-}
-
 #ifndef COBS_SELECT_STAGES
 #define COBS_SELECT_STAGES 2
 #endif
@@ -465,32 +304,6 @@ inline int sel_max_segments(int units, int nGc) {
     return std::min(std::min(nGc, kSelMaxSeg), kSelGridCap / std::max(1, units) + 2);
 }
 
-// Running best-first list of one warp (lane j = j-th best), with the k-th best as the bar
-// a newcomer must beat. Groups with no lane above the bar cost one ballot.
-struct RunList {
-    float s;
-    int i;
-    float ts;
-    int ti;
-    __device__ void init() {
-        s = -INFINITY;
-        i = kInvalid;
-        ts = -INFINITY;
-        ti = kInvalid;
-    }
-    __device__ void bar(int k) {
-        ts = __shfl_sync(kFull, s, k - 1);
-        ti = __shfl_sync(kFull, i, k - 1);
-    }
-    // one candidate per lane (invalid lanes carry (-inf, kInvalid))
-    __device__ void add(float sc, int bi, int k, int lane) {
-        const unsigned up = __ballot_sync(kFull, bi != kInvalid && better(sc, bi, ts, ti));
-        if (up == 0u) return;
-        warp_sort_best_first(sc, bi, lane);
-        warp_merge_best_first(s, i, sc, bi, lane);
-        bar(k);
-    }
-};
 
 // grid (G_sel), one warp per CTA, persistent. CTA c scores the summary groups of its stream-K
 // range in order: each group (32 blocks, 2 d 32 floats) arrives by one bulk (TMA) copy into a

@@ -79,7 +79,12 @@ typedef enum {
 
 typedef enum { COBS_F32 = 0, COBS_BF16 = 1 } cobs_dtype;
 
-typedef enum { COBS_WS_SELECT = 0, COBS_WS_DECODE = 1, COBS_WS_PREFILL = 2 } cobs_workspace_kind;
+typedef enum {
+    COBS_WS_SELECT = 0,
+    COBS_WS_DECODE = 1,
+    COBS_WS_PREFILL = 2,
+    COBS_WS_STEP = 3 /* cobs_decode_step */
+} cobs_workspace_kind;
 
 /* Second-order statistic kept per block ([COBS] §2.2/§2.3: the block covariance Sigma_b, compressed):
  *   COBS_VAR_CHANNEL    the per-channel population variance var_{b,c} (the diagonal of Sigma_b);
@@ -191,6 +196,31 @@ cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const v
                                     const void* V, const void* Kc, const void* Vc,
                                     const int32_t* idx, const float* gates, void* O,
                                     void* workspace, size_t ws_bytes, cobs_stream_t stream);
+
+/*
+ * One decode step, enqueued as one unit: the summary update of cobs_build_summaries from t_begin,
+ * then the block selection of cobs_select (prefill = 0), then cobs_sparse_attn_decode, with the
+ * arguments, layouts and results of those three calls ([COBS] §2.2/§2.3 summaries and
+ * second-order selection; [NSA-181] the three paths and their gates). idx and O are written as
+ * the separate calls write them (the same indices bit for bit, the same attention up to float32
+ * summation order).
+ * For bf16 with d in {64, 128} and the COBS_VAR_CHANNEL or COBS_VAR_ISOTROPIC summaries the
+ * selection and the attention run as one persistent kernel (one CTA per SM): the summaries, the
+ * window and compressed tokens and the selected blocks are read back to back, and a unit's
+ * selected blocks are read as soon as its selection is complete. Other shapes run the separate
+ * kernels.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_STEP) bytes (sized for the current device's
+ *              SM count), ZERO-FILLED before its first use and again before it is used with
+ *              other params or after a call that set the device error flag; a completed call
+ *              leaves it ready for the next one. Calls that share one workspace must not run
+ *              concurrently.
+ * Errors: those of the three calls. A wait on another CTA's result is bounded: if it gives up
+ * (kernel resources held by other work for more than about 0.1 s), the device error flag is set.
+ */
+cobs_status cobs_decode_step(const cobs_params* p, const void* Q, const void* K, const void* V,
+                             const float* Pk, const float* Pv, int32_t t_begin, float* summaries,
+                             void* Kc, void* Vc, int32_t* idx, const float* gates, void* O,
+                             void* workspace, size_t ws_bytes, cobs_stream_t stream);
 
 /*
  * Decode attention without a workspace. The paper has no counterpart to this call: it exists
