@@ -1,32 +1,39 @@
 // Decode step, bf16: block selection and the three-branch decode attention in one persistent
 // kernel, so that the summaries, the window, the compressed tokens and the selected blocks
-// stream through HBM back to back instead of in three dependent launches.
+// stream through HBM back to back instead of in dependent launches.
 //
 // What is computed is exactly cobs_select (decode) followed by cobs_sparse_attn_decode:
 // COBS (gist.science explainer §2.3) ranks the complete blocks by the second-order score and
 // keeps the top-k per GQA group; the NSA paths (Janus issue #181: compression, selection,
 // sliding window) are attended with softmaxes of their own and mixed by the gates. Decode is
-// bound by the KV-cache read (explainer, "Problemstellung"), so the kernel is scheduled for HBM:
+// bound by the KV-cache read (explainer, "Problemstellung"), so the kernel is scheduled for HBM,
+// and nothing on a streaming warp's path waits for a global-memory round trip (under a
+// saturated HBM each one costs microseconds):
 //
-// * One CTA per SM, 4 warps, each warp an independent worker with a private 3-stage ring of
-//   shared-memory tiles filled by bulk / TMA copies (no multicast).
+// * One CTA per SM: 7 streaming warps and 1 helper warp, two warps per scheduler (so that one's
+//   latencies hide behind the other's work, with up to 255 registers each). Every streaming warp
+//   has a private 3-stage ring of 8 KiB shared-memory tiles filled by bulk / TMA copies (no
+//   multicast). An attention tile is 16 keys of K and V; a summary group (32 blocks) is four
+//   tiles: two halves of its means, two of its variances.
 // * The work is three phases, each cut into contiguous per-warp ranges (stream-K), and every
-//   warp walks its ranges in phase order:
-//     S  the summary groups of every unit (32 blocks; the mean half and the variance half of
-//        a group are two tiles): canonical float32 scores and a warp top-k list;
+//   streaming warp walks its ranges in phase order:
+//     S  the summary groups of every unit: canonical float32 scores (the four channel chains
+//        run on across a group's tiles) and a warp top-k list per unit;
 //     A  the window and compressed-token tiles of every unit (they do not depend on S);
 //     B  the tiles of the selected blocks of every unit.
-//   The range of phase A is sized so that every warp streams the same number of tiles in all.
-// * A unit's selection may be cut across warps: each deposits its segment list, and the last
-//   to arrive (a per-unit counter) merges them, writes idx and publishes the unit with the
-//   launch's epoch number. A phase-B tile of the unit waits for that flag (bounded) before it
-//   reads idx; every warp finishes its own phase-S segments before it waits on any flag, and
-//   phase S itself waits on nothing, so the waits cannot form a cycle.
-// * An attention piece (the tiles of one (unit, branch) a warp covers) leaves a partial
-//   record (m, l, o); the last piece of a (unit, branch) folds its records into the gated
-//   branch output, and the last branch of a unit sums the branches into O. The counters are
-//   re-armed by the warps that complete them, and the epoch advances when the last CTA ends.
+//   The ranges of phase A are sized so that every warp streams the same number of tiles.
+// * A unit's selection may be cut across warps: each deposits its sorted segment list with
+//   plain 64-bit stores that carry the launch's epoch tag next to the block index (no fence,
+//   no counter). The helper warp of every CTA merges the segments of the units its streaming
+//   warps need in phase B (polling until every word carries this launch's tag), writes idx
+//   for the units whose first selected tile it holds, and publishes the block indices in shared
+//   memory behind one mbarrier per unit.
+// * An attention piece (the tiles of one (unit, branch) a warp covers) leaves a partial record
+//   (m, l, o) with plain stores. The launch is cooperative (every CTA resident): after a grid
+//   barrier (an arrival counter, bounded wait) every CTA folds the records of a share of the
+//   (unit, head) pairs, applies the gates and writes O; CTA 0 then advances the epoch.
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "dims.h"
@@ -37,8 +44,27 @@
 namespace cobs {
 namespace {
 
-constexpr int kStepWarps = 4;   // workers per CTA
-constexpr int kStepStages = 3;  // ring depth per worker
+#ifndef COBS_STEP_WARPS
+#define COBS_STEP_WARPS 7
+#endif
+#ifndef COBS_STEP_STAGES
+#define COBS_STEP_STAGES 3
+#endif
+constexpr int kStepWarps = COBS_STEP_WARPS;    // streaming warps per CTA (with the helper, two per scheduler)
+constexpr int kStepStages = COBS_STEP_STAGES;  // ring depth per streaming warp
+constexpr int kStepThreads = (kStepWarps + 1) * 32;
+#ifndef COBS_STEP_TK
+#define COBS_STEP_TK 16
+#endif
+constexpr int kStepTK = COBS_STEP_TK;    // keys per attention tile (16 or 32)
+constexpr int kParts = 32 / kStepTK;     // tiles per half of a summary group (means or variances)
+constexpr uint32_t kIdxBits = 25;                      // block index field of a segment word
+constexpr uint32_t kIdxNone = (1u << kIdxBits) - 1u;   // an empty entry
+constexpr uint32_t kTagMask = 0x7Fu;                   // epoch tag field (7 bits)
+
+// Bytes of one ring stage: the K and V halves of a kStepTK-key tile (= one part of a summary group).
+template <int D>
+constexpr size_t step_stage_bytes() { return (size_t)2 * (D / 64) * kStepTK * 128; }
 
 struct StepArgs {
     const __nv_bfloat16* Q;
@@ -47,27 +73,21 @@ struct StepArgs {
     int32_t* idx;
     __nv_bfloat16* O;
     int* err;
-    // workspace (control words at the start)
-    unsigned* ctl;       // [0] epoch of the last completed launch, [1] CTAs finished in this launch
-    unsigned* ready;     // [units] epoch at which idx[u] was published
-    unsigned* sel_cnt;   // [units] selection segments deposited
-    unsigned* br_cnt;    // [units][3] attention pieces flushed, per branch
-    unsigned* unit_cnt;  // [units] branches finalised
-    float* seg_s;        // [units][maxseg][32] segment lists (scores, best first)
-    int* seg_i;          // [units][maxseg][32] (block indices)
-    float* rec;          // [units][3][maxw][G][D + 4] attention partial records
-    float* bout;         // [units][3][G][D] gated branch outputs
+    // workspace
+    unsigned* ctl;                // [0] epoch of the last completed step, [1] grid-barrier arrivals
+    unsigned long long* seg;      // [units][maxseg][32] segment lists: score bits << 32 | tag << 25 | index
+    float* rec;                   // [units][3][maxw][G][D + 4] attention partial records
     // shape
     int units, G, T, k, W, nB, nC, nG, nGc, ncand, iso, D;
     int tS, tW, tC, tA;  // tiles per unit: selected blocks, window, compressed tokens, tW + tC
-    int tpg;             // ring tiles per summary group (2: means + variances, 1: isotropic)
+    int tpg;             // ring tiles per summary group (2 kParts: means + variances, kParts: isotropic)
     int gfloats;         // floats per stored summary group
-    int nwarps;
+    int nwarps;          // streaming warps in the grid
     long long nS, nA, nBt, tot;  // phase sizes (groups, tiles, tiles) and tpg nS + nA + nBt
     int balanced;        // phase A sized so that every warp's total is equal
     int dense[3];        // phase S, A, B: every warp's range is nonempty (else at most one element each)
-    int nbr;             // branches with tiles (selected blocks always; window, compressed tokens if any)
     int maxseg, maxw;
+    int maxbu;           // most phase-B units any CTA holds
     float isd, c2, sl2;
     // reciprocals of the divisors of the partition arithmetic (exact quotients: see div_floor)
     double inv_nw, inv_nS, inv_nA, inv_nBt;
@@ -143,214 +163,110 @@ __host__ __device__ __forceinline__ int branch_pieces(const StepArgs& a, int u, 
 __host__ __device__ __forceinline__ int sel_segments(const StepArgs& a, int u) {
     return run_pieces<0>(a, (long long)u * a.nGc, a.nGc);
 }
+// Phase-B units of CTA c: [first, last] (last < first when its warps hold no phase-B tile).
+__host__ __device__ __forceinline__ void cta_bunits(const StepArgs& a, int c, int* first, int* last) {
+    const long long z0 = fB(a, (long long)c * kStepWarps), z1 = fB(a, (long long)(c + 1) * kStepWarps);
+    if (z1 <= z0) { *first = 0; *last = -1; return; }
+    *first = (int)(z0 / a.tS);
+    *last = (int)((z1 - 1) / a.tS);
+}
 
 struct Item {
-    int kind;       // 0 summary means (or isotropic tile), 1 summary variances, 2 attention tile
+    int kind;       // 0 summary means, 1 summary variances, 2 attention tile
     int unit;
     int a;          // summary group (kinds 0, 1) or branch (kind 2)
+    int part;       // summary tiles: the part (channel range) of the half
     int row;        // attention: first row of K / V (branches 0, 1) or Kc / Vc (branch 2)
     unsigned mask;  // attention: valid keys of the tile (0: nothing to load)
 };
 
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ int ld_relaxed(const int* p) {
-    int v;
-    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+
+__device__ __forceinline__ unsigned long long seg_word(float s, int i, unsigned tag) {
+    const uint32_t ix = i == kInvalid ? kIdxNone : (uint32_t)i;
+    return ((unsigned long long)__float_as_uint(s) << 32) | ((unsigned long long)(tag & kTagMask) << kIdxBits) | ix;
 }
 
-// Bounded wait for a published flag (one thread). False (and kErrWaitTimeout recorded) if it
-// did not arrive within kWaitLimitNs.
-__device__ __forceinline__ bool wait_flag(const unsigned* f, unsigned want, int* err) {
-    if (ld_acquire(f) == want) return true;
-    const uint64_t t0 = global_ns();
-    for (uint32_t i = 0; i < kMaxWaitIters; ++i) {
-        __nanosleep(128);
-        if (ld_acquire(f) == want) return true;
-        if (global_ns() - t0 > kWaitLimitNs) break;
-    }
-    report_error(err, kErrWaitTimeout);
-    return false;
+// Deposit the sorted segment list of warp v for unit u (one 64-bit store per lane, tagged).
+__device__ __forceinline__ void sel_deposit(const StepArgs& a, int v, long long r0, int u, const RunList& rl,
+                                            unsigned ep, int lane) {
+    const int slot = run_slot<0>(a, v, r0, (long long)u * a.nGc);
+    a.seg[((size_t)u * a.maxseg + slot) * 32 + lane] = seg_word(rl.s, rl.i, ep);
 }
 
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
-    return x;
-}
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
-    return x;
-}
+// Helper warp: the merged top-k of unit u from its deposited segment lists, sorted by block index
+// (-1 padded) into out[0 .. k). The segments are loaded 16 at a time (one round trip) and polled
+// (bounded) until every word carries this launch's tag, staged in shared memory (hbuf, [16][32]
+// words) and merged one by one; a segment whose best entry does not beat the current k-th best is
+// skipped.
+constexpr int kHelperRound = 16;
 
-// Selection segment of unit u held by warp v (list rl): write idx directly when the warp held the
-// whole unit; else deposit it, and if it is the last to arrive, merge all segments of the unit
-// and write idx. Either way the writer publishes the unit with the epoch.
-__device__ void sel_finish(const StepArgs& a, int v, long long r0, int u, const RunList& rl, unsigned ep,
-                           int lane) {
-    const int nseg = sel_segments(a, u);
-    float s = rl.s;
-    int i = rl.i;
-    if (nseg > 1) {
-        const int slot = run_slot<0>(a, v, r0, (long long)u * a.nGc);
-        const size_t base = ((size_t)u * a.maxseg + slot) * 32;
-        a.seg_s[base + lane] = s;
-        a.seg_i[base + lane] = i;
-        __threadfence();
-        __syncwarp();
-        unsigned old = 0;
-        if (lane == 0) old = atomicAdd(&a.sel_cnt[u], 1u);
-        old = __shfl_sync(kFull, old, 0);
-        if (old != (unsigned)(nseg - 1)) return;
-        __threadfence();
-        // the other segments, 16 at a time; a segment whose best entry does not beat the current
-        // k-th best cannot contribute and costs one comparison
-        float ts = __shfl_sync(kFull, s, a.k - 1);
-        int ti = __shfl_sync(kFull, i, a.k - 1);
-        for (int j0 = 0; j0 < nseg; j0 += 16) {
-            float bs[16];
-            int bi[16];
+__device__ void helper_merge(const StepArgs& a, int u, unsigned ep, int lane, int* out, unsigned long long* hbuf) {
+    float s = -INFINITY;
+    int i = kInvalid;
+    if (a.nGc > 0) {
+        const int nseg = sel_segments(a, u);
+        float ts = -INFINITY;
+        int ti = kInvalid;
+        const unsigned tag = ep & kTagMask;
+        for (int j0 = 0; j0 < nseg; j0 += kHelperRound) {
+            const int nj = min(kHelperRound, nseg - j0);
+            const uint64_t t0 = global_ns();
+            for (uint32_t it = 0;; ++it) {
+                unsigned long long w[kHelperRound];
+                bool ready = true;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const int j = j0 + q;
-                bs[q] = -INFINITY;
-                bi[q] = kInvalid;
-                if (j < nseg && j != slot) {
-                    const size_t o = ((size_t)u * a.maxseg + j) * 32 + lane;
-                    bs[q] = __ldcg(a.seg_s + o);
-                    bi[q] = __ldcg(a.seg_i + o);
+                for (int q = 0; q < kHelperRound; ++q)
+                    w[q] = q < nj ? ld_relaxed_u64(a.seg + ((size_t)u * a.maxseg + j0 + q) * 32 + lane) : 0ull;
+#pragma unroll
+                for (int q = 0; q < kHelperRound; ++q)
+                    if (q < nj) ready &= (uint32_t)((w[q] >> kIdxBits) & kTagMask) == tag;
+                const bool all = __all_sync(kFull, ready);
+                const bool late = !all && (it >= kMaxWaitIters || global_ns() - t0 > kWaitLimitNs);
+                if (all || late) {
+                    if (late && lane == 0) report_error(a.err, kErrWaitTimeout);
+#pragma unroll
+                    for (int q = 0; q < kHelperRound; ++q) hbuf[q * 32 + lane] = w[q];
+                    break;
                 }
+                __nanosleep(500);
             }
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const float b0s = __shfl_sync(kFull, bs[q], 0);
-                const int b0i = __shfl_sync(kFull, bi[q], 0);
+            __syncwarp();
+#pragma unroll 1
+            for (int q = 0; q < nj; ++q) {
+                const unsigned long long w = hbuf[q * 32 + lane];
+                const uint32_t ix = (uint32_t)w & kIdxNone;
+                const float bs = __uint_as_float((uint32_t)(w >> 32));
+                const int bi = ix == kIdxNone ? kInvalid : (int)ix;
+                const float b0s = __shfl_sync(kFull, bs, 0);
+                const int b0i = __shfl_sync(kFull, bi, 0);
                 if (b0i == kInvalid || !better(b0s, b0i, ts, ti)) continue;  // uniform
-                warp_merge_best_first(s, i, bs[q], bi[q], lane);
+                warp_merge_best_first(s, i, bs, bi, lane);
                 ts = __shfl_sync(kFull, s, a.k - 1);
                 ti = __shfl_sync(kFull, i, a.k - 1);
             }
+            __syncwarp();
         }
-        if (lane == 0) a.sel_cnt[u] = 0u;  // re-armed for the next launch
     }
     const int key = warp_sort_asc(lane < a.k ? i : kInvalid, lane);
-    if (lane < a.k) a.idx[(size_t)u * a.k + lane] = key == kInvalid ? -1 : key;
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release(&a.ready[u], ep);
+    if (lane < a.k) out[lane] = key == kInvalid ? -1 : key;
 }
 
-// Fold the records of unit u's branch br into the gated branch output bout[u][br] (all heads):
-// o_h = g_{h,br} * (sum_j 2^(m_j - M) o_j) / (sum_j 2^(m_j - M) l_j), zero for an empty branch.
-// Heads in fours; lane = D/32 consecutive channels; pieces 32 at a time (lane = piece for the
-// maxima and sums), the running maximum rescaled between chunks.
+// Partial record of warp v's piece of (unit u, branch br): (m, l) per head in scaled log2 units
+// and the unnormalised o, plain stores (folded by every CTA after the grid barrier).
 template <int D>
-__device__ void finalize_branch(const StepArgs& a, int u, int br, int np, int lane) {
-    constexpr int CPL = D / 32;  // channels per lane
-    constexpr int RF = D + 4;
-    const size_t rs = (size_t)a.G * RF;  // floats per record slot
-    const float* base = a.rec + ((size_t)u * 3 + br) * a.maxw * rs;
-    const int gate_col = br == 0 ? 1 : (br == 1 ? 2 : 0);  // gates are (cmp, slc, win)
-    for (int h0 = 0; h0 < a.G; h0 += 4) {
-        float M[4], Ls[4], acc[4][CPL];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            M[q] = -INFINITY;
-            Ls[q] = 0.0f;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[q][c] = 0.0f;
-        }
-        for (int c0 = 0; c0 < np; c0 += 32) {
-            const int nj = min(32, np - c0);
-            float mj[4], lj[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                mj[q] = -INFINITY;
-                lj[q] = 0.0f;
-                if (lane < nj && h0 + q < a.G) {
-                    const float* r = base + (size_t)(c0 + lane) * rs + (size_t)(h0 + q) * RF;
-                    mj[q] = __ldcg(r);
-                    lj[q] = __ldcg(r + 1);
-                }
-            }
-            float fj[4], sc[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float nM = fmaxf(M[q], warp_max(mj[q]));
-                sc[q] = (M[q] == -INFINITY || nM == -INFINITY) ? 0.0f : exp2f(M[q] - nM);
-                fj[q] = (mj[q] == -INFINITY) ? 0.0f : exp2f(mj[q] - nM);
-                Ls[q] = Ls[q] * sc[q] + warp_sum(lj[q] * fj[q]);
-                M[q] = nM;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) acc[q][c] *= sc[q];
-            }
-#pragma unroll 4
-            for (int j = 0; j < nj; ++j) {
-                const float* r = base + (size_t)(c0 + j) * rs + 4 + lane * CPL;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float f = __shfl_sync(kFull, fj[q], j);
-                    if (h0 + q < a.G) {
-                        float o[CPL];
-                        if constexpr (CPL == 4) {
-                            const float4 t = __ldcg(reinterpret_cast<const float4*>(r + (size_t)(h0 + q) * RF));
-                            o[0] = t.x; o[1] = t.y; o[2] = t.z; o[3] = t.w;
-                        } else {
-                            const float2 t = __ldcg(reinterpret_cast<const float2*>(r + (size_t)(h0 + q) * RF));
-                            o[0] = t.x; o[1] = t.y;
-                        }
-#pragma unroll
-                        for (int c = 0; c < CPL; ++c) acc[q][c] = fmaf(f, o[c], acc[q][c]);
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int h = h0 + q;
-            if (h >= a.G) break;
-            const float g = a.gates[((size_t)u * a.G + h) * 3 + gate_col];
-            const float w = Ls[q] > 0.0f ? g / Ls[q] : 0.0f;
-            float* out = a.bout + (((size_t)u * 3 + br) * a.G + h) * D + lane * CPL;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) out[c] = acc[q][c] * w;
-        }
-    }
-}
-
-// Sum the finalised branch outputs of unit u into O (bf16).
-template <int D>
-__device__ void finalize_unit(const StepArgs& a, int u, int lane) {
-    constexpr int CPL = D / 32;
-    for (int h = 0; h < a.G; ++h) {
-        float s[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) s[c] = 0.0f;
-#pragma unroll
-        for (int br = 0; br < 3; ++br) {
-            if ((br == 1 && a.tW == 0) || (br == 2 && a.tC == 0)) continue;  // branches without tiles
-            const float* src = a.bout + (((size_t)u * 3 + br) * a.G + h) * D + lane * CPL;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) s[c] += __ldcg(src + c);
-        }
-        __nv_bfloat16* o = a.O + ((size_t)u * a.G + h) * D + lane * CPL;
-#pragma unroll
-        for (int c = 0; c < CPL; c += 2) *reinterpret_cast<__nv_bfloat162*>(o + c) = __floats2bfloat162_rn(s[c], s[c + 1]);
-    }
-}
-
-// Partial record of warp v's piece of (unit u, branch br); the last piece of the branch
-// finalises it, and the last branch of the unit writes O.
-template <int D>
-__device__ void att_flush(const StepArgs& a, int v, long long rstart, int u, int br, WState<D>& st, int lane) {
+__device__ __forceinline__ void att_flush(const StepArgs& a, int v, long long rstart, int u, int br, WState<D>& st,
+                                          int lane) {
     constexpr int RF = D + 4;
     float l0 = st.l0, l1 = st.l1;
     l0 += __shfl_xor_sync(kFull, l0, 1);
@@ -359,7 +275,6 @@ __device__ void att_flush(const StepArgs& a, int v, long long rstart, int u, int
     l1 += __shfl_xor_sync(kFull, l1, 2);
     long long x0, len;
     branch_run(a, u, br, &x0, &len);
-    const int np = br == 0 ? run_pieces<2>(a, x0, len) : run_pieces<1>(a, x0, len);
     const int slot = br == 0 ? run_slot<2>(a, v, rstart, x0) : run_slot<1>(a, v, rstart, x0);
     float* rec = a.rec + (((size_t)u * 3 + br) * a.maxw + (size_t)slot) * a.G * RF;
     const int r0 = lane >> 2, r1 = r0 + 8, c = 2 * (lane & 3);
@@ -378,277 +293,459 @@ __device__ void att_flush(const StepArgs& a, int v, long long rstart, int u, int
         if (r0 < a.G) *reinterpret_cast<float2*>(rec + r0 * RF + 4 + nd * 8 + c) = make_float2(st.o[nd][0], st.o[nd][1]);
         if (r1 < a.G) *reinterpret_cast<float2*>(rec + r1 * RF + 4 + nd * 8 + c) = make_float2(st.o[nd][2], st.o[nd][3]);
     }
-    __threadfence();
-    __syncwarp();
-    unsigned old = 0;
-    if (lane == 0) old = atomicAdd(&a.br_cnt[(size_t)u * 3 + br], 1u);
-    old = __shfl_sync(kFull, old, 0);
-    if (old != (unsigned)(np - 1)) return;
-    __threadfence();
-    finalize_branch<D>(a, u, br, np, lane);
-    if (lane == 0) a.br_cnt[(size_t)u * 3 + br] = 0u;
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) old = atomicAdd(&a.unit_cnt[u], 1u);
-    old = __shfl_sync(kFull, old, 0);
-    if (old != (unsigned)(a.nbr - 1)) return;
-    __threadfence();
-    finalize_unit<D>(a, u, lane);
-    if (lane == 0) a.unit_cnt[u] = 0u;
 }
 
+// The same record from the keys-as-rows state (thread t holds heads 2 (t % 4), + 1 and channels
+// mt 16 + t / 4 (+ 8) of O^T).
 template <int D>
-__global__ void __launch_bounds__(kStepWarps * 32, 1) decode_step_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                          const __grid_constant__ CUtensorMap tmV,
-                                                                          const __grid_constant__ CUtensorMap tmKc,
-                                                                          const __grid_constant__ CUtensorMap tmVc,
-                                                                          StepArgs a) {
-    constexpr int kBox = kTK * 128;        // one 64-column box of a 32-row tile
+__device__ __forceinline__ void att_flush_t(const StepArgs& a, int v, long long rstart, int u, int br, WStateT<D>& st,
+                                            int lane) {
+    constexpr int RF = D + 4;
+    float l0 = st.l[0], l1 = st.l[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(kFull, l0, o);
+        l1 += __shfl_xor_sync(kFull, l1, o);
+    }
+    long long x0, len;
+    branch_run(a, u, br, &x0, &len);
+    const int slot = br == 0 ? run_slot<2>(a, v, rstart, x0) : run_slot<1>(a, v, rstart, x0);
+    float* rec = a.rec + (((size_t)u * 3 + br) * a.maxw + (size_t)slot) * a.G * RF;
+    const int g = lane >> 2, h0 = 2 * (lane & 3);
+    const bool in0 = h0 < a.G, in1 = h0 + 1 < a.G;
+    if (g == 0) {
+        if (in0) {
+            rec[h0 * RF + 0] = st.m[0];
+            rec[h0 * RF + 1] = l0;
+        }
+        if (in1) {
+            rec[(h0 + 1) * RF + 0] = st.m[1];
+            rec[(h0 + 1) * RF + 1] = l1;
+        }
+    }
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        if (in0) {
+            rec[h0 * RF + 4 + mt * 16 + g] = st.o[mt][0];
+            rec[h0 * RF + 4 + mt * 16 + g + 8] = st.o[mt][2];
+        }
+        if (in1) {
+            rec[(h0 + 1) * RF + 4 + mt * 16 + g] = st.o[mt][1];
+            rec[(h0 + 1) * RF + 4 + mt * 16 + g + 8] = st.o[mt][3];
+        }
+    }
+}
+
+// Fold the records of (unit, head h) into O, by all NW warps of the CTA (after the grid barrier):
+// NW/2 warps take the selected-block records (every (NW/2)-th), NW/8 (at least one) the window
+// records, the rest the compressed-token records; each folds up to 8 records per round trip into
+// (M, L, acc); warp 0 then combines the warps of each branch, applies the gates (cmp, slc, win) and
+// writes O. wM, wL [NW] and wO [NW][D] are shared-memory scratch.
+template <int D, int NW>
+__device__ void merge_head(const StepArgs& a, int unit, int h, float* wM, float* wL, float* wO) {
+    constexpr int RF = D + 4;
+    constexpr int CPL = D / 32;  // channels per lane
+    constexpr int kBatch = 8;
+    constexpr int kS = NW / 2 > 0 ? NW / 2 : 1, kW = NW / 8 > 0 ? NW / 8 : 1, kC = NW - kS - kW;
+    static_assert(kC >= 1, "at least one warp per branch");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int br = warp < kS ? 0 : (warp < kS + kW ? 1 : 2);
+    const int sl0 = warp < kS ? warp : (warp < kS + kW ? warp - kS : warp - kS - kW);
+    const int step = warp < kS ? kS : (warp < kS + kW ? kW : kC);
+    const int np = branch_pieces(a, unit, br);
+    const size_t rs = (size_t)a.G * RF;
+    const float* base = a.rec + ((size_t)unit * 3 + br) * a.maxw * rs + (size_t)h * RF;
+    float M = -INFINITY, Lsum = 0.0f, acc[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[c] = 0.0f;
+    for (int sl = sl0; sl < np; sl += kBatch * step) {
+        float m[kBatch], l[kBatch], o[kBatch][CPL];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int s = sl + q * step;
+            m[q] = -INFINITY;
+            l[q] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[q][c] = 0.0f;
+            if (s < np) {
+                const float* r = base + (size_t)s * rs;
+                m[q] = __ldcg(r);
+                l[q] = __ldcg(r + 1);
+                if constexpr (CPL == 4) {
+                    const float4 v4 = __ldcg(reinterpret_cast<const float4*>(r + 4 + lane * 4));
+                    o[q][0] = v4.x; o[q][1] = v4.y; o[q][2] = v4.z; o[q][3] = v4.w;
+                } else {
+                    const float2 v2 = __ldcg(reinterpret_cast<const float2*>(r + 4 + lane * 2));
+                    o[q][0] = v2.x; o[q][1] = v2.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            if (m[q] == -INFINITY) continue;
+            const float nM = fmaxf(M, m[q]);
+            const float fa = M == -INFINITY ? 0.0f : exp2f(M - nM);  // maxima are in log2 units
+            const float fb = exp2f(m[q] - nM);
+            Lsum = Lsum * fa + l[q] * fb;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[c] = acc[c] * fa + o[q][c] * fb;
+            M = nM;
+        }
+    }
+    if (lane == 0) {
+        wM[warp] = M;
+        wL[warp] = Lsum;
+    }
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) wO[warp * D + lane * CPL + c] = acc[c];
+    __syncthreads();
+    if (warp == 0) {
+        const int hq_row = unit * a.G + h;
+        const float* gate = a.gates + (size_t)hq_row * 3;
+        float out[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) out[c] = 0.0f;
+        // branch b2: selected blocks, window, compressed tokens: consecutive warp ranges
+        for (int b2 = 0; b2 < 3; ++b2) {
+            const int w0 = b2 == 0 ? 0 : (b2 == 1 ? kS : kS + kW), w1 = b2 == 0 ? kS : (b2 == 1 ? kS + kW : NW);
+            float GM = -INFINITY;
+            for (int w = w0; w < w1; ++w) GM = fmaxf(GM, wM[w]);
+            if (GM == -INFINITY) continue;
+            float GL = 0.0f, sum[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) sum[c] = 0.0f;
+            for (int w = w0; w < w1; ++w) {
+                if (wM[w] == -INFINITY) continue;
+                const float f = exp2f(wM[w] - GM);
+                GL += wL[w] * f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) sum[c] += wO[w * D + lane * CPL + c] * f;
+            }
+            if (!(GL > 0.0f)) continue;
+            const float gw = gate[b2 == 0 ? 1 : (b2 == 1 ? 2 : 0)] / GL;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) out[c] += gw * sum[c];
+        }
+        __nv_bfloat16* o = a.O + (size_t)hq_row * D + lane * CPL;
+#pragma unroll
+        for (int c = 0; c < CPL; c += 2)
+            *reinterpret_cast<__nv_bfloat162*>(o + c) = __floats2bfloat162_rn(out[c], out[c + 1]);
+    }
+    __syncthreads();  // the scratch is free for the next (unit, head)
+}
+
+// TR: keys as the mma rows (groups of at most 8 heads), else the heads as the rows.
+template <int D, bool TR>
+__global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                       const __grid_constant__ CUtensorMap tmV,
+                                                                       const __grid_constant__ CUtensorMap tmKc,
+                                                                       const __grid_constant__ CUtensorMap tmVc,
+                                                                       StepArgs a) {
+    constexpr int kBox = kStepTK * 128;    // one 64-column box of a 16-row tile
     constexpr int kMat = (D / 64) * kBox;  // K or V part of an attention tile
-    constexpr int kStage = 2 * kMat;       // = D * 128 bytes = one half of a summary group
-    static_assert(kStage == D * 32 * 4, "an attention tile and a summary half-group fill one stage");
+    constexpr int kStage = 2 * kMat;       // one K + V tile
+    static_assert(kStage == step_stage_bytes<D>(), "the launch sizes the rings with the same stage bytes");
+    static_assert(kStage * kParts == D * 32 * 4, "an attention tile and a summary part fill one stage");
+    constexpr int kPartC = D / kParts;     // channels of a summary part
+    constexpr bool kIL = D == 128;         // K / V tiles as one [rows][2][64] box (both column halves)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bars[kStepWarps][kStepStages];
     __shared__ __align__(16) float qsm[kStepWarps][2][D];         // group query: Qsum, Q2
     __shared__ __align__(16) float iso_sm[kStepWarps][kStepStages][32];
     __shared__ float q2t_sm[kStepWarps];
     __shared__ Item desc[kStepWarps][kStepStages];
+    __shared__ __align__(16) unsigned long long hbuf[kHelperRound * 32];  // helper staging
+    __shared__ float mM[kStepWarps + 1], mL[kStepWarps + 1];              // record merge scratch
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    unsigned char* ring = base + (size_t)warp * kStepStages * kStage;
-    uint64_t* bar = bars[warp];
-    const int v = blockIdx.x * kStepWarps + warp;
+    // phase-B block indices published by the helper warp: [maxbu][32] int, then [maxbu] mbarriers
+    int* bidx = reinterpret_cast<int*>(base + (size_t)kStepWarps * kStepStages * kStage);
+    uint64_t* ubar = reinterpret_cast<uint64_t*>(bidx + (size_t)a.maxbu * 32);
     const unsigned ep = *reinterpret_cast<volatile unsigned*>(a.ctl) + 1u;
+    int bu_first, bu_last;
+    cta_bunits(a, blockIdx.x, &bu_first, &bu_last);
 
-    // this warp's ranges
-    const long long s0 = fS(a, v), s1 = fS(a, v + 1);
-    const long long a0 = fA(a, v), a1 = fA(a, v + 1);
-    const long long b0 = fB(a, v), b1 = fB(a, v + 1);
-    const int nSi = (int)(s1 - s0) * a.tpg, nAi = (int)(a1 - a0), nBi = (int)(b1 - b0);
-    const int n = nSi + nAi + nBi;
-
-    if (lane == 0) {
-        for (int s = 0; s < kStepStages; ++s) mbar_init(&bar[s], 1);
+    if (threadIdx.x == 0) {
+        for (int j = 0; j <= bu_last - bu_first; ++j) mbar_init(&ubar[j], 32);  // every helper lane arrives
         fence_barrier_init();
     }
-    // no complete block: every list is empty (written by the first warps)
-    if (a.nGc == 0)
-        for (int u = v; u < a.units; u += a.nwarps) {
-            if (lane < a.k) a.idx[(size_t)u * a.k + lane] = -1;
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(&a.ready[u], ep);
-        }
-    __syncwarp();
+    __syncthreads();
 
-    const int t = a.T - 1;
-    int ready_u = -1;
-    // descriptor of this warp's item i (uniform across the warp)
-    auto item_at = [&](int i) {
-        Item it;
-        it.row = 0;
-        it.mask = 0u;
-        if (i < nSi) {
-            const int x = (int)s0 + (a.tpg == 2 ? i >> 1 : i);
-            it.kind = a.tpg == 2 ? i & 1 : 0;
-            it.unit = x / a.nGc;
-            it.a = x - it.unit * a.nGc;
-            it.mask = 1u;
-        } else if (i < nSi + nAi) {
-            const int y = (int)a0 + (i - nSi);
-            it.kind = 2;
-            it.unit = y / a.tA;
-            const int l = y - it.unit * a.tA;
-            if (l < a.tW) {
-                it.a = 1;
-                const int r0 = max(0, t - a.W + 1) + l * kTK;
-                it.row = it.unit * a.T + r0;
-                const int nk = min(kTK, t + 1 - r0);
-                it.mask = nk >= 32 ? kFull : ((1u << nk) - 1u);
-            } else {
-                it.a = 2;
-                const int c0 = (l - a.tW) * kTK;
-                it.row = it.unit * a.nC + c0;
-                const int nk = min(kTK, a.nC - c0);
-                it.mask = nk >= 32 ? kFull : ((1u << nk) - 1u);
-            }
-        } else {
-            const int z = (int)b0 + (i - nSi - nAi);
-            it.kind = 2;
-            it.a = 0;
-            it.unit = z / a.tS;
-            const int l = z - it.unit * a.tS;
-            int bi = -1;
-            if (lane == 0) {
-                if (it.unit != ready_u) wait_flag(&a.ready[it.unit], ep, a.err);  // gives up after a bound
-                bi = ld_relaxed(a.idx + (size_t)it.unit * a.k + l / (64 / kTK));
-            }
-            ready_u = it.unit;
-            bi = __shfl_sync(kFull, bi, 0);
-            if (bi >= 0) {
-                if (bi >= a.nB) {
-                    if (lane == 0) report_error(a.err, kErrBadIndex);
-                } else {
-                    it.row = it.unit * a.T + bi * 64 + (l % (64 / kTK)) * kTK;
-                    it.mask = kTK == 32 ? kFull : 0xFFFFu;
-                }
-            }
+    // ------------------------------------------------------------------ helper warp
+    if (warp == kStepWarps) {
+        for (int u = bu_first; u <= bu_last; ++u) {
+            int* out = bidx + (size_t)(u - bu_first) * 32;
+            helper_merge(a, u, ep, lane, out, hbuf);
+            // the CTA that holds the unit's first selected tile writes idx
+            if (lane < a.k && fB(a, (long long)blockIdx.x * kStepWarps) <= (long long)u * a.tS)
+                a.idx[(size_t)u * a.k + lane] = out[lane];
+            mbar_arrive(&ubar[u - bu_first]);  // each lane releases the indices it wrote
         }
-        return it;
-    };
-    uint32_t phase = 0;    // bit s: parity of the next completion of stage s
-    bool ok = true;        // false after a timed-out wait (uniform across the warp)
-    uint32_t pending = 0;  // stages with a copy in flight (lane 0's view)
-    auto issue = [&](const Item& it, int s) {  // lane 0 only
-        unsigned char* dst = ring + (size_t)s * kStage;
-        if (it.kind < 2 || it.mask != 0u) pending |= 1u << s;
-        if (it.kind < 2) {
-            const float* g = a.summ + ((size_t)it.unit * a.nG + it.a) * a.gfloats;
-            if (it.kind == 0) {
-                mbar_arrive_expect_tx(&bar[s], kStage + (a.iso ? 128u : 0u));
-                bulk_g2s(dst, g, kStage, &bar[s]);
-                if (a.iso) bulk_g2s(iso_sm[warp][s], g + D * 32, 128, &bar[s]);
-            } else {
-                mbar_arrive_expect_tx(&bar[s], kStage);
-                bulk_g2s(dst, g + D * 32, kStage, &bar[s]);
-            }
-            return;
-        }
-        if (it.mask == 0u) return;
-        const CUtensorMap* mk = it.a == 2 ? &tmKc : &tmK;
-        const CUtensorMap* mv = it.a == 2 ? &tmVc : &tmV;
-        mbar_arrive_expect_tx(&bar[s], kStage);
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-            tma_load_2d(dst + h * kBox, mk, h * 64, it.row, &bar[s]);
-            tma_load_2d(dst + kMat + h * kBox, mv, h * 64, it.row, &bar[s]);
-        }
-    };
+    } else {
+        // ------------------------------------------------------------------ streaming warps
+        unsigned char* ring = base + (size_t)warp * kStepStages * kStage;
+        uint64_t* bar = bars[warp];
+        const int v = blockIdx.x * kStepWarps + warp;
+        const long long s0 = fS(a, v), s1 = fS(a, v + 1);
+        const long long a0 = fA(a, v), a1 = fA(a, v + 1);
+        const long long b0 = fB(a, v), b1 = fB(a, v + 1);
+        const int nSi = (int)(s1 - s0) * a.tpg, nAi = (int)(a1 - a0), nBi = (int)(b1 - b0);
+        const int n = nSi + nAi + nBi;
 
-    int next_issue = 0;
-    bool sel_flushed = nSi == 0;
-    // issue every item whose stage is free; a phase-B item only once this warp's own selection
-    // segments are deposited (its descriptor may wait on a unit that one of them completes)
-    auto issue_ahead = [&](int consumed) {
-        while (next_issue < n && next_issue < consumed + kStepStages &&
-               (next_issue < nSi + nAi || sel_flushed)) {
-            const Item it = item_at(next_issue);
-            const int s = next_issue % kStepStages;
-            if (lane == 0) {
-                desc[warp][s] = it;
-                fence_proxy_async();
-                if (ok) issue(it, s);  // after a timed-out wait nothing more is loaded
-            }
-            ++next_issue;
+        if (lane == 0) {
+            for (int s = 0; s < kStepStages; ++s) mbar_init(&bar[s], 1);
+            fence_barrier_init();
         }
         __syncwarp();
-    };
 
-    RunList rl;
-    rl.init();
-    int sel_u = -1;
-    float apart = 0.0f;
-    WState<D> st;
-    st.init();
-    uint32_t qa[D / 16][4];
-    int att_u = -1, att_br = -1, q_u = -1;
-
-    issue_ahead(0);
-    for (int i = 0; i < n; ++i) {
-        issue_ahead(i);
-        const int s = i % kStepStages;
-        const Item it = desc[warp][s];
-        const unsigned char* stage = ring + (size_t)s * kStage;
-        if (it.kind < 2) {
-            if (it.unit != sel_u) {
-                if (sel_u >= 0) sel_finish(a, v, s0, sel_u, rl, ep, lane);
-                __syncwarp();  // every lane is done with the previous unit's group query
-                rl.init();
-                sel_u = it.unit;
-                // group query of the unit: lane l forms channels [l D/32, (l + 1) D/32)
-                group_query_chunk<__nv_bfloat16, D / 32>(a.Q + (size_t)sel_u * a.G * D, a.G, D, lane * (D / 32), true,
-                                                         &qsm[warp][0][lane * (D / 32)],
-                                                         &qsm[warp][1][lane * (D / 32)]);
-                __syncwarp();
-                if (a.iso) {
-                    if (lane == 0) q2t_sm[warp] = q2_total<D>(qsm[warp][1]);
-                    __syncwarp();
-                }
-            }
-            if (ok) ok = mbar_wait(&bar[s], (phase >> s) & 1u, a.err);
-            ok = __all_sync(kFull, ok);
-            if (ok) pending &= ~(1u << s);
-            phase ^= 1u << s;
-            const float* tile = reinterpret_cast<const float*>(stage);
-            const int b = it.a * 32 + lane;
-            bool done_group = false;
-            float sc = -INFINITY;
-            if (it.kind == 0) {
-                apart = ok ? score_mean_part<D>(tile, qsm[warp][0], lane) : 0.0f;
-                if (a.iso) {
-                    sc = score_combine(apart, __fmul_rn(q2t_sm[warp], iso_sm[warp][s][lane]), a.isd, a.c2);
-                    done_group = true;
+        const int t = a.T - 1;
+        uint32_t phase = 0;    // bit s: parity of the next completion of stage s
+        bool ok = true;        // false after a timed-out wait (uniform across the warp)
+        uint32_t pending = 0;  // stages with a copy in flight (lane 0's view)
+        int ready_u = -1;      // phase-B unit whose indices this warp has seen published
+        // descriptor of this warp's item i (uniform across the warp); element indices fit in int32
+        // descriptor of item i; a phase-B item first waits for its unit's published indices
+        auto item_at = [&](int i) {
+            Item it;
+            it.row = 0;
+            it.mask = 0u;
+            if (i < nSi) {
+                const int x = (int)s0 + i / a.tpg;
+                const int r = i - (i / a.tpg) * a.tpg;
+                it.kind = r / kParts;
+                it.part = r % kParts;
+                it.unit = x / a.nGc;
+                it.a = x - it.unit * a.nGc;
+                it.mask = 1u;
+            } else if (i < nSi + nAi) {
+                const int y = (int)a0 + (i - nSi);
+                it.kind = 2;
+                it.unit = y / a.tA;
+                const int l = y - it.unit * a.tA;
+                if (l < a.tW) {
+                    it.a = 1;
+                    const int r0 = max(0, t - a.W + 1) + l * kStepTK;
+                    it.row = it.unit * a.T + r0;
+                    const int nk = min(kStepTK, t + 1 - r0);
+                    it.mask = nk >= 32 ? kFull : ((1u << nk) - 1u);
+                } else {
+                    it.a = 2;
+                    const int c0 = (l - a.tW) * kStepTK;
+                    it.row = it.unit * a.nC + c0;
+                    const int nk = min(kStepTK, a.nC - c0);
+                    it.mask = nk >= 32 ? kFull : ((1u << nk) - 1u);
                 }
             } else {
-                const float vpart = ok ? score_var_part<D>(tile, qsm[warp][1], lane) : 0.0f;
-                sc = score_combine(apart, vpart, a.isd, a.c2);
-                done_group = true;
-            }
-            if (done_group) {
-                const bool valid = ok && b < a.ncand;
-                rl.add(valid ? sc : -INFINITY, valid ? b : kInvalid, a.k, lane);
-            }
-            if (i == nSi - 1) {  // the last summary tile of this warp: deposit / publish now
-                __syncwarp();
-                sel_finish(a, v, s0, sel_u, rl, ep, lane);
-                sel_u = -1;
-                sel_flushed = true;
-            }
-        } else {
-            if (it.unit != att_u || it.a != att_br) {
-                if (att_u >= 0) att_flush<D>(a, v, att_br == 0 ? b0 : a0, att_u, att_br, st, lane);
-                st.init();
-                att_u = it.unit;
-                att_br = it.a;
-                if (att_u != q_u) {
-                    load_q<D>(a.Q + (size_t)att_u * a.G * D, a.G, qa, lane);
-                    q_u = att_u;
+                const int z = (int)b0 + (i - nSi - nAi);
+                it.kind = 2;
+                it.a = 0;
+                it.unit = z / a.tS;
+                const int l = z - it.unit * a.tS;
+                const int j = it.unit - bu_first;  // this CTA's slot of the unit
+                if (it.unit != ready_u) {
+                    if (ok) ok = mbar_wait(&ubar[j], 0, a.err);  // the helper published the unit's indices
+                    ok = __all_sync(kFull, ok);
+                    ready_u = it.unit;
+                }
+                const int bi = ok ? bidx[(size_t)j * 32 + l / (64 / kStepTK)] : -1;
+                if (bi >= 0) {
+                    if (bi >= a.nB) {
+                        if (lane == 0) report_error(a.err, kErrBadIndex);
+                    } else {
+                        it.row = it.unit * a.T + bi * 64 + (l % (64 / kStepTK)) * kStepTK;
+                        it.mask = kStepTK == 32 ? kFull : 0xFFFFu;
+                    }
                 }
             }
-            if (it.mask != 0u) {
+            return it;
+        };
+        auto issue = [&](const Item& it, int s) {  // lane 0 only
+            unsigned char* dst = ring + (size_t)s * kStage;
+            if (it.kind < 2) {
+                pending |= 1u << s;
+                const float* g = a.summ + ((size_t)it.unit * a.nG + it.a) * a.gfloats;
+                // the isotropic scalars come with the last part of the means
+                const bool iso_here = a.iso && it.part == kParts - 1;
+                mbar_arrive_expect_tx(&bar[s], kStage + (iso_here ? 128u : 0u));
+                bulk_g2s(dst, g + (size_t)it.kind * D * 32 + (size_t)it.part * (kStage / 4), kStage, &bar[s]);
+                if (iso_here) bulk_g2s(iso_sm[warp][s], g + D * 32, 128, &bar[s]);
+                return;
+            }
+            if (it.mask == 0u) return;
+            pending |= 1u << s;
+            const CUtensorMap* mk = it.a == 2 ? &tmKc : &tmK;
+            const CUtensorMap* mv = it.a == 2 ? &tmVc : &tmV;
+            mbar_arrive_expect_tx(&bar[s], kStage);
+            if (kIL) {  // one 3-D box per tensor: rows it.row .. it.row + 15, both column halves
+                tma_load_3d(dst, mk, 0, 0, it.row, &bar[s]);
+                tma_load_3d(dst + kMat, mv, 0, 0, it.row, &bar[s]);
+            } else {
+                tma_load_2d(dst, mk, 0, it.row, &bar[s]);
+                tma_load_2d(dst + kMat, mv, 0, it.row, &bar[s]);
+            }
+        };
+
+
+        int next_issue = 0;
+        bool sel_done = nSi == 0;  // this warp's selection segments are all deposited
+        // issue every item whose stage is free (item i uses stage i % kStepStages); a phase-B item only
+        // once this warp's own segments are deposited (the helper it waits for may need them)
+        auto issue_ahead = [&](int consumed) {
+            while (next_issue < n && next_issue < consumed + kStepStages && (next_issue < nSi + nAi || sel_done)) {
+                const Item it = item_at(next_issue);
+                const int s = next_issue % kStepStages;
+                if (lane == 0) {
+                    desc[warp][s] = it;
+                    fence_proxy_async();
+                    if (ok) issue(it, s);  // after a timed-out wait nothing more is loaded
+                }
+                ++next_issue;
+            }
+            __syncwarp();
+        };
+
+        RunList rl;
+        rl.init();
+        int sel_u = -1;
+        float apart = 0.0f;
+        float ch[4] = {0.f, 0.f, 0.f, 0.f};  // the four canonical chains of the current half
+        std::conditional_t<TR, WStateT<D>, WState<D>> st;
+        st.init();
+        uint32_t qa[D / 16][TR ? 2 : 4];
+        int att_u = -1, att_br = -1, q_u = -1;
+
+        issue_ahead(0);
+        for (int i = 0; i < n; ++i) {
+            issue_ahead(i);
+            const int s = i % kStepStages;
+            const Item it = desc[warp][s];
+            const unsigned char* stage = ring + (size_t)s * kStage;
+            if (it.kind < 2) {
+                if (it.unit != sel_u) {
+                    if (sel_u >= 0) sel_deposit(a, v, s0, sel_u, rl, ep, lane);
+                    __syncwarp();  // every lane is done with the previous unit's group query
+                    rl.init();
+                    sel_u = it.unit;
+                    // group query of the unit: lane l forms channels [l D/32, (l + 1) D/32)
+                    group_query_chunk<__nv_bfloat16, D / 32>(a.Q + (size_t)sel_u * a.G * D, a.G, D, lane * (D / 32), true,
+                                                             &qsm[warp][0][lane * (D / 32)],
+                                                             &qsm[warp][1][lane * (D / 32)]);
+                    __syncwarp();
+                    if (a.iso) {
+                        if (lane == 0) q2t_sm[warp] = q2_total<D>(qsm[warp][1]);
+                        __syncwarp();
+                    }
+                }
                 if (ok) ok = mbar_wait(&bar[s], (phase >> s) & 1u, a.err);
                 ok = __all_sync(kFull, ok);
                 if (ok) pending &= ~(1u << s);
                 phase ^= 1u << s;
-                if (ok) tile_mma<D>(st, qa, stage, stage + kMat, it.mask, a.sl2, lane);
+                const float* tile = reinterpret_cast<const float*>(stage);
+                const int b = it.a * 32 + lane;
+                bool done_group = false;
+                float sc = -INFINITY;
+                if (it.part == 0) ch[0] = ch[1] = ch[2] = ch[3] = 0.0f;
+                // channels [part kPartC, (part + 1) kPartC) of the means (Qsum) or variances (Q2)
+                if (ok) score_chains<kPartC / 4>(tile, qsm[warp][it.kind] + it.part * kPartC, lane, ch);
+                if (it.part == kParts - 1) {
+                    const float half_sum = combine4(ch[0], ch[1], ch[2], ch[3]);
+                    if (it.kind == 0) {
+                        apart = half_sum;
+                        if (a.iso) {
+                            sc = score_combine(apart, __fmul_rn(q2t_sm[warp], iso_sm[warp][s][lane]), a.isd, a.c2);
+                            done_group = true;
+                        }
+                    } else {
+                        sc = score_combine(apart, half_sum, a.isd, a.c2);
+                        done_group = true;
+                    }
+                }
+                if (done_group) {
+                    const bool valid = ok && b < a.ncand;
+                    rl.add(valid ? sc : -INFINITY, valid ? b : kInvalid, a.k, lane);
+                }
+                if (i == nSi - 1) {  // the last summary tile of this warp
+                    sel_deposit(a, v, s0, sel_u, rl, ep, lane);
+                    sel_u = -1;
+                    sel_done = true;
+                }
+            } else {
+                if (it.unit != att_u || it.a != att_br) {
+                    if (att_u >= 0) {
+                        if constexpr (TR) att_flush_t<D>(a, v, att_br == 0 ? b0 : a0, att_u, att_br, st, lane);
+                        else att_flush<D>(a, v, att_br == 0 ? b0 : a0, att_u, att_br, st, lane);
+                    }
+                    st.init();
+                    att_u = it.unit;
+                    att_br = it.a;
+                    if (att_u != q_u) {
+                        if constexpr (TR) load_qt<D>(a.Q + (size_t)att_u * a.G * D, a.G, qa, lane);
+                        else load_q<D>(a.Q + (size_t)att_u * a.G * D, a.G, qa, lane);
+                        q_u = att_u;
+                    }
+                }
+                if (it.mask != 0u) {
+                    if (ok) ok = mbar_wait(&bar[s], (phase >> s) & 1u, a.err);
+                    ok = __all_sync(kFull, ok);
+                    if (ok) pending &= ~(1u << s);
+                    phase ^= 1u << s;
+                    if (ok) {
+                        if constexpr (TR) tile_mma_t<D, kStepTK, kIL>(st, qa, stage, stage + kMat, it.mask, a.sl2, lane);
+                        else tile_mma<D, kStepTK, kIL>(st, qa, stage, stage + kMat, it.mask, a.sl2, lane);
+                    }
+                }
             }
+            __syncwarp();
         }
-        __syncwarp();
+        if (att_u >= 0) {
+            if constexpr (TR) att_flush_t<D>(a, v, att_br == 0 ? b0 : a0, att_u, att_br, st, lane);
+            else att_flush<D>(a, v, att_br == 0 ? b0 : a0, att_u, att_br, st, lane);
+        }
+        // after a timed-out wait: let the copies still in flight land (bounded) before the CTA exits
+        if (lane == 0 && !ok)
+            for (int s = 0; s < kStepStages; ++s)
+                if ((pending >> s) & 1u) mbar_wait(&bar[s], (phase >> s) & 1u, nullptr);
     }
-    if (att_u >= 0) att_flush<D>(a, v, att_br == 0 ? b0 : a0, att_u, att_br, st, lane);
-    // after a timed-out wait: let the copies still in flight land (bounded) before the CTA exits
-    if (lane == 0 && !ok)
-        for (int s = 0; s < kStepStages; ++s)
-            if ((pending >> s) & 1u) mbar_wait(&bar[s], (phase >> s) & 1u, nullptr);
 
-    // the last CTA to finish advances the epoch (the next launch on the stream reads it)
+    // ------------------------------------------------------------------ grid barrier, record merge
+    // Every CTA is resident (cooperative launch, one per SM). The arrival counter ctl[1] grows by
+    // the grid size per step, so this step's barrier is complete at ep x gridDim.x arrivals.
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned old = atomicAdd(&a.ctl[1], 1u);
-        if (old == gridDim.x - 1) {
-            a.ctl[1] = 0u;
-            __threadfence();
-            a.ctl[0] = ep;
+        __threadfence();  // this CTA's records and idx are visible before its arrival
+        atomicAdd(&a.ctl[1], 1u);
+        const unsigned target = ep * gridDim.x;
+        const uint64_t t0 = global_ns();
+        bool late = false;
+        for (uint32_t it = 0; (int)(ld_acquire_u32(&a.ctl[1]) - target) < 0; ++it) {
+            if (it >= kMaxWaitIters || global_ns() - t0 > kWaitLimitNs) {
+                late = true;
+                break;
+            }
+            __nanosleep(64);
         }
+        if (late) report_error(a.err, kErrWaitTimeout);
+        __threadfence();
+        mM[0] = late ? 1.0f : 0.0f;
     }
+    __syncthreads();
+    const bool merge_ok = mM[0] == 0.0f;
+    __syncthreads();
+    if (merge_ok) {
+        float* wO = reinterpret_cast<float*>(base);  // the rings are free: [kStepWarps + 1][D]
+        for (int p = blockIdx.x; p < a.units * a.G; p += gridDim.x)
+            merge_head<D, kStepWarps + 1>(a, p / a.G, p % a.G, mM, mL, wO);
+    }
+    // the epoch advances once every CTA has passed the barrier (all read it at their start)
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&a.ctl[0], 1u);
+
 }
 
-// Workspace layout: control words, then the counters, segment lists, records and branch outputs
-// (each region 256-byte aligned).
+// Workspace layout: the control word, the segment lists and the attention records (each region
+// 256-byte aligned).
 struct StepLayout {
-    size_t ctl, ready, sel_cnt, br_cnt, unit_cnt, seg_s, seg_i, rec, bout, total;
+    size_t ctl, seg, rec, total;
 };
 
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -657,14 +754,8 @@ StepLayout step_layout(const StepArgs& a) {
     StepLayout L;
     size_t o = 0;
     L.ctl = o; o = al256(o + 2 * sizeof(unsigned));
-    L.ready = o; o = al256(o + (size_t)a.units * sizeof(unsigned));
-    L.sel_cnt = o; o = al256(o + (size_t)a.units * sizeof(unsigned));
-    L.br_cnt = o; o = al256(o + (size_t)a.units * 3 * sizeof(unsigned));
-    L.unit_cnt = o; o = al256(o + (size_t)a.units * sizeof(unsigned));
-    L.seg_s = o; o = al256(o + (size_t)a.units * a.maxseg * 32 * sizeof(float));
-    L.seg_i = o; o = al256(o + (size_t)a.units * a.maxseg * 32 * sizeof(int));
+    L.seg = o; o = al256(o + (size_t)a.units * a.maxseg * 32 * sizeof(unsigned long long));
     L.rec = o; o = al256(o + (size_t)a.units * 3 * a.maxw * a.G * (a.D + 4) * sizeof(float));
-    L.bout = o; o = al256(o + (size_t)a.units * 3 * a.G * a.D * sizeof(float));
     L.total = o;
     return L;
 }
@@ -676,18 +767,17 @@ StepArgs make_step_args(const Dims& m) {
     a.ncand = m.nB;  // decode at T - 1: every complete block is a candidate
     a.nGc = (a.ncand + 31) / 32;
     a.iso = m.iso;
-    a.tpg = m.iso ? 1 : 2;
+    a.tpg = (m.iso ? 1 : 2) * kParts;
     a.gfloats = (int)m.group_floats();
-    a.tS = m.k * (64 / kTK);
-    a.tW = (std::min(m.W, m.T) + kTK - 1) / kTK;
-    a.tC = (m.nC + kTK - 1) / kTK;
+    a.tS = m.k * (64 / kStepTK);
+    a.tW = (std::min(m.W, m.T) + kStepTK - 1) / kStepTK;
+    a.tC = (m.nC + kStepTK - 1) / kStepTK;
     a.tA = a.tW + a.tC;
     a.nwarps = sm_count() * kStepWarps;
     a.nS = (long long)a.units * a.nGc;
     a.nA = (long long)a.units * a.tA;
     a.nBt = (long long)a.units * a.tS;
     a.tot = a.tpg * a.nS + a.nA + a.nBt;
-    a.nbr = 1 + (a.tW > 0) + (a.tC > 0);
     a.inv_nw = 1.0 / a.nwarps;
     a.inv_nS = a.nS > 0 ? 1.0 / (double)a.nS : 0.0;
     a.inv_nA = a.nA > 0 ? 1.0 / (double)a.nA : 0.0;
@@ -706,6 +796,12 @@ StepArgs make_step_args(const Dims& m) {
         if (a.nGc > 0) a.maxseg = std::max(a.maxseg, sel_segments(a, u));
         for (int br = 0; br < 3; ++br) a.maxw = std::max(a.maxw, branch_pieces(a, u, br));
     }
+    a.maxbu = 1;
+    for (int c = 0; c < a.nwarps / kStepWarps; ++c) {
+        int f, l;
+        cta_bunits(a, c, &f, &l);
+        a.maxbu = std::max(a.maxbu, l - f + 1);
+    }
     float isd, c2;
     score_constants(m.d, m.alpha, &isd, &c2);
     a.isd = isd;
@@ -714,35 +810,66 @@ StepArgs make_step_args(const Dims& m) {
     return a;
 }
 
+// Dynamic shared memory: the rings, then the phase-B index table and its mbarriers, plus the
+// alignment slack of the ring base.
 template <int D>
-size_t step_smem() { return (size_t)kStepWarps * kStepStages * D * 128 + 1024; }
+size_t step_smem(const StepArgs& a) {
+    return (size_t)kStepWarps * kStepStages * step_stage_bytes<D>() +
+           (size_t)a.maxbu * (32 * sizeof(int) + sizeof(uint64_t)) + 1024;
+}
 
-template <int D>
+template <int D, bool TR>
 cudaError_t launch_step_d(const Dims& m, StepArgs a, const void* K, const void* V, const void* Kc, const void* Vc,
                           cudaStream_t s) {
     CUtensorMap tk, tv, tkc, tvc;
     const uint64_t kvrows = (uint64_t)m.units() * m.T;
     const uint64_t crows = m.nC > 0 ? (uint64_t)m.units() * m.nC : kvrows;
-    if (!encode_tmap_bf16_2d(&tk, K, kvrows, D, kTK) || !encode_tmap_bf16_2d(&tv, V, kvrows, D, kTK) ||
-        !encode_tmap_bf16_2d(&tkc, m.nC > 0 ? Kc : K, crows, D, kTK) ||
-        !encode_tmap_bf16_2d(&tvc, m.nC > 0 ? Vc : V, crows, D, kTK))
+    // d = 128: a [rows][2][64] view (row pitch 256 bytes, half pitch 128) read in boxes of
+    // kStepTK rows x both halves; d = 64: [rows][64] in boxes of kStepTK rows
+    auto enc = [&](CUtensorMap* map, const void* base, uint64_t rows) {
+        if (D == 128) {
+            const uint64_t dims[3] = {64, 2, rows};
+            const uint64_t strides[2] = {128, 256};
+            const uint32_t box[3] = {64, 2, (uint32_t)kStepTK};
+            return encode_tmap_bf16_3d(map, base, dims, strides, box);
+        }
+        return encode_tmap_bf16_2d(map, base, rows, D, kStepTK);
+    };
+    if (!enc(&tk, K, kvrows) || !enc(&tv, V, kvrows) || !enc(&tkc, m.nC > 0 ? Kc : K, crows) ||
+        !enc(&tvc, m.nC > 0 ? Vc : V, crows))
         return cudaErrorInvalidValue;
-    const size_t smem = step_smem<D>();
-    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = step_smem<D>(a);
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_step_kernel<D, TR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_step_kernel<D>, kStepWarps * 32, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_step_kernel<D, TR>, kStepThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorNotSupported;
+    // cooperative: every CTA resident at once (the record merge follows a grid barrier)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.nwarps / kStepWarps);
+    cfg.blockDim = dim3(kStepThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     count_launch();
-    decode_step_kernel<D><<<a.nwarps / kStepWarps, kStepWarps * 32, smem, s>>>(tk, tv, tkc, tvc, a);
-    return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<D, TR>, tk, tv, tkc, tvc, a);
 }
 
 }  // namespace
 
 bool decode_step_supported(const Dims& m) {
-    return m.dtype == COBS_BF16 && !m.lr && (m.d == 128 || m.d == 64) && m.L == 64;
+    // the phase-B index table of a CTA must fit beside the rings (checked on the host sizes)
+    if (!(m.dtype == COBS_BF16 && !m.lr && (m.d == 128 || m.d == 64) && m.L == 64 &&
+          (long long)m.nB < (1ll << kIdxBits) - 1))
+        return false;
+    const StepArgs a = make_step_args(m);
+    return (m.d == 128 ? step_smem<128>(a) : step_smem<64>(a)) <= 200 * 1024;
 }
 
 size_t decode_step_workspace_bytes(const Dims& m) {
@@ -763,15 +890,12 @@ cudaError_t launch_decode_step(const Dims& m, const void* Q, const float* summ, 
     a.O = static_cast<__nv_bfloat16*>(O);
     a.err = err;
     a.ctl = reinterpret_cast<unsigned*>(w + L.ctl);
-    a.ready = reinterpret_cast<unsigned*>(w + L.ready);
-    a.sel_cnt = reinterpret_cast<unsigned*>(w + L.sel_cnt);
-    a.br_cnt = reinterpret_cast<unsigned*>(w + L.br_cnt);
-    a.unit_cnt = reinterpret_cast<unsigned*>(w + L.unit_cnt);
-    a.seg_s = reinterpret_cast<float*>(w + L.seg_s);
-    a.seg_i = reinterpret_cast<int*>(w + L.seg_i);
+    a.seg = reinterpret_cast<unsigned long long*>(w + L.seg);
     a.rec = reinterpret_cast<float*>(w + L.rec);
-    a.bout = reinterpret_cast<float*>(w + L.bout);
-    return m.d == 128 ? launch_step_d<128>(m, a, K, V, Kc, Vc, s) : launch_step_d<64>(m, a, K, V, Kc, Vc, s);
+    // groups of at most 8 heads: keys as the mma rows
+    if (m.G <= 8)
+        return m.d == 128 ? launch_step_d<128, true>(m, a, K, V, Kc, Vc, s) : launch_step_d<64, true>(m, a, K, V, Kc, Vc, s);
+    return m.d == 128 ? launch_step_d<128, false>(m, a, K, V, Kc, Vc, s) : launch_step_d<64, false>(m, a, K, V, Kc, Vc, s);
 }
 
 }  // namespace cobs

@@ -193,23 +193,33 @@ struct RunList {
     }
 };
 
+// Continue the four canonical chains over NC4 consecutive channel quads: chain j adds
+// fma(q_c, x_c, .) for the channels c = j (mod 4) in ascending order. x: [NC4][32][4]
+// channel-interleaved values of the group's 32 blocks (lane = block); q: the NC4 * 4 matching
+// query values. Feeding a group's channel quads in ascending order, in one call or several,
+// gives the same chains.
+template <int NC4>
+__device__ __forceinline__ void score_chains(const float* x, const float* q, int lane, float (&c)[4]) {
+    const float4* x4 = reinterpret_cast<const float4*>(x) + lane;
+#pragma unroll 8
+    for (int c4 = 0; c4 < NC4; ++c4) {
+        const float4 m = x4[c4 * 32];
+        const float4 qq = reinterpret_cast<const float4*>(q)[c4];
+        c[0] = __fmaf_rn(qq.x, m.x, c[0]);
+        c[1] = __fmaf_rn(qq.y, m.y, c[1]);
+        c[2] = __fmaf_rn(qq.z, m.z, c[2]);
+        c[3] = __fmaf_rn(qq.w, m.w, c[3]);
+    }
+}
+
 // The mean half of the canonical score: a = (s0 + s1) + (s2 + s3), chain j summing
 // fma(Qsum_c, mu_c, .) over the channels c = j (mod 4) in ascending order. mu: the group's
 // [D/4][32][4] channel-interleaved means (lane = block).
 template <int D>
 __device__ __forceinline__ float score_mean_part(const float* mu, const float* qs, int lane) {
-    const float4* mu4 = reinterpret_cast<const float4*>(mu) + lane;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 8
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 m = mu4[c4 * 32];
-        const float4 q = reinterpret_cast<const float4*>(qs)[c4];
-        a0 = __fmaf_rn(q.x, m.x, a0);
-        a1 = __fmaf_rn(q.y, m.y, a1);
-        a2 = __fmaf_rn(q.z, m.z, a2);
-        a3 = __fmaf_rn(q.w, m.w, a3);
-    }
-    return combine4(a0, a1, a2, a3);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    score_chains<D / 4>(mu, qs, lane, c);
+    return combine4(c[0], c[1], c[2], c[3]);
 }
 
 // The variance half: v = four-chain sum of fma(Q2_c, var_c, .) in the same order.
