@@ -297,8 +297,8 @@ def decode_config(w, args, R=None, world=1):
         cfg["rank"] = args.rank
     if args.variance == "subspace":
         cfg.update(sub=args.sub, queries="concentrated in the subspace (leak 0.1)")
-    cfg["step"] = ("cobs_decode_step: summary update at T-1, then selection + decode attention in one kernel; "
-                   "one CUDA graph")
+    cfg["step"] = ("cobs_decode_step: summary update at T-1, selection, then the decode attention as a "
+                   "programmatic dependent of the selection; one CUDA graph")
     cfg["l2"] = f"{R or max(1, args.copies)} KV-cache copies rotated between steps (working set > L2)"
     cfg["parallelism"] = f"dp{world} (independent decode batches per GPU)"
     return cfg
@@ -541,8 +541,9 @@ def measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=True, c
 
     # ---- per-call durations: graphs of one part of the step each, replayed one at a time on the
     # launching stream with the same copy rotation (cold, isolated figures: no overlap with the
-    # neighbouring kernels): the summary update alone; the fused selection + attention kernel alone
-    # (cobs_decode_step with nothing to update); and the three separate calls of the unfused step ----
+    # neighbouring kernels, so they add up to more than the step, whose attention grid overlaps the
+    # selection as its programmatic dependent): the three separate calls; and the one-kernel
+    # alternative (cobs_decode_step_fused with nothing to update) ----
     def timed_parts(build_parts, nparts):
         graphs_, evs_ = [], []
         for r in range(R):
@@ -573,39 +574,47 @@ def measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=True, c
                                                  bufs[r].Vc)
 
     def fused_only(r):
-        return lambda: cobs.cobs_decode_step(p, tQ, Ks[r], Vs[r], tPk, tPv, w.T, bufs[r].summaries, bufs[r].Kc,
-                                             bufs[r].Vc, bufs[r].idx, tg, bufs[r].O, bufs[r].ws_step)
+        return lambda: cobs.cobs_decode_step_fused(p, tQ, Ks[r], Vs[r], tPk, tPv, w.T, bufs[r].summaries,
+                                                   bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg, bufs[r].O,
+                                                   bufs[r].ws_step_fused)
 
-    t_upd, t_fused = timed_parts(lambda r: [upd(r), fused_only(r)], 2)
-    t_upd2, t_sel, t_att = timed_parts(lambda r: [
+    has_fused = bufs[0].ws_step_fused is not None
+    t_fused = timed_parts(lambda r: [fused_only(r)], 1)[0] if has_fused else None
+    t_upd, t_sel, t_att = timed_parts(lambda r: [
         upd(r),
         lambda: cobs.cobs_select(p, tQ, bufs[r].summaries, 0, bufs[r].idx, bufs[r].ws_select),
         lambda: cobs.cobs_sparse_attn_decode(p, tQ, Ks[r], Vs[r], bufs[r].Kc, bufs[r].Vc, bufs[r].idx, tg,
                                              bufs[r].O, bufs[r].ws_attn)], 3)
-    # the unfused step (three calls, five kernels) as one graph, for comparison with the headline
-    ugraphs = []
-    for r in range(R):
-        gr = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gr, stream=stream):
-            cobs.decode_step(p, tQ, Ks[r], Vs[r], tPk, tPv, tg, bufs[r], t_begin=w.T - 1, fused=False)
-        ugraphs.append(gr)
-    torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        for i in range(R):
-            ugraphs[i].replay()
-        e0.record(stream)
-        for i in range(steps):
-            ugraphs[i % R].replay()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    ms_unfused = e0.elapsed_time(e1) / steps
-    del ugraphs
+    # the same step through the three separate calls, and through the one-kernel alternative, each
+    # as one graph per copy, for comparison with the headline
+    def step_graph_ms(path):
+        ugraphs = []
+        for r in range(R):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                cobs.decode_step(p, tQ, Ks[r], Vs[r], tPk, tPv, tg, bufs[r], t_begin=w.T - 1, path=path)
+            ugraphs.append(gr)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            for i in range(R):
+                ugraphs[i].replay()
+            e0.record(stream)
+            for i in range(steps):
+                ugraphs[i % R].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        del ugraphs
+        return e0.elapsed_time(e1) / steps
+
+    ms_calls = step_graph_ms("calls")
+    ms_fused = step_graph_ms("fused") if has_fused else None
 
     e2e = None
     if with_e2e:
         e2e = measure_e2e(w, p, Q, g, Ks, Vs, bufs, tPk, tPv, tQ, tg, stream, dev, cobs, R, steps)
-    out = {"ms": ms, "clocks": clk_summary, "t_upd": t_upd, "t_fused": t_fused, "t_upd2": t_upd2, "t_sel": t_sel,
-           "t_att": t_att, "ms_unfused": ms_unfused, "e2e": e2e, "launches_per_step": launches_per_step,
+    out = {"ms": ms, "clocks": clk_summary, "t_upd": t_upd, "t_fused": t_fused, "t_sel": t_sel,
+           "t_att": t_att, "ms_calls": ms_calls, "ms_fused": ms_fused, "e2e": e2e,
+           "launches_per_step": launches_per_step,
            "device_error": cobs.device_error(), "idx0": idx0, "O0": O0, "idx_a0": idx_a0,
            "host": (K, V, Q, g, Pk, Pv, basis)}
     del graphs[:], Ks, Vs, bufs
@@ -690,23 +699,46 @@ def oracle_parity(w, idx_g, O_g, res_units, tol):
             "fp64_near_ties": len(gaps), "fp64_near_tie_max_rel_gap": max(gaps) if gaps else None}
 
 
+def decode_roofline(by, m, peak, peak_kind):
+    """Roofline of the step's dominant kernel, the three-branch decode attention (the largest share
+    of the step's bytes), timed alone."""
+    att_gbs = by["attn"] / (m["t_att"] * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "decode_stream_kernel (three-branch decode attention)",
+            "achieved": att_gbs, "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
+            "peak_kind": f"{peak_kind} (copy, read + write)", "algorithmic_bytes_per_launch": by["attn"],
+            "timing": "CUDA events around cobs_sparse_attn_decode alone (graph per copy, replayed on the "
+                      "launching stream, median)",
+            "traffic": recorded_traffic("decode_attention")}
+
+
+def decode_calls(by, m, peak):
+    """Per-call durations and the alternative schedules of the same step."""
+    out = {"build_summaries_update": m["t_upd"], "select": m["t_sel"], "sparse_attn_decode": m["t_att"],
+           "select_gbs": by["select"] / (m["t_sel"] * 1e-3) / 1e9,
+           "attn_gbs": by["attn"] / (m["t_att"] * 1e-3) / 1e9,
+           "separate_calls_ms_per_step": m["ms_calls"]}
+    if m["t_fused"] is not None:
+        gbs = (by["select"] + by["attn"]) / (m["t_fused"] * 1e-3) / 1e9
+        out["fused"] = {"ms_per_step": m["ms_fused"], "decode_step_kernel": m["t_fused"], "kernel_gbs": gbs,
+                        "kernel_frac": gbs / peak,
+                        "definition": "cobs_decode_step_fused: selection and attention in one persistent kernel"}
+    return out
+
+
 def decode_subrecord(name, args, dev, cobs, world, steps=50, warmup=5, R=4):
     """A decode workload other than the headline one, measured the same way (no end-to-end
-    pass): step time, the fused kernel's roofline, traffic ratios, oracle parity on two units."""
+    pass): step time, the attention kernel's roofline, traffic ratios, oracle parity on two units."""
     import synth
     w = synth.WORKLOADS[name]
     m = measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=False, clocks=False)
     by = decode_bytes(w, m["idx0"], args.variance, args.rank, args.sub)
     peak, peak_kind = read_peaks()
-    fused_gbs = (by["select"] + by["attn"]) / (m["t_fused"] * 1e-3) / 1e9
+    hbm = by["total"] / (m["ms"] * 1e-3) / 1e9
     rec = {"workload": name, "config": decode_config(w, args, R, world), "ms_per_step": m["ms"],
            "value": w.B * w.Hq * world / (m["ms"] * 1e-3), "unit": "query-heads/s",
-           "hbm_gbs": by["total"] / (m["ms"] * 1e-3) / 1e9, "hbm_bytes_per_step": by["total"],
-           "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": fused_gbs, "peak": peak,
-                        "unit": "GB/s", "frac": fused_gbs / peak, "peak_kind": peak_kind,
-                        "algorithmic_bytes_per_launch": by["select"] + by["attn"]},
-           "calls_ms": {"build_summaries_update": m["t_upd"], "decode_step_kernel": m["t_fused"],
-                        "unfused_ms_per_step": m["ms_unfused"], "select": m["t_sel"], "sparse_attn_decode": m["t_att"]},
+           "hbm_gbs": hbm, "hbm_bytes_per_step": by["total"], "step_frac": hbm / peak,
+           "roofline": decode_roofline(by, m, peak, peak_kind),
+           "calls_ms": decode_calls(by, m, peak),
            "traffic": traffic_ratios(w, m["idx0"], m["idx_a0"], args.variance, args.rank, args.sub),
            "gpu_launches": m["launches_per_step"] * steps, "steps": steps, "device_error": m["device_error"]}
     if not args.no_cpu_baseline:
@@ -763,8 +795,6 @@ def run_ours(args):
     qheads = w.B * w.Hq * world
     by = decode_bytes(w, idx0, args.variance, args.rank, args.sub)
     peak, peak_kind = read_peaks()
-    fused_gbs = (by["select"] + by["attn"]) / (m["t_fused"] * 1e-3) / 1e9
-    att_gbs = by["attn"] / (m["t_att"] * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": qheads / (ms * 1e-3), "unit": "query-heads/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -772,18 +802,9 @@ def run_ours(args):
         "config": decode_config(w, args, R, world),
         "hbm_gbs": by["total"] / (ms * 1e-3) / 1e9,
         "hbm_bytes_per_step": by["total"],
-        "roofline": {"bound": "hbm", "kernel": "decode_step_kernel (selection + three-branch attention, one launch)",
-                     "achieved": fused_gbs, "peak": peak, "unit": "GB/s", "frac": fused_gbs / peak,
-                     "peak_kind": f"{peak_kind} (copy, read + write)",
-                     "algorithmic_bytes_per_launch": by["select"] + by["attn"],
-                     "timing": "CUDA events around the kernel alone (graph per copy, replayed on the launching "
-                               "stream, median)",
-                     "traffic": recorded_traffic("decode_step")},
-        "calls_ms": {"build_summaries_update": m["t_upd"], "decode_step_kernel": m["t_fused"],
-                     "unfused": {"ms_per_step": m["ms_unfused"], "build_summaries_update": m["t_upd2"],
-                                 "select": m["t_sel"], "sparse_attn_decode": m["t_att"],
-                                 "select_gbs": by["select"] / (m["t_sel"] * 1e-3) / 1e9,
-                                 "attn_gbs": att_gbs, "attn_frac": att_gbs / peak}},
+        "step_frac": by["total"] / (ms * 1e-3) / 1e9 / peak,
+        "roofline": decode_roofline(by, m, peak, peak_kind),
+        "calls_ms": decode_calls(by, m, peak),
         "traffic": traffic_ratios(w, idx0, m["idx_a0"], args.variance, args.rank, args.sub),
         "e2e": {"value": qheads / (e2e["ms"] * 1e-3), "unit": "query-heads/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["ms"],

@@ -28,11 +28,13 @@ COBS_WS_SELECT = 0
 COBS_WS_DECODE = 1
 COBS_WS_PREFILL = 2
 COBS_WS_STEP = 3
+COBS_WS_STEP_FUSED = 4
 
 EXPORTED = [
     "cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
     "cobs_sparse_attn_decode_noalloc", "cobs_workspace_bytes", "cobs_summaries_elems", "cobs_status_string", "cobs_last_error",
     "cobs_device_error", "cobs_launch_count", "cobs_version", "cobs_block_log_mass", "cobs_decode_step",
+    "cobs_decode_step_fused",
 ]
 
 
@@ -64,8 +66,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.cobs_sparse_attn_decode_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.cobs_block_log_mass.argtypes = [P, vp, vp, vp, vp]
     lib.cobs_decode_step.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.cobs_decode_step_fused.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for f in ("cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
-              "cobs_sparse_attn_decode_noalloc", "cobs_block_log_mass", "cobs_decode_step"):
+              "cobs_sparse_attn_decode_noalloc", "cobs_block_log_mass", "cobs_decode_step", "cobs_decode_step_fused"):
         getattr(lib, f).restype = ctypes.c_int
     lib.cobs_workspace_bytes.argtypes = [P, i32]
     lib.cobs_workspace_bytes.restype = sz
@@ -204,6 +207,16 @@ def cobs_decode_step(p: Params, Q, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, idx
                                  _ptr(workspace), nbytes, _stream(stream)))
 
 
+def cobs_decode_step_fused(p: Params, Q, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, idx, gates, O, workspace,
+                           stream=None):
+    """The same step with the selection and the attention in one persistent kernel."""
+    cp = p.c()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.cobs_decode_step_fused(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(Pk), _ptr(Pv),
+                                       int(t_begin), _ptr(summaries), _ptr(Kc), _ptr(Vc), _ptr(idx), _ptr(gates),
+                                       _ptr(O), _ptr(workspace), nbytes, _stream(stream)))
+
+
 def cobs_sparse_attn_decode_noalloc(p: Params, Q, K, V, Kc, Vc, idx, gates, O, stream=None):
     """Decode attention using the library's built-in device scratch instead of a workspace,
     for callers that cannot provide device memory of their own (see include/cobs.h)."""
@@ -237,6 +250,7 @@ class Buffers:
     ws_select: torch.Tensor
     ws_attn: torch.Tensor
     ws_step: torch.Tensor | None = None
+    ws_step_fused: torch.Tensor | None = None  # None: a shape cobs_decode_step_fused does not take
 
 
 def alloc(p: Params, prefill: bool, device="cuda") -> Buffers:
@@ -254,16 +268,25 @@ def alloc(p: Params, prefill: bool, device="cuda") -> Buffers:
                           dtype=torch.uint8, device=device)
     ws_step = None if prefill else torch.zeros(max(16, workspace_bytes(p, COBS_WS_STEP)), dtype=torch.uint8,
                                                device=device)
-    return Buffers(summ, Kc, Vc, idx, O, ws_sel, ws_attn, ws_step)
+    nf = 0 if prefill else workspace_bytes(p, COBS_WS_STEP_FUSED)
+    ws_fused = torch.zeros(nf, dtype=torch.uint8, device=device) if nf else None
+    return Buffers(summ, Kc, Vc, idx, O, ws_sel, ws_attn, ws_step, ws_fused)
 
 
-def decode_step(p: Params, Q, K, V, Pk, Pv, gates, buf: Buffers, t_begin: int, stream=None, fused: bool = True):
+def decode_step(p: Params, Q, K, V, Pk, Pv, gates, buf: Buffers, t_begin: int, stream=None, path: str = "step"):
     """Summaries update from t_begin, selection and attention for the query at T - 1: one
-    cobs_decode_step call, or (fused=False) the three separate calls."""
-    if fused:
+    cobs_decode_step call (path "step"), one cobs_decode_step_fused call ("fused"), or the three
+    separate calls ("calls")."""
+    if path == "step":
         cobs_decode_step(p, Q, K, V, Pk, Pv, t_begin, buf.summaries, buf.Kc, buf.Vc, buf.idx, gates, buf.O,
                          buf.ws_step, stream)
         return
+    if path == "fused":
+        cobs_decode_step_fused(p, Q, K, V, Pk, Pv, t_begin, buf.summaries, buf.Kc, buf.Vc, buf.idx, gates, buf.O,
+                               buf.ws_step_fused, stream)
+        return
+    if path != "calls":
+        raise ValueError(f"unknown decode step path {path!r}")
     cobs_build_summaries(p, K, V, Pk, Pv, t_begin, buf.summaries, buf.Kc, buf.Vc, stream)
     cobs_select(p, Q, buf.summaries, 0, buf.idx, buf.ws_select, stream)
     cobs_sparse_attn_decode(p, Q, K, V, buf.Kc, buf.Vc, buf.idx, gates, buf.O, buf.ws_attn, stream)

@@ -131,17 +131,15 @@ void score_constants(int d, float alpha, float* isd, float* c2) {
 namespace {
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Decode step workspace: the fused kernel's control words, lists and records, or (for the shapes
-// it does not take) the selection workspace followed by the decode-attention workspace.
+// Decode step workspace: the selection workspace followed by the decode-attention workspace.
 size_t step_workspace_bytes(const cobs::Dims& m) {
-    if (cobs::decode_step_supported(m)) return cobs::decode_step_workspace_bytes(m);
     return al256(cobs::select_workspace_bytes(m, 0)) + cobs::decode_workspace_bytes(m);
 }
 }  // namespace
 
 extern "C" {
 
-int32_t cobs_version(void) { return 101; }
+int32_t cobs_version(void) { return 102; }
 
 int64_t cobs_launch_count(int32_t reset) {
     return reset ? cobs::g_launches.exchange(0) : cobs::g_launches.load();
@@ -177,6 +175,7 @@ size_t cobs_workspace_bytes(const cobs_params* p, int32_t which) {
         case COBS_WS_DECODE: return cobs::decode_workspace_bytes(m);
         case COBS_WS_PREFILL: return cobs::prefill_workspace_bytes(m);
         case COBS_WS_STEP: return step_workspace_bytes(m);
+        case COBS_WS_STEP_FUSED: return cobs::decode_step_workspace_bytes(m);  // 0: shape not taken
     }
     return 0;
 }
@@ -275,34 +274,61 @@ cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const v
     return COBS_OK;
 }
 
-cobs_status cobs_decode_step(const cobs_params* p, const void* Q, const void* K, const void* V, const float* Pk,
-                             const float* Pv, int32_t t_begin, float* summaries, void* Kc, void* Vc, int32_t* idx,
-                             const float* gates, void* O, void* workspace, size_t ws_bytes, cobs_stream_t stream) {
+// Checks shared by the two decode-step entry points.
+static cobs_status step_common(const cobs_params* p, const void* Q, const void* K, const void* V, const float* Pk,
+                               const float* Pv, int32_t t_begin, float* summaries, void* Kc, void* Vc,
+                               int32_t* idx, const float* gates, void* O, void* workspace) {
     COBS_TRY(attn_common(p, Q, K, V, Kc, Vc, idx, gates, O));
     COBS_TRY(check_ptr(Pk, "Pk", true));
     COBS_TRY(check_ptr(Pv, "Pv", true));
     COBS_TRY(check_ptr(summaries, "summaries"));
     if (p->variance == COBS_VAR_SUBSPACE) COBS_TRY(check_ptr(p->basis, "basis"));
     if (t_begin < 0 || t_begin > p->T) return fail(COBS_ERR_INVALID_ARG, "t_begin %d outside [0, T]", t_begin);
+    COBS_TRY(check_ptr(workspace, "workspace"));
+    return COBS_OK;
+}
+
+cobs_status cobs_decode_step(const cobs_params* p, const void* Q, const void* K, const void* V, const float* Pk,
+                             const float* Pv, int32_t t_begin, float* summaries, void* Kc, void* Vc, int32_t* idx,
+                             const float* gates, void* O, void* workspace, size_t ws_bytes, cobs_stream_t stream) {
+    COBS_TRY(step_common(p, Q, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, idx, gates, O, workspace));
     const cobs::Dims m = cobs::make_dims(*p);
     const size_t need = step_workspace_bytes(m);
-    COBS_TRY(check_ptr(workspace, "workspace"));
     if (ws_bytes < need) return fail(COBS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
     int* flag = nullptr;
     COBS_TRY(device_flag(&flag));
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cobs::launch_summaries(m, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, s, flag);
     if (e != cudaSuccess) return cuda_fail(e, "cobs_decode_step: summary update launch");
-    if (cobs::decode_step_supported(m)) {
-        e = cobs::launch_decode_step(m, Q, summaries, K, V, Kc, Vc, idx, gates, O, workspace, s, flag);
-        if (e != cudaSuccess) return cuda_fail(e, "cobs_decode_step launch");
-        return COBS_OK;
-    }
     unsigned char* w = static_cast<unsigned char*>(workspace);
     e = cobs::launch_select(m, Q, summaries, 0, idx, w, s, flag);
     if (e != cudaSuccess) return cuda_fail(e, "cobs_decode_step: selection launch");
-    e = cobs::launch_decode(m, Q, K, V, Kc, Vc, idx, gates, O, w + al256(cobs::select_workspace_bytes(m, 0)), s, flag);
+    // the attention grid follows the selection grids as their programmatic dependent
+    e = cobs::launch_decode(m, Q, K, V, Kc, Vc, idx, gates, O, w + al256(cobs::select_workspace_bytes(m, 0)), s, flag,
+                            true);
     if (e != cudaSuccess) return cuda_fail(e, "cobs_decode_step: attention launch");
+    return COBS_OK;
+}
+
+cobs_status cobs_decode_step_fused(const cobs_params* p, const void* Q, const void* K, const void* V,
+                                   const float* Pk, const float* Pv, int32_t t_begin, float* summaries, void* Kc,
+                                   void* Vc, int32_t* idx, const float* gates, void* O, void* workspace,
+                                   size_t ws_bytes, cobs_stream_t stream) {
+    COBS_TRY(step_common(p, Q, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, idx, gates, O, workspace));
+    const cobs::Dims m = cobs::make_dims(*p);
+    if (!cobs::decode_step_supported(m))
+        return fail(COBS_ERR_UNSUPPORTED,
+                    "cobs_decode_step_fused takes bf16, d in {64, 128}, block 64 and the per-channel or isotropic "
+                    "summaries (with its rings and index tables in shared memory); use cobs_decode_step");
+    const size_t need = cobs::decode_step_workspace_bytes(m);
+    if (ws_bytes < need) return fail(COBS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    int* flag = nullptr;
+    COBS_TRY(device_flag(&flag));
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cobs::launch_summaries(m, K, V, Pk, Pv, t_begin, summaries, Kc, Vc, s, flag);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_decode_step_fused: summary update launch");
+    e = cobs::launch_decode_step(m, Q, summaries, K, V, Kc, Vc, idx, gates, O, workspace, s, flag);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_decode_step_fused launch");
     return COBS_OK;
 }
 

@@ -381,8 +381,9 @@ size_t decode_workspace_bytes(const Dims& m) {
 
 cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                           const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
-                          cudaStream_t s, int* err) {
-    if (m.dtype == COBS_BF16) return launch_decode_stream(m, Q, K, V, Kc, Vc, idx, gates, O, ws, s, err);
+                          cudaStream_t s, int* err, bool after_select) {
+    if (m.dtype == COBS_BF16)
+        return launch_decode_stream(m, Q, K, V, Kc, Vc, idx, gates, O, ws, after_select, s, err);
     AttnArgs a = make_args(m, Q, K, V, Kc, Vc, idx, gates, O, ws, err, 1, kCKf);
     return m.d == 128 ? launch_decode_d<128>(m, a, s) : launch_decode_d<64>(m, a, s);
 }

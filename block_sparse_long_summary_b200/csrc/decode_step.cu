@@ -10,11 +10,11 @@
 // and nothing on a streaming warp's path waits for a global-memory round trip (under a
 // saturated HBM each one costs microseconds):
 //
-// * One CTA per SM: 7 streaming warps and 1 helper warp, two warps per scheduler (so that one's
-//   latencies hide behind the other's work, with up to 255 registers each). Every streaming warp
-//   has a private 3-stage ring of 8 KiB shared-memory tiles filled by bulk / TMA copies (no
-//   multicast). An attention tile is 16 keys of K and V; a summary group (32 blocks) is four
-//   tiles: two halves of its means, two of its variances.
+// * One CTA per SM: 4 streaming warps (one per scheduler) and 1 helper warp. Every streaming
+//   warp has a private 3-stage ring of 16 KiB shared-memory tiles (d = 128) filled by bulk / TMA
+//   copies (no multicast). An attention tile is 32 keys of K and V; a summary group (32 blocks)
+//   is two tiles: its means and its variances. (Each warp's path is latency-bound: larger tiles
+//   cost fewer per-tile steps per byte, which measured faster than more warps with 16-key tiles.)
 // * The work is three phases, each cut into contiguous per-warp ranges (stream-K), and every
 //   streaming warp walks its ranges in phase order:
 //     S  the summary groups of every unit: canonical float32 scores (the four channel chains
@@ -45,18 +45,18 @@ namespace cobs {
 namespace {
 
 #ifndef COBS_STEP_WARPS
-#define COBS_STEP_WARPS 7
+#define COBS_STEP_WARPS 4
 #endif
 #ifndef COBS_STEP_STAGES
 #define COBS_STEP_STAGES 3
 #endif
-constexpr int kStepWarps = COBS_STEP_WARPS;    // streaming warps per CTA (with the helper, two per scheduler)
+constexpr int kStepWarps = COBS_STEP_WARPS;    // streaming warps per CTA (one per scheduler; the helper is the fifth)
 constexpr int kStepStages = COBS_STEP_STAGES;  // ring depth per streaming warp
 constexpr int kStepThreads = (kStepWarps + 1) * 32;
 #ifndef COBS_STEP_TK
-#define COBS_STEP_TK 16
+#define COBS_STEP_TK 32
 #endif
-constexpr int kStepTK = COBS_STEP_TK;    // keys per attention tile (16 or 32)
+constexpr int kStepTK = COBS_STEP_TK;    // keys per attention tile (16 or 32; a ring stage is 16 KiB at d = 128)
 constexpr int kParts = 32 / kStepTK;     // tiles per half of a summary group (means or variances)
 constexpr uint32_t kIdxBits = 25;                      // block index field of a segment word
 constexpr uint32_t kIdxNone = (1u << kIdxBits) - 1u;   // an empty entry
@@ -88,15 +88,33 @@ struct StepArgs {
     int dense[3];        // phase S, A, B: every warp's range is nonempty (else at most one element each)
     int maxseg, maxw;
     int maxbu;           // most phase-B units any CTA holds
+    int mgroups;         // record merge: warp groups per CTA (pairs folded at once)
     float isd, c2, sl2;
     // reciprocals of the divisors of the partition arithmetic (exact quotients: see div_floor)
     double inv_nw, inv_nS, inv_nA, inv_nBt;
+    // the same divisors' 32-bit multipliers floor((2^32 - 1) / n), set when every numerator of the
+    // partition arithmetic is below 2^32 (else 0: the double path)
+    uint32_t mg_nw, mg_nS, mg_nA, mg_nBt;
 };
 
-// floor(x / n) for 0 <= x < 2^50 and 1 <= n < 2^40 without an integer division: the double
-// quotient estimate x * (1/n) is within 1 of the true quotient, and one integer remainder check
-// corrects it. (64-bit integer division is a long dependent instruction sequence on the GPU.)
-__host__ __device__ __forceinline__ long long div_floor(long long x, long long n, double inv) {
+// floor(x / n) for 0 <= x < 2^50 and 1 <= n < 2^40 without an integer division. (Integer division
+// and the 64-bit integer <-> double conversions are long dependent instruction sequences on the
+// GPU, and the partition arithmetic sits on every warp's path.) With a multiplier mg =
+// floor((2^32 - 1) / n) and x < 2^32, the high word of x mg is within 2 below the quotient
+// (x mg / 2^32 > x / n - x / (n 2^32) - x / 2^32 > x / n - 2); two remainder checks correct it.
+// Otherwise the double quotient estimate x * (1/n) is within 1 of the true quotient, and one
+// remainder check corrects it.
+__host__ __device__ __forceinline__ long long div_floor(long long x, long long n, double inv, uint32_t mg) {
+#ifdef __CUDA_ARCH__
+    if (mg != 0u) {
+        const uint32_t xx = (uint32_t)x, nn = (uint32_t)n;
+        uint32_t q = __umulhi(xx, mg);
+        uint32_t r = xx - q * nn;
+        if (r >= nn) { ++q; r -= nn; }
+        if (r >= nn) ++q;
+        return q;
+    }
+#endif
     long long q = (long long)((double)x * inv);
     long long r = x - q * n;
     if (r < 0) { --q; r += n; }
@@ -106,18 +124,19 @@ __host__ __device__ __forceinline__ long long div_floor(long long x, long long n
 
 // Per-warp ranges of the three phases: warp v takes [f(v), f(v + 1)) of each.
 __host__ __device__ __forceinline__ long long fS(const StepArgs& a, long long v) {
-    return div_floor(v * a.nS, a.nwarps, a.inv_nw);
+    return div_floor(v * a.nS, a.nwarps, a.inv_nw, a.mg_nw);
 }
 __host__ __device__ __forceinline__ long long fB(const StepArgs& a, long long v) {
-    return div_floor(v * a.nBt, a.nwarps, a.inv_nw);
+    return div_floor(v * a.nBt, a.nwarps, a.inv_nw, a.mg_nw);
 }
 __host__ __device__ __forceinline__ long long fA(const StepArgs& a, long long v) {
-    if (!a.balanced) return div_floor(v * a.nA, a.nwarps, a.inv_nw);
-    return div_floor(v * a.tot, a.nwarps, a.inv_nw) - a.tpg * fS(a, v) - fB(a, v);
+    if (!a.balanced) return div_floor(v * a.nA, a.nwarps, a.inv_nw, a.mg_nw);
+    return div_floor(v * a.tot, a.nwarps, a.inv_nw, a.mg_nw) - a.tpg * fS(a, v) - fB(a, v);
 }
 // The largest v with floor(v n / N) <= x: v = ceil((x + 1) N / n) - 1 (at most N - 1).
-__host__ __device__ __forceinline__ int floor_part_inverse(long long x, long long n, double inv_n, int N) {
-    const long long v = div_floor((x + 1) * N + n - 1, n, inv_n) - 1;
+__host__ __device__ __forceinline__ int floor_part_inverse(long long x, long long n, double inv_n, uint32_t mg_n,
+                                                           int N) {
+    const long long v = div_floor((x + 1) * N + n - 1, n, inv_n, mg_n) - 1;
     return (int)(v < N - 1 ? v : N - 1);
 }
 // The warp whose range of phase PH holds element x (the largest v with f(v) <= x). The floor
@@ -125,9 +144,9 @@ __host__ __device__ __forceinline__ int floor_part_inverse(long long x, long lon
 // than tpg + 2, so the closed-form inverse of that floor partition is a few steps from the answer.
 template <int PH>
 __host__ __device__ __forceinline__ int warp_of(const StepArgs& a, long long x) {
-    if (PH == 0) return floor_part_inverse(x, a.nS, a.inv_nS, a.nwarps);
-    if (PH == 2) return floor_part_inverse(x, a.nBt, a.inv_nBt, a.nwarps);
-    int v = floor_part_inverse(x, a.nA, a.inv_nA, a.nwarps);
+    if (PH == 0) return floor_part_inverse(x, a.nS, a.inv_nS, a.mg_nS, a.nwarps);
+    if (PH == 2) return floor_part_inverse(x, a.nBt, a.inv_nBt, a.mg_nBt, a.nwarps);
+    int v = floor_part_inverse(x, a.nA, a.inv_nA, a.mg_nA, a.nwarps);
     if (!a.balanced) return v;
     while (v > 0 && fA(a, v) > x) --v;
     while (v < a.nwarps - 1 && fA(a, v + 1) <= x) ++v;
@@ -144,10 +163,12 @@ __host__ __device__ __forceinline__ int run_pieces(const StepArgs& a, long long 
     if (!a.dense[PH]) return (int)len;
     return warp_of<PH>(a, x0 + len - 1) - warp_of<PH>(a, x0) + 1;
 }
-// Slot (0 .. pieces - 1) of the piece of warp v, whose range of the phase starts at r0.
+// Slot (0 .. pieces - 1) of the piece of warp v, whose range of the phase starts at r0. A run that
+// starts inside the range (x0 >= r0) has its first piece there: slot 0, nothing to invert.
 template <int PH>
 __host__ __device__ __forceinline__ int run_slot(const StepArgs& a, int v, long long r0, long long x0) {
-    return a.dense[PH] ? v - warp_of<PH>(a, x0) : (int)((r0 > x0 ? r0 : x0) - x0);
+    if (x0 >= r0) return 0;
+    return a.dense[PH] ? v - warp_of<PH>(a, x0) : (int)(r0 - x0);
 }
 // Run of unit u's branch br (0 selected blocks: phase B; 1 window, 2 compressed tokens: phase A).
 __host__ __device__ __forceinline__ void branch_run(const StepArgs& a, int u, int br, long long* x0, long long* len) {
@@ -336,102 +357,88 @@ __device__ __forceinline__ void att_flush_t(const StepArgs& a, int v, long long 
     }
 }
 
-// Fold the records of (unit, head h) into O, by all NW warps of the CTA (after the grid barrier):
-// NW/2 warps take the selected-block records (every (NW/2)-th), NW/8 (at least one) the window
-// records, the rest the compressed-token records; each folds up to 8 records per round trip into
-// (M, L, acc); warp 0 then combines the warps of each branch, applies the gates (cmp, slc, win) and
-// writes O. wM, wL [NW] and wO [NW][D] are shared-memory scratch.
-template <int D, int NW>
-__device__ void merge_head(const StepArgs& a, int unit, int h, float* wM, float* wL, float* wO) {
-    constexpr int RF = D + 4;
-    constexpr int CPL = D / 32;  // channels per lane
-    constexpr int kBatch = 8;
-    constexpr int kS = NW / 2 > 0 ? NW / 2 : 1, kW = NW / 8 > 0 ? NW / 8 : 1, kC = NW - kS - kW;
-    static_assert(kC >= 1, "at least one warp per branch");
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int br = warp < kS ? 0 : (warp < kS + kW ? 1 : 2);
-    const int sl0 = warp < kS ? warp : (warp < kS + kW ? warp - kS : warp - kS - kW);
-    const int step = warp < kS ? kS : (warp < kS + kW ? kW : kC);
-    const int np = branch_pieces(a, unit, br);
-    const size_t rs = (size_t)a.G * RF;
-    const float* base = a.rec + ((size_t)unit * 3 + br) * a.maxw * rs + (size_t)h * RF;
-    float M = -INFINITY, Lsum = 0.0f, acc[CPL];
+// Record merge (after the grid barrier). The CTA's NW warps form ng groups of NW / ng warps; in
+// round r, group g folds pair p = blockIdx.x + (r ng + g) gridDim.x, p = unit G + head. The
+// records of a pair (its selected-block, window and compressed-token pieces, in that order) are
+// dealt to the group's warps in turn; each warp stages its records in its share of the free rings
+// (16-byte asynchronous copies, as many per round trip as fit), folds them in order (maxima in
+// log2 units) and leaves one (M, L, acc) per branch. The group's first warp then combines its warps per branch,
+// applies the gates (cmp, slc, win) and writes O. The loops are kept rolled: this code runs once
+// per launch, from a cold instruction cache.
+
+// Groups of the record merge: a power of two, at most nw (every group has at least one warp), and
+// no more than the pairs of the busiest CTA need.
+inline int merge_groups(const StepArgs& a, int grid, int nw) {
+    const long long pairs = (long long)a.units * a.G;
+    const long long per = (pairs + grid - 1) / grid;  // pairs of the busiest CTA
+    int ng = 1;
+    while (ng * 2 <= nw && ng < per) ng *= 2;
+    return ng;
+}
+
+// Running (M, L, acc) of one branch; fold one record (m, l, o) into it.
+template <int CPL>
+struct MergeAcc {
+    float M, L, o[CPL];
+    __device__ __forceinline__ void init() {
+        M = -INFINITY;
+        L = 0.0f;
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[c] = 0.0f;
-    for (int sl = sl0; sl < np; sl += kBatch * step) {
-        float m[kBatch], l[kBatch], o[kBatch][CPL];
+        for (int c = 0; c < CPL; ++c) o[c] = 0.0f;
+    }
+    __device__ __forceinline__ void fold(float m, float l, const float (&x)[CPL]) {
+        const float nM = fmaxf(M, m);
+        const float fa = M == -INFINITY ? 0.0f : exp2f(M - nM);
+        const float fb = exp2f(m - nM);
+        L = L * fa + l * fb;
 #pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int s = sl + q * step;
-            m[q] = -INFINITY;
-            l[q] = 0.0f;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) o[q][c] = 0.0f;
-            if (s < np) {
-                const float* r = base + (size_t)s * rs;
-                m[q] = __ldcg(r);
-                l[q] = __ldcg(r + 1);
-                if constexpr (CPL == 4) {
-                    const float4 v4 = __ldcg(reinterpret_cast<const float4*>(r + 4 + lane * 4));
-                    o[q][0] = v4.x; o[q][1] = v4.y; o[q][2] = v4.z; o[q][3] = v4.w;
-                } else {
-                    const float2 v2 = __ldcg(reinterpret_cast<const float2*>(r + 4 + lane * 2));
-                    o[q][0] = v2.x; o[q][1] = v2.y;
-                }
-            }
+        for (int c = 0; c < CPL; ++c) o[c] = o[c] * fa + x[c] * fb;
+        M = nM;
+    }
+    __device__ __forceinline__ void store(float* wM, float* wL, float* wO, int slot, int lane) const {
+        if (lane == 0) {
+            wM[slot] = M;
+            wL[slot] = L;
         }
 #pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            if (m[q] == -INFINITY) continue;
-            const float nM = fmaxf(M, m[q]);
-            const float fa = M == -INFINITY ? 0.0f : exp2f(M - nM);  // maxima are in log2 units
-            const float fb = exp2f(m[q] - nM);
-            Lsum = Lsum * fa + l[q] * fb;
+        for (int c = 0; c < CPL; ++c) wO[(size_t)slot * (CPL * 32) + lane * CPL + c] = o[c];
+    }
+};
+
+// The group's first warp: combine warps w0 .. w0 + gsize - 1 per branch, gate and write O.
+template <int D>
+__device__ void merge_pair_finish(const StepArgs& a, int pair, int w0, int gsize, const float* gate,
+                                  const float* wM, const float* wL, const float* wO) {
+    constexpr int CPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    float out[CPL];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[c] = acc[c] * fa + o[q][c] * fb;
-            M = nM;
+    for (int c = 0; c < CPL; ++c) out[c] = 0.0f;
+#pragma unroll
+    for (int b = 0; b < 3; ++b) {
+        float GM = -INFINITY;
+        for (int w = w0; w < w0 + gsize; ++w) GM = fmaxf(GM, wM[w * 3 + b]);
+        if (GM == -INFINITY) continue;
+        float GL = 0.0f, sum[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) sum[c] = 0.0f;
+        for (int w = w0; w < w0 + gsize; ++w) {
+            const float mw = wM[w * 3 + b];
+            if (mw == -INFINITY) continue;
+            const float f = exp2f(mw - GM);
+            GL += wL[w * 3 + b] * f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) sum[c] += wO[((size_t)w * 3 + b) * D + lane * CPL + c] * f;
         }
+        if (!(GL > 0.0f)) continue;
+        const float gw = gate[b == 0 ? 1 : (b == 1 ? 2 : 0)] / GL;  // gates are stored (cmp, slc, win)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) out[c] += gw * sum[c];
     }
-    if (lane == 0) {
-        wM[warp] = M;
-        wL[warp] = Lsum;
-    }
+    __nv_bfloat16* o = a.O + (size_t)pair * D + lane * CPL;  // pair = unit G + head = query-head row
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) wO[warp * D + lane * CPL + c] = acc[c];
-    __syncthreads();
-    if (warp == 0) {
-        const int hq_row = unit * a.G + h;
-        const float* gate = a.gates + (size_t)hq_row * 3;
-        float out[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) out[c] = 0.0f;
-        // branch b2: selected blocks, window, compressed tokens: consecutive warp ranges
-        for (int b2 = 0; b2 < 3; ++b2) {
-            const int w0 = b2 == 0 ? 0 : (b2 == 1 ? kS : kS + kW), w1 = b2 == 0 ? kS : (b2 == 1 ? kS + kW : NW);
-            float GM = -INFINITY;
-            for (int w = w0; w < w1; ++w) GM = fmaxf(GM, wM[w]);
-            if (GM == -INFINITY) continue;
-            float GL = 0.0f, sum[CPL];
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) sum[c] = 0.0f;
-            for (int w = w0; w < w1; ++w) {
-                if (wM[w] == -INFINITY) continue;
-                const float f = exp2f(wM[w] - GM);
-                GL += wL[w] * f;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) sum[c] += wO[w * D + lane * CPL + c] * f;
-            }
-            if (!(GL > 0.0f)) continue;
-            const float gw = gate[b2 == 0 ? 1 : (b2 == 1 ? 2 : 0)] / GL;
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) out[c] += gw * sum[c];
-        }
-        __nv_bfloat16* o = a.O + (size_t)hq_row * D + lane * CPL;
-#pragma unroll
-        for (int c = 0; c < CPL; c += 2)
-            *reinterpret_cast<__nv_bfloat162*>(o + c) = __floats2bfloat162_rn(out[c], out[c + 1]);
-    }
-    __syncthreads();  // the scratch is free for the next (unit, head)
+    for (int c = 0; c < CPL; c += 2)
+        *reinterpret_cast<__nv_bfloat162*>(o + c) = __floats2bfloat162_rn(out[c], out[c + 1]);
 }
 
 // TR: keys as the mma rows (groups of at most 8 heads), else the heads as the rows.
@@ -446,6 +453,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     constexpr int kStage = 2 * kMat;       // one K + V tile
     static_assert(kStage == step_stage_bytes<D>(), "the launch sizes the rings with the same stage bytes");
     static_assert(kStage * kParts == D * 32 * 4, "an attention tile and a summary part fill one stage");
+    static_assert((size_t)(kStepWarps + 1) * 3 * D * 4 <= (size_t)kStepWarps * kStepStages * kStage,
+                  "the merge scratch fits in the rings");
     constexpr int kPartC = D / kParts;     // channels of a summary part
     constexpr bool kIL = D == 128;         // K / V tiles as one [rows][2][64] box (both column halves)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -455,7 +464,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     __shared__ float q2t_sm[kStepWarps];
     __shared__ Item desc[kStepWarps][kStepStages];
     __shared__ __align__(16) unsigned long long hbuf[kHelperRound * 32];  // helper staging
-    __shared__ float mM[kStepWarps + 1], mL[kStepWarps + 1];              // record merge scratch
+    __shared__ float wM[(kStepWarps + 1) * 3], wL[(kStepWarps + 1) * 3];  // record merge scratch
+    __shared__ float gsm[(kStepWarps + 1) * 3];                           // gates of the first merge round
+    __shared__ int merge_ok;
+    __shared__ int npc[(kStepWarps + 1) * 3];  // pieces of each branch of the first merge round's pairs
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char* base = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -481,6 +493,11 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
             if (lane < a.k && fB(a, (long long)blockIdx.x * kStepWarps) <= (long long)u * a.tS)
                 a.idx[(size_t)u * a.k + lane] = out[lane];
             mbar_arrive(&ubar[u - bu_first]);  // each lane releases the indices it wrote
+        }
+        // while the streaming warps finish: the piece counts of the first merge round's pairs
+        if (lane < a.mgroups * 3) {
+            const long long p = blockIdx.x + (long long)(lane / 3) * gridDim.x;
+            if (p < (long long)a.units * a.G) npc[lane] = branch_pieces(a, (int)(p / a.G), lane % 3);
         }
     } else {
         // ------------------------------------------------------------------ streaming warps
@@ -711,6 +728,10 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
     // ------------------------------------------------------------------ grid barrier, record merge
     // Every CTA is resident (cooperative launch, one per SM). The arrival counter ctl[1] grows by
     // the grid size per step, so this step's barrier is complete at ep x gridDim.x arrivals.
+    constexpr int kNW = kStepWarps + 1;
+    const int ng = min(max(a.mgroups, 1), kNW), gsize = kNW / ng;  // gsize >= 1 (the loops step by it)
+    const int grp = warp / gsize, gw = warp - grp * gsize;  // warps past ng groups (kNW % ng) stay idle
+    const long long pairs = (long long)a.units * a.G;
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();  // this CTA's records and idx are visible before its arrival
@@ -727,15 +748,85 @@ __global__ void __launch_bounds__(kStepThreads, 1) decode_step_kernel(const __gr
         }
         if (late) report_error(a.err, kErrWaitTimeout);
         __threadfence();
-        mM[0] = late ? 1.0f : 0.0f;
+        merge_ok = late ? 0 : 1;
+    } else if (threadIdx.x < 1 + ng * 3) {  // meanwhile: the gates of the first round's pairs
+        const int g = (threadIdx.x - 1) / 3, j = (threadIdx.x - 1) % 3;
+        const long long p = blockIdx.x + (long long)g * gridDim.x;
+        if (p < pairs) gsm[g * 3 + j] = __ldg(a.gates + p * 3 + j);
     }
     __syncthreads();
-    const bool merge_ok = mM[0] == 0.0f;
-    __syncthreads();
     if (merge_ok) {
-        float* wO = reinterpret_cast<float*>(base);  // the rings are free: [kStepWarps + 1][D]
-        for (int p = blockIdx.x; p < a.units * a.G; p += gridDim.x)
-            merge_head<D, kStepWarps + 1>(a, p / a.G, p % a.G, mM, mL, wO);
+        constexpr int CPL = D / 32;
+        constexpr int kRecBytes = (D + 4) * 4;  // one head's record: m, l, 2 pad, o[D]
+        constexpr int kRecChunks = kRecBytes / 16;
+        constexpr size_t kRingBytes = (size_t)kStepWarps * kStepStages * kStage;
+        constexpr size_t kScratch = (size_t)kNW * 3 * D * 4;
+        constexpr int kCap = (int)((kRingBytes - kScratch) / kNW / kRecBytes);  // records per warp per round trip
+        static_assert(kRecBytes % 16 == 0 && kCap >= 1, "records are staged in 16-byte pieces");
+        float* wO = reinterpret_cast<float*>(base + kRingBytes - kScratch);  // [kNW][3][D]
+        unsigned char* mine = base + (size_t)warp * kCap * kRecBytes;      // this warp's staging slots
+        const size_t rs = (size_t)a.G * (D + 4);
+        for (int r = 0;; ++r) {
+            const long long p0 = blockIdx.x + (long long)r * ng * gridDim.x;
+            if (p0 >= pairs) break;  // uniform across the CTA
+            const long long p = p0 + (long long)grp * gridDim.x;
+            const int pair = grp < ng && p < pairs ? (int)p : -1;
+            if (lane == 0)
+                for (int b = 0; b < 3; ++b) wM[warp * 3 + b] = -INFINITY;
+            MergeAcc<CPL> acc;
+            acc.init();
+            int cb = 0;  // branch of acc
+            if (pair >= 0) {
+                const int unit = pair / a.G, h = pair - unit * a.G;
+                const int n0 = r == 0 ? npc[grp * 3] : branch_pieces(a, unit, 0);
+                const int n01 = n0 + (r == 0 ? npc[grp * 3 + 1] : branch_pieces(a, unit, 1));
+                const int nr = n01 + (r == 0 ? npc[grp * 3 + 2] : branch_pieces(a, unit, 2));
+                const float* rbase = a.rec + (size_t)unit * 3 * a.maxw * rs + (size_t)h * (D + 4);
+                // this warp's records: gw, gw + gsize, ...; kCap of them per round trip
+#pragma unroll 1
+                for (int x0 = gw; x0 < nr; x0 += kCap * gsize) {
+                    int nx = 0;
+#pragma unroll 1
+                    for (int x = x0; x < nr && nx < kCap; x += gsize, ++nx) {
+                        const int b = x < n0 ? 0 : (x < n01 ? 1 : 2);
+                        const int sl = x - (b == 0 ? 0 : (b == 1 ? n0 : n01));
+                        const unsigned char* src =
+                            reinterpret_cast<const unsigned char*>(rbase + ((size_t)b * a.maxw + sl) * rs);
+                        for (int j = lane; j < kRecChunks; j += 32)
+                            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                                             smem_addr(mine + (size_t)nx * kRecBytes + j * 16)),
+                                         "l"(src + j * 16)
+                                         : "memory");
+                    }
+                    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+                    __syncwarp();
+#pragma unroll 1
+                    for (int q = 0; q < nx; ++q) {
+                        const int x = x0 + q * gsize;
+                        const int b = x < n0 ? 0 : (x < n01 ? 1 : 2);
+                        if (b != cb) {
+                            acc.store(wM, wL, wO, warp * 3 + cb, lane);
+                            acc.init();
+                            cb = b;
+                        }
+                        const float* rp = reinterpret_cast<const float*>(mine + (size_t)q * kRecBytes);
+                        const float m = rp[0];
+                        if (m == -INFINITY) continue;
+                        float o[CPL];
+#pragma unroll
+                        for (int c = 0; c < CPL; ++c) o[c] = rp[4 + lane * CPL + c];
+                        acc.fold(m, rp[1], o);
+                    }
+                    __syncwarp();  // the slots are read before the next copies
+                }
+            }
+            acc.store(wM, wL, wO, warp * 3 + cb, lane);
+            __syncthreads();
+            if (gw == 0 && pair >= 0)
+                merge_pair_finish<D>(a, pair, warp, gsize, r == 0 ? gsm + grp * 3 : a.gates + (size_t)pair * 3, wM,
+                                     wL, wO);
+            __syncthreads();
+        }
     }
     // the epoch advances once every CTA has passed the barrier (all read it at their start)
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&a.ctl[0], 1u);
@@ -782,6 +873,14 @@ StepArgs make_step_args(const Dims& m) {
     a.inv_nS = a.nS > 0 ? 1.0 / (double)a.nS : 0.0;
     a.inv_nA = a.nA > 0 ? 1.0 / (double)a.nA : 0.0;
     a.inv_nBt = a.nBt > 0 ? 1.0 / (double)a.nBt : 0.0;
+    // 32-bit division multipliers when every numerator fits: v n <= nwarps tot and
+    // (x + 1) nwarps + n - 1 <= (nwarps + 1) tot
+    const bool narrow = (unsigned long long)(a.nwarps + 1) * (unsigned long long)(a.tot + 1) < (1ull << 32);
+    auto mg = [&](long long n) { return narrow && n > 0 ? (uint32_t)(0xFFFFFFFFull / (unsigned long long)n) : 0u; };
+    a.mg_nw = mg(a.nwarps);
+    a.mg_nS = mg(a.nS);
+    a.mg_nA = mg(a.nA);
+    a.mg_nBt = mg(a.nBt);
     // balanced phase-A ranges when every warp's is nonempty (strictly increasing starts)
     a.balanced = 1;
     for (long long v = 0; v < a.nwarps; ++v)
@@ -796,6 +895,7 @@ StepArgs make_step_args(const Dims& m) {
         if (a.nGc > 0) a.maxseg = std::max(a.maxseg, sel_segments(a, u));
         for (int br = 0; br < 3; ++br) a.maxw = std::max(a.maxw, branch_pieces(a, u, br));
     }
+    a.mgroups = merge_groups(a, a.nwarps / kStepWarps, kStepWarps + 1);
     a.maxbu = 1;
     for (int c = 0; c < a.nwarps / kStepWarps; ++c) {
         int f, l;

@@ -5,10 +5,14 @@
 // the window and the compressed tokens are read ("Problemstellung": decode is bound by the
 // KV-cache read). How it is scheduled:
 //
-// * Every (batch, KV-head) unit contributes its tiles in the order SLC (2 tiles per
-//   selected block), WIN (the window rows in 32-row tiles), CMP (compressed tokens in
-//   32-row tiles). The tiles of all units form one sequence that is cut into equal,
-//   contiguous ranges, one per warp, so every SM streams the same number of bytes.
+// * Every (batch, KV-head) unit contributes its tiles in the order WIN (the window rows in
+//   32-row tiles), CMP (compressed tokens in 32-row tiles), SLC (2 tiles per selected
+//   block). The tiles of all units form one sequence that is cut into equal, contiguous
+//   ranges, one per warp, so every SM streams the same number of bytes.
+// * After a selection in the same stream (the decode step) the grid is launched as a
+//   programmatic dependent of the selection: the window and compressed-token tiles, which
+//   do not depend on it, stream while it finishes; a warp waits for the selection grid
+//   (griddepcontrol.wait) before it reads its first selected-block index.
 // * Each warp is its own producer: TMA 2-D loads (128-byte swizzle, no multicast) of the
 //   K and V halves of a tile into a private 3-stage ring, an mbarrier per stage.
 // * The G query heads of the unit are the m16 rows of mma.sync tiles (rows >= G are zero);
@@ -52,8 +56,9 @@ struct StreamArgs {
 
 __host__ __device__ __forceinline__ int rec_floats(int D) { return D + 4; }  // m, l, pad, pad, o[D]
 
+// Branch br's tiles within a unit: WIN [0, tW), CMP [tW, tW + tC), SLC [tW + tC, tpu).
 __host__ __device__ __forceinline__ int branch_begin(const StreamArgs& a, int br) {
-    return br == 0 ? 0 : (br == 1 ? a.tS : a.tS + a.tW);
+    return br == 1 ? 0 : (br == 2 ? a.tW : a.tW + a.tC);
 }
 __host__ __device__ __forceinline__ int branch_len(const StreamArgs& a, int br) {
     return br == 0 ? a.tS : (br == 1 ? a.tW : a.tC);
@@ -65,13 +70,19 @@ struct Tile {
     uint32_t mask;     // valid keys of the tile
 };
 
-// Tile gt of the global sequence. Uniform across the warp.
-__device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt) {
+// Tile gt of the global sequence. Uniform across the warp. Before the first selected-block
+// index it reads, the warp waits for the grid it depends on (the selection), once.
+__device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt, bool& waited) {
     Tile tl;
     tl.unit = (int)(gt / a.tpu);
     int l = (int)(gt - (long long)tl.unit * a.tpu);
     const int t = a.T - 1;
-    if (l < a.tS) {
+    if (l >= a.tW + a.tC) {
+        if (!waited) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            waited = true;
+        }
+        l -= a.tW + a.tC;
         tl.br = 0;
         tl.j = l;
         const int bi = a.idx[(size_t)tl.unit * a.k + l / (64 / kTK)];
@@ -85,16 +96,16 @@ __device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt) {
                 tl.mask = kTK == 32 ? kFull : 0xFFFFu;
             }
         }
-    } else if (l < a.tS + a.tW) {
+    } else if (l < a.tW) {
         tl.br = 1;
-        tl.j = l - a.tS;
+        tl.j = l;
         const int r0 = max(0, t - a.W + 1) + tl.j * kTK;
         tl.row = tl.unit * a.T + r0;
         const int n = min(kTK, t + 1 - r0);
         tl.mask = n >= 32 ? kFull : ((1u << n) - 1u);  // n <= kTK
     } else {
         tl.br = 2;
-        tl.j = l - a.tS - a.tW;
+        tl.j = l - a.tW;
         const int c0 = tl.j * kTK;
         tl.row = tl.unit * a.nC + c0;
         const int n = min(kTK, a.nC - c0);
@@ -180,8 +191,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
     // descriptors of the next kStages tiles, in registers: a selected block's index is read
     // when its tile is prefetched, not when it is consumed
     Tile tq[kStages];
+    bool waited = false;
 #pragma unroll
-    for (int j = 0; j < kStages; ++j) tq[j] = j < n ? tile_at(a, g0 + j) : Tile{0, 0, 0, 0, 0u};
+    for (int j = 0; j < kStages; ++j) tq[j] = j < n ? tile_at(a, g0 + j, waited) : Tile{0, 0, 0, 0, 0u};
     if (lane == 0) {
 #pragma unroll
         for (int j = 0; j < kStages; ++j)
@@ -201,7 +213,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
 #pragma unroll
         for (int j = 0; j + 1 < kStages; ++j) tq[j] = tq[j + 1];
         const bool more = i + kStages < n;
-        tq[kStages - 1] = more ? tile_at(a, g0 + i + kStages) : Tile{0, 0, 0, 0, 0u};
+        tq[kStages - 1] = more ? tile_at(a, g0 + i + kStages, waited) : Tile{0, 0, 0, 0, 0u};
         if (tl.unit != cur.unit || tl.br != cur.br) {
             flush<D>(a, v, cur.unit, cur.br, st, lane);
             st.init();
@@ -324,7 +336,7 @@ size_t stream_smem() { return (size_t)kWarps * kStages * 2 * (D / 64) * kTK * 12
 
 template <int D>
 cudaError_t launch_stream_d(const Dims& m, StreamArgs a, const void* K, const void* V, const void* Kc, const void* Vc,
-                            cudaStream_t s) {
+                            bool after_select, cudaStream_t s) {
     CUtensorMap tk, tv, tkc, tvc;
     const uint64_t kvrows = (uint64_t)m.units() * m.T;
     const uint64_t crows = m.nC > 0 ? (uint64_t)m.units() * m.nC : kvrows;
@@ -337,9 +349,21 @@ cudaError_t launch_stream_d(const Dims& m, StreamArgs a, const void* K, const vo
     if (e != cudaSuccess) return e;
     const long long nwarps = (a.total + a.tpw - 1) / a.tpw;
     const int grid = (int)((nwarps + kWarps - 1) / kWarps);
-    count_launch();
-    decode_stream_kernel<D><<<grid, kWarps * 32, smem, s>>>(tk, tv, tkc, tvc, a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kWarps * 32);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = after_select ? 1 : 0;  // else: after whatever precedes it, in stream order
+        count_launch();
+        e = cudaLaunchKernelEx(&cfg, decode_stream_kernel<D>, tk, tv, tkc, tvc, a);
+        if (e != cudaSuccess) return e;
+    }
     // the merge grid may launch while the decode grid drains; it waits for it on the device
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(m.G, m.units());
@@ -364,7 +388,7 @@ size_t decode_stream_workspace_bytes(const Dims& m) {
 
 cudaError_t launch_decode_stream(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                                  const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
-                                 cudaStream_t s, int* err) {
+                                 bool after_select, cudaStream_t s, int* err) {
     StreamArgs a = make_stream_args(m);
     a.Q = static_cast<const __nv_bfloat16*>(Q);
     a.idx = idx;
@@ -372,7 +396,8 @@ cudaError_t launch_decode_stream(const Dims& m, const void* Q, const void* K, co
     a.O = static_cast<__nv_bfloat16*>(O);
     a.rec = static_cast<float*>(ws);
     a.err = err;
-    return m.d == 128 ? launch_stream_d<128>(m, a, K, V, Kc, Vc, s) : launch_stream_d<64>(m, a, K, V, Kc, Vc, s);
+    return m.d == 128 ? launch_stream_d<128>(m, a, K, V, Kc, Vc, after_select, s)
+                      : launch_stream_d<64>(m, a, K, V, Kc, Vc, after_select, s);
 }
 
 }  // namespace cobs

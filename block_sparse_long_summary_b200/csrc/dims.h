@@ -69,12 +69,14 @@ cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int p
 
 size_t decode_workspace_bytes(const Dims& m);
 size_t decode_stream_workspace_bytes(const Dims& m);
+// after_select: launched as a programmatic dependent of the selection grids just before it in the
+// stream (the decode step); it then reads K, V, Kc and Vc before they complete and idx after.
 cudaError_t launch_decode_stream(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                                  const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
-                                 cudaStream_t s, int* err);
+                                 bool after_select, cudaStream_t s, int* err);
 cudaError_t launch_decode(const Dims& m, const void* Q, const void* K, const void* V, const void* Kc,
                           const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
-                          cudaStream_t s, int* err);
+                          cudaStream_t s, int* err, bool after_select = false);
 
 // Decode with the library's fixed device scratch in place of a workspace (no allocation).
 size_t noalloc_scratch_bytes();

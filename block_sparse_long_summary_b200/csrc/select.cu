@@ -449,6 +449,9 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
 __global__ void __launch_bounds__(256) select_merge_kernel(const float* __restrict__ ws_s,
                                                            const int* __restrict__ ws_i, int32_t* __restrict__ idx,
                                                            int nGc, long long n, int grid, int k, int maxseg) {
+    // a dependent grid (the decode step's attention) may be scheduled now; it waits for this grid
+    // to complete before it reads idx
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ float ls[kSelMaxSeg][32];
     __shared__ int li[kSelMaxSeg][32];

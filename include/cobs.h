@@ -83,7 +83,8 @@ typedef enum {
     COBS_WS_SELECT = 0,
     COBS_WS_DECODE = 1,
     COBS_WS_PREFILL = 2,
-    COBS_WS_STEP = 3 /* cobs_decode_step */
+    COBS_WS_STEP = 3,      /* cobs_decode_step */
+    COBS_WS_STEP_FUSED = 4 /* cobs_decode_step_fused (0 bytes: a shape it does not take) */
 } cobs_workspace_kind;
 
 /* Second-order statistic kept per block ([COBS] §2.2/§2.3: the block covariance Sigma_b, compressed):
@@ -204,23 +205,40 @@ cobs_status cobs_sparse_attn_decode(const cobs_params* p, const void* Q, const v
  * second-order selection; [NSA-181] the three paths and their gates). idx and O are written as
  * the separate calls write them (the same indices bit for bit, the same attention up to float32
  * summation order).
- * For bf16 with d in {64, 128} and the COBS_VAR_CHANNEL or COBS_VAR_ISOTROPIC summaries the
- * selection and the attention run as one persistent kernel (one CTA per SM): the summaries, the
- * window and compressed tokens and the selected blocks are read back to back, and a unit's
- * selected blocks are read as soon as its selection is complete. Other shapes run the separate
- * kernels.
- *   workspace: >= cobs_workspace_bytes(p, COBS_WS_STEP) bytes (sized for the current device's
- *              SM count), ZERO-FILLED before its first use and again before it is used with
- *              other params or after a call that set the device error flag; a completed call
- *              leaves it ready for the next one. Calls that share one workspace must not run
- *              concurrently.
- * Errors: those of the three calls. A wait on another CTA's result is bounded: if it gives up
- * (kernel resources held by other work for more than about 0.1 s), the device error flag is set.
+ * The attention grid is launched as a programmatic dependent of the selection grids: its window
+ * and compressed-token tiles, which do not depend on idx, stream while the selection finishes,
+ * and it reads idx only after the selection grids have completed.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_STEP) bytes; no initial contents are needed.
+ *              Calls that share one workspace must not run concurrently.
+ * Errors: those of the three calls.
  */
 cobs_status cobs_decode_step(const cobs_params* p, const void* Q, const void* K, const void* V,
                              const float* Pk, const float* Pv, int32_t t_begin, float* summaries,
                              void* Kc, void* Vc, int32_t* idx, const float* gates, void* O,
                              void* workspace, size_t ws_bytes, cobs_stream_t stream);
+
+/*
+ * The same decode step with the selection and the attention in one persistent kernel (one CTA per
+ * SM, cooperative launch): the summaries, the window and compressed tokens and the selected blocks
+ * are read back to back, and a unit's selected blocks are read as soon as its selection is
+ * complete; after a grid barrier every CTA folds a share of the split-K partial results. Results
+ * are those of cobs_decode_step. It is an alternative schedule of the same work: on the seeded
+ * decode workloads it measures slower than cobs_decode_step.
+ * Takes bf16, d in {64, 128}, block 64 and the COBS_VAR_CHANNEL or COBS_VAR_ISOTROPIC summaries
+ * (when its per-CTA tables fit in shared memory); other shapes return COBS_ERR_UNSUPPORTED.
+ *   workspace: >= cobs_workspace_bytes(p, COBS_WS_STEP_FUSED) bytes (sized for the current
+ *              device's SM count), ZERO-FILLED before its first use and again before it is used
+ *              with other params or after a call that set the device error flag; a completed call
+ *              leaves it ready for the next one. Calls that share one workspace must not run
+ *              concurrently.
+ * Errors: those of cobs_decode_step. A wait on another CTA's result is bounded: if it gives up
+ * (kernel resources held by other work for more than about 0.1 s), the device error flag is set.
+ */
+cobs_status cobs_decode_step_fused(const cobs_params* p, const void* Q, const void* K,
+                                   const void* V, const float* Pk, const float* Pv,
+                                   int32_t t_begin, float* summaries, void* Kc, void* Vc,
+                                   int32_t* idx, const float* gates, void* O, void* workspace,
+                                   size_t ws_bytes, cobs_stream_t stream);
 
 /*
  * Decode attention without a workspace. The paper has no counterpart to this call: it exists

@@ -23,7 +23,7 @@ int main(void) {
     p.alpha = 1.0f; p.dtype = COBS_BF16; p.variance = COBS_VAR_CHANNEL; p.rank = 0;
     p.sub = 0; p.basis = NULL;
 
-    CHECK(cobs_version() == 101);
+    CHECK(cobs_version() == 102);
     CHECK(strcmp(cobs_status_string(COBS_OK), "ok") == 0);
     /* 64 units x 16 groups of 32 blocks x (means + variances) */
     CHECK(cobs_summaries_elems(&p) == (size_t)64 * 16 * 2 * 128 * 32);

@@ -93,14 +93,15 @@ def summaries_blocks(flat, p):
     return a.reshape(p.B, p.Hkv, nG * 32, 2, p.d)[:, :, :nB]
 
 
-def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel", rank=4, basis=None, fused=True):
-    """The decode step through cobs_decode_step (fused=True) or the three separate calls."""
+def run_decode(w, K, V, Q, gates, Pk, Pv, variance="channel", rank=4, basis=None, path="step"):
+    """The decode step through cobs_decode_step (path "step"), cobs_decode_step_fused ("fused") or
+    the three separate calls ("calls")."""
     C = cobs()
     p = params_of(w, variance, rank, basis)
     buf = C.alloc(p, prefill=False)
     C.device_error(reset=True)
     C.decode_step(p, dev(Q, w.dtype), dev(K, w.dtype), dev(V, w.dtype), dev(Pk, "f32"), dev(Pv, "f32"),
-                  torch.from_numpy(gates).cuda(), buf, t_begin=0, fused=fused)
+                  torch.from_numpy(gates).cuda(), buf, t_begin=0, path=path)
     torch.cuda.synchronize()
     return p, buf
 

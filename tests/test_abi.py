@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.version() == 101
+    assert lib.version() == 102
     assert lib._lib.cobs_status_string(0) == b"ok"
     assert lib._lib.cobs_status_string(-1) == b"invalid argument"
 

@@ -63,11 +63,11 @@ def test_tiny_fp32_decode():
     ("tiny", dict(T=1000 + 23, Hq=3, Hkv=1, d=128)),               # float32, ragged, d = 128
     ("tiny", dict(T=5000, Hq=8, Hkv=2, topk=7, window=300)),        # float32, odd k
 ])
-@pytest.mark.parametrize("fused", [True, False], ids=["step", "calls"])
-def test_decode_shapes(name, over, fused):
+@pytest.mark.parametrize("path", ["step", "calls"])
+def test_decode_shapes(name, over, path):
     w = synth.WORKLOADS[name].replace(**over)
     K, V, Q, g, Pk, Pv = inputs_decode(w)
-    p, buf = run_decode(w, K, V, Q, g, Pk, Pv, fused=fused)
+    p, buf = run_decode(w, K, V, Q, g, Pk, Pv, path=path)
     assert cobs().device_error() == 0
     units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     _check_units(w, K, V, Q, g, Pk, Pv, p, buf, units)
