@@ -318,25 +318,30 @@ float cobs_oracle_bf16_rn(float x) {
     return v.f;
 }
 
+/* The E2M1 form of n vectors of len numbers each (the rule above, one scale per vector):
+ * x [n][len] -> codes [n][len] (0..15), scales [n], xq [n][len] (the dequantized values). */
+void cobs_oracle_fp4_vectors(const float* x, int64_t n, int len, uint8_t* codes, float* scales, float* xq) {
+    for (int64_t r = 0; r < n; ++r) {
+        const float* v = x + r * len;
+        float a = 0.0f;
+        for (int c = 0; c < len; ++c) a = fmaxf(a, fabsf(v[c]));
+        const float s = a / 6.0f;
+        scales[r] = s;
+        for (int c = 0; c < len; ++c) {
+            const int code = s > 0.0f ? cobs_oracle_e2m1_code(v[c] / s) : 0;
+            codes[r * len + c] = (uint8_t)code;
+            const float m = (code & 8) ? -kE2M1[code & 7] : kE2M1[code & 7];
+            xq[r * len + c] = m * s;
+        }
+    }
+}
+
 /* mu: [nb][d] -> mu_q [nb][d]; u: [nb][R][d] -> codes [nb][R][d] (0..15), scales [nb][R], u_q [nb][R][d]. */
 void cobs_oracle_lowrank_fp4_f32(const float* mu, const float* u, int64_t nb, int d, int R, float* mu_q,
                                  uint8_t* codes, float* scales, float* u_q) {
-    for (int64_t b = 0; b < nb; ++b) {
+    for (int64_t b = 0; b < nb; ++b)
         for (int c = 0; c < d; ++c) mu_q[b * d + c] = cobs_oracle_bf16_rn(mu[b * d + c]);
-        for (int j = 0; j < R; ++j) {
-            const float* x = u + (b * R + j) * (int64_t)d;
-            float a = 0.0f;
-            for (int c = 0; c < d; ++c) a = fmaxf(a, fabsf(x[c]));
-            const float s = a / 6.0f;
-            scales[b * R + j] = s;
-            for (int c = 0; c < d; ++c) {
-                const int code = s > 0.0f ? cobs_oracle_e2m1_code(x[c] / s) : 0;
-                codes[(b * R + j) * (int64_t)d + c] = (uint8_t)code;
-                const float m = (code & 8) ? -kE2M1[code & 7] : kE2M1[code & 7];
-                u_q[(b * R + j) * (int64_t)d + c] = m * s;
-            }
-        }
-    }
+    cobs_oracle_fp4_vectors(u, nb * R, d, codes, scales, u_q);
 }
 
 /*
@@ -353,6 +358,21 @@ void cobs_oracle_lowrank_fp4_f32(const float* mu, const float* u, int64_t nb, in
 void cobs_oracle_subspace_project(const float* P, const float* x, int64_t n, int d, int s, float* out) {
     for (int64_t r = 0; r < n; ++r)
         for (int i = 0; i < s; ++i) out[r * s + i] = dot4s(P + i, x + r * d, d, s, 1);
+}
+
+/*
+ * Query subspace with FP4 coordinates and a BF16 mean (COBS §2.3 applies the three compressions
+ * together; §4.1 reports this form as "Subspace, r=4, FP4"): the subspace summaries above, then
+ *   mean: mu'_c = RN_bf16(mu_c);  projected vector j: the E2M1 rule above over its s coordinates
+ *   (a = max_i |u~_{j,i}|, scale a / 6), u~'_{j,i} = (+-m) * scale;  lambda_j stays float32.
+ * The score is the subspace score of (mu', u~', lambda).
+ * mu: [nb][d] -> mu_q; ut: [nb][R][s] -> codes [nb][R][s], scales [nb][R], ut_q [nb][R][s].
+ */
+void cobs_oracle_subspace_fp4_f32(const float* mu, const float* ut, int64_t nb, int d, int s, int R, float* mu_q,
+                                  uint8_t* codes, float* scales, float* ut_q) {
+    for (int64_t b = 0; b < nb; ++b)
+        for (int c = 0; c < d; ++c) mu_q[b * d + c] = cobs_oracle_bf16_rn(mu[b * d + c]);
+    cobs_oracle_fp4_vectors(ut, nb * R, s, codes, scales, ut_q);
 }
 
 /* q: [G][d]; qsum: [d]; mu: [nb][d]; ut: [nb][R][s]; lam: [nb][R]; P: [d][s]; S: [nb] */

@@ -22,7 +22,8 @@ order (compressed, selected, window). For the compressed covariance forms of [CO
 the low-rank eigenpairs come from a fixed float32 subspace iteration (pinned against
 numpy's eigh); FP4 keeps one float32 scale max|u|/6 per eigenvector; the query-subspace
 basis is given by the caller, and both the eigenvectors and the query heads are projected
-on it.
+on it; the three together (the form §4.1 reports) quantize the projected coordinates with
+the same FP4 rule and keep the mean in bf16.
 
 Nothing here is blocked, fused or reordered: each function follows the definition it
 cites, with numpy's matmul, sum and sort as the only library steps.
@@ -87,6 +88,10 @@ def _c():
         lib.cobs_oracle_subspace_project.restype = None
         lib.cobs_oracle_subspace_scores.argtypes = [vp, vp, i32, vp, vp, vp, i64, i32, i32, i32, vp, f32, f32, vp]
         lib.cobs_oracle_subspace_scores.restype = None
+        lib.cobs_oracle_fp4_vectors.argtypes = [vp, i64, i32, vp, vp, vp]
+        lib.cobs_oracle_fp4_vectors.restype = None
+        lib.cobs_oracle_subspace_fp4_f32.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp, vp, vp]
+        lib.cobs_oracle_subspace_fp4_f32.restype = None
         _clib = lib
     return _clib
 
@@ -262,6 +267,46 @@ def canonical_summaries_subspace(K32: np.ndarray, L: int, R: int, P: np.ndarray)
     return Subspace((mu, ut, lam, P))
 
 
+def fp4_vectors(x: np.ndarray):
+    """E2M1 form of the rows of x [n, len] (one scale per row, canonical_fp32.c): (codes uint8,
+    scales float32 [n], dequantized float32 [n, len])."""
+    x = _f32c(x)
+    n, ln = x.shape
+    codes = np.zeros((n, ln), np.uint8)
+    scales = np.zeros(n, np.float32)
+    xq = np.zeros((n, ln), np.float32)
+    if n:
+        _c().cobs_oracle_fp4_vectors(x.ctypes.data, n, ln, codes.ctypes.data, scales.ctypes.data, xq.ctypes.data)
+    return codes, scales, xq
+
+
+class SubspaceFP4(tuple):
+    """Query-subspace summaries with FP4 coordinates: (mu_q [nB, d] bf16 values as float32, codes
+    [nB, R, s] uint8, scales [nB, R] float32, lam [nB, R] float32, ut_q [nB, R, s] the dequantized
+    coordinates, P [d, s])."""
+
+    def dequantized(self) -> Subspace:
+        mu_q, _, _, lam, ut_q, P = self
+        return Subspace((mu_q, ut_q, lam, P))
+
+
+def canonical_summaries_subspace_fp4(K32: np.ndarray, L: int, R: int, P: np.ndarray) -> SubspaceFP4:
+    """The query-subspace summaries with the mean rounded to bf16 and each projected eigenvector's
+    s coordinates stored in E2M1 with one float32 scale (max |u~| / 6): the three compressions of
+    [COBS] §2.3 together, the form [COBS] §4.1 reports as "Subspace, r=4, FP4"."""
+    mu, ut, lam, P = canonical_summaries_subspace(K32, L, R, P)
+    nB, d = mu.shape
+    sdim = ut.shape[2]
+    mu_q = np.zeros_like(mu)
+    codes = np.zeros((nB, R, sdim), np.uint8)
+    scales = np.zeros((nB, R), np.float32)
+    ut_q = np.zeros_like(ut)
+    if nB:
+        _c().cobs_oracle_subspace_fp4_f32(mu.ctypes.data, np.ascontiguousarray(ut).ctypes.data, nB, d, sdim, R,
+                                          mu_q.ctypes.data, codes.ctypes.data, scales.ctypes.data, ut_q.ctypes.data)
+    return SubspaceFP4((mu_q, codes, scales, lam, ut_q, P))
+
+
 def canonical_scores_subspace(q_group32: np.ndarray, summ: Subspace, alpha: float) -> np.ndarray:
     """float32 group scores [nB] with query-subspace summaries (canonical_fp32.c)."""
     mu, ut, lam, P = summ
@@ -407,12 +452,17 @@ def head_scores_lowrank(q: np.ndarray, mu: np.ndarray, u: np.ndarray, lam: np.nd
 
 def group_scores_subspace(qs: np.ndarray, mu, u, lam, P, alpha: float) -> np.ndarray:
     """Query-subspace per-group score: sum_h [q_h.mu/sqrt(d) + alpha/2 sum_j lam_j ((P^T q_h).(P^T u_j))^2 / d]."""
+    return group_scores_subspace_coords(qs, mu, u @ P, lam, P, alpha)
+
+
+def group_scores_subspace_coords(qs: np.ndarray, mu, ut, lam, P, alpha: float) -> np.ndarray:
+    """The same score from the eigenvectors' subspace coordinates ut [nB, R, s] as stored (for
+    the FP4 form: the dequantized coordinates and the bf16 mean), float64."""
     d = qs.shape[-1]
-    up = u @ P                      # [nB, R, s]
     out = 0.0
     for q in qs:
         qp = P.T @ q
-        out = out + (mu @ q) / np.sqrt(d) + alpha * 0.5 * ((up @ qp) ** 2 * lam).sum(axis=-1) / d
+        out = out + (mu @ q) / np.sqrt(d) + alpha * 0.5 * ((ut @ qp) ** 2 * lam).sum(axis=-1) / d
     return out
 
 
@@ -550,6 +600,8 @@ def select_decode(w, q_group32: np.ndarray, summ: np.ndarray):
 
     summ: canonical summaries [nB, 2, d] (per-channel variance), [nB, d + 1] (isotropic) or a
     LowRank triple (mean, eigenvectors, eigenvalues)."""
+    if isinstance(summ, SubspaceFP4):
+        summ = summ.dequantized()
     if isinstance(summ, Subspace):
         S = canonical_scores_subspace(q_group32, summ, w.alpha)
         return top_k(S, n_candidates(w.T - 1, w.block), w.topk), S
@@ -571,7 +623,8 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
 
     variance: "channel" (per-channel variance summaries), "isotropic" (one scalar per block),
     "lowrank" / "lowrank_fp4" (the rank leading eigenpairs of each block's covariance) or
-    "subspace" (those eigenpairs with the eigenvectors as coordinates in basis [d, s]).
+    "subspace" (those eigenpairs with the eigenvectors as coordinates in basis [d, s]) or
+    "subspace_fp4" (those coordinates in E2M1 with one scale per vector, the mean in bf16).
 
     Returns dict with idx [B, Hkv, k], O [B, Hq, d] (float64; rows of unlisted units are NaN),
     summ, Kc, Vc per computed unit, and near-tie reports (b, h, relative gap) for the units where
@@ -596,6 +649,8 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
             sel_summ = canonical_summaries_lowrank_fp4(K.astype(np.float32), w.block, rank)
         elif variance == "subspace":
             sel_summ = canonical_summaries_subspace(K.astype(np.float32), w.block, rank, basis)
+        elif variance == "subspace_fp4":
+            sel_summ = canonical_summaries_subspace_fp4(K.astype(np.float32), w.block, rank, basis)
         else:
             sel_summ = summ
         sel, _ = select_decode(w, qs.astype(np.float32), sel_summ)
@@ -608,6 +663,10 @@ def decode(w, K_all, V_all, Q, gates, Pk, Pv, units=None, variance="channel", ra
         elif variance == "subspace":
             S64 = group_scores_subspace(qs, *block_eigenpairs(K, w.block, rank), np.asarray(basis, np.float64),
                                         w.alpha)
+        elif variance == "subspace_fp4":  # the float64 score of the stored (quantized) form
+            mu_q, _, _, lam_q, ut_q, _ = sel_summ
+            S64 = group_scores_subspace_coords(qs, mu_q.astype(np.float64), ut_q.astype(np.float64),
+                                               lam_q.astype(np.float64), np.asarray(basis, np.float64), w.alpha)
         else:
             S64 = group_scores(qs, mu, var, w.alpha)
         gap = near_tie_gap(S64, sel, n_candidates(t, w.block), w.topk)

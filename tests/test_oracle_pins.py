@@ -843,3 +843,91 @@ def test_subspace_decode_with_identity_basis_is_low_rank_decode():
     b = O.decode(w, K, V, Q, g, Pk, Pv, variance="subspace", rank=4, basis=np.eye(w.d, dtype=np.float32))
     assert np.array_equal(a["idx"], b["idx"])
     assert np.array_equal(a["O"], b["O"])
+
+
+# ---------------------------------------------------------------- query subspace with FP4 coordinates
+
+def test_subspace_fp4_with_the_identity_basis_is_the_fp4_low_rank_form():
+    """P = I (s = d): the projected coordinates are the eigenvectors exactly, so every stored field
+    (bf16 mean, codes, scales, eigenvalues, dequantized vectors) and every score equal the FP4
+    low-rank form's, bit for bit."""
+    rng = np.random.default_rng(61)
+    L, d, R, nB, G = 64, 32, 3, 12, 4
+    K = _aniso_blocks(rng, nB, L, d, [2.0, 1.2, 0.7, 0.4], 0.05).astype(np.float32)
+    I = np.eye(d, dtype=np.float32)
+    sub = O.canonical_summaries_subspace_fp4(K, L, R, I)
+    lr = O.canonical_summaries_lowrank_fp4(K, L, R)
+    for x, y in zip(sub[:5], lr):
+        assert np.array_equal(x, y)
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    assert np.array_equal(O.canonical_scores_subspace(q, sub.dequantized(), 1.0),
+                          O.canonical_scores_lowrank(q, lr.dequantized(), 1.0))
+
+
+def test_fp4_vectors_are_exact_on_the_e2m1_grid():
+    """Rows whose entries are E2M1 magnitudes times a power of two whose largest magnitude is 6:
+    the scale is that power of two exactly and every entry round-trips exactly, with the code of
+    its magnitude index and sign (worked by hand from the E2M1 table 0, .5, 1, 1.5, 2, 3, 4, 6)."""
+    x = np.array([[6.0, -3.0, 0.5, 0.0, 1.5, -6.0, 4.0, -0.5],
+                  [0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0]], np.float32)
+    x[0] *= 0.125
+    codes, scales, xq = O.fp4_vectors(x)
+    assert scales.tolist() == [0.125, 0.0]
+    assert codes[0].tolist() == [7, 8 | 5, 1, 0, 3, 8 | 7, 6, 8 | 1]
+    assert codes[1].tolist() == [0] * 8
+    assert np.array_equal(xq, x)
+
+
+def test_subspace_fp4_coordinates_within_the_e2m1_grid_bound():
+    """The dequantized subspace coordinates differ from the float32 ones by at most half the E2M1
+    gap at their magnitude (0.25, 0.5 or 1 times the scale); the scale is max |u~| / 6; the mean is
+    the bf16 rounding of the float32 mean (8 significant bits: relative error at most half an ulp,
+    2^-8); eigenvalues unchanged."""
+    rng = np.random.default_rng(62)
+    L, d, R, nB, s = 64, 128, 4, 8, 84
+    K = _aniso_blocks(rng, nB, L, d, [3.0, 2.0, 1.4, 1.0, 0.5], 0.05).astype(np.float32)
+    P = _orthonormal(rng, d, s).astype(np.float32)
+    mu, ut, lam, _ = O.canonical_summaries_subspace(K, L, R, P)
+    mu_q, codes, scales, lam_q, ut_q, _ = O.canonical_summaries_subspace_fp4(K, L, R, P)
+    assert np.array_equal(lam_q, lam)
+    assert codes.shape == (nB, R, s) and codes.max() <= 15
+    sc = scales[..., None].astype(np.float64)
+    err = np.abs(ut_q.astype(np.float64) - ut.astype(np.float64))
+    half_gap = np.where(np.abs(ut) / sc > 4, 1.0, np.where(np.abs(ut) / sc > 2, 0.5, 0.25))
+    assert np.all(err <= half_gap * sc * (1 + 1e-6) + 1e-12)
+    assert np.allclose(scales, np.abs(ut).max(axis=-1) / 6, rtol=1e-7)
+    rel = np.abs(mu_q.astype(np.float64) - mu) / np.maximum(np.abs(mu.astype(np.float64)), 1e-30)
+    assert np.all(rel <= 2.0 ** -8)
+
+
+def test_subspace_fp4_canonical_scores_match_float64_of_the_stored_form():
+    """The float32 canonical scores of the stored (dequantized) form agree with the float64 score of
+    the same stored numbers to float32 rounding (a relative bound on the summed terms)."""
+    rng = np.random.default_rng(63)
+    L, d, R, nB, G, s = 64, 128, 4, 40, 4, 84
+    K = _aniso_blocks(rng, nB, L, d, [3.0, 2.0, 1.4, 1.0, 0.5], 0.05).astype(np.float32)
+    P = _orthonormal(rng, d, s).astype(np.float32)
+    summ = O.canonical_summaries_subspace_fp4(K, L, R, P)
+    q = rng.standard_normal((G, d)).astype(np.float32)
+    S32 = O.canonical_scores_subspace(q, summ.dequantized(), 1.0).astype(np.float64)
+    mu_q, _, _, lam, ut_q, _ = summ
+    S64 = O.group_scores_subspace_coords(q.astype(np.float64), mu_q.astype(np.float64), ut_q.astype(np.float64),
+                                         lam.astype(np.float64), P.astype(np.float64), 1.0)
+    # magnitude of the summed terms: |q||mu| / sqrt(d) per head + the covariance term
+    scale = np.abs(S64) + np.linalg.norm(q, axis=1).sum() * np.linalg.norm(mu_q, axis=1) / np.sqrt(d) + 1.0
+    assert np.all(np.abs(S32 - S64) <= 64 * 2.0 ** -24 * scale)
+
+
+def test_subspace_fp4_selection_tracks_the_float32_subspace_selection():
+    """On anisotropic blocks with queries in the subspace, the FP4 coordinates select nearly the same
+    blocks as the float32 subspace coordinates."""
+    rng = np.random.default_rng(64)
+    L, d, R, nB, G, k, s = 64, 128, 4, 96, 4, 16, 84
+    K = _aniso_blocks(rng, nB, L, d, [3.0, 2.0, 1.4, 1.0, 0.6, 0.4], 0.05).astype(np.float32)
+    K += (rng.standard_normal((nB, 1, d)) * rng.uniform(0.2, 1.5, (nB, 1, 1))).repeat(L, axis=1).reshape(nB * L, d).astype(np.float32)
+    P = _orthonormal(rng, d, s).astype(np.float32)
+    q = (P @ rng.standard_normal((s, G))).T.astype(np.float32)
+    s32 = O.canonical_scores_subspace(q, O.canonical_summaries_subspace(K, L, R, P), 1.0)
+    s4 = O.canonical_scores_subspace(q, O.canonical_summaries_subspace_fp4(K, L, R, P).dequantized(), 1.0)
+    a, b = set(O.top_k(s32, nB, k).tolist()), set(O.top_k(s4, nB, k).tolist())
+    assert len(a & b) >= 13
