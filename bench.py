@@ -42,7 +42,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode32k", choices=["decode32k", "decode128k", "prefill32k", "sweep"])
     ap.add_argument("--contexts", default=None, help="sweep: comma-separated context lengths (default 8k .. 1M)")
-    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank", "lowrank_fp4", "subspace"],
+    ap.add_argument("--variance", choices=["channel", "isotropic", "lowrank", "lowrank_fp4", "subspace",
+                                           "subspace_fp4"],
                     default="channel",
                     help="second-order statistic of the summaries (per-channel variance, one scalar per block, "
                          "or the leading eigenpairs of each block's covariance)")
@@ -181,7 +182,8 @@ def summary_block_bytes(d, variance, rank, sub):
     """Summary bytes per selection block for each second-order form."""
     return {"isotropic": (d + 1) * 4, "lowrank": (d + rank * d + rank) * 4,
             "lowrank_fp4": 2 * d + rank * d // 2 + 8 * rank,
-            "subspace": (d + rank * sub + rank) * 4}.get(variance, 2 * d * 4)
+            "subspace": (d + rank * sub + rank) * 4,
+            "subspace_fp4": 2 * d + rank * (-(-sub // 32) * 32) // 2 + 8 * rank}.get(variance, 2 * d * 4)
 
 
 def decode_bytes(w, idx, variance="channel", rank=4, sub=84):
@@ -205,7 +207,7 @@ def decode_bytes(w, idx, variance="channel", rank=4, sub=84):
     attn += w.B * w.Hq * d * esz * 2 + w.B * w.Hq * 3 * 4 + units * w.topk * 4   # Q, O, gates, idx
     per_block = summary_block_bytes(d, variance, rank, sub)
     select = units * w.nB * per_block + w.B * w.Hq * d * esz + units * w.topk * 4
-    if variance == "subspace":
+    if variance in ("subspace", "subspace_fp4"):
         select += d * sub * 4   # the basis
     # summary update for the appended token: the completed block (64 K rows) and the last
     # compressed token (cmp_block K and V rows), plus their outputs
@@ -293,9 +295,9 @@ def decode_config(w, args, R=None, world=1):
     cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "topk": w.topk,
            "window": w.window, "cmp_block": w.cmp_block, "cmp_stride": w.cmp_stride, "alpha": w.alpha,
            "variance": args.variance}
-    if args.variance in ("lowrank", "lowrank_fp4", "subspace"):
+    if args.variance in ("lowrank", "lowrank_fp4", "subspace", "subspace_fp4"):
         cfg["rank"] = args.rank
-    if args.variance == "subspace":
+    if args.variance in ("subspace", "subspace_fp4"):
         cfg.update(sub=args.sub, queries="concentrated in the subspace (leak 0.1)")
     cfg["step"] = ("cobs_decode_step: summary update at T-1, selection, then the decode attention as a "
                    "programmatic dependent of the selection; one CUDA graph")
@@ -471,7 +473,7 @@ def measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=True, c
     import torch
     import torch.distributed as dist
     import synth
-    basis = synth.subspace_basis(w, args.sub) if args.variance == "subspace" else None
+    basis = synth.subspace_basis(w, args.sub) if args.variance in ("subspace", "subspace_fp4") else None
     p = cobs.Params(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, T=w.T, topk=w.topk, window=w.window, block=w.block,
                     cmp_block=w.cmp_block, cmp_stride=w.cmp_stride, alpha=w.alpha, dtype=w.dtype,
                     variance=args.variance, rank=args.rank,
@@ -891,7 +893,7 @@ def sweep_rows(args, dev, cobs, contexts):
     rows = []
     stream = torch.cuda.Stream(device=dev)
 
-    basis = synth.subspace_basis(base, args.sub) if args.variance == "subspace" else None
+    basis = synth.subspace_basis(base, args.sub) if args.variance in ("subspace", "subspace_fp4") else None
     tbasis = torch.from_numpy(basis).to(dev) if basis is not None else None
     qbasis = synth.subspace_basis(base, args.sub) if (basis is not None or args.subspace_queries) else None
 
@@ -997,7 +999,7 @@ def run_sweep(args):
     peak, peak_kind = read_peaks()
     n_rec = min(8, base.B)
     rows = sweep_rows(args, dev, cobs, contexts)
-    basis_used = args.variance == "subspace" or args.subspace_queries
+    basis_used = args.variance in ("subspace", "subspace_fp4") or args.subspace_queries
     top = rows[-1]
     line = {"metric": "selector GB/s over context length (decode selection, 64 x 8 units, top-16)",
             "value": top["gbs"], "unit": "GB/s", "n_gpus": 1, "steps": top["steps"], "warmup": max(3, args.warmup),

@@ -24,6 +24,7 @@ COBS_ERR_WORKSPACE = -4
 COBS_F32 = 0
 COBS_BF16 = 1
 COBS_VAR_CHANNEL, COBS_VAR_ISOTROPIC, COBS_VAR_LOWRANK, COBS_VAR_LOWRANK_FP4, COBS_VAR_SUBSPACE = 0, 1, 2, 3, 4
+COBS_VAR_SUBSPACE_FP4 = 5
 COBS_WS_SELECT = 0
 COBS_WS_DECODE = 1
 COBS_WS_PREFILL = 2
@@ -104,15 +105,16 @@ class Params:
     cmp_stride: int = 16
     alpha: float = 1.0
     dtype: str = "bf16"
-    variance: str = "channel"   # "channel", "isotropic", "lowrank", "lowrank_fp4" or "subspace"
+    variance: str = "channel"   # "channel", "isotropic", "lowrank", "lowrank_fp4", "subspace", "subspace_fp4"
     rank: int = 4               # eigenpairs per block for the low-rank forms
-    sub: int = 84               # "subspace": coordinates kept per eigenvector
-    basis: object = dataclasses.field(default=None, compare=False, repr=False)  # "subspace": [d, sub] f32 CUDA
+    sub: int = 84               # "subspace(_fp4)": coordinates kept per eigenvector
+    basis: object = dataclasses.field(default=None, compare=False, repr=False)  # "subspace(_fp4)": [d, sub] f32
 
     def c(self) -> cobs_params:
         var = {"channel": COBS_VAR_CHANNEL, "isotropic": COBS_VAR_ISOTROPIC, "lowrank": COBS_VAR_LOWRANK,
-               "lowrank_fp4": COBS_VAR_LOWRANK_FP4, "subspace": COBS_VAR_SUBSPACE}[self.variance]
-        sub = var == COBS_VAR_SUBSPACE
+               "lowrank_fp4": COBS_VAR_LOWRANK_FP4, "subspace": COBS_VAR_SUBSPACE,
+               "subspace_fp4": COBS_VAR_SUBSPACE_FP4}[self.variance]
+        sub = var in (COBS_VAR_SUBSPACE, COBS_VAR_SUBSPACE_FP4)
         if sub and self.basis is not None and (self.basis.dtype != torch.float32 or
                                                 tuple(self.basis.shape) != (self.d, self.sub)):
             raise ValueError("basis must be a float32 [d, sub] tensor")

@@ -55,6 +55,11 @@ cobs_status device_flag(int** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The query-subspace summaries (float32 or FP4 coordinates) take a basis.
+bool uses_basis(const cobs_params* p) {
+    return p->variance == COBS_VAR_SUBSPACE || p->variance == COBS_VAR_SUBSPACE_FP4;
+}
+
 cobs_status validate(const cobs_params* p) {
     if (p == nullptr) return fail(COBS_ERR_INVALID_ARG, "params is NULL");
     if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->T < 1)
@@ -73,13 +78,11 @@ cobs_status validate(const cobs_params* p) {
         return fail(COBS_ERR_INVALID_ARG, "need 1 <= cmp_stride <= cmp_block (got %d, %d)", p->cmp_stride,
                     p->cmp_block);
     if (p->dtype != COBS_F32 && p->dtype != COBS_BF16) return fail(COBS_ERR_INVALID_ARG, "dtype %d", p->dtype);
-    if (p->variance < COBS_VAR_CHANNEL || p->variance > COBS_VAR_SUBSPACE)
+    if (p->variance < COBS_VAR_CHANNEL || p->variance > COBS_VAR_SUBSPACE_FP4)
         return fail(COBS_ERR_INVALID_ARG, "variance %d (a cobs_variance value)", p->variance);
-    if ((p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4 ||
-         p->variance == COBS_VAR_SUBSPACE) &&
-        (p->rank < 1 || p->rank > 8))
+    if (p->variance >= COBS_VAR_LOWRANK && (p->rank < 1 || p->rank > 8))
         return fail(COBS_ERR_UNSUPPORTED, "rank %d (supported: 1 .. 8)", p->rank);
-    if (p->variance == COBS_VAR_SUBSPACE) {
+    if (uses_basis(p)) {
         if (p->sub < 4 || p->sub > p->d || p->sub % 4 != 0)
             return fail(COBS_ERR_UNSUPPORTED, "subspace dimension %d (a multiple of 4 in 4 .. d)", p->sub);
     }
@@ -201,7 +204,7 @@ cobs_status cobs_build_summaries(const cobs_params* p, const void* K, const void
     COBS_TRY(check_ptr(Pk, "Pk", true));
     COBS_TRY(check_ptr(Pv, "Pv", true));
     COBS_TRY(check_ptr(summaries, "summaries"));
-    if (p->variance == COBS_VAR_SUBSPACE) COBS_TRY(check_ptr(p->basis, "basis"));
+    if (uses_basis(p)) COBS_TRY(check_ptr(p->basis, "basis"));
     const cobs::Dims m = cobs::make_dims(*p);
     if (m.nC > 0) {
         COBS_TRY(check_ptr(Kc, "Kc"));
@@ -223,9 +226,8 @@ cobs_status cobs_select(const cobs_params* p, const void* Q, const float* summar
     COBS_TRY(check_ptr(idx, "idx"));
     if (prefill != 0 && prefill != 1) return fail(COBS_ERR_INVALID_ARG, "prefill must be 0 or 1");
     if (prefill) COBS_TRY(validate_prefill_rows(p));
-    if (p->variance == COBS_VAR_SUBSPACE && !prefill) COBS_TRY(check_ptr(p->basis, "basis"));
-    if (prefill && (p->variance == COBS_VAR_LOWRANK || p->variance == COBS_VAR_LOWRANK_FP4 ||
-                    p->variance == COBS_VAR_SUBSPACE))
+    if (uses_basis(p) && !prefill) COBS_TRY(check_ptr(p->basis, "basis"));
+    if (prefill && p->variance >= COBS_VAR_LOWRANK)
         return fail(COBS_ERR_UNSUPPORTED, "prefill selection with low-rank summaries");
     const cobs::Dims m = cobs::make_dims(*p);
     const size_t need = cobs::select_workspace_bytes(m, prefill);
@@ -282,7 +284,7 @@ static cobs_status step_common(const cobs_params* p, const void* Q, const void* 
     COBS_TRY(check_ptr(Pk, "Pk", true));
     COBS_TRY(check_ptr(Pv, "Pv", true));
     COBS_TRY(check_ptr(summaries, "summaries"));
-    if (p->variance == COBS_VAR_SUBSPACE) COBS_TRY(check_ptr(p->basis, "basis"));
+    if (uses_basis(p)) COBS_TRY(check_ptr(p->basis, "basis"));
     if (t_begin < 0 || t_begin > p->T) return fail(COBS_ERR_INVALID_ARG, "t_begin %d outside [0, T]", t_begin);
     COBS_TRY(check_ptr(workspace, "workspace"));
     return COBS_OK;

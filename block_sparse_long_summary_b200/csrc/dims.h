@@ -18,14 +18,16 @@ struct Dims {
     int dtype;    // cobs_dtype
     int iso;      // summaries keep one variance scalar per block (COBS_VAR_ISOTROPIC)
     int lr;       // eigenpairs per block (COBS_VAR_LOWRANK / _FP4), else 0
-    int fp4;      // low-rank summaries stored as FP4 eigenvectors and a bf16 mean
-    int sub;      // COBS_VAR_SUBSPACE: eigenvectors kept as sub coordinates in the basis, else 0
-    const float* basis;  // COBS_VAR_SUBSPACE: [d][sub] float32 device array
+    int fp4;      // low-rank summaries stored as FP4 eigenvectors (or coordinates) and a bf16 mean
+    int sub;      // COBS_VAR_SUBSPACE(_FP4): eigenvectors kept as sub coordinates in the basis, else 0
+    const float* basis;  // COBS_VAR_SUBSPACE(_FP4): [d][sub] float32 device array
     int units() const { return B * Hkv; }
     // floats of one 32-block summary group: means and per-channel variances, means and one
     // scalar per block, or means, lr eigenvectors and lr eigenvalues per block
+    // FP4 codes per vector and block: d, or sub rounded up to a multiple of 32
+    int code_width() const { return sub ? (sub + 31) / 32 * 32 : d; }
     size_t group_floats() const {
-        if (lr && fp4) return (size_t)8 * (2 * d + lr * d / 2 + 8 * lr);
+        if (lr && fp4) return (size_t)8 * (2 * d + lr * code_width() / 2 + 8 * lr);
         if (lr && sub) return (size_t)32 * (d + lr * sub + lr);
         if (lr) return (size_t)32 * (d + lr * d + lr);
         return iso ? (size_t)(d + 1) * 32 : (size_t)2 * d * 32;
@@ -41,13 +43,11 @@ inline Dims make_dims(const cobs_params& p) {
     m.nG = m.nB > 0 ? (m.nB + 31) / 32 : 1;
     m.nC = (p.cmp_stride > 0 && p.T >= p.cmp_block) ? (p.T - p.cmp_block) / p.cmp_stride + 1 : 0;
     m.alpha = p.alpha; m.dtype = p.dtype; m.iso = p.variance == COBS_VAR_ISOTROPIC;
-    m.lr = (p.variance == COBS_VAR_LOWRANK || p.variance == COBS_VAR_LOWRANK_FP4 ||
-            p.variance == COBS_VAR_SUBSPACE)
-               ? p.rank
-               : 0;
-    m.fp4 = p.variance == COBS_VAR_LOWRANK_FP4;
-    m.sub = p.variance == COBS_VAR_SUBSPACE ? p.sub : 0;
-    m.basis = p.variance == COBS_VAR_SUBSPACE ? p.basis : nullptr;
+    m.lr = p.variance >= COBS_VAR_LOWRANK ? p.rank : 0;
+    m.fp4 = p.variance == COBS_VAR_LOWRANK_FP4 || p.variance == COBS_VAR_SUBSPACE_FP4;
+    const bool subspace = p.variance == COBS_VAR_SUBSPACE || p.variance == COBS_VAR_SUBSPACE_FP4;
+    m.sub = subspace ? p.sub : 0;
+    m.basis = subspace ? p.basis : nullptr;
     return m;
 }
 

@@ -198,13 +198,18 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
     return out;
 }
 
-// Canonical low-rank score from FP4 summaries: the bf16 means and the dequantized eigenvectors
-// u'_c = value(code_c) * scale_j (one rounded multiply), then the low-rank score's sums. Tile
-// bytes: bf16 means [D/8][32][8], codes of vector j [D/32][32][16] (channel 2i in the low nibble
-// of byte i), scales [R][32] f32, eigenvalues [R][32] f32.
-template <int D>
-__device__ __forceinline__ float block_score_lr_fp4(const float* tile, const float* qs, const float* qh, int G, int R,
-                                                    int lane, float isd, float c2) {
+// Canonical low-rank score from FP4 summaries: the bf16 means and the dequantized vectors
+// u'_i = value(code_i) * scale_j (one rounded multiply), then the low-rank score's sums. Tile
+// bytes: bf16 means [D/8][32][8], codes of vector j [CW/32][32][16] (entry 2i in the low nibble
+// of byte i), scales [R][32] f32, eigenvalues [R][32] f32. SUB = false: the vectors are the
+// eigenvectors (CW = S = D) and qh the heads [G][D]; SUB = true: the S coordinates of the
+// eigenvectors in the query subspace (CW = S rounded up to 32, codes past S zero) and qh the
+// projected heads [G][S] (S a multiple of 4: coordinate i to chain i mod 4, as the channels).
+template <int D, bool SUB>
+__device__ __forceinline__ float block_score_fp4(const float* tile, const float* qs, const float* qh, int G, int R,
+                                                 int S_, int lane, float isd, float c2) {
+    const int S = SUB ? S_ : D;
+    const int CW = SUB ? (S_ + 31) / 32 * 32 : D;
     const unsigned char* t8 = reinterpret_cast<const unsigned char*>(tile);
     float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
@@ -218,12 +223,12 @@ __device__ __forceinline__ float block_score_lr_fp4(const float* tile, const flo
             a[t & 3] = __fmaf_rn(qs[8 * c8 + t], mu, a[t & 3]);
         }
     }
-    const float* scl = reinterpret_cast<const float*>(t8 + (size_t)64 * D + (size_t)R * 16 * D);
+    const float* scl = reinterpret_cast<const float*>(t8 + (size_t)64 * D + (size_t)R * 16 * CW);
     const float* lam = scl + R * 32;
     float v = 0.0f;
     for (int j = 0; j < R; ++j) {
         const float sj = scl[j * 32 + lane];
-        const unsigned char* cj = t8 + (size_t)64 * D + (size_t)j * 16 * D;
+        const unsigned char* cj = t8 + (size_t)64 * D + (size_t)j * 16 * CW;
         // heads in fours: each 32-channel chunk is decoded once per four heads
         // (u'_c = value * scale, one rounded multiply)
         float e = 0.0f;
@@ -231,7 +236,7 @@ __device__ __forceinline__ float block_score_lr_fp4(const float* tile, const flo
             float p[4][4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) p[h][0] = p[h][1] = p[h][2] = p[h][3] = 0.0f;
-            for (int w = 0; w < D / 32; ++w) {
+            for (int w = 0; w < CW / 32; ++w) {
                 const uint4 wv = *reinterpret_cast<const uint4*>(cj + ((size_t)w * 32 + lane) * 16);
                 const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
                 float u[32];
@@ -244,9 +249,10 @@ __device__ __forceinline__ float block_score_lr_fp4(const float* tile, const flo
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     if (hb + h < G) {
-                        const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)(hb + h) * D) + w * 8;
+                        const float4* q4 = reinterpret_cast<const float4*>(qh + (size_t)(hb + h) * S) + w * 8;
 #pragma unroll
                         for (int t4 = 0; t4 < 8; ++t4) {
+                            if (SUB && w * 32 + t4 * 4 >= S) break;  // past the S coordinates
                             const float4 q = q4[t4];
                             p[h][0] = __fmaf_rn(q.x, u[4 * t4 + 0], p[h][0]);
                             p[h][1] = __fmaf_rn(q.y, u[4 * t4 + 1], p[h][1]);
@@ -282,7 +288,7 @@ constexpr int group_floats() { return ISO ? (D + 1) * 32 : 2 * D * 32; }
 #define COBS_SELECT_CTAS_PER_SM 3
 #endif
 constexpr int kSelStages = COBS_SELECT_STAGES;
-// At most this many one-warp selection CTAs per SM (twice as many for the FP4 low-rank
+// At most this many one-warp selection CTAs per SM (twice as many for the FP4
 // summaries, whose scoring is bound by arithmetic and whose tiles are small); the grid takes the
 // smaller of this and the number that fit an SM with the mode's shared memory (2 for the float32
 // low-rank summaries), so that every CTA is resident from the start.
@@ -316,7 +322,8 @@ inline int sel_max_segments(int units, int nGc) {
 // floats per group, one ring stage, the group's query heads in shared memory after the ring),
 // 3: low-rank with FP4 eigenvectors and bf16 means (as 2, with the ring of the other modes),
 // 4: query subspace (as 2, with the projected heads qt_ws [units][G][S] written by
-// project_queries_kernel, which this grid waits for, in place of the heads).
+// project_queries_kernel, which this grid waits for, in place of the heads), 5: query subspace
+// with FP4 coordinates and bf16 means (as 3, with the projected heads of 4).
 template <typename T, int D, int MODE>
 __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__ Q, const float* __restrict__ summ,
                                                            int32_t* __restrict__ idx, float* __restrict__ ws_s,
@@ -330,6 +337,7 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
     __shared__ float q2t_sm;
     constexpr bool ISO = MODE == 1;
     constexpr int kStg = (MODE == 2 || MODE == 4) ? 1 : kSelStages;
+    constexpr bool kProj = MODE == 4 || MODE == 5;  // the projected heads of project_queries_kernel
     const int kTileFloats = MODE >= 2 ? tile_floats : group_floats<D, ISO>();
     const uint32_t kTileBytes = (uint32_t)kTileFloats * 4;
     // the merge grid may be scheduled now; it still waits for this grid to complete
@@ -402,7 +410,7 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
                 if (lane == 0) q2t_sm = q2_total<D>(qsm[1]);
                 __syncwarp();
             }
-            if (MODE == 4) {  // the group's projected heads, after the ring
+            if (kProj) {  // the group's projected heads, after the ring
                 float* qh = tiles + kStg * kTileFloats;
                 if (x == x0) asm volatile("griddepcontrol.wait;" ::: "memory");  // qt_ws is complete
                 for (int e = lane; e < G * S; e += 32) qh[e] = __ldcg(qt_ws + (size_t)u * G * S + e);
@@ -421,8 +429,9 @@ __global__ void __launch_bounds__(32) select_decode_kernel(const T* __restrict__
         if (ok) {
             const float* tl = tiles + st * kTileFloats;
             const float* qh = tiles + kStg * kTileFloats;
-            const float s_all = MODE == 4 ? block_score_sub<D>(tl, qsm[0], qh, G, R, S, lane, isd, c2)
-                                : MODE == 3 ? block_score_lr_fp4<D>(tl, qsm[0], qh, G, R, lane, isd, c2)
+            const float s_all = MODE == 5   ? block_score_fp4<D, true>(tl, qsm[0], qh, G, R, S, lane, isd, c2)
+                                : MODE == 4 ? block_score_sub<D>(tl, qsm[0], qh, G, R, S, lane, isd, c2)
+                                : MODE == 3 ? block_score_fp4<D, false>(tl, qsm[0], qh, G, R, D, lane, isd, c2)
                                 : MODE == 2 ? block_score_sub<D>(tl, qsm[0], qh, G, R, D, lane, isd, c2)
                                 : ISO       ? block_score_iso<D>(tl, qsm[0], q2t_sm, lane, isd, c2)
                                             : block_score<D>(tl, qsm[0], qsm[1], lane, isd, c2);
@@ -669,6 +678,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         const size_t smem = MODE == 2   ? tile_bytes + (size_t)kMaxGroup * D * 4
                             : MODE == 3 ? (size_t)kSelStages * tile_bytes + (size_t)kMaxGroup * D * 4
                             : MODE == 4 ? tile_bytes + (size_t)m.G * m.sub * 4
+                            : MODE == 5 ? (size_t)kSelStages * tile_bytes + (size_t)m.G * m.sub * 4
                                         : (size_t)kSelStages * tile_bytes;
         if (smem > 227 * 1024) return cudaErrorNotSupported;
         cudaError_t e = cudaFuncSetAttribute(select_decode_kernel<T, D, MODE>,
@@ -677,7 +687,7 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         int per_sm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_decode_kernel<T, D, MODE>, 32, smem);
         if (e != cudaSuccess) return e;
-        per_sm = std::max(1, std::min(per_sm, MODE == 3 ? 2 * kSelCtasPerSm : kSelCtasPerSm));
+        per_sm = std::max(1, std::min(per_sm, (MODE == 3 || MODE == 5) ? 2 * kSelCtasPerSm : kSelCtasPerSm));
         // grid: the resident CTAs of every SM and at least one group each. A unit's groups then
         // meet at most min(nGc, ceil(grid / units) + 1) <= maxseg ranges (grid <= kSelGridCap).
         long long grid = std::min<long long>((long long)sm_count() * per_sm, kSelGridCap);
@@ -687,8 +697,9 @@ cudaError_t launch_select_t(const Dims& m, const T* Q, const float* summ, int pr
         grid = std::max<long long>(1, grid);
         float* ws_s = static_cast<float*>(ws);
         int* ws_i = reinterpret_cast<int*>(ws_s + (size_t)m.units() * maxseg * m.k);
-        float* qt_ws = MODE == 4 ? select_qt_region(m, ws) : nullptr;
-        if (MODE == 4 && n > 0) {  // the projected heads, then the selection grid as their dependent
+        constexpr bool kProj = MODE == 4 || MODE == 5;
+        float* qt_ws = kProj ? select_qt_region(m, ws) : nullptr;
+        if (kProj && n > 0) {  // the projected heads, then the selection grid as their dependent
             count_launch();
             project_queries_kernel<T, D><<<dim3(m.units(), (m.G * m.sub + 63) / 64), 256, 0, s>>>(Q, m.basis, m.G,
                                                                                                    m.sub, qt_ws);
@@ -769,7 +780,8 @@ cudaError_t launch_select_v(const Dims& m, const void* Q, const float* summ, int
 
 cudaError_t launch_select(const Dims& m, const void* Q, const float* summ, int prefill, int32_t* idx, void* ws,
                           cudaStream_t s, int* err) {
-    if (m.sub) return launch_select_v<4>(m, Q, summ, prefill, idx, ws, s, err);
+    if (m.sub) return m.fp4 ? launch_select_v<5>(m, Q, summ, prefill, idx, ws, s, err)
+                            : launch_select_v<4>(m, Q, summ, prefill, idx, ws, s, err);
     if (m.lr) return m.fp4 ? launch_select_v<3>(m, Q, summ, prefill, idx, ws, s, err)
                            : launch_select_v<2>(m, Q, summ, prefill, idx, ws, s, err);
     return m.iso ? launch_select_v<1>(m, Q, summ, prefill, idx, ws, s, err)

@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
     }
     __syncthreads();
     const int ln = j & 31;
-    if (S > 0) {
+    if (S > 0 && !fp4) {
         // query-subspace form: eigenvector jj kept as u~_i = four-chain sum over c of P[c][i] u_c
         // (i < S), in the [S/4][32][4] interleaving
         const size_t gf = (size_t)32 * (D + R * S + R);
@@ -235,16 +235,20 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
         if (c < R) base[(size_t)(1 + R) * D * 32 + (size_t)c * 32 + ln] = lam_sh[ord_sh[c]];
         return;
     }
-    // FP4 layout (bytes): bf16 means [D/8][32][8], E2M1 codes of vector jj [D/32][32][16]
-    // (channel 2i in the low nibble of byte i), scales [R][32] f32, eigenvalues [R][32] f32
-    const size_t gbytes = (size_t)32 * (2 * D + R * D / 2 + 8 * R);
+    // FP4 layout (bytes): bf16 means [D/8][32][8], E2M1 codes of vector jj [CW/32][32][16]
+    // (entry 2i in the low nibble of byte i), scales [R][32] f32, eigenvalues [R][32] f32. The
+    // vector is the eigenvector (CW = D), or its S coordinates in the query subspace (the
+    // projection of the float32 form above; CW = S rounded up to 32, the codes past S zero).
+    const int CW = S > 0 ? (S + 31) / 32 * 32 : D;
+    const size_t gbytes = (size_t)32 * (2 * D + R * CW / 2 + 8 * R);
     unsigned char* g8 = reinterpret_cast<unsigned char*>(summ) + ((size_t)unit * nG + (size_t)(j >> 5)) * gbytes;
     const __nv_bfloat16 mb = __float2bfloat16_rn(mu_c);
     *reinterpret_cast<__nv_bfloat16*>(g8 + ((size_t)(c / 8) * 32 + ln) * 16 + (c % 8) * 2) = mb;
-    float* scl = reinterpret_cast<float*>(g8 + (size_t)64 * D + (size_t)R * 16 * D);
+    float* scl = reinterpret_cast<float*>(g8 + (size_t)64 * D + (size_t)R * 16 * CW);
     float* lamo = scl + R * 32;
+    const bool live = S == 0 || c < S;  // thread c holds an entry of the vector
     for (int jj = 0; jj < R; ++jj) {
-        const float x = V[c][ord_sh[jj]];
+        const float x = S == 0 ? V[c][ord_sh[jj]] : (live ? lr_dot4(Pb + c, &V[0][ord_sh[jj]], D, S, kLrMaxR + 1) : 0.0f);
         red[c] = fabsf(x);
         __syncthreads();
         for (int o = D / 2; o > 0; o >>= 1) {  // max is exact in any order
@@ -252,10 +256,10 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
             __syncthreads();
         }
         const float sc = __fdiv_rn(red[0], 6.0f);
-        code_sh[c] = sc > 0.0f ? e2m1_code(__fdiv_rn(x, sc)) : 0;
+        code_sh[c] = live && sc > 0.0f ? e2m1_code(__fdiv_rn(x, sc)) : 0;
         __syncthreads();
-        if ((c & 1) == 0)
-            g8[(size_t)64 * D + (size_t)jj * 16 * D + ((size_t)(c / 32) * 32 + ln) * 16 + (c % 32) / 2] =
+        if ((c & 1) == 0 && c < CW)
+            g8[(size_t)64 * D + (size_t)jj * 16 * CW + ((size_t)(c / 32) * 32 + ln) * 16 + (c % 32) / 2] =
                 (unsigned char)(code_sh[c] | (code_sh[c + 1] << 4));
         if (c == 0) {
             scl[jj * 32 + ln] = sc;

@@ -50,6 +50,10 @@
  *                  variance = COBS_VAR_SUBSPACE (rank R, sub s): [B, Hkv, nG, 32 (d + R s + R)]
  *                  float32: the means as above, then the s coordinates of eigenvector j < R in a
  *                  [s/4, 32, 4] interleaving, then the R eigenvalues [R, 32].
+ *                  variance = COBS_VAR_SUBSPACE_FP4 (rank R, sub s; sp = s rounded up to a
+ *                  multiple of 32): the COBS_VAR_LOWRANK_FP4 layout with the codes of the s
+ *                  coordinates of projected eigenvector j in [sp/32, 32, 16] bytes (coordinates
+ *                  s .. sp - 1 have code 0): 8 (2d + R sp / 2 + 8 R) float32 elements per group.
  *                  (32 consecutive blocks are interleaved channel-by-channel so that one
  *                  group is one contiguous copy and lane b%32 reads its block's channels.)
  * - GQA: query head h belongs to KV head h / (Hq / Hkv).
@@ -109,13 +113,19 @@ typedef enum {
  *                       per block); the query heads are projected the same way, q~ = P^T q (float32,
  *                       four-chain sums over the d channels), and the score term is
  *                       alpha/2 * sum_j lambda_j (q~ . u~_j)^2 / d. Exact for queries inside span(P)
- *                       when P has orthonormal columns. Decode selection only. */
+ *                       when P has orthonormal columns. Decode selection only.
+ *   COBS_VAR_SUBSPACE_FP4  the three compressions of [COBS] §2.3 together (the form its §4.1 reports
+ *                       as "Subspace, r=4, FP4"): the COBS_VAR_SUBSPACE coordinates of each
+ *                       eigenvector in FP4 (E2M1, one float32 scale max|u~|/6 per vector, the
+ *                       COBS_VAR_LOWRANK_FP4 rounding) and the mean in bf16; the score uses the
+ *                       dequantized values. Decode selection only. */
 typedef enum {
     COBS_VAR_CHANNEL = 0,
     COBS_VAR_ISOTROPIC = 1,
     COBS_VAR_LOWRANK = 2,
     COBS_VAR_LOWRANK_FP4 = 3,
-    COBS_VAR_SUBSPACE = 4
+    COBS_VAR_SUBSPACE = 4,
+    COBS_VAR_SUBSPACE_FP4 = 5
 } cobs_variance;
 
 /* Problem statement ([COBS] §2.3, [SKILL] "Method"): block size, compression block and
@@ -135,8 +145,8 @@ typedef struct {
     int32_t dtype;      /* cobs_dtype of Q, K, V, Kc, Vc, O */
     int32_t variance;   /* cobs_variance: the second-order statistic of the summaries */
     int32_t rank;       /* eigenpairs per block for the low-rank forms (1 .. 8); ignored otherwise */
-    int32_t sub;        /* COBS_VAR_SUBSPACE: subspace dimension s (a multiple of 4, 4 .. d); else ignored */
-    const float* basis; /* COBS_VAR_SUBSPACE: device array [d][sub] float32, the basis P of the query
+    int32_t sub;        /* COBS_VAR_SUBSPACE(_FP4): subspace dimension s (a multiple of 4, 4 .. d); else ignored */
+    const float* basis; /* COBS_VAR_SUBSPACE(_FP4): device array [d][sub] float32, the basis P of the query
                            subspace (orthonormal columns expected, not checked), read by
                            cobs_build_summaries and cobs_select and owned by the caller; else ignored */
 } cobs_params;

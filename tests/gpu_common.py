@@ -29,7 +29,7 @@ def f64(t):
 
 
 def params_of(w, variance="channel", rank=4, basis=None):
-    """basis: the query-subspace basis [d, s] (numpy float32) for variance "subspace"."""
+    """basis: the query-subspace basis [d, s] (numpy float32) for variance "subspace(_fp4)"."""
     C = cobs()
     extra = {}
     if basis is not None:
@@ -39,24 +39,29 @@ def params_of(w, variance="channel", rank=4, basis=None):
                     rank=rank, **extra)
 
 
-def summaries_blocks(flat, p):
+def summaries_blocks(flat, p, check_padding=True):
     """Device summaries (channel-interleaved groups of 32 blocks) -> [B, Hkv, nB, 2, d] float32
     (per-channel variance) or [B, Hkv, nB, d + 1] (isotropic: means, then the block's scalar)."""
     nB = p.T // p.block
     nG = max(1, -(-nB // 32))
-    if p.variance == "lowrank_fp4":
+    if p.variance in ("lowrank_fp4", "subspace_fp4"):
+        # codes of cw entries per vector: the d channels, or the sub coordinates padded to 32
         R, d = p.rank, p.d
-        gb = 32 * (2 * d + R * d // 2 + 8 * R)
+        n = p.sub if p.variance == "subspace_fp4" else d
+        cw = -(-n // 32) * 32
+        gb = 32 * (2 * d + R * cw // 2 + 8 * R)
         raw = flat[: p.B * p.Hkv * nG * gb // 4].cpu().numpy().view(np.uint8).reshape(p.B, p.Hkv, nG, gb)
         mub = raw[..., :64 * d].copy().view(np.uint16).reshape(p.B, p.Hkv, nG, d // 8, 32, 8)
         mu = (mub.astype(np.uint32) << 16).view(np.float32).transpose(0, 1, 2, 4, 3, 5).reshape(p.B, p.Hkv, nG * 32, d)
-        cb = raw[..., 64 * d:64 * d + R * 16 * d].reshape(p.B, p.Hkv, nG, R, d // 32, 32, 16)
-        codes = np.stack([cb & 15, cb >> 4], axis=-1).reshape(p.B, p.Hkv, nG, R, d // 32, 32, 32)
-        codes = codes.transpose(0, 1, 2, 5, 3, 4, 6).reshape(p.B, p.Hkv, nG * 32, R, d)
-        tail = raw[..., 64 * d + R * 16 * d:].copy().view(np.float32).reshape(p.B, p.Hkv, nG, 2, R, 32)
+        cb = raw[..., 64 * d:64 * d + R * 16 * cw].reshape(p.B, p.Hkv, nG, R, cw // 32, 32, 16)
+        codes = np.stack([cb & 15, cb >> 4], axis=-1).reshape(p.B, p.Hkv, nG, R, cw // 32, 32, 32)
+        codes = codes.transpose(0, 1, 2, 5, 3, 4, 6).reshape(p.B, p.Hkv, nG * 32, R, cw)
+        if check_padding:
+            assert not codes[:, :, :nB, :, n:].any(), "codes past the stored entries must be zero"
+        tail = raw[..., 64 * d + R * 16 * cw:].copy().view(np.float32).reshape(p.B, p.Hkv, nG, 2, R, 32)
         scales = tail[..., 0, :, :].transpose(0, 1, 2, 4, 3).reshape(p.B, p.Hkv, nG * 32, R)
         lam = tail[..., 1, :, :].transpose(0, 1, 2, 4, 3).reshape(p.B, p.Hkv, nG * 32, R)
-        return mu[:, :, :nB], codes[:, :, :nB].astype(np.uint8), scales[:, :, :nB], lam[:, :, :nB]
+        return mu[:, :, :nB], codes[:, :, :nB, :, :n].astype(np.uint8), scales[:, :, :nB], lam[:, :, :nB]
     if p.variance == "subspace":
         R, d, S = p.rank, p.d, p.sub
         gf = 32 * (d + R * S + R)

@@ -116,6 +116,8 @@ def test_workspace_sizes(lib):
     (dict(variance="subspace", rank=4, sub=82), -2),   # not a multiple of 4
     (dict(variance="subspace", rank=4, sub=0), -2),
     (dict(variance="subspace", rank=4, sub=132), -2),  # more than d
+    (dict(variance="subspace_fp4", rank=4, sub=82), -2),
+    (dict(variance="subspace_fp4", rank=9, sub=84), -2),
 ])
 def test_summary_form_validation(lib, kw, status):
     p = _p(**kw)
@@ -128,14 +130,15 @@ def test_summary_form_validation(lib, kw, status):
 
 def test_unknown_variance_rejected(lib):
     cp = _p().c()
-    cp.variance = 5
+    cp.variance = 6   # one past COBS_VAR_SUBSPACE_FP4
     fake = ctypes.c_void_p(256)
     assert lib._lib.cobs_build_summaries(ctypes.byref(cp), fake, fake, None, None, 0, fake, fake, fake, None) == -1
     assert b"variance" in lib._lib.cobs_last_error()
 
 
-def test_subspace_needs_a_basis(lib):
-    p = _p(variance="subspace", rank=4, sub=84)   # no basis: sizing works, compute calls refuse
+@pytest.mark.parametrize("variance", ["subspace", "subspace_fp4"])
+def test_subspace_needs_a_basis(lib, variance):
+    p = _p(variance=variance, rank=4, sub=84)   # no basis: sizing works, compute calls refuse
     assert lib.summaries_elems(p) > 0
     cp = p.c()
     fake = ctypes.c_void_p(256)
@@ -158,6 +161,9 @@ def test_summary_sizes_of_every_form(lib):
     assert lib.summaries_elems(_p(variance="lowrank", rank=4, **kw)) == units * nG * 32 * (d + 4 * d + 4)
     assert lib.summaries_elems(_p(variance="lowrank_fp4", rank=3, **kw)) == units * nG * 8 * (2 * d + 3 * d // 2 + 24)
     assert lib.summaries_elems(_p(variance="subspace", rank=4, sub=84, **kw)) == units * nG * 32 * (d + 4 * 84 + 4)
+    # FP4 coordinates: 84 codes padded to 96 per vector
+    assert lib.summaries_elems(_p(variance="subspace_fp4", rank=4, sub=84, **kw)) == units * nG * 8 * (2 * d + 4 * 96 // 2
+                                                                                                        + 32)
     # the query-subspace form's selection workspace adds the projected heads [units, G, s] float32
     ws_lr = lib.workspace_bytes(_p(variance="lowrank", rank=4, **kw), lib.COBS_WS_SELECT)
     ws_sub = lib.workspace_bytes(_p(variance="subspace", rank=4, sub=84, **kw), lib.COBS_WS_SELECT)

@@ -65,7 +65,8 @@ def test_prefill_flops_match_a_per_position_count():
 
 
 @pytest.mark.parametrize("variance,rank,sub", [("channel", 0, 0), ("isotropic", 0, 0), ("lowrank", 4, 0),
-                                               ("lowrank_fp4", 3, 0), ("subspace", 4, 84)])
+                                               ("lowrank_fp4", 3, 0), ("subspace", 4, 84),
+                                               ("subspace_fp4", 4, 84), ("subspace_fp4", 2, 64)])
 def test_summary_bytes_per_block_match_the_library_layout(variance, rank, sub):
     from block_sparse_long_summary_b200 import build as B
     B.build()
