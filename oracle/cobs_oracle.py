@@ -443,6 +443,29 @@ def block_eigenpairs(K: np.ndarray, L: int, R: int):
     return mu, u, lam
 
 
+def query_basis(Q: np.ndarray, s: int):
+    """The query subspace of [COBS] §2.3: the eigenvectors of the queries' second moment
+    M = (1/n) sum_i q_i q_i^T (rows of Q [n, d], float64) for its s largest eigenvalues, as the
+    columns of P [d, s] in descending eigenvalue order (numpy's eigh), each column's sign fixed so
+    that its largest-magnitude entry (the first such on ties) is positive. Returns (P, eigenvalues
+    [s]).
+
+    The pages say the subspace is spanned by the top eigenvectors of the query second moment but
+    not how it is estimated: reading, the second moment of the sample of queries the caller
+    passes (for example a prefill's queries)."""
+    Q = np.asarray(Q, np.float64)
+    n, d = Q.shape
+    M = Q.T @ Q / n
+    w, V = np.linalg.eigh(M)
+    order = np.argsort(-w, kind="stable")[:s]
+    P = V[:, order].copy()
+    for k in range(s):
+        i = int(np.argmax(np.abs(P[:, k])))
+        if P[i, k] < 0:
+            P[:, k] = -P[:, k]
+    return P, w[order]
+
+
 def head_scores_lowrank(q: np.ndarray, mu: np.ndarray, u: np.ndarray, lam: np.ndarray, alpha: float) -> np.ndarray:
     """Low-rank per-head score: q.mu_b/sqrt(d) + alpha * 1/2 * sum_j lam_j (q . u_j)^2 / d
     (the second cumulant 1/2 q^T Sigma_b q / d with Sigma_b ~ sum_j lam_j u_j u_j^T)."""

@@ -931,3 +931,58 @@ def test_subspace_fp4_selection_tracks_the_float32_subspace_selection():
     s4 = O.canonical_scores_subspace(q, O.canonical_summaries_subspace_fp4(K, L, R, P).dequantized(), 1.0)
     a, b = set(O.top_k(s32, nB, k).tolist()), set(O.top_k(s4, nB, k).tolist())
     assert len(a & b) >= 13
+
+
+# ---------------------------------------------------------------- query-subspace basis from queries
+
+def test_query_basis_recovers_an_exactly_diagonal_second_moment():
+    """Rows +-c_k u_k of an orthonormal U: M = (1/n) sum_k 2 c_k^2 u_k u_k^T exactly, so the basis is
+    the u_k of the s largest c_k (each with its largest-magnitude entry made positive) and the
+    eigenvalues are 2 c_k^2 / n."""
+    rng = np.random.default_rng(71)
+    d, s = 16, 5
+    U, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    c = np.linspace(3.0, 0.5, d)
+    rows = np.concatenate([c[:, None] * U.T, -c[:, None] * U.T])   # [2d, d]
+    rows = rows[rng.permutation(2 * d)]
+    P, lam = O.query_basis(rows, s)
+    n = 2 * d
+    assert np.allclose(lam, 2 * c[:s] ** 2 / n, rtol=1e-12)
+    for k in range(s):
+        u = U[:, k] * np.sign(U[np.argmax(np.abs(U[:, k])), k])
+        assert np.allclose(P[:, k], u, atol=1e-10), k
+
+
+def test_query_basis_two_dimensional_closed_form():
+    """d = 2: the leading eigenvalue of [[a, b], [b, c]] is (a + c)/2 + sqrt(((a - c)/2)^2 + b^2) and
+    its eigenvector is at angle atan2(2b, a - c)/2."""
+    Q = np.array([[1.0, 2.0], [3.0, -1.0], [0.5, 0.25], [-2.0, 1.5]])
+    a, b, c = (Q[:, 0] ** 2).mean(), (Q[:, 0] * Q[:, 1]).mean(), (Q[:, 1] ** 2).mean()
+    P, lam = O.query_basis(Q, 1)
+    assert lam[0] == pytest.approx((a + c) / 2 + math.sqrt(((a - c) / 2) ** 2 + b * b), rel=1e-12)
+    th = 0.5 * math.atan2(2 * b, a - c)
+    v = np.array([math.cos(th), math.sin(th)])
+    v = v * np.sign(v[np.argmax(np.abs(v))])
+    assert np.allclose(P[:, 0], v, atol=1e-12)
+
+
+def test_query_basis_planted_subspace_and_invariances():
+    """Queries drawn in a planted s-dimensional subspace with distinct scales plus small isotropic
+    noise: the basis spans the planted subspace (projectors agree to sampling error); permuting the
+    rows leaves the basis unchanged and scaling them by 2 multiplies the eigenvalues by 4; the
+    columns are orthonormal with the sign rule."""
+    rng = np.random.default_rng(72)
+    d, s, n = 64, 12, 40000
+    P0, _ = np.linalg.qr(rng.standard_normal((d, s)))
+    sig = np.linspace(3.0, 1.5, s)
+    Q = (rng.standard_normal((n, s)) * sig) @ P0.T + 0.05 * rng.standard_normal((n, d))
+    P, lam = O.query_basis(Q, s)
+    assert np.abs(P @ P.T - P0 @ P0.T).max() < 0.02
+    assert np.allclose(lam, sig ** 2 + 0.05 ** 2, rtol=0.05)
+    assert np.allclose(P.T @ P, np.eye(s), atol=1e-12)
+    for k in range(s):
+        assert P[np.argmax(np.abs(P[:, k])), k] > 0
+    P2, lam2 = O.query_basis(Q[rng.permutation(n)], s)
+    assert np.allclose(P2, P, atol=1e-9) and np.allclose(lam2, lam, rtol=1e-12)
+    P3, lam3 = O.query_basis(2 * Q, s)
+    assert np.allclose(P3, P, atol=1e-9) and np.allclose(lam3, 4 * lam, rtol=1e-12)
