@@ -18,7 +18,8 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libcobs.so")
-SOURCES = ["api.cu", "summary.cu", "select.cu", "decode.cu", "decode_stream.cu", "decode_step.cu", "tma.cu", "prefill.cu", "mass.cu"]
+SOURCES = ["api.cu", "summary.cu", "select.cu", "decode.cu", "decode_stream.cu", "decode_step.cu", "tma.cu", "prefill.cu",
+           "mass.cu", "basis.cu"]
 HEADERS = ["common.cuh", "attn.cuh", "dims.h", "tma.h", "tc.cuh", "select_core.cuh", "stream_tile.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

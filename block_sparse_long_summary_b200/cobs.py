@@ -30,12 +30,13 @@ COBS_WS_DECODE = 1
 COBS_WS_PREFILL = 2
 COBS_WS_STEP = 3
 COBS_WS_STEP_FUSED = 4
+COBS_WS_BASIS = 5
 
 EXPORTED = [
     "cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
     "cobs_sparse_attn_decode_noalloc", "cobs_workspace_bytes", "cobs_summaries_elems", "cobs_status_string", "cobs_last_error",
     "cobs_device_error", "cobs_launch_count", "cobs_version", "cobs_block_log_mass", "cobs_decode_step",
-    "cobs_decode_step_fused",
+    "cobs_decode_step_fused", "cobs_query_basis",
 ]
 
 
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.cobs_block_log_mass.argtypes = [P, vp, vp, vp, vp]
     lib.cobs_decode_step.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.cobs_decode_step_fused.argtypes = [P, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.cobs_query_basis.argtypes = [P, vp, ctypes.c_int64, vp, vp, vp, sz, vp]
+    lib.cobs_query_basis.restype = ctypes.c_int
     for f in ("cobs_build_summaries", "cobs_select", "cobs_sparse_attn_decode", "cobs_sparse_attn_prefill",
               "cobs_sparse_attn_decode_noalloc", "cobs_block_log_mass", "cobs_decode_step", "cobs_decode_step_fused"):
         getattr(lib, f).restype = ctypes.c_int
@@ -217,6 +220,25 @@ def cobs_decode_step_fused(p: Params, Q, K, V, Pk, Pv, t_begin, summaries, Kc, V
     _check(_lib.cobs_decode_step_fused(ctypes.byref(cp), _ptr(Q), _ptr(K), _ptr(V), _ptr(Pk), _ptr(Pv),
                                        int(t_begin), _ptr(summaries), _ptr(Kc), _ptr(Vc), _ptr(idx), _ptr(gates),
                                        _ptr(O), _ptr(workspace), nbytes, _stream(stream)))
+
+
+def cobs_query_basis(p: Params, Q, n, basis, eigenvalues, workspace, stream=None):
+    """Query-subspace basis [d, p.sub] (and eigenvalues, or None) from n query rows of Q."""
+    cp = p.c()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.cobs_query_basis(ctypes.byref(cp), _ptr(Q), int(n), _ptr(basis), _ptr(eigenvalues), _ptr(workspace),
+                                 nbytes, _stream(stream)))
+
+
+def query_basis(p: Params, Q, stream=None):
+    """Allocate and compute the basis [d, p.sub] float32 and eigenvalues [p.sub] from the rows of Q
+    (any shape [..., d] in p's storage type)."""
+    rows = Q.reshape(-1, p.d)
+    basis = torch.empty((p.d, p.sub), dtype=torch.float32, device=Q.device)
+    evals = torch.empty(p.sub, dtype=torch.float32, device=Q.device)
+    ws = torch.empty(max(16, workspace_bytes(p, COBS_WS_BASIS)), dtype=torch.uint8, device=Q.device)
+    cobs_query_basis(p, rows, rows.shape[0], basis, evals, ws, stream)
+    return basis, evals
 
 
 def cobs_sparse_attn_decode_noalloc(p: Params, Q, K, V, Kc, Vc, idx, gates, O, stream=None):

@@ -179,6 +179,7 @@ size_t cobs_workspace_bytes(const cobs_params* p, int32_t which) {
         case COBS_WS_PREFILL: return cobs::prefill_workspace_bytes(m);
         case COBS_WS_STEP: return step_workspace_bytes(m);
         case COBS_WS_STEP_FUSED: return cobs::decode_step_workspace_bytes(m);  // 0: shape not taken
+        case COBS_WS_BASIS: return cobs::basis_workspace_bytes(m);
     }
     return 0;
 }
@@ -381,6 +382,26 @@ cobs_status cobs_block_log_mass(const cobs_params* p, const void* Q, const void*
     if (m.G > 16) return fail(COBS_ERR_UNSUPPORTED, "cobs_block_log_mass supports at most 16 query heads per group");
     cudaError_t e = cobs::launch_block_log_mass(m, Q, K, out, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "cobs_block_log_mass launch");
+    return COBS_OK;
+}
+
+cobs_status cobs_query_basis(const cobs_params* p, const void* Q, int64_t n, float* basis, float* eigenvalues,
+                             void* workspace, size_t ws_bytes, cobs_stream_t stream) {
+    COBS_TRY(validate(p));
+    if (p->sub < 4 || p->sub > p->d || p->sub % 4 != 0)
+        return fail(COBS_ERR_UNSUPPORTED, "subspace dimension %d (a multiple of 4 in 4 .. d)", p->sub);
+    if (n < 1) return fail(COBS_ERR_INVALID_ARG, "n = %lld query rows (at least one)", (long long)n);
+    COBS_TRY(check_ptr(Q, "Q"));
+    COBS_TRY(check_ptr(basis, "basis"));
+    COBS_TRY(check_ptr(eigenvalues, "eigenvalues", true));
+    COBS_TRY(check_ptr(workspace, "workspace"));
+    const cobs::Dims m = cobs::make_dims(*p);
+    cobs::Dims mb = m;
+    mb.sub = p->sub;  // the basis width, whatever the params' summary form
+    const size_t need = cobs::basis_workspace_bytes(mb);
+    if (ws_bytes < need) return fail(COBS_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+    cudaError_t e = cobs::launch_query_basis(mb, Q, (long long)n, basis, eigenvalues, workspace, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cobs_query_basis launch");
     return COBS_OK;
 }
 

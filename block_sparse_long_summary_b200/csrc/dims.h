@@ -101,6 +101,12 @@ cudaError_t launch_prefill(const Dims& m, const void* Q, const void* K, const vo
                            const void* Vc, const int32_t* idx, const float* gates, void* O, void* ws,
                            cudaStream_t s, int* err);
 
+// Query-subspace basis from n query rows [n][d]: the eigenvectors of their second moment for the
+// m.sub largest eigenvalues, basis [d][m.sub] float32 (evals [m.sub], may be null).
+size_t basis_workspace_bytes(const Dims& m);
+cudaError_t launch_query_basis(const Dims& m, const void* Q, long long n, float* basis, float* evals, void* ws,
+                               cudaStream_t s);
+
 // Evaluation only: ln of the exact attention mass of every complete block, out [B, Hq, nB] f32
 // (cudaErrorNotSupported if G > 16).
 cudaError_t launch_block_log_mass(const Dims& m, const void* Q, const void* K, float* out, cudaStream_t s);

@@ -88,7 +88,8 @@ typedef enum {
     COBS_WS_DECODE = 1,
     COBS_WS_PREFILL = 2,
     COBS_WS_STEP = 3,      /* cobs_decode_step */
-    COBS_WS_STEP_FUSED = 4 /* cobs_decode_step_fused (0 bytes: a shape it does not take) */
+    COBS_WS_STEP_FUSED = 4, /* cobs_decode_step_fused (0 bytes: a shape it does not take) */
+    COBS_WS_BASIS = 5       /* cobs_query_basis */
 } cobs_workspace_kind;
 
 /* Second-order statistic kept per block ([COBS] §2.2/§2.3: the block covariance Sigma_b, compressed):
@@ -283,6 +284,29 @@ cobs_status cobs_sparse_attn_prefill(const cobs_params* p, const void* Q, const 
                                      const void* V, const void* Kc, const void* Vc,
                                      const int32_t* idx, const float* gates, void* O,
                                      void* workspace, size_t ws_bytes, cobs_stream_t stream);
+
+/*
+ * The query subspace for COBS_VAR_SUBSPACE(_FP4) from a sample of queries ([COBS] §2.3: the
+ * covariance is kept in the subspace spanned by the top eigenvectors of the queries' second
+ * moment). M = (1/n) sum_i q_i q_i^T over the n rows of Q [n, d] (storage type of p->dtype; any
+ * query vectors, for example a prefill's Q [B, T, Hq, d] as n = B T Hq rows), accumulated in
+ * float32 per range of rows and summed over the ranges in double; then a cyclic Jacobi
+ * eigendecomposition of M in float32 on the GPU.
+ *   basis       [d, p->sub] float32 (row-major, the layout of cobs_params.basis): the
+ *               eigenvectors of the p->sub largest eigenvalues as orthonormal columns, in
+ *               descending eigenvalue order, each with its largest-magnitude entry positive.
+ *   eigenvalues [p->sub] float32 in the same order, or NULL.
+ *   workspace   >= cobs_workspace_bytes(p, COBS_WS_BASIS) bytes (sized for the current
+ *               device's SM count); no initial contents are needed.
+ * Only p->d, p->dtype and p->sub are used (the rest must still validate). Errors:
+ * COBS_ERR_UNSUPPORTED unless p->sub is a multiple of 4 in 4 .. d; COBS_ERR_INVALID_ARG for
+ * n < 1 or NULL / misaligned pointers; COBS_ERR_WORKSPACE. Eigenvectors of eigenvalues that
+ * (nearly) coincide are any orthonormal basis of their eigenspace; the spanned subspace is
+ * well defined when the p->sub-th and (p->sub + 1)-th eigenvalues are apart.
+ */
+cobs_status cobs_query_basis(const cobs_params* p, const void* Q, int64_t n, float* basis,
+                             float* eigenvalues, void* workspace, size_t ws_bytes,
+                             cobs_stream_t stream);
 
 /*
  * Evaluation only (no step of the decode or prefill path calls it): the log of the exact
