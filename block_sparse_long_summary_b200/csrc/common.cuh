@@ -81,12 +81,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 #ifndef COBS_WAIT_TRY
 #define COBS_WAIT_TRY 1
 #endif
-#if COBS_WAIT_TRY
-// One hardware wait of at most about kSuspendHintNs: the warp is woken when the phase completes.
-constexpr uint32_t kSuspendHintNs = 1000;
 // Give up after this long (far above any legitimate wait of these kernels), or after
 // kMaxWaitIters hardware waits, whichever comes first.
 constexpr uint64_t kWaitLimitNs = 100000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+#if COBS_WAIT_TRY
+// One hardware wait of at most about kSuspendHintNs: the warp is woken when the phase completes.
+#ifndef COBS_SUSPEND_HINT_NS
+#define COBS_SUSPEND_HINT_NS 1000
+#endif
+constexpr uint32_t kSuspendHintNs = COBS_SUSPEND_HINT_NS;
 
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t done;
@@ -98,12 +108,6 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
         : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return done != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
