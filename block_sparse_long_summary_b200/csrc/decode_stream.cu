@@ -5,14 +5,15 @@
 // the window and the compressed tokens are read ("Problemstellung": decode is bound by the
 // KV-cache read). How it is scheduled:
 //
-// * Every (batch, KV-head) unit contributes its tiles in the order WIN (the window rows in
-//   32-row tiles), CMP (compressed tokens in 32-row tiles), SLC (2 tiles per selected
-//   block). The tiles of all units form one sequence that is cut into equal, contiguous
-//   ranges, one per warp, so every SM streams the same number of bytes.
+// * The tiles form two sequences: phase A, every (batch, KV-head) unit's WIN tiles (the window
+//   rows in 32-row tiles) then its CMP tiles (compressed tokens in 32-row tiles), unit after
+//   unit; phase B, every unit's SLC tiles (2 per selected block). Each phase is cut into
+//   equal, contiguous ranges, one per warp, and every warp streams its phase-A range and then
+//   its phase-B range, so every SM streams the same number of bytes in each phase.
 // * After a selection in the same stream (the decode step) the grid is launched as a
-//   programmatic dependent of the selection: the window and compressed-token tiles, which
-//   do not depend on it, stream while it finishes; a warp waits for the selection grid
-//   (griddepcontrol.wait) before it reads its first selected-block index.
+//   programmatic dependent of the selection: phase A, which does not depend on it, streams
+//   while the selection runs; a warp waits for the selection grid (griddepcontrol.wait)
+//   before it reads its first selected-block index.
 // * Each warp is its own producer: TMA 2-D loads (128-byte swizzle, no multicast) of the
 //   K and V halves of a tile into a private 2-stage ring, an mbarrier per stage (2 stages of
 //   16 KiB per warp: the 128 KiB a CTA holds leave room on the SM for the selection grid the
@@ -49,19 +50,21 @@ struct StreamArgs {
     float* rec;
     int* err;
     int Hq, Hkv, G, T, L, k, W, nB, nC;
-    int tS, tW, tC, tpu;  // tiles per unit: SLC, WIN, CMP, total
-    long long total;      // units * tpu
-    int tpw;              // tiles per warp
+    int tS, tW, tC, tAu;  // tiles per unit: SLC, WIN, CMP, WIN + CMP
+    long long nA, nBt;    // tiles of phase A (units * tAu) and phase B (units * tS)
+    int tpwA, tpwB;       // tiles per warp in each phase
     int maxw;             // record slots per (unit, branch)
     float sl2;            // log2(e) / sqrt(d)
 };
 
 __host__ __device__ __forceinline__ int rec_floats(int D) { return D + 4; }  // m, l, pad, pad, o[D]
 
-// Branch br's tiles within a unit: WIN [0, tW), CMP [tW, tW + tC), SLC [tW + tC, tpu).
-__host__ __device__ __forceinline__ int branch_begin(const StreamArgs& a, int br) {
-    return br == 1 ? 0 : (br == 2 ? a.tW : a.tW + a.tC);
+// First tile of (unit, br) in its phase's sequence and that phase's tiles per warp: WIN
+// [0, tW) and CMP [tW, tAu) of the unit's phase-A tiles, SLC [0, tS) of its phase-B tiles.
+__host__ __device__ __forceinline__ long long piece_begin(const StreamArgs& a, int unit, int br) {
+    return br == 0 ? (long long)unit * a.tS : (long long)unit * a.tAu + (br == 2 ? a.tW : 0);
 }
+__host__ __device__ __forceinline__ int phase_tpw(const StreamArgs& a, int br) { return br == 0 ? a.tpwB : a.tpwA; }
 __host__ __device__ __forceinline__ int branch_len(const StreamArgs& a, int br) {
     return br == 0 ? a.tS : (br == 1 ? a.tW : a.tC);
 }
@@ -72,19 +75,20 @@ struct Tile {
     uint32_t mask;     // valid keys of the tile
 };
 
-// Tile gt of the global sequence. Uniform across the warp. Before the first selected-block
-// index it reads, the warp waits for the grid it depends on (the selection), once.
+// Tile gt of the joint numbering (phase A in [0, nA), phase B from nA). Uniform across the
+// warp. Before the first selected-block index it reads, the warp waits for the grid it depends
+// on (the selection), once.
 __device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt, bool& waited) {
     Tile tl;
-    tl.unit = (int)(gt / a.tpu);
-    int l = (int)(gt - (long long)tl.unit * a.tpu);
     const int t = a.T - 1;
-    if (l >= a.tW + a.tC) {
+    if (gt >= a.nA) {
         if (!waited) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
             waited = true;
         }
-        l -= a.tW + a.tC;
+        const long long q = gt - a.nA;
+        tl.unit = (int)(q / a.tS);
+        const int l = (int)(q - (long long)tl.unit * a.tS);
         tl.br = 0;
         tl.j = l;
         const int bi = a.idx[(size_t)tl.unit * a.k + l / (64 / kTK)];
@@ -98,7 +102,11 @@ __device__ __forceinline__ Tile tile_at(const StreamArgs& a, long long gt, bool&
                 tl.mask = kTK == 32 ? kFull : 0xFFFFu;
             }
         }
-    } else if (l < a.tW) {
+        return tl;
+    }
+    tl.unit = (int)(gt / a.tAu);
+    const int l = (int)(gt - (long long)tl.unit * a.tAu);
+    if (l < a.tW) {
         tl.br = 1;
         tl.j = l;
         const int r0 = max(0, t - a.W + 1) + tl.j * kTK;
@@ -124,7 +132,7 @@ __device__ __forceinline__ void flush(const StreamArgs& a, long long v, int unit
     l0 += __shfl_xor_sync(kFull, l0, 2);
     l1 += __shfl_xor_sync(kFull, l1, 1);
     l1 += __shfl_xor_sync(kFull, l1, 2);
-    const long long first_v = ((long long)unit * a.tpu + branch_begin(a, br)) / a.tpw;
+    const long long first_v = piece_begin(a, unit, br) / phase_tpw(a, br);
     float* rec = a.rec + (((size_t)unit * 3 + br) * a.maxw + (size_t)(v - first_v)) * a.G * rec_floats(D);
     const int r0 = lane >> 2, r1 = r0 + 8, c = 2 * (lane & 3);
     if ((lane & 3) == 0) {
@@ -167,10 +175,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
     // the merge grid may be scheduled now; it still waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long v = (long long)blockIdx.x * kWarps + warp;
-    const long long g0 = v * a.tpw;
-    const long long g1 = min(a.total, g0 + a.tpw);
-    if (g0 >= g1) return;
-    const int n = (int)(g1 - g0);
+    // this warp's ranges: [a0, a0 + nAw) of phase A, then [b0, b0 + nBw) of phase B
+    const long long a0 = v * a.tpwA, b0 = v * a.tpwB;
+    const int nAw = (int)max(0LL, min(a.nA, a0 + a.tpwA) - a0);
+    const int nBw = (int)max(0LL, min(a.nBt, b0 + a.tpwB) - b0);
+    const int n = nAw + nBw;
+    if (n == 0) return;
+    auto gt_of = [&](int i) -> long long { return i < nAw ? a0 + i : a.nA + b0 + (i - nAw); };
 
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(&bar[s], 1);
@@ -195,7 +206,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
     Tile tq[kStages];
     bool waited = false;
 #pragma unroll
-    for (int j = 0; j < kStages; ++j) tq[j] = j < n ? tile_at(a, g0 + j, waited) : Tile{0, 0, 0, 0, 0u};
+    for (int j = 0; j < kStages; ++j) tq[j] = j < n ? tile_at(a, gt_of(j), waited) : Tile{0, 0, 0, 0, 0u};
     if (lane == 0) {
 #pragma unroll
         for (int j = 0; j < kStages; ++j)
@@ -215,7 +226,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
 #pragma unroll
         for (int j = 0; j + 1 < kStages; ++j) tq[j] = tq[j + 1];
         const bool more = i + kStages < n;
-        tq[kStages - 1] = more ? tile_at(a, g0 + i + kStages, waited) : Tile{0, 0, 0, 0, 0u};
+        tq[kStages - 1] = more ? tile_at(a, gt_of(i + kStages), waited) : Tile{0, 0, 0, 0, 0u};
         if (tl.unit != cur.unit || tl.br != cur.br) {
             flush<D>(a, v, cur.unit, cur.br, st, lane);
             st.init();
@@ -237,35 +248,41 @@ __global__ void __launch_bounds__(kWarps * 32) decode_stream_kernel(const __grid
     flush<D>(a, v, cur.unit, cur.br, st, lane);
 }
 
-// grid (G, units), 4 warps. Warp 0 folds the SLC records of the (unit, head), warp 1 the WIN
-// records, warps 2 and 3 the even and odd CMP records; each warp issues the loads of 4 records
-// at a time. Warp 0 then combines, applies the gates (cmp, slc, win) and writes O. Launched as a
-// programmatic dependent of the decode kernel: it waits for that grid before reading records.
+// grid (G, units), 8 warps per (unit, head): warps 0-2 fold the SLC records (every third slot),
+// warp 3 the WIN records, warps 4-7 the CMP records (every fourth slot); each warp keeps the
+// loads of 8 records in flight. Warp 0 then combines the warps of each branch, applies the
+// gates (cmp, slc, win) and writes O. Launched as a programmatic dependent of the decode
+// kernel: it waits for that grid before reading records.
+constexpr int kMergeWarps = 8;
+constexpr int kMergeBatch = 8;
+__host__ __device__ __forceinline__ int merge_branch(int w) { return w < 3 ? 0 : (w == 3 ? 1 : 2); }
+
 template <int D>
-__global__ void __launch_bounds__(128) decode_stream_merge(StreamArgs a) {
+__global__ void __launch_bounds__(kMergeWarps * 32) decode_stream_merge(StreamArgs a) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float wM[4], wL[4];
-    __shared__ float wO[4][D];
+    __shared__ float wM[kMergeWarps], wL[kMergeWarps];
+    __shared__ float wO[kMergeWarps][D];
     const int h = blockIdx.x, unit = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int hq_row = unit * a.G + h;  // = b * Hq + g * G + h
     const int c0 = lane * 4;
-    const int br = warp < 2 ? warp : 2;
+    const int br = merge_branch(warp);
     const int len = branch_len(a, br);
     int nslots = 0;
     if (len > 0) {
-        const long long s0 = (long long)unit * a.tpu + branch_begin(a, br);
-        nslots = (int)((s0 + len - 1) / a.tpw - s0 / a.tpw) + 1;
+        const long long s0 = piece_begin(a, unit, br);
+        const int tpw = phase_tpw(a, br);
+        nslots = (int)((s0 + len - 1) / tpw - s0 / tpw) + 1;
     }
-    const int sl0 = warp < 2 ? 0 : warp - 2, step = warp < 2 ? 1 : 2;
+    const int sl0 = br == 0 ? warp : (br == 1 ? 0 : warp - 4), step = br == 0 ? 3 : (br == 1 ? 1 : 4);
     const float* base = a.rec + ((size_t)unit * 3 + br) * a.maxw * a.G * rec_floats(D) + (size_t)h * rec_floats(D);
     const size_t rs = (size_t)a.G * rec_floats(D);
     float M = -INFINITY, Lsum = 0.0f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int sl = sl0; sl < nslots; sl += 4 * step) {
-        float m[4], l[4];
-        float4 o[4];
+    for (int sl = sl0; sl < nslots; sl += kMergeBatch * step) {
+        float m[kMergeBatch], l[kMergeBatch];
+        float4 o[kMergeBatch];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < kMergeBatch; ++q) {
             const int s = sl + q * step;
             m[q] = -INFINITY;
             l[q] = 0.0f;
@@ -278,7 +295,7 @@ __global__ void __launch_bounds__(128) decode_stream_merge(StreamArgs a) {
             }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < kMergeBatch; ++q) {
             if (m[q] == -INFINITY) continue;
             const float nM = fmaxf(M, m[q]);
             const float fa = M == -INFINITY ? 0.0f : exp2f(M - nM);  // maxima are in log2 units
@@ -301,18 +318,22 @@ __global__ void __launch_bounds__(128) decode_stream_merge(StreamArgs a) {
     if (warp != 0 || c0 >= D) return;
     const float* gate = a.gates + (size_t)hq_row * 3;
     float out[4] = {0.f, 0.f, 0.f, 0.f};
-    // branch results: SLC = warp 0, WIN = warp 1, CMP = warps 2 + 3
+    // branch results: SLC = warps 0-2, WIN = warp 3, CMP = warps 4-7
     for (int b2 = 0; b2 < 3; ++b2) {
-        const int w0 = b2, w1 = b2 == 2 ? 3 : b2;
-        const float GM = fmaxf(wM[w0], wM[w1]);
+        const int w0 = b2 == 0 ? 0 : (b2 == 1 ? 3 : 4), w1 = b2 == 0 ? 3 : (b2 == 1 ? 4 : kMergeWarps);
+        float GM = -INFINITY;
+        for (int w = w0; w < w1; ++w) GM = fmaxf(GM, wM[w]);
         if (GM == -INFINITY) continue;
-        const float f0 = wM[w0] == -INFINITY ? 0.0f : exp2f(wM[w0] - GM);
-        const float f1 = (w1 == w0 || wM[w1] == -INFINITY) ? 0.0f : exp2f(wM[w1] - GM);
-        const float GL = wL[w0] * f0 + (w1 == w0 ? 0.0f : wL[w1] * f1);
+        float GL = 0.0f, ob[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int w = w0; w < w1; ++w) {
+            if (wM[w] == -INFINITY) continue;
+            const float f = exp2f(wM[w] - GM);
+            GL += wL[w] * f;
+            for (int j = 0; j < 4; ++j) ob[j] += wO[w][c0 + j] * f;
+        }
         if (!(GL > 0.0f)) continue;
         const float gw = gate[b2 == 0 ? 1 : (b2 == 1 ? 2 : 0)] / GL;  // gates are (cmp, slc, win)
-        for (int j = 0; j < 4; ++j)
-            out[j] += gw * (wO[w0][c0 + j] * f0 + (w1 == w0 ? 0.0f : wO[w1][c0 + j] * f1));
+        for (int j = 0; j < 4; ++j) out[j] += gw * ob[j];
     }
     __nv_bfloat16* o = a.O + (size_t)hq_row * D + c0;
     for (int j = 0; j < 4; ++j) o[j] = __float2bfloat16_rn(out[j]);
@@ -324,11 +345,14 @@ StreamArgs make_stream_args(const Dims& m) {
     a.tS = m.k * (m.L / kTK);
     a.tW = (std::min(m.W, m.T) + kTK - 1) / kTK;
     a.tC = (m.nC + kTK - 1) / kTK;
-    a.tpu = a.tS + a.tW + a.tC;
-    a.total = (long long)m.units() * a.tpu;
+    a.tAu = a.tW + a.tC;
+    a.nA = (long long)m.units() * a.tAu;
+    a.nBt = (long long)m.units() * a.tS;
     const long long warps_wanted = (long long)sm_count() * kWarps;
-    a.tpw = (int)std::max<long long>(1, (a.total + warps_wanted - 1) / warps_wanted);
-    a.maxw = std::max(a.tS, std::max(a.tW, a.tC)) / a.tpw + 2;
+    a.tpwA = (int)std::max<long long>(1, (a.nA + warps_wanted - 1) / warps_wanted);
+    a.tpwB = (int)std::max<long long>(1, (a.nBt + warps_wanted - 1) / warps_wanted);
+    // pieces of one (unit, branch): at most len / tpw + 2 warps meet its tiles
+    a.maxw = std::max(a.tS / a.tpwB, std::max(a.tW, a.tC) / a.tpwA) + 2;
     a.sl2 = 1.4426950408889634f / sqrtf((float)m.d);
     return a;
 }
@@ -349,7 +373,7 @@ cudaError_t launch_stream_d(const Dims& m, StreamArgs a, const void* K, const vo
     const size_t smem = stream_smem<D>();
     cudaError_t e = cudaFuncSetAttribute(decode_stream_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const long long nwarps = (a.total + a.tpw - 1) / a.tpw;
+    const long long nwarps = std::max((a.nA + a.tpwA - 1) / a.tpwA, (a.nBt + a.tpwB - 1) / a.tpwB);
     const int grid = (int)((nwarps + kWarps - 1) / kWarps);
     {
         cudaLaunchConfig_t cfg = {};
@@ -369,7 +393,7 @@ cudaError_t launch_stream_d(const Dims& m, StreamArgs a, const void* K, const vo
     // the merge grid may launch while the decode grid drains; it waits for it on the device
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(m.G, m.units());
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(kMergeWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
