@@ -86,9 +86,56 @@ __global__ void __launch_bounds__(128) summaries_kernel(const T* __restrict__ K,
 //   channels l, l + 32, ... with fma, then a five-level xor butterfly of adds), V = W;
 //   then T = Y V and lambda_j = (four-chain sum of T[., j]^2) / L, pairs ordered by lambda
 //   descending (ties: lower j).
-// grid (blocks to build, units), D threads (thread = channel).
+// grid (blocks to build, units), kLrThreads threads: thread c < D owns channel c for the mean and
+// the outputs; in the products T = Y V and W = Y^T T a thread takes one chain of one row of Y
+// (or column of Y) against all R columns, the four chains in four neighbouring lanes, combined
+// by two shuffles in the canonical order (s0 + s1) + (s2 + s3); one warp orthonormalises.
 constexpr int kLrIters = 24;
 constexpr int kLrMaxR = 8;
+constexpr int kLrThreads = 512;
+constexpr int kLrPitch = 4;  // Y rows padded by 4 floats: the lanes of a product read distinct banks
+
+// Chain q of the four-chain dots of one row x (stride sx) against the R columns of a
+// row-major [n][kLrMaxR] matrix y (16-byte aligned rows): s[jj] = fma over the terms i = q,
+// q + 4, ... below n in ascending order, from +0. Then the chains of the four neighbouring
+// lanes q = 0..3 are combined as (s0 + s1) + (s2 + s3): every lane of the quad ends with the
+// same values as lr_dot4(x, y + jj, n, sx, kLrMaxR).
+__device__ __forceinline__ void lr_quad_dots(const float* x, const float* y, int n, int sx, int q, int R,
+                                             float (&s)[kLrMaxR]) {
+#pragma unroll
+    for (int jj = 0; jj < kLrMaxR; ++jj) s[jj] = 0.0f;
+    if (R <= 4) {
+#pragma unroll 4
+        for (int i = q; i < n; i += 4) {
+            const float xv = x[i * sx];
+            const float4 a = *reinterpret_cast<const float4*>(y + i * kLrMaxR);
+            s[0] = __fmaf_rn(xv, a.x, s[0]);
+            s[1] = __fmaf_rn(xv, a.y, s[1]);
+            s[2] = __fmaf_rn(xv, a.z, s[2]);
+            s[3] = __fmaf_rn(xv, a.w, s[3]);
+        }
+    } else {
+#pragma unroll 4
+        for (int i = q; i < n; i += 4) {
+            const float xv = x[i * sx];
+            const float4 a = *reinterpret_cast<const float4*>(y + i * kLrMaxR);
+            const float4 b = *reinterpret_cast<const float4*>(y + i * kLrMaxR + 4);
+            s[0] = __fmaf_rn(xv, a.x, s[0]);
+            s[1] = __fmaf_rn(xv, a.y, s[1]);
+            s[2] = __fmaf_rn(xv, a.z, s[2]);
+            s[3] = __fmaf_rn(xv, a.w, s[3]);
+            s[4] = __fmaf_rn(xv, b.x, s[4]);
+            s[5] = __fmaf_rn(xv, b.y, s[5]);
+            s[6] = __fmaf_rn(xv, b.z, s[6]);
+            s[7] = __fmaf_rn(xv, b.w, s[7]);
+        }
+    }
+#pragma unroll
+    for (int jj = 0; jj < kLrMaxR; ++jj) {
+        const float v = __fadd_rn(s[jj], __shfl_xor_sync(0xffffffffu, s[jj], 1));  // s0 + s1, s2 + s3
+        s[jj] = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 2));                 // (s0 + s1) + (s2 + s3)
+    }
+}
 
 __device__ __forceinline__ float lr_v0(int c, int j) {
     const uint32_t h = (uint32_t)c * 2654435761u + (uint32_t)(j + 1) * 40503u;
@@ -126,74 +173,121 @@ __device__ __forceinline__ int e2m1_code(float x) {
     return best == 0 ? 0 : ((x < 0.0f ? 8 : 0) | best);
 }
 
+// Modified Gram-Schmidt of the R columns of W[D][kLrMaxR + 1] into V[D][kLrMaxR], by one warp holding every
+// column in registers (lane l: channels l, l + 32, ...). Each "32-lane" dot sums its lane's
+// channels in ascending order with fma, then adds across lanes by a five-level xor butterfly;
+// column i is normalised (sqrt, divide; zero if its norm is zero) once the projections on the
+// columns before it are removed, and then its projection is removed from every later column.
+// Every column sees the same operations in the same order as in the column-by-column form
+// (projections on columns 0, 1, ... in turn, then the normalisation), so the result is the
+// same bit for bit; the dots of the later columns against column i are independent, so their
+// butterflies run side by side.
+template <int D>
+__device__ __forceinline__ void lr_orthonormalize(const float (*W)[kLrMaxR + 1], float (*V)[kLrMaxR], int R,
+                                                  int lane) {
+    constexpr int kPer = D / 32;
+    float w[kLrMaxR][kPer];
+#pragma unroll
+    for (int jj = 0; jj < kLrMaxR; ++jj)
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) w[jj][q] = jj < R ? W[lane + 32 * q][jj] : 0.0f;
+#pragma unroll
+    for (int i = 0; i < kLrMaxR; ++i) {
+        if (i >= R) break;
+        float nn = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) nn = __fmaf_rn(w[i][q], w[i][q], nn);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) nn = __fadd_rn(nn, __shfl_xor_sync(0xffffffffu, nn, o));
+        const float n = __fsqrt_rn(nn);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) w[i][q] = n > 0.0f ? __fdiv_rn(w[i][q], n) : 0.0f;
+        float p[kLrMaxR];
+#pragma unroll
+        for (int jj = i + 1; jj < kLrMaxR; ++jj) {
+            p[jj] = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) p[jj] = __fmaf_rn(w[i][q], w[jj][q], p[jj]);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int jj = i + 1; jj < kLrMaxR; ++jj) p[jj] = __fadd_rn(p[jj], __shfl_xor_sync(0xffffffffu, p[jj], o));
+#pragma unroll
+        for (int jj = i + 1; jj < kLrMaxR; ++jj)
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) w[jj][q] = __fmaf_rn(-p[jj], w[i][q], w[jj][q]);
+    }
+#pragma unroll
+    for (int jj = 0; jj < kLrMaxR; ++jj)
+#pragma unroll
+        for (int q = 0; q < kPer; ++q)
+            if (jj < R) V[lane + 32 * q][jj] = w[jj][q];
+}
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
+__global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
                                                     int fp4, const float* __restrict__ Pb, int S,
                                                     float* __restrict__ summ) {
-    __shared__ float Y[kBlock][D + 1];  // +1: rows on different banks
-    // rows of kLrMaxR + 1 floats: thread c's row starts on bank 9c mod 32, so the per-thread row
-    // accesses of a warp are free of bank conflicts
-    __shared__ float V[D][kLrMaxR + 1], W[D][kLrMaxR + 1];
-    __shared__ float Tm[kBlock][kLrMaxR];
-    __shared__ float bcast;
+    __shared__ float Y[kBlock][D + kLrPitch];
+    // W: rows of kLrMaxR + 1 floats (lane l's row starts on bank 9 l mod 32: the orthonormalising
+    // warp reads it free of bank conflicts); V and T: 16-byte aligned rows of kLrMaxR floats,
+    // read a row at a time by the products
+    __shared__ float W[D][kLrMaxR + 1];
+    __shared__ __align__(16) float V[D][kLrMaxR];
+    __shared__ __align__(16) float Tm[kBlock][kLrMaxR];
     __shared__ int ord_sh[kLrMaxR];
     __shared__ float lam_sh[kLrMaxR];
     __shared__ float red[D];
     __shared__ int code_sh[D];
     const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+    const bool ch = c < D;  // this thread owns channel c
     const int unit = blockIdx.y;
     const int j = j_begin + blockIdx.x;
-    float mu_c;
-    // canonical mean of channel c (rows ascending), then the centred rows
+    float mu_c = 0.0f;
+    // the block's rows (as float) staged in Y by every thread, coalesced
     {
-        const T* rows = K + ((size_t)unit * Tctx + (size_t)j * kBlock) * D + c;
-        float x[kBlock];
-#pragma unroll
-        for (int r = 0; r < kBlock; ++r) x[r] = Elem<T>::load(rows + (size_t)r * D);
+        const T* rows = K + ((size_t)unit * Tctx + (size_t)j * kBlock) * D;
+        for (int e = c; e < kBlock * D; e += kLrThreads) Y[e / D][e % D] = Elem<T>::load(rows + e);
+    }
+    __syncthreads();
+    // canonical mean of channel c (rows ascending), then the centred rows
+    if (ch) {
         float sum = 0.0f;
-#pragma unroll
-        for (int r = 0; r < kBlock; ++r) sum = __fadd_rn(sum, x[r]);
+#pragma unroll 16
+        for (int r = 0; r < kBlock; ++r) sum = __fadd_rn(sum, Y[r][c]);
         const float mu = __fmul_rn(sum, 1.0f / kBlock);
-#pragma unroll
-        for (int r = 0; r < kBlock; ++r) Y[r][c] = __fsub_rn(x[r], mu);
+#pragma unroll 16
+        for (int r = 0; r < kBlock; ++r) Y[r][c] = __fsub_rn(Y[r][c], mu);
         mu_c = mu;
         for (int jj = 0; jj < R; ++jj) V[c][jj] = lr_v0(c, jj);
     }
     __syncthreads();
-    // "32-lane" dot of columns a and b of W (warp 0 computes, every thread reads the result)
-    auto wdot = [&](int a, int b) -> float {
-        if (warp == 0) {
-            float p = 0.0f;
-            for (int cc = lane; cc < D; cc += 32) p = __fmaf_rn(W[cc][a], W[cc][b], p);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
-            if (lane == 0) bcast = p;
-        }
-        __syncthreads();
-        const float v = bcast;
-        __syncthreads();
-        return v;
-    };
     for (int it = 0; it <= kLrIters; ++it) {
-        for (int o = c; o < kBlock * R; o += D) {
-            const int r = o / R, jj = o % R;
-            Tm[r][jj] = lr_dot4(&Y[r][0], &V[0][jj], D, 1, kLrMaxR + 1);
+        // T[r][.] = four-chain dots over the channels of row r of Y and the columns of V (threads
+        // 4 r + q, whole warps)
+        if (c < 4 * kBlock) {
+            float sv[kLrMaxR];
+            lr_quad_dots(&Y[c >> 2][0], &V[0][0], D, 1, c & 3, R, sv);
+            if ((c & 3) == 0)
+#pragma unroll
+                for (int jj = 0; jj < kLrMaxR; ++jj)
+                    if (jj < R) Tm[c >> 2][jj] = sv[jj];
         }
         __syncthreads();
         if (it == kLrIters) break;
-        for (int jj = 0; jj < R; ++jj) W[c][jj] = lr_dot4(&Y[0][c], &Tm[0][jj], kBlock, D + 1, kLrMaxR);
-        __syncthreads();
-        for (int jj = 0; jj < R; ++jj) {
-            for (int i = 0; i < jj; ++i) {
-                const float p = wdot(i, jj);
-                W[c][jj] = __fmaf_rn(-p, W[c][i], W[c][jj]);
-                __syncthreads();
-            }
-            const float n = __fsqrt_rn(wdot(jj, jj));
-            W[c][jj] = n > 0.0f ? __fdiv_rn(W[c][jj], n) : 0.0f;
-            __syncthreads();
+        // W[cc][.] = four-chain dots over the rows of column cc of Y and the columns of T
+        // (threads 4 cc + q, whole warps)
+        if (c < 4 * D) {
+            float sw[kLrMaxR];
+            lr_quad_dots(&Y[0][c >> 2], &Tm[0][0], kBlock, D + kLrPitch, c & 3, R, sw);
+            if ((c & 3) == 0)
+#pragma unroll
+                for (int jj = 0; jj < kLrMaxR; ++jj)
+                    if (jj < R) W[c >> 2][jj] = sw[jj];
         }
-        for (int jj = 0; jj < R; ++jj) V[c][jj] = W[c][jj];
+        __syncthreads();
+        if (warp == 0) lr_orthonormalize<D>(W, V, R, lane);
         __syncthreads();
     }
     if (c < R) lam_sh[c] = __fmul_rn(lr_dot4(&Tm[0][c], &Tm[0][c], kBlock, kLrMaxR, kLrMaxR), 1.0f / kBlock);
@@ -217,11 +311,11 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
         // (i < S), in the [S/4][32][4] interleaving
         const size_t gf = (size_t)32 * (D + R * S + R);
         float* base = summ + ((size_t)unit * nG + (size_t)(j >> 5)) * gf;
-        base[((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = mu_c;
-        for (int o = c; o < R * S; o += D) {
+        if (ch) base[((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = mu_c;
+        for (int o = c; o < R * S; o += kLrThreads) {
             const int jj = o / S, i = o % S;
             base[(size_t)32 * D + (size_t)jj * S * 32 + ((size_t)(i / 4) * 32 + ln) * 4 + (i & 3)] =
-                lr_dot4(Pb + i, &V[0][ord_sh[jj]], D, S, kLrMaxR + 1);
+                lr_dot4(Pb + i, &V[0][ord_sh[jj]], D, S, kLrMaxR);
         }
         if (c < R) base[(size_t)32 * (D + R * S) + (size_t)c * 32 + ln] = lam_sh[ord_sh[c]];
         return;
@@ -229,6 +323,7 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
     if (!fp4) {
         const size_t gf = (size_t)32 * (D + R * D + R);
         float* base = summ + (size_t)unit * nG * gf + (size_t)(j >> 5) * gf;
+        if (!ch) return;
         base[((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = mu_c;
         for (int jj = 0; jj < R; ++jj)
             base[(size_t)(1 + jj) * D * 32 + ((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = V[c][ord_sh[jj]];
@@ -242,21 +337,24 @@ __global__ void __launch_bounds__(D) lowrank_kernel(const T* __restrict__ K, int
     const int CW = S > 0 ? (S + 31) / 32 * 32 : D;
     const size_t gbytes = (size_t)32 * (2 * D + R * CW / 2 + 8 * R);
     unsigned char* g8 = reinterpret_cast<unsigned char*>(summ) + ((size_t)unit * nG + (size_t)(j >> 5)) * gbytes;
-    const __nv_bfloat16 mb = __float2bfloat16_rn(mu_c);
-    *reinterpret_cast<__nv_bfloat16*>(g8 + ((size_t)(c / 8) * 32 + ln) * 16 + (c % 8) * 2) = mb;
+    if (ch) {
+        const __nv_bfloat16 mb = __float2bfloat16_rn(mu_c);
+        *reinterpret_cast<__nv_bfloat16*>(g8 + ((size_t)(c / 8) * 32 + ln) * 16 + (c % 8) * 2) = mb;
+    }
     float* scl = reinterpret_cast<float*>(g8 + (size_t)64 * D + (size_t)R * 16 * CW);
     float* lamo = scl + R * 32;
-    const bool live = S == 0 || c < S;  // thread c holds an entry of the vector
+    const bool live = ch && (S == 0 || c < S);  // thread c holds an entry of the vector
     for (int jj = 0; jj < R; ++jj) {
-        const float x = S == 0 ? V[c][ord_sh[jj]] : (live ? lr_dot4(Pb + c, &V[0][ord_sh[jj]], D, S, kLrMaxR + 1) : 0.0f);
-        red[c] = fabsf(x);
+        const float x = !live ? 0.0f
+                        : S == 0 ? V[c][ord_sh[jj]] : lr_dot4(Pb + c, &V[0][ord_sh[jj]], D, S, kLrMaxR);
+        if (ch) red[c] = fabsf(x);
         __syncthreads();
         for (int o = D / 2; o > 0; o >>= 1) {  // max is exact in any order
             if (c < o) red[c] = fmaxf(red[c], red[c + o]);
             __syncthreads();
         }
         const float sc = __fdiv_rn(red[0], 6.0f);
-        code_sh[c] = live && sc > 0.0f ? e2m1_code(__fdiv_rn(x, sc)) : 0;
+        if (ch) code_sh[c] = live && sc > 0.0f ? e2m1_code(__fdiv_rn(x, sc)) : 0;
         __syncthreads();
         if ((c & 1) == 0 && c < CW)
             g8[(size_t)64 * D + (size_t)jj * 16 * CW + ((size_t)(c / 32) * 32 + ln) * 16 + (c % 32) / 2] =
@@ -669,10 +767,10 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
         count_launch();
         if (m.lr) {
             if (m.d == 128)
-                lowrank_kernel<T, 128><<<dim3(nbuild, units), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                lowrank_kernel<T, 128><<<dim3(nbuild, units), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
                     m.basis, m.sub, summ);
             else
-                lowrank_kernel<T, 64><<<dim3(nbuild, units), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                lowrank_kernel<T, 64><<<dim3(nbuild, units), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
                     m.basis, m.sub, summ);
         } else {
             summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
@@ -722,10 +820,10 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
     if (nj > 0 && m.lr) {
         count_launch();
         if (m.d == 128)
-            lowrank_kernel<T, 128><<<dim3(1, m.units()), 128, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+            lowrank_kernel<T, 128><<<dim3(1, m.units()), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
                 m.basis, m.sub, summ);
         else
-            lowrank_kernel<T, 64><<<dim3(1, m.units()), 64, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+            lowrank_kernel<T, 64><<<dim3(1, m.units()), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
                 m.basis, m.sub, summ);
         *e = cudaGetLastError();
     }
