@@ -86,13 +86,16 @@ __global__ void __launch_bounds__(128) summaries_kernel(const T* __restrict__ K,
 //   channels l, l + 32, ... with fma, then a five-level xor butterfly of adds), V = W;
 //   then T = Y V and lambda_j = (four-chain sum of T[., j]^2) / L, pairs ordered by lambda
 //   descending (ties: lower j).
-// grid (blocks to build, units), kLrThreads threads: thread c < D owns channel c for the mean and
+// grid (blocks to build, units), NT threads (kLrThreadsWide for a few blocks, where the latency of
+// one block is the cost; kLrThreadsNarrow for many, where several CTAs share an SM): thread c < D
+// owns channel c for the mean and
 // the outputs; in the products T = Y V and W = Y^T T a thread takes one chain of one row of Y
 // (or column of Y) against all R columns, the four chains in four neighbouring lanes, combined
 // by two shuffles in the canonical order (s0 + s1) + (s2 + s3); one warp orthonormalises.
 constexpr int kLrIters = 24;
 constexpr int kLrMaxR = 8;
-constexpr int kLrThreads = 512;
+constexpr int kLrThreadsWide = 512;
+constexpr int kLrThreadsNarrow = 128;
 constexpr int kLrPitch = 4;  // Y rows padded by 4 floats: the lanes of a product read distinct banks
 
 // Chain q of the four-chain dots of one row x (stride sx) against the R columns of a
@@ -225,8 +228,8 @@ __device__ __forceinline__ void lr_orthonormalize(const float (*W)[kLrMaxR + 1],
             if (jj < R) V[lane + 32 * q][jj] = w[jj][q];
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
+template <typename T, int D, int NT>
+__global__ void __launch_bounds__(NT, 1) lowrank_kernel(const T* __restrict__ K, int Tctx, int nG, int j_begin, int R,
                                                     int fp4, const float* __restrict__ Pb, int S,
                                                     float* __restrict__ summ) {
     __shared__ float Y[kBlock][D + kLrPitch];
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const T* __restr
     // the block's rows (as float) staged in Y by every thread, coalesced
     {
         const T* rows = K + ((size_t)unit * Tctx + (size_t)j * kBlock) * D;
-        for (int e = c; e < kBlock * D; e += kLrThreads) Y[e / D][e % D] = Elem<T>::load(rows + e);
+        for (int e = c; e < kBlock * D; e += NT) Y[e / D][e % D] = Elem<T>::load(rows + e);
     }
     __syncthreads();
     // canonical mean of channel c (rows ascending), then the centred rows
@@ -264,27 +267,27 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const T* __restr
     }
     __syncthreads();
     for (int it = 0; it <= kLrIters; ++it) {
-        // T[r][.] = four-chain dots over the channels of row r of Y and the columns of V (threads
-        // 4 r + q, whole warps)
-        if (c < 4 * kBlock) {
+        // T[r][.] = four-chain dots over the channels of row r of Y and the columns of V (tasks
+        // 4 r + q; NT and 4 L are multiples of 32, so whole warps take whole quads)
+        for (int t = c; t < 4 * kBlock; t += NT) {
             float sv[kLrMaxR];
-            lr_quad_dots(&Y[c >> 2][0], &V[0][0], D, 1, c & 3, R, sv);
-            if ((c & 3) == 0)
+            lr_quad_dots(&Y[t >> 2][0], &V[0][0], D, 1, t & 3, R, sv);
+            if ((t & 3) == 0)
 #pragma unroll
                 for (int jj = 0; jj < kLrMaxR; ++jj)
-                    if (jj < R) Tm[c >> 2][jj] = sv[jj];
+                    if (jj < R) Tm[t >> 2][jj] = sv[jj];
         }
         __syncthreads();
         if (it == kLrIters) break;
         // W[cc][.] = four-chain dots over the rows of column cc of Y and the columns of T
-        // (threads 4 cc + q, whole warps)
-        if (c < 4 * D) {
+        // (tasks 4 cc + q)
+        for (int t = c; t < 4 * D; t += NT) {
             float sw[kLrMaxR];
-            lr_quad_dots(&Y[0][c >> 2], &Tm[0][0], kBlock, D + kLrPitch, c & 3, R, sw);
-            if ((c & 3) == 0)
+            lr_quad_dots(&Y[0][t >> 2], &Tm[0][0], kBlock, D + kLrPitch, t & 3, R, sw);
+            if ((t & 3) == 0)
 #pragma unroll
                 for (int jj = 0; jj < kLrMaxR; ++jj)
-                    if (jj < R) W[c >> 2][jj] = sw[jj];
+                    if (jj < R) W[t >> 2][jj] = sw[jj];
         }
         __syncthreads();
         if (warp == 0) lr_orthonormalize<D>(W, V, R, lane);
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kLrThreads, 1) lowrank_kernel(const T* __restr
         const size_t gf = (size_t)32 * (D + R * S + R);
         float* base = summ + ((size_t)unit * nG + (size_t)(j >> 5)) * gf;
         if (ch) base[((size_t)(c / 4) * 32 + ln) * 4 + (c & 3)] = mu_c;
-        for (int o = c; o < R * S; o += kLrThreads) {
+        for (int o = c; o < R * S; o += NT) {
             const int jj = o / S, i = o % S;
             base[(size_t)32 * D + (size_t)jj * S * 32 + ((size_t)(i / 4) * 32 + ln) * 4 + (i & 3)] =
                 lr_dot4(Pb + i, &V[0][ord_sh[jj]], D, S, kLrMaxR);
@@ -756,6 +759,29 @@ __global__ void __launch_bounds__(256) append_kernel(const T* __restrict__ K, co
     }
 }
 
+// The low-rank summaries of blocks [j_begin, j_begin + nbuild) of every unit: wide CTAs while the
+// grid leaves SMs idle (the decode step's one block per unit), narrow ones, several per SM, else.
+template <typename T>
+void launch_lowrank(const Dims& m, const T* K, int nbuild, int j_begin, float* summ, cudaStream_t s) {
+    const dim3 grid(nbuild, m.units());
+    const bool wide = (long long)nbuild * m.units() < (long long)sm_count();
+    if (m.d == 128) {
+        if (wide)
+            lowrank_kernel<T, 128, kLrThreadsWide><<<grid, kLrThreadsWide, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                                                                                m.basis, m.sub, summ);
+        else
+            lowrank_kernel<T, 128, kLrThreadsNarrow><<<grid, kLrThreadsNarrow, 0, s>>>(K, m.T, m.nG, j_begin, m.lr,
+                                                                                    m.fp4, m.basis, m.sub, summ);
+    } else {
+        if (wide)
+            lowrank_kernel<T, 64, kLrThreadsWide><<<grid, kLrThreadsWide, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
+                                                                               m.basis, m.sub, summ);
+        else
+            lowrank_kernel<T, 64, kLrThreadsNarrow><<<grid, kLrThreadsNarrow, 0, s>>>(K, m.T, m.nG, j_begin, m.lr,
+                                                                                   m.fp4, m.basis, m.sub, summ);
+    }
+}
+
 template <typename T>
 cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const float* Pk, const float* Pv,
                                int t_begin, float* summ, T* Kc, T* Vc, cudaStream_t s) {
@@ -766,12 +792,7 @@ cudaError_t launch_summaries_t(const Dims& m, const T* K, const T* V, const floa
     if (nbuild > 0) {
         count_launch();
         if (m.lr) {
-            if (m.d == 128)
-                lowrank_kernel<T, 128><<<dim3(nbuild, units), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
-                    m.basis, m.sub, summ);
-            else
-                lowrank_kernel<T, 64><<<dim3(nbuild, units), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
-                    m.basis, m.sub, summ);
+            launch_lowrank(m, K, nbuild, j_begin, summ, s);
         } else {
             summaries_kernel<T><<<dim3(nbuild, units), m.d, 0, s>>>(K, m.T, m.d, m.nG, j_begin, m.iso, summ);
         }
@@ -819,12 +840,7 @@ bool try_append(const Dims& m, const T* K, const T* V, const float* Pk, const fl
     }
     if (nj > 0 && m.lr) {
         count_launch();
-        if (m.d == 128)
-            lowrank_kernel<T, 128><<<dim3(1, m.units()), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
-                m.basis, m.sub, summ);
-        else
-            lowrank_kernel<T, 64><<<dim3(1, m.units()), kLrThreads, 0, s>>>(K, m.T, m.nG, j_begin, m.lr, m.fp4,
-                m.basis, m.sub, summ);
+        launch_lowrank(m, K, 1, j_begin, summ, s);
         *e = cudaGetLastError();
     }
     return true;
