@@ -110,16 +110,16 @@ def source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
+def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on the
-    current sources (else None)."""
+    current sources and on `workload` (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel)
-    if not ent or ent.get("source_hash") != source_hash(kernel):
+    if not ent or ent.get("source_hash") != source_hash(kernel) or ent.get("workload") != workload:
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -439,7 +439,7 @@ def bench_prefill(w, steps, warmup, dev, cobs):
         # the burst peak; the sustained one beside it
         "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": att_tf, "peak": burst,
                      "unit": "TFLOP/s", "frac": att_tf / burst, "peak_kind": f"{kind} burst bf16",
-                     "frac_of_sustained": att_tf / sustained, "traffic": recorded_traffic("prefill_tc")},
+                     "frac_of_sustained": att_tf / sustained, "traffic": recorded_traffic("prefill_tc", traffic_key(w))},
         "summary_build_gbs": (kv_bytes + buf.summaries.numel() * 4 + 2 * buf.Kc.numel() * 2) / (t_sum * 1e-3) / 1e9,
         "gpu_launches": launches,
         "steps": steps,
@@ -703,7 +703,12 @@ def oracle_parity(w, idx_g, O_g, res_units, tol):
             "fp64_near_ties": len(gaps), "fp64_near_tie_max_rel_gap": max(gaps) if gaps else None}
 
 
-def decode_roofline(by, m, peak, peak_kind):
+def traffic_key(w) -> str:
+    """The workload a recorded ncu capture must have been taken on to stand for this run."""
+    return f"{w.name} B={w.B} T={w.T}"
+
+
+def decode_roofline(by, m, peak, peak_kind, workload):
     """Roofline of the step's dominant kernel, the three-branch decode attention (the largest share
     of the step's bytes), timed alone."""
     att_gbs = by["attn"] / (m["t_att"] * 1e-3) / 1e9
@@ -712,7 +717,7 @@ def decode_roofline(by, m, peak, peak_kind):
             "peak_kind": f"{peak_kind} (copy, read + write)", "algorithmic_bytes_per_launch": by["attn"],
             "timing": "CUDA events around cobs_sparse_attn_decode alone (graph per copy, replayed on the "
                       "launching stream, median)",
-            "traffic": recorded_traffic("decode_attention")}
+            "traffic": recorded_traffic("decode_attention", workload)}
 
 
 def decode_calls(by, m, peak):
@@ -741,7 +746,7 @@ def decode_subrecord(name, args, dev, cobs, world, steps=50, warmup=5, R=4):
     rec = {"workload": name, "config": decode_config(w, args, R, world), "ms_per_step": m["ms"],
            "value": w.B * w.Hq * world / (m["ms"] * 1e-3), "unit": "query-heads/s",
            "hbm_gbs": hbm, "hbm_bytes_per_step": by["total"], "step_frac": hbm / peak,
-           "roofline": decode_roofline(by, m, peak, peak_kind),
+           "roofline": decode_roofline(by, m, peak, peak_kind, traffic_key(w)),
            "calls_ms": decode_calls(by, m, peak),
            "traffic": traffic_ratios(w, m["idx0"], m["idx_a0"], args.variance, args.rank, args.sub),
            "gpu_launches": m["launches_per_step"] * steps, "steps": steps, "device_error": m["device_error"]}
@@ -807,7 +812,7 @@ def run_ours(args):
         "hbm_gbs": by["total"] / (ms * 1e-3) / 1e9,
         "hbm_bytes_per_step": by["total"],
         "step_frac": by["total"] / (ms * 1e-3) / 1e9 / peak,
-        "roofline": decode_roofline(by, m, peak, peak_kind),
+        "roofline": decode_roofline(by, m, peak, peak_kind, traffic_key(w)),
         "calls_ms": decode_calls(by, m, peak),
         "traffic": traffic_ratios(w, idx0, m["idx_a0"], args.variance, args.rank, args.sub),
         "e2e": {"value": qheads / (e2e["ms"] * 1e-3), "unit": "query-heads/s", "h2d_bytes_per_step": e2e["h2d"],
@@ -1015,7 +1020,7 @@ def run_sweep(args):
                        "recall_on": f"first {n_rec} sequences x {base.Hkv} KV heads"},
             "roofline": {"bound": "hbm", "kernel": "select_decode_kernel", "achieved": top["gbs"], "peak": peak,
                          "unit": "GB/s", "frac": top["frac"], "peak_kind": peak_kind,
-                         "traffic": recorded_traffic("select_decode")},
+                         "traffic": recorded_traffic("select_decode", "sweep")},
             "sweep": rows, "gpu_launches": sum(r["gpu_launches"] for r in rows), "device_error": cobs.device_error()}
     if rank == 0:
         print(json.dumps(line), flush=True)
