@@ -571,7 +571,9 @@ def measure_decode(w, args, dev, cobs, world, R, steps, warmup, with_e2e=True, c
                     e = evs_[r]
                     out.append([e[j].elapsed_time(e[j + 1]) for j in range(nparts)])
         del graphs_
-        return [statistics.median(x[j] for x in out) for j in range(nparts)]
+        # the mean, not the median: event pairs recorded inside a graph resolve about 2 us, so
+        # single samples fall on that grid and only their mean resolves the launch's duration
+        return [statistics.fmean(x[j] for x in out) for j in range(nparts)]
 
     def upd(r):
         return lambda: cobs.cobs_build_summaries(p, Ks[r], Vs[r], tPk, tPv, w.T - 1, bufs[r].summaries, bufs[r].Kc,
@@ -716,7 +718,7 @@ def decode_roofline(by, m, peak, peak_kind, workload):
             "achieved": att_gbs, "peak": peak, "unit": "GB/s", "frac": att_gbs / peak,
             "peak_kind": f"{peak_kind} (copy, read + write)", "algorithmic_bytes_per_launch": by["attn"],
             "timing": "CUDA events around cobs_sparse_attn_decode alone (graph per copy, replayed on the "
-                      "launching stream, median)",
+                      "launching stream, mean over the timed replays)",
             "traffic": recorded_traffic("decode_attention", workload)}
 
 
