@@ -96,7 +96,7 @@ constexpr int kLrIters = 24;
 constexpr int kLrMaxR = 8;
 constexpr int kLrThreadsWide = 512;
 constexpr int kLrThreadsNarrow = 128;
-constexpr int kLrPitch = 4;  // Y rows padded by 4 floats: the lanes of a product read distinct banks
+constexpr int kLrPitch = 4;  // Y rows padded by 4 floats: T = Y V reads distinct banks, W = Yt T two lanes a bank
 
 // Chain q of the four-chain dots of one row x (stride sx) against the R columns of a
 // row-major [n][kLrMaxR] matrix y (16-byte aligned rows): s[jj] = fma over the terms i = q,
