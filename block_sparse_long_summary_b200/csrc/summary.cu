@@ -185,18 +185,16 @@ __device__ __forceinline__ int e2m1_code(float x) {
 // (projections on columns 0, 1, ... in turn, then the normalisation), so the result is the
 // same bit for bit; the dots of the later columns against column i are independent, so their
 // butterflies run side by side.
-template <int D>
-__device__ __forceinline__ void lr_orthonormalize(const float (*W)[kLrMaxR + 1], float (*V)[kLrMaxR], int R,
-                                                  int lane) {
+template <int D, int R>
+__device__ __forceinline__ void lr_orthonormalize_r(const float (*W)[kLrMaxR + 1], float (*V)[kLrMaxR], int lane) {
     constexpr int kPer = D / 32;
-    float w[kLrMaxR][kPer];
+    float w[R][kPer];
 #pragma unroll
-    for (int jj = 0; jj < kLrMaxR; ++jj)
+    for (int jj = 0; jj < R; ++jj)
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) w[jj][q] = jj < R ? W[lane + 32 * q][jj] : 0.0f;
+        for (int q = 0; q < kPer; ++q) w[jj][q] = W[lane + 32 * q][jj];
 #pragma unroll
-    for (int i = 0; i < kLrMaxR; ++i) {
-        if (i >= R) break;
+    for (int i = 0; i < R; ++i) {
         float nn = 0.0f;
 #pragma unroll
         for (int q = 0; q < kPer; ++q) nn = __fmaf_rn(w[i][q], w[i][q], nn);
@@ -205,9 +203,9 @@ __device__ __forceinline__ void lr_orthonormalize(const float (*W)[kLrMaxR + 1],
         const float n = __fsqrt_rn(nn);
 #pragma unroll
         for (int q = 0; q < kPer; ++q) w[i][q] = n > 0.0f ? __fdiv_rn(w[i][q], n) : 0.0f;
-        float p[kLrMaxR];
+        float p[R];
 #pragma unroll
-        for (int jj = i + 1; jj < kLrMaxR; ++jj) {
+        for (int jj = i + 1; jj < R; ++jj) {
             p[jj] = 0.0f;
 #pragma unroll
             for (int q = 0; q < kPer; ++q) p[jj] = __fmaf_rn(w[i][q], w[jj][q], p[jj]);
@@ -215,17 +213,33 @@ __device__ __forceinline__ void lr_orthonormalize(const float (*W)[kLrMaxR + 1],
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-            for (int jj = i + 1; jj < kLrMaxR; ++jj) p[jj] = __fadd_rn(p[jj], __shfl_xor_sync(0xffffffffu, p[jj], o));
+            for (int jj = i + 1; jj < R; ++jj) p[jj] = __fadd_rn(p[jj], __shfl_xor_sync(0xffffffffu, p[jj], o));
 #pragma unroll
-        for (int jj = i + 1; jj < kLrMaxR; ++jj)
+        for (int jj = i + 1; jj < R; ++jj)
 #pragma unroll
             for (int q = 0; q < kPer; ++q) w[jj][q] = __fmaf_rn(-p[jj], w[i][q], w[jj][q]);
     }
 #pragma unroll
-    for (int jj = 0; jj < kLrMaxR; ++jj)
+    for (int jj = 0; jj < R; ++jj)
 #pragma unroll
-        for (int q = 0; q < kPer; ++q)
-            if (jj < R) V[lane + 32 * q][jj] = w[jj][q];
+        for (int q = 0; q < kPer; ++q) V[lane + 32 * q][jj] = w[jj][q];
+}
+
+// The rank is a launch argument (1..kLrMaxR); each rank gets its own fully unrolled routine, so
+// that no dot, shuffle or update is spent on columns past R.
+template <int D>
+__device__ __forceinline__ void lr_orthonormalize(const float (*W)[kLrMaxR + 1], float (*V)[kLrMaxR], int R,
+                                                  int lane) {
+    switch (R) {
+        case 1: lr_orthonormalize_r<D, 1>(W, V, lane); break;
+        case 2: lr_orthonormalize_r<D, 2>(W, V, lane); break;
+        case 3: lr_orthonormalize_r<D, 3>(W, V, lane); break;
+        case 4: lr_orthonormalize_r<D, 4>(W, V, lane); break;
+        case 5: lr_orthonormalize_r<D, 5>(W, V, lane); break;
+        case 6: lr_orthonormalize_r<D, 6>(W, V, lane); break;
+        case 7: lr_orthonormalize_r<D, 7>(W, V, lane); break;
+        default: lr_orthonormalize_r<D, kLrMaxR>(W, V, lane); break;
+    }
 }
 
 template <typename T, int D, int NT>
